@@ -1,0 +1,356 @@
+"""Benchmark of the GALE 1-bit MoE expert layer on B200.
+
+Workload: one routed-expert MoE layer at decode batch 1 -- 256 GALE-1bit
+SwiGLU experts, w1/w3 [2048 x 4096], w2 [4096 x 2048] (about 1.07 GB packed,
+all resident), top-6 routing with gates softmax-normalised over the selected
+six, bf16 hidden states N(0,1) [1 x 4096].  A step is one gale_moe_forward
+call: routing permute, FWHT of x, fused w1/w3 GEMV + SwiGLU, FWHT of h, w2
+GEMV, gate-weighted combine.  Every step uses a fresh routing from a seeded
+pool, and L2 is flushed (a write larger than L2) between timed steps, outside
+the timed events.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+For N > 1 launch under torch.distributed.run: every rank runs its own replica
+(weak scaling, no collective on the data path); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gale_synth as gs  # noqa: E402
+
+METRIC = "MoE expert-layer tokens/s and packed-expert HBM GB/s (% of B200 roofline)"
+UNIT = "tokens/s"
+D_MODEL, D_FF, N_EXPERTS, TOP_K = 4096, 2048, 256, 6
+WORKLOAD = ("moe_layer_decode: 256 GALE-1bit experts (w1/w3 [2048x4096], w2 [4096x2048]), "
+            "top-6 softmax routing, bf16 hidden [B x 4096]")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ----------------------------------------------------------------------------
+# clocks sampling (nvidia-smi during the timed region)
+# ----------------------------------------------------------------------------
+
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader",
+                                          "-i", str(self.index), "-lms", "200"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1].split()[0]))
+                    smax.append(float(parts[2].split()[0]))
+                except ValueError:
+                    continue
+                for n, v in zip(names[1:], parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# the layer on the device
+# ----------------------------------------------------------------------------
+
+def build_layer(torch, G, layer_id: int = 0):
+    """Pack 256 seeded experts into one resident device buffer (gale_pack)."""
+    stride = G.gale_expert_bytes(D_MODEL, D_FF)
+    buf = torch.empty(N_EXPERTS * stride, dtype=torch.uint8, device="cuda")
+    l1 = G.gale_pack_layout(D_FF, D_MODEL)["total"]
+    offs = [0, l1, 2 * l1]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for e in range(N_EXPERTS):
+        for m, c in enumerate(gs.expert_canonical(D_MODEL, D_FF, layer=layer_id, expert=e)):
+            dev = {k: torch.from_numpy(np.ascontiguousarray(v)).cuda()
+                   for k, v in (("signs", c["signs"]), ("s_blk", c["s_blk"].view(np.uint16)),
+                                ("s_row", c["s_row"].view(np.uint16)), ("idx", c["idx"]), ("q", c["q"]))}
+            G.gale_pack(dev["signs"], dev["s_blk"], dev["s_row"], dev["idx"], dev["q"], c["rows"], c["cols"],
+                        buf[e * stride + offs[m]:], status)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError("gale_pack reported invalid outliers")
+    return buf, stride
+
+
+def routing_pool(n: int, B: int, tag0: int):
+    pool = []
+    for i in range(n):
+        lg = gs.router_logits(B, N_EXPERTS, tag=tag0 + i)
+        ids, gates = gs.route_topk(lg, TOP_K)
+        bits, _ = gs.hidden_bf16(B, D_MODEL, tag=tag0 + i)
+        pool.append((bits, ids, gates, len(np.unique(ids))))
+    return pool
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import bit_expert_gemv_b200 as G
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
+    G.lib()
+    buf, stride = build_layer(torch, G)
+    layer = G.make_layer(buf, stride, N_EXPERTS, D_MODEL, D_FF)
+    expert_bytes = stride
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size if hasattr(
+        torch.cuda.get_device_properties(local), "L2_cache_size") else 126 * 2 ** 20
+    flush = torch.empty(max(2 * l2, 256 * 2 ** 20), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def measure(B, steps, warmup, tag0):
+        pool = routing_pool(steps + warmup, B, tag0 + 7919 * rank)
+        dev = [(torch.from_numpy(b).view(torch.bfloat16).cuda(), torch.from_numpy(i).cuda(),
+                torch.from_numpy(g).cuda(), nd) for b, i, g, nd in pool]
+        ws = torch.empty(G.gale_moe_workspace_size(layer, B, TOP_K), dtype=torch.uint8, device="cuda")
+        out = torch.empty(B, D_MODEL, dtype=torch.float32, device="cuda")
+        for s in range(warmup):
+            x, ids, gates, _ = dev[s]
+            G.gale_moe_forward(layer, x, ids, gates, out, ws)
+        torch.cuda.synchronize()
+        if int(ws[:4].view(torch.int32).item()) != 0:
+            raise RuntimeError("device status after warm-up")
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for s in range(steps):
+            x, ids, gates, _ = dev[warmup + s]
+            flush.zero_()
+            ev[s][0].record(stream)
+            G.gale_moe_forward(layer, x, ids, gates, out, ws)
+            ev[s][1].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        times = [a.elapsed_time(b) * 1e-3 for a, b in ev]
+        total = sum(times)
+        n_bytes = sum(dev[warmup + s][3] for s in range(steps)) * expert_bytes
+        return total, n_bytes, times
+
+    def measure_e2e(B, steps, warmup, tag0):
+        """Through the public API with host buffers: pinned H2D of x, ids and
+        gates, the layer, and a D2H of the output, every step."""
+        pool = routing_pool(steps + warmup, B, tag0 + 7919 * rank)
+        host = [(torch.from_numpy(b).view(torch.bfloat16).pin_memory(), torch.from_numpy(i).pin_memory(),
+                 torch.from_numpy(g).pin_memory()) for b, i, g, _ in pool]
+        xd = torch.empty(B, D_MODEL, dtype=torch.bfloat16, device="cuda")
+        idd = torch.empty(B, TOP_K, dtype=torch.int32, device="cuda")
+        gd = torch.empty(B, TOP_K, dtype=torch.float32, device="cuda")
+        ws = torch.empty(G.gale_moe_workspace_size(layer, B, TOP_K), dtype=torch.uint8, device="cuda")
+        out = torch.empty(B, D_MODEL, dtype=torch.float32, device="cuda")
+        out_h = torch.empty(B, D_MODEL, dtype=torch.float32).pin_memory()
+
+        def step(s):
+            x, i, g = host[s]
+            xd.copy_(x, non_blocking=True)
+            idd.copy_(i, non_blocking=True)
+            gd.copy_(g, non_blocking=True)
+            G.gale_moe_forward(layer, xd, idd, gd, out, ws)
+            out_h.copy_(out, non_blocking=True)
+
+        for s in range(warmup):
+            step(s)
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for s in range(steps):
+            flush.zero_()
+            ev[s][0].record(stream)
+            step(warmup + s)
+            ev[s][1].record(stream)
+        torch.cuda.synchronize()
+        total = sum(a.elapsed_time(b) * 1e-3 for a, b in ev)
+        h2d = B * D_MODEL * 2 + B * TOP_K * 4 * 2
+        d2h = B * D_MODEL * 4
+        return total, h2d, d2h
+
+    clocks = Clocks(local)
+    clocks.start()
+    t1, bytes1, times1 = measure(1, args.steps, args.warmup, 10_000)
+    clocks_info = clocks.stop()
+    t8, bytes8, _ = measure(8, max(args.steps // 2, 3), args.warmup, 20_000)
+    te, h2d, d2h = measure_e2e(1, args.steps, args.warmup, 30_000)
+
+    # max over ranks of the device time
+    tt = torch.tensor([t1, t8, te], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    t1, t8, te = [float(v) for v in tt.tolist()]
+    tokens = 1 * args.steps * world
+    value = tokens / t1
+    gbs = bytes1 * world / t1 / 1e9
+    peak, peak_kind = peaks()
+    avg_launch = t1 / args.steps
+    achieved = bytes1 / args.steps / avg_launch / 1e9
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * t1 / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": 1, "experts": N_EXPERTS, "top_k": TOP_K,
+                   "d_model": D_MODEL, "d_ff": D_FF, "packed_bytes_per_expert": expert_bytes,
+                   "l2": "flushed between timed steps (write of 2x L2, outside the events)",
+                   "routing": "fresh seeded routing every step", "parallelism": f"replicas{world}"},
+        "hbm_gbs": gbs,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                     "kernel": "gale_moe_forward (whole layer)"},
+        "b8": {"tokens_per_s": 8 * max(args.steps // 2, 3) * world / t8,
+               "hbm_gbs": bytes8 * world / t8 / 1e9, "frac": bytes8 * world / t8 / 1e9 / peak},
+        "e2e": {"value": tokens / te, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clocks_info,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timings
+# ----------------------------------------------------------------------------
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_step(O, B, tag):
+    lg = gs.router_logits(B, N_EXPERTS, tag=tag)
+    ids, gates = gs.route_topk(lg, TOP_K)
+    _, xv = gs.hidden_bf16(B, D_MODEL, tag=tag)
+    cache = {}
+
+    def dense(e):
+        if e not in cache:
+            cs = gs.expert_canonical(D_MODEL, D_FF, expert=e)
+            cache[e] = [O.dequant_packed(O.pack(c), c["rows"], c["cols"]) for c in cs]
+        return cache[e]
+
+    O.moe_layer(dense, xv, ids, gates)
+    return B
+
+
+def cpu_baseline(budget_s: float):
+    from oracle import gale_oracle as O
+    t0 = time.perf_counter()
+    toks = 0
+    n = 0
+    while time.perf_counter() - t0 < budget_s and n < 64:
+        toks += oracle_step(O, 1, 50_000 + n)
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": toks / dt, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": f"{n} decode-B1 layer steps (6 experts each, unpack + dense fp64 dequant + FWHT + "
+                      f"SwiGLU + combine), {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from oracle import gale_oracle as O
+    for s in range(args.warmup):
+        oracle_step(O, 1, 60_000 + s)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        oracle_step(O, 1, 70_000 + s)
+    dt = time.perf_counter() - t0
+    value = args.steps / dt
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": 1, "experts": N_EXPERTS, "top_k": TOP_K},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+                         "sample": f"{args.steps} decode-B1 layer steps"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="gale", choices=["gale", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

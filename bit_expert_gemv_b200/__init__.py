@@ -1,0 +1,191 @@
+"""Python binding of libgale, the sm_100a GALE 1-bit routed-expert library.
+
+Argument marshalling only: every function forwards torch tensors (device
+memory owned by the caller) as raw pointers to the C ABI declared in
+``include/gale.h``, under the same names.  There is no CPU fallback: if the
+library is missing, loading it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgale.so")
+
+GALE_OK = 0
+GALE_ERR_ARG = -1
+GALE_ERR_ALIGN = -2
+GALE_ERR_WORKSPACE = -3
+GALE_ERR_CUDA = -4
+GALE_ERR_TIMEOUT = -5
+GALE_ERR_UNSUPPORTED = -6
+
+GALE_F32, GALE_BF16, GALE_F16 = 0, 1, 2
+GALE_MODE_PLAIN, GALE_MODE_SWIGLU = 0, 1
+GALE_FLAG_RESIDUAL_RMSNORM = 1
+
+# every symbol include/gale.h declares
+EXPORTS = (
+    "gale_status_string", "gale_pack_layout", "gale_expert_bytes", "gale_pack", "gale_unpack",
+    "gale_fwht1024", "gale_expert_gemv", "gale_route_permute", "gale_moe_workspace_size",
+    "gale_moe_forward", "gale_selftest_scratch_bytes", "gale_selftest",
+)
+
+
+class GaleError(RuntimeError):
+    def __init__(self, code: int, where: str = ""):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)}" if where else status_string(code))
+
+
+class gale_layout(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int32), ("cols", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("offset", ctypes.c_int64 * 5),
+                ("size", ctypes.c_int64 * 5), ("total", ctypes.c_int64)]
+
+
+class gale_matrix(ctypes.Structure):
+    _fields_ = [("packed", ctypes.c_void_p), ("rows", ctypes.c_int32), ("cols", ctypes.c_int32)]
+
+
+class gale_layer(ctypes.Structure):
+    _fields_ = [("base", ctypes.c_void_p), ("expert_stride", ctypes.c_int64),
+                ("n_experts", ctypes.c_int32), ("d_model", ctypes.c_int32),
+                ("d_ff", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgale.so (built in-tree by ``bit_expert_gemv_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run `python -m bit_expert_gemv_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        sig = {
+            "gale_status_string": (ctypes.c_char_p, [i32]),
+            "gale_pack_layout": (i32, [i32, i32, ctypes.POINTER(gale_layout)]),
+            "gale_expert_bytes": (i64, [i32, i32]),
+            "gale_pack": (i32, [vp, vp, vp, vp, vp, i32, i32, vp, vp, vp]),
+            "gale_unpack": (i32, [vp, i32, i32, vp, vp]),
+            "gale_fwht1024": (i32, [vp, i32, vp, i32, i64, i32, vp]),
+            "gale_expert_gemv": (i32, [ctypes.POINTER(gale_matrix), ctypes.POINTER(gale_matrix), vp, i32,
+                                       vp, i32, vp]),
+            "gale_route_permute": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp]),
+            "gale_moe_workspace_size": (sz, [ctypes.POINTER(gale_layer), i32, i32]),
+            "gale_moe_forward": (i32, [ctypes.POINTER(gale_layer), vp, vp, vp, i32, i32, vp, i32, i32,
+                                       ctypes.c_float, vp, sz, vp]),
+            "gale_selftest_scratch_bytes": (sz, []),
+            "gale_selftest": (i32, [vp, vp]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().gale_status_string(int(code)).decode()
+
+
+def _check(rc: int, where: str):
+    if rc != GALE_OK:
+        raise GaleError(rc, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    return {torch.float32: GALE_F32, torch.bfloat16: GALE_BF16, torch.float16: GALE_F16}[t.dtype]
+
+
+# ----------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ----------------------------------------------------------------------------
+
+def gale_pack_layout(rows: int, cols: int) -> dict:
+    out = gale_layout()
+    _check(lib().gale_pack_layout(rows, cols, ctypes.byref(out)), "gale_pack_layout")
+    return {"rows": out.rows, "cols": out.cols, "k": out.k, "offsets": list(out.offset),
+            "sizes": list(out.size), "total": out.total}
+
+
+def gale_expert_bytes(d_model: int, d_ff: int) -> int:
+    return int(lib().gale_expert_bytes(d_model, d_ff))
+
+
+def gale_pack(signs, s_blk, s_row, idx, q, rows: int, cols: int, dst, status, stream=None):
+    _check(lib().gale_pack(_ptr(signs), _ptr(s_blk), _ptr(s_row), _ptr(idx), _ptr(q), rows, cols,
+                           _ptr(dst), _ptr(status), _stream(stream)), "gale_pack")
+
+
+def gale_unpack(packed, rows: int, cols: int, dense, stream=None):
+    _check(lib().gale_unpack(_ptr(packed), rows, cols, _ptr(dense), _stream(stream)), "gale_unpack")
+
+
+def gale_fwht1024(x, y, stream=None):
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols else 0
+    _check(lib().gale_fwht1024(_ptr(x), _dtype_code(x), _ptr(y), _dtype_code(y), rows, cols,
+                               _stream(stream)), "gale_fwht1024")
+
+
+def gale_expert_gemv(W, rows: int, cols: int, x_rot, y, W3=None, mode: int = GALE_MODE_PLAIN,
+                     stream=None):
+    a = gale_matrix(_ptr(W), rows, cols)
+    b = gale_matrix(_ptr(W3), rows, cols) if W3 is not None else None
+    ntok = x_rot.numel() // cols
+    _check(lib().gale_expert_gemv(ctypes.byref(a), ctypes.byref(b) if b is not None else None,
+                                  _ptr(x_rot), ntok, _ptr(y), mode, _stream(stream)), "gale_expert_gemv")
+
+
+def gale_route_permute(ids, n_experts: int, counts, offsets, perm, status, stream=None):
+    B, K = ids.shape
+    _check(lib().gale_route_permute(_ptr(ids), B, K, n_experts, _ptr(counts), _ptr(offsets), _ptr(perm),
+                                    _ptr(status), _stream(stream)), "gale_route_permute")
+
+
+def make_layer(base, expert_stride: int, n_experts: int, d_model: int, d_ff: int) -> gale_layer:
+    return gale_layer(_ptr(base), expert_stride, n_experts, d_model, d_ff, 0)
+
+
+def gale_moe_workspace_size(layer: gale_layer, B: int, K: int) -> int:
+    return int(lib().gale_moe_workspace_size(ctypes.byref(layer), B, K))
+
+
+def gale_moe_forward(layer: gale_layer, x, ids, gates, out, ws, flags: int = 0, eps: float = 1e-6,
+                     stream=None):
+    B, K = ids.shape
+    _check(lib().gale_moe_forward(ctypes.byref(layer), _ptr(x), _ptr(ids), _ptr(gates), B, K, _ptr(out),
+                                  _dtype_code(out), flags, eps, _ptr(ws), ws.numel() * ws.element_size(),
+                                  _stream(stream)), "gale_moe_forward")
+
+
+def gale_selftest_scratch_bytes() -> int:
+    return int(lib().gale_selftest_scratch_bytes())
+
+
+def gale_selftest(scratch, stream=None) -> int:
+    return int(lib().gale_selftest(_ptr(scratch), _stream(stream)))

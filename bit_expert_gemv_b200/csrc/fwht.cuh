@@ -1,0 +1,31 @@
+// Unnormalised Walsh-Hadamard butterflies over one 1024-block held by a warp:
+// v[i] of lane l is element 32*i + l.  Natural (Sylvester) order.
+#pragma once
+
+namespace gale {
+
+__device__ __forceinline__ void fwht1024_warp(float (&v)[32], int lane) {
+    // strides 1..16: partner lane differs in bit s
+#pragma unroll
+    for (int s = 0; s < 5; ++s) {
+        const bool upper = (lane >> s) & 1;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            float o = __shfl_xor_sync(0xffffffffu, v[i], 1 << s);
+            v[i] = upper ? (o - v[i]) : (v[i] + o);
+        }
+    }
+    // strides 32..512: partner register differs in bit s
+#pragma unroll
+    for (int s = 0; s < 5; ++s) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (i & (1 << s)) continue;
+            float a = v[i], b = v[i | (1 << s)];
+            v[i] = a + b;
+            v[i | (1 << s)] = a - b;
+        }
+    }
+}
+
+}  // namespace gale

@@ -1,0 +1,249 @@
+// gale_moe_forward: one routed-expert layer,
+//   y[t] = sum_k gates[t,k] * W2_e H( silu(W1_e H x[t]) * (W3_e H x[t]) ),  e = ids[t,k]
+// (SwiGLU experts over GALE 1-bit packed records, top-K routing).
+//
+// Stages: routing permute -> FWHT(x) -> grouped w1/w3 GEMV + SwiGLU ->
+// FWHT(h) -> grouped w2 GEMV -> deterministic gate-weighted combine in fixed
+// k order (optionally + residual and RMSNorm).
+#include "common.cuh"
+#include "gemv_simple.cuh"
+#include "moe.cuh"
+#include "route.cuh"
+
+namespace gale {
+
+constexpr int kGWarps = 8;
+constexpr int kGRowsPerWarp = 8;
+constexpr int kGRowsPerCta = kGWarps * kGRowsPerWarp;
+
+MoeWs carve_ws(void* ws, const gale_layer& L, int B, int K) {
+    MoeWs w{};
+    char* p = static_cast<char*>(ws);
+    int64_t o = 0;
+    auto take = [&](int64_t bytes) {
+        char* q = p ? p + o : nullptr;
+        o = align_up(o + bytes, 256);
+        return q;
+    };
+    const int64_t BK = int64_t(B) * K;
+    w.status = reinterpret_cast<int32_t*>(take(256));
+    w.counts = reinterpret_cast<int32_t*>(take(4 * int64_t(L.n_experts)));
+    w.offsets = reinterpret_cast<int32_t*>(take(4 * (int64_t(L.n_experts) + 1)));
+    w.perm = reinterpret_cast<int32_t*>(take(4 * BK));
+    w.pos_of_pair = reinterpret_cast<int32_t*>(take(4 * BK));
+    w.active = reinterpret_cast<int32_t*>(take(4 * int64_t(L.n_experts)));
+    w.n_active = reinterpret_cast<int32_t*>(take(4));
+    w.x_rot = reinterpret_cast<float*>(take(4 * int64_t(B) * L.d_model));
+    w.h = reinterpret_cast<float*>(take(4 * BK * L.d_ff));
+    w.o = reinterpret_cast<float*>(take(4 * BK * L.d_model));
+    w.bytes = size_t(o);
+    return w;
+}
+
+// Grouped GEMV: CTA (row tile, active slot).  The slot's expert e processes
+// its pairs in permuted order; w1/w3 read x_rot of the pair's token, w2 reads
+// the pair's own rotated hidden row.
+template <bool SWIGLU>
+__global__ void __launch_bounds__(256) moe_group_gemv_kernel(GroupArgs g) {
+    extern __shared__ float xs[];
+    const int slot = blockIdx.y;
+    if (slot >= *g.n_active) return;
+    const int e = g.active[slot];
+    const int n_e = g.counts[e];
+    const int off = g.offsets[e];
+    const char* rec = static_cast<const char*>(g.base) + int64_t(e) * g.expert_stride;
+    const MatView a = make_view(rec + g.mat_off_a, g.rows, g.cols);
+    const MatView b = make_view(rec + g.mat_off_b, g.rows, g.cols);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int cols = g.cols;
+    for (int t0 = 0; t0 < n_e; t0 += g.chunk) {
+        const int nt = min(g.chunk, n_e - t0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < nt * cols; i += blockDim.x) {
+            const int ti = i / cols, c = i - ti * cols;
+            const int64_t src_row = SWIGLU ? int64_t(g.perm[off + t0 + ti] / g.K) : int64_t(off + t0 + ti);
+            xs[i] = g.x[src_row * cols + c];
+        }
+        __syncthreads();
+        for (int i = 0; i < kGRowsPerWarp; ++i) {
+            const int r = blockIdx.x * kGRowsPerCta + i * kGWarps + warp;
+            if (r >= g.rows) break;
+            float acc[kSimpleNT];
+            row_dot_simple(a, r, xs, nt, acc, lane);
+            if (SWIGLU) {
+                float acc3[kSimpleNT];
+                row_dot_simple(b, r, xs, nt, acc3, lane);
+#pragma unroll
+                for (int t = 0; t < kSimpleNT; ++t) acc[t] = silu(acc[t]) * acc3[t];
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int t = 0; t < kSimpleNT; ++t)
+                    if (t < nt) g.out[int64_t(off + t0 + t) * g.rows + r] = acc[t];
+            }
+        }
+    }
+}
+
+// One CTA per token: y = sum_k gates[t,k] * o[pos(t,k)] in fixed k order,
+// then either stored, or v = x + y normalised (RMSNorm, unit weight) to bf16.
+__global__ void __launch_bounds__(256) moe_combine_kernel(CombineArgs c) {
+    extern __shared__ float red[];
+    const int t = blockIdx.x;
+    const int d = c.d_model;
+    float ss = 0.f;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+        float y = 0.f;
+        for (int k = 0; k < c.K; ++k) {
+            const int pos = c.pos_of_pair[t * c.K + k];
+            if (pos >= 0) y = fmaf(c.gates[t * c.K + k], c.o[int64_t(pos) * d + i], y);
+        }
+        if (c.fuse_norm) {
+            const float v = bf16_to_f32(c.x[int64_t(t) * d + i]) + y;
+            c.scratch[int64_t(t) * d + i] = v;
+            ss = fmaf(v, v, ss);
+        } else {
+            store_from_f32(c.out, c.out_dtype, int64_t(t) * d + i, y);
+        }
+    }
+    if (!c.fuse_norm) return;
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+        v = warp_sum(v);
+        if (threadIdx.x == 0) red[0] = v;
+    }
+    __syncthreads();
+    const float inv = rsqrtf(red[0] / float(d) + c.eps);
+    for (int i = threadIdx.x; i < d; i += blockDim.x)
+        store_from_f32(c.out, GALE_BF16, int64_t(t) * d + i, c.scratch[int64_t(t) * d + i] * inv);
+}
+
+int validate_layer(const gale_layer* L) {
+    if (!L || !L->base || L->n_experts < 1 || L->n_experts > 1024) return GALE_ERR_ARG;
+    if (!valid_cols(L->d_model) || !valid_cols(L->d_ff) || L->d_model > 16384 || L->d_ff > 16384)
+        return GALE_ERR_ARG;
+    const int64_t eb = 2 * make_layout(L->d_ff, L->d_model).total + make_layout(L->d_model, L->d_ff).total;
+    if (L->expert_stride < eb || L->expert_stride % 256) return GALE_ERR_ARG;
+    if (!aligned(L->base, 256)) return GALE_ERR_ALIGN;
+    return GALE_OK;
+}
+
+int launch_group_gemv(bool swiglu, GroupArgs g, int max_slots, cudaStream_t st) {
+    const int chunk_cap = int((200 * 1024) / (int64_t(g.cols) * 4));
+    g.chunk = chunk_cap < 1 ? 1 : (chunk_cap > kSimpleNT ? kSimpleNT : chunk_cap);
+    const size_t smem = size_t(g.chunk) * g.cols * sizeof(float);
+    dim3 grid((g.rows + kGRowsPerCta - 1) / kGRowsPerCta, max_slots);
+    if (swiglu) {
+        GALE_CUDA_TRY(cudaFuncSetAttribute(moe_group_gemv_kernel<true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+        moe_group_gemv_kernel<true><<<grid, 256, smem, st>>>(g);
+    } else {
+        GALE_CUDA_TRY(cudaFuncSetAttribute(moe_group_gemv_kernel<false>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+        moe_group_gemv_kernel<false><<<grid, 256, smem, st>>>(g);
+    }
+    GALE_LAUNCH_CHECK();
+    return GALE_OK;
+}
+
+}  // namespace gale
+
+extern "C" size_t gale_moe_workspace_size(const gale_layer* layer, int B, int K) {
+    if (gale::validate_layer(layer) == GALE_ERR_ARG || B < 0 || K < 1 || K > 16) return 0;
+    return gale::carve_ws(nullptr, *layer, B, K).bytes;
+}
+
+extern "C" int gale_moe_forward(const gale_layer* layer, const uint16_t* x, const int32_t* ids,
+                                const float* gates, int B, int K, void* out, int out_dtype, int flags,
+                                float eps, void* ws, size_t ws_bytes, void* stream) {
+    using namespace gale;
+    int rc = validate_layer(layer);
+    if (rc != GALE_OK) return rc;
+    if (B < 0 || K < 1 || K > 16 || K > layer->n_experts) return GALE_ERR_ARG;
+    if (flags & ~GALE_FLAG_RESIDUAL_RMSNORM) return GALE_ERR_ARG;
+    const bool fuse = flags & GALE_FLAG_RESIDUAL_RMSNORM;
+    if (out_dtype != GALE_F32 && out_dtype != GALE_BF16) return GALE_ERR_ARG;
+    if (fuse && (out_dtype != GALE_BF16 || !(eps >= 0.f))) return GALE_ERR_ARG;
+    if (!ws) return GALE_ERR_WORKSPACE;
+    const gale_layer& L = *layer;
+    MoeWs w = carve_ws(ws, L, B, K);
+    if (ws_bytes < w.bytes) return GALE_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return GALE_ERR_ALIGN;
+    cudaStream_t st = as_stream(stream);
+    GALE_CUDA_TRY(cudaMemsetAsync(w.status, 0, sizeof(int32_t), st));
+    if (B == 0) return GALE_OK;
+    if (!x || !ids || !gates || !out) return GALE_ERR_ARG;
+    if (!aligned(x, 4) || !aligned(ids, 4) || !aligned(gates, 4) || !aligned(out, 4)) return GALE_ERR_ALIGN;
+    const int64_t BK = int64_t(B) * K;
+    if (BK > (1 << 24)) return GALE_ERR_UNSUPPORTED;
+
+    GALE_CUDA_TRY(cudaMemsetAsync(w.pos_of_pair, 0xFF, size_t(BK) * 4, st));
+    RouteArgs ra{};
+    ra.ids = ids;
+    ra.B = B;
+    ra.K = K;
+    ra.E = L.n_experts;
+    ra.counts = w.counts;
+    ra.offsets = w.offsets;
+    ra.perm = w.perm;
+    ra.pos_of_pair = w.pos_of_pair;
+    ra.active = w.active;
+    ra.n_active = w.n_active;
+    ra.status = w.status;
+    rc = launch_route_permute(ra, st);
+    if (rc != GALE_OK) return rc;
+
+    rc = gale_fwht1024(x, GALE_BF16, w.x_rot, GALE_F32, B, L.d_model, stream);
+    if (rc != GALE_OK) return rc;
+
+    const int64_t w1_bytes = make_layout(L.d_ff, L.d_model).total;
+    const int max_slots = int(BK < L.n_experts ? BK : L.n_experts);
+    GroupArgs g{};
+    g.base = L.base;
+    g.expert_stride = L.expert_stride;
+    g.counts = w.counts;
+    g.offsets = w.offsets;
+    g.perm = w.perm;
+    g.active = w.active;
+    g.n_active = w.n_active;
+    g.K = K;
+    g.rows = L.d_ff;
+    g.cols = L.d_model;
+    g.mat_off_a = 0;
+    g.mat_off_b = w1_bytes;
+    g.x = w.x_rot;
+    g.out = w.h;
+    rc = launch_group_gemv(true, g, max_slots, st);
+    if (rc != GALE_OK) return rc;
+
+    rc = gale_fwht1024(w.h, GALE_F32, w.h, GALE_F32, BK, L.d_ff, stream);
+    if (rc != GALE_OK) return rc;
+
+    g.rows = L.d_model;
+    g.cols = L.d_ff;
+    g.mat_off_a = 2 * w1_bytes;
+    g.mat_off_b = 2 * w1_bytes;
+    g.x = w.h;
+    g.out = w.o;
+    rc = launch_group_gemv(false, g, max_slots, st);
+    if (rc != GALE_OK) return rc;
+
+    CombineArgs c{};
+    c.o = w.o;
+    c.pos_of_pair = w.pos_of_pair;
+    c.gates = gates;
+    c.x = x;
+    c.K = K;
+    c.d_model = L.d_model;
+    c.out = out;
+    c.out_dtype = out_dtype;
+    c.fuse_norm = fuse;
+    c.eps = eps;
+    c.scratch = w.x_rot;   // x_rot is dead by now; reused for v = x + y
+    moe_combine_kernel<<<B, 256, 32 * sizeof(float), st>>>(c);
+    GALE_LAUNCH_CHECK();
+    return GALE_OK;
+}

@@ -1,0 +1,220 @@
+/*
+ * gale.h -- C ABI of libgale, the sm_100a (B200) implementation of the
+ * decode-time GALE 1-bit routed-expert forward.
+ *
+ * The format (DeepSeek-V4-Flash -- GALE 1-bit experts, "What is in the pack",
+ * routed-experts row; the same on the DeepSeek-V4-Pro-671B-GALE-1bit-v4 card,
+ * weights table): every expert matrix W [rows x cols] is stored in the domain
+ * rotated by a blocked FWHT-1024 along its input dimension (cols), as one sign
+ * bit per weight, one fp16 scale per 128-weight block along the row, and 1 %
+ * of the columns of every row as int4 outliers with a per-row fp16 scale.
+ * The outlier value replaces the signed weight at its column.
+ *
+ * Conventions shared by every entry point
+ *  - C linkage, no exceptions, no exit().  Every call returns an int status:
+ *    GALE_OK (0) or a negative GALE_ERR_* code.
+ *  - All memory is owned by the caller.  Pointers named "device" must point
+ *    to CUDA device memory of the current device; nothing is allocated or
+ *    freed by the library, which keeps only a per-device attribute cache.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous on that stream unless stated; launch
+ *    failures return GALE_ERR_CUDA.  Errors found on the device (bad expert
+ *    ids, unsorted outlier columns) are written to a caller-provided int32
+ *    status word in device memory, which the caller reads after the stream
+ *    has been synchronised.  The library never traps a kernel.
+ *  - Dtype codes: GALE_F32, GALE_BF16, GALE_F16.  All multi-byte values are
+ *    little-endian.
+ */
+#ifndef GALE_H
+#define GALE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define GALE_OK               0
+#define GALE_ERR_ARG         -1   /* invalid argument or device-detected invalid input */
+#define GALE_ERR_ALIGN       -2   /* a pointer lacks the alignment the call needs */
+#define GALE_ERR_WORKSPACE   -3   /* workspace missing or too small */
+#define GALE_ERR_CUDA        -4   /* a CUDA runtime call or launch failed */
+#define GALE_ERR_TIMEOUT     -5   /* a bounded device-side wait ran out */
+#define GALE_ERR_UNSUPPORTED -6   /* shape or device not supported */
+
+/* element types */
+#define GALE_F32  0
+#define GALE_BF16 1
+#define GALE_F16  2
+
+/* gale_expert_gemv modes */
+#define GALE_MODE_PLAIN  0        /* y = Q(W) x_rot */
+#define GALE_MODE_SWIGLU 1        /* y = silu(Q(W) x_rot) * (Q(W3) x_rot) */
+
+/* gale_moe_forward flags */
+#define GALE_FLAG_RESIDUAL_RMSNORM 1  /* out = bf16(RMSNorm(x + y)), unit weight */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gale_status_string(int status);
+
+/* ---------------------------------------------------------------------------
+ * Packed-matrix layout.
+ *
+ * A packed matrix of `rows` x `cols` weights (cols a multiple of 1024, which
+ * is also a multiple of the 128-weight scale block) holds five sections, each
+ * starting on a 256-byte boundary (the manifest of the pack records "sections"
+ * per matrix: DeepSeek-V4-Flash -- GALE 1-bit experts, "Files"):
+ *   0 signs : rows*cols/8 bytes of uint32 words, row-major; column c of row r
+ *             is bit (c % 32) of word r*(cols/32) + c/32; a set bit means -1.
+ *   1 s_blk : fp16 [rows][cols/128], the scale of weights 128b..128b+127.
+ *   2 s_row : fp16 [rows], the outlier scale of each row.
+ *   3 idx   : uint16 [rows][k], outlier columns, strictly ascending per row.
+ *   4 q     : int4 two's complement; value j of row r is nibble n = r*k + j,
+ *             stored in byte n/2, low nibble first.
+ * k = nearest integer to cols/100 (41 for 4096 columns, 20 for 2048): the
+ * count that reproduces the card's 1.329 bits/weight and 46.0 GB.  Sign bits
+ * under outlier columns are stored and ignored.  An expert record is
+ * w1 || w3 || w2 (w1, w3: [d_ff x d_model], w2: [d_model x d_ff]), with no
+ * padding between matrices.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+    int32_t rows;
+    int32_t cols;
+    int32_t k;            /* outliers per row */
+    int32_t reserved;
+    int64_t offset[5];    /* byte offset of each section from the record start */
+    int64_t size[5];      /* byte size of each section (without padding) */
+    int64_t total;        /* bytes of the whole matrix record (256-aligned) */
+} gale_layout;
+
+/* Fills *out for a rows x cols matrix.  Host only, no CUDA call.
+ * Errors: GALE_ERR_ARG if out is NULL, rows < 1, cols < 1024,
+ * cols % 1024 != 0 or cols > 65536 (idx is uint16). */
+int gale_pack_layout(int rows, int cols, gale_layout* out);
+
+/* Bytes of one expert record w1 || w3 || w2, or 0 on invalid sizes. */
+int64_t gale_expert_bytes(int d_model, int d_ff);
+
+/* Packs a matrix from canonical unpacked device arrays into `dst` (device,
+ * gale_layout.total bytes, 16-byte aligned; padding bytes are zeroed):
+ *   signs uint8 [rows][cols] (0 = +1, nonzero = -1), s_blk fp16 bits
+ *   [rows][cols/128], s_row fp16 bits [rows], idx uint16 [rows][k],
+ *   q int8 [rows][k] in [-8, 7].
+ * `status` (device int32) is set to 0 by the call, then to GALE_ERR_ARG by
+ * the kernel if any row's idx is not strictly ascending and < cols, or a q
+ * value is out of range; the bytes of such rows are then unspecified. */
+int gale_pack(const uint8_t* signs, const uint16_t* s_blk, const uint16_t* s_row,
+              const uint16_t* idx, const int8_t* q, int rows, int cols,
+              void* dst, int32_t* status, void* stream);
+
+/* Dense dequantisation Q(W_rot) of a packed matrix (device) into
+ * dense fp32 [rows][cols] (device): sign * s_blk, then outliers replaced by
+ * q * s_row.  Every value is exact in fp32.  Reads idx without validation:
+ * pass only records produced by gale_pack with status 0. */
+int gale_unpack(const void* packed, int rows, int cols, float* dense, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Blocked FWHT-1024 (the rotation; DeepSeek-V4-Pro-671B-GALE-1bit-v4 card,
+ * knobs paragraph, butterfly Walsh-Hadamard transform).
+ * y[r, 1024b + i] = (1/32) * sum_j H[i, j] * x[r, 1024b + j], H the Sylvester
+ * Hadamard matrix of order 1024 in natural order (H[i,j] = (-1)^popcount(i&j)).
+ * x: device [rows][cols] of x_dtype; y: device [rows][cols] of y_dtype
+ * (GALE_F32, GALE_BF16 or GALE_F16; the sums are taken in fp32 and rounded
+ * to y_dtype once).  y may alias x when the dtypes are equal.
+ * Errors: GALE_ERR_ARG for cols % 1024 != 0, rows < 0, bad dtypes;
+ * GALE_ERR_ALIGN for pointers not 4-byte aligned.  rows == 0 is a no-op.
+ * ------------------------------------------------------------------------- */
+int gale_fwht1024(const void* x, int x_dtype, void* y, int y_dtype, int64_t rows, int cols,
+                  void* stream);
+
+/* ---------------------------------------------------------------------------
+ * One packed matrix (or a SwiGLU w1/w3 pair) times rotated activations
+ * (DeepSeek-V4-Pro-671B-GALE-1bit-v4 card, knobs paragraph: the direct GEMV
+ * straight from the packed record, signs, block scales and int4 outliers
+ * decoded in registers).
+ * ------------------------------------------------------------------------- */
+typedef struct {
+    const void* packed;   /* device, 16-byte aligned record */
+    int32_t rows;
+    int32_t cols;
+} gale_matrix;
+
+/* x_rot: device fp32 [ntok][W.cols], already rotated (gale_fwht1024).
+ * y: device fp32 [ntok][W.rows].
+ * mode GALE_MODE_PLAIN : y = Q(W) x_rot (W3 must be NULL).
+ * mode GALE_MODE_SWIGLU: y = silu(Q(W) x_rot) * (Q(W3) x_rot), W3 of the
+ *                        same shape as W.
+ * 1 <= ntok <= 64.  Accumulation is fp32.
+ * Errors: GALE_ERR_ARG (shapes, mode, ntok), GALE_ERR_ALIGN. */
+int gale_expert_gemv(const gale_matrix* W, const gale_matrix* W3, const float* x_rot,
+                     int ntok, float* y, int mode, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Routing permute: groups the B*K (token, slot) pairs by expert, stable in
+ * pair order (pair index p = t*K + k).
+ *   ids    : device int32 [B][K], expert ids in [0, E), distinct within a token
+ *   counts : device int32 [E]      pairs per expert
+ *   offsets: device int32 [E + 1]  exclusive prefix sum of counts
+ *   perm   : device int32 [B*K]    pair indices sorted by (expert, p)
+ *   status : device int32, set to 0 by the call, GALE_ERR_ARG if an id is out
+ *            of range or repeated within a token (such pairs are dropped).
+ * 1 <= K <= 16, 1 <= E <= 1024, B >= 0.  Bit-exact and deterministic.
+ * ------------------------------------------------------------------------- */
+int gale_route_permute(const int32_t* ids, int B, int K, int E, int32_t* counts,
+                       int32_t* offsets, int32_t* perm, int32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * One routed-expert MoE layer.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+    const void* base;       /* device; expert e's record at base + e*expert_stride */
+    int64_t expert_stride;  /* bytes, >= gale_expert_bytes(d_model, d_ff), multiple of 256 */
+    int32_t n_experts;      /* E, 1..1024 */
+    int32_t d_model;        /* hidden size, multiple of 1024 */
+    int32_t d_ff;           /* expert intermediate size, multiple of 1024 */
+    int32_t reserved;
+} gale_layer;
+
+/* Workspace bytes gale_moe_forward needs for B tokens and top-K routing. */
+size_t gale_moe_workspace_size(const gale_layer* layer, int B, int K);
+
+/* y[t] = sum_{k<K} gates[t,k] * expert_{ids[t,k]}(x[t]), where
+ * expert_e(x) = Q(W2_e) H( silu(Q(W1_e) H x) * (Q(W3_e) H x) ) with H the
+ * blocked FWHT-1024 (SwiGLU expert, top-K routed experts of the layer; the
+ * card's "43 layers x 256 experts", "experts touched per token 258 (43 x 6)").
+ * The K contributions are summed in fixed k order (deterministic, no atomics).
+ *   x     : device bf16 bits [B][d_model]
+ *   ids   : device int32 [B][K];   gates : device fp32 [B][K]
+ *   out   : device [B][d_model] of out_dtype (GALE_F32 or GALE_BF16)
+ *   flags : 0, or GALE_FLAG_RESIDUAL_RMSNORM: out = bf16(v / sqrt(mean(v^2) + eps))
+ *           with v = x + y (post-norm residual step of an expert-only layer
+ *           chain; out_dtype must be GALE_BF16).
+ *   ws    : device workspace of at least gale_moe_workspace_size() bytes,
+ *           256-byte aligned.  Its first int32 is the device status word:
+ *           the call resets it to 0; kernels set GALE_ERR_ARG (bad ids) or
+ *           GALE_ERR_TIMEOUT (a bounded wait ran out).  Read it after the
+ *           stream is synchronised.  Calls sharing one workspace must not
+ *           overlap on the device.
+ * Tokens per expert choose the kernel: decode batches stream the packed
+ * signs through the fused GEMV; prefill-sized groups use the tensor-core
+ * tile path.  Both compute the same function.
+ * Errors: GALE_ERR_ARG, GALE_ERR_ALIGN, GALE_ERR_WORKSPACE, GALE_ERR_CUDA. */
+int gale_moe_forward(const gale_layer* layer, const uint16_t* x, const int32_t* ids,
+                     const float* gates, int B, int K, void* out, int out_dtype, int flags,
+                     float eps, void* ws, size_t ws_bytes, void* stream);
+
+/* Built-in parity self-check on tiny shapes (the card's "optional fast paths
+ * verify themselves at startup" -- without any fallback).  Synchronous:
+ * allocates nothing itself but needs `scratch` of gale_selftest_scratch_bytes()
+ * device bytes.  Returns GALE_OK when the GPU results match the host-side
+ * expectations built into the library. */
+size_t gale_selftest_scratch_bytes(void);
+int gale_selftest(void* scratch, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GALE_H */

@@ -1,0 +1,258 @@
+"""GPU parity: every entry point of libgale against the fp64 oracle.
+
+Bit-exact for packing, dense dequantisation and the routing permute; within
+a relative L2 error of 2e-3 (bf16 activations, fp32 accumulation) for the
+expert GEMV, the SwiGLU expert and the MoE layer; FWHT within fp32 rounding.
+"""
+import numpy as np
+import pytest
+
+import gale_synth as gs
+from oracle import gale_oracle as O
+
+from .helpers import REL_L2_TOL, Layer, gpu_pack, rel_l2, to_dev
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+G = pytest.importorskip("bit_expert_gemv_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    G.lib()
+
+
+def _empty_u8(n):
+    return torch.zeros(n, dtype=torch.uint8, device="cuda")
+
+
+# ----------------------------------------------------------------------------
+# pack / unpack
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rows,cols", [(1, 1024), (37, 2048), (100, 3072), (2048, 4096), (4096, 2048)])
+def test_pack_bit_exact(rows, cols):
+    c = gs.matrix_canonical(rows, cols, expert=rows + cols)
+    want = O.pack(c)
+    dst = _empty_u8(G.gale_pack_layout(rows, cols)["total"])
+    status = gpu_pack(c, dst)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert np.array_equal(dst.cpu().numpy(), want)
+
+
+def test_pack_rejects_unsorted_idx():
+    c = gs.matrix_canonical(8, 1024, expert=1)
+    c["idx"] = c["idx"].copy()
+    c["idx"][3, 4] = c["idx"][3, 3]
+    dst = _empty_u8(G.gale_pack_layout(8, 1024)["total"])
+    status = gpu_pack(c, dst)
+    torch.cuda.synchronize()
+    assert int(status.item()) == G.GALE_ERR_ARG
+
+
+@pytest.mark.parametrize("rows,cols", [(3, 1024), (129, 2048), (2048, 4096)])
+def test_unpack_bit_exact(rows, cols):
+    c = gs.matrix_canonical(rows, cols, expert=5)
+    dst = _empty_u8(G.gale_pack_layout(rows, cols)["total"])
+    gpu_pack(c, dst)
+    dense = torch.empty(rows, cols, dtype=torch.float32, device="cuda")
+    G.gale_unpack(dst, rows, cols, dense)
+    torch.cuda.synchronize()
+    want = O.dequant(c)
+    assert np.array_equal(dense.cpu().numpy().astype(np.float64), want)
+
+
+# ----------------------------------------------------------------------------
+# FWHT
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rows,cols", [(1, 1024), (3, 4096), (37, 2048), (0, 1024)])
+def test_fwht_f32(rows, cols):
+    x = np.stack([gs.x_f32(cols, tag=100 + r) for r in range(rows)]) if rows else np.zeros((0, cols), np.float32)
+    xd = to_dev(x.astype(np.float32))
+    y = torch.empty_like(xd)
+    G.gale_fwht1024(xd, y)
+    torch.cuda.synchronize()
+    if rows:
+        want = O.fwht_blocked(x.astype(np.float64))
+        assert np.max(np.abs(y.cpu().numpy() - want)) < 2e-5 * max(1.0, np.max(np.abs(want)))
+
+
+def test_fwht_bf16_in_place_involution():
+    bits, vals = gs.hidden_bf16(5, 4096, tag=9)
+    xd = to_dev(bits, torch.bfloat16)
+    y = torch.empty(5, 4096, dtype=torch.float32, device="cuda")
+    G.gale_fwht1024(xd, y)
+    want = O.fwht_blocked(vals.astype(np.float64))
+    z = y.clone()
+    G.gale_fwht1024(z, z)      # in place, back to x
+    torch.cuda.synchronize()
+    assert np.max(np.abs(y.cpu().numpy() - want)) < 2e-5 * np.max(np.abs(want))
+    assert np.max(np.abs(z.cpu().numpy() - vals)) < 1e-5
+
+
+# ----------------------------------------------------------------------------
+# expert GEMV
+# ----------------------------------------------------------------------------
+
+def _packed_dev(c):
+    dst = _empty_u8(G.gale_pack_layout(c["rows"], c["cols"])["total"])
+    gpu_pack(c, dst)
+    return dst
+
+
+@pytest.mark.parametrize("rows,cols,ntok", [(2048, 4096, 1), (4096, 2048, 1), (100, 1024, 3), (37, 2048, 8),
+                                             (300, 4096, 5), (64, 3072, 64), (17, 1024, 9)])
+def test_gemv_plain(rows, cols, ntok):
+    c = gs.matrix_canonical(rows, cols, expert=rows, matrix=gs.W2)
+    W = _packed_dev(c)
+    x = np.stack([gs.x_f32(cols, tag=t) for t in range(ntok)])
+    y = torch.empty(ntok, rows, dtype=torch.float32, device="cuda")
+    G.gale_expert_gemv(W, rows, cols, to_dev(x), y)
+    torch.cuda.synchronize()
+    want = O.gemv(O.dequant(c), x.astype(np.float64))
+    assert rel_l2(y.cpu().numpy(), want) < REL_L2_TOL
+
+
+@pytest.mark.parametrize("rows,cols,ntok", [(2048, 4096, 1), (2048, 4096, 8), (200, 2048, 2), (48, 1024, 33)])
+def test_gemv_swiglu(rows, cols, ntok):
+    c1 = gs.matrix_canonical(rows, cols, expert=7, matrix=gs.W1)
+    c3 = gs.matrix_canonical(rows, cols, expert=7, matrix=gs.W3)
+    W1, W3 = _packed_dev(c1), _packed_dev(c3)
+    x = np.stack([gs.x_f32(cols, tag=50 + t) for t in range(ntok)])
+    y = torch.empty(ntok, rows, dtype=torch.float32, device="cuda")
+    G.gale_expert_gemv(W1, rows, cols, to_dev(x), y, W3=W3, mode=G.GALE_MODE_SWIGLU)
+    torch.cuda.synchronize()
+    want = O.swiglu_hidden(O.dequant(c1), O.dequant(c3), x.astype(np.float64))
+    assert rel_l2(y.cpu().numpy(), want) < REL_L2_TOL
+
+
+def test_gemv_unit_scale_integer_exact():
+    """All-unit-scale pack and integer x: the product is an exact integer sum,
+    so the GPU must match the oracle bit for bit."""
+    rows, cols = 64, 2048
+    c = gs.matrix_canonical(rows, cols, expert=11)
+    c["s_blk"] = np.ones_like(c["s_blk"])
+    c["s_row"] = np.ones_like(c["s_row"])
+    W = _packed_dev(c)
+    x = np.random.default_rng(3).integers(-8, 9, size=(2, cols)).astype(np.float32)
+    y = torch.empty(2, rows, dtype=torch.float32, device="cuda")
+    G.gale_expert_gemv(W, rows, cols, to_dev(x), y)
+    torch.cuda.synchronize()
+    want = O.gemv(O.dequant(c), x.astype(np.float64))
+    assert np.array_equal(y.cpu().numpy().astype(np.float64), want)
+
+
+# ----------------------------------------------------------------------------
+# routing permute
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,K,E,skew", [(1, 6, 256, 0.0), (8, 6, 256, 0.0), (64, 6, 256, 0.5),
+                                         (4096, 6, 256, 0.5), (3, 2, 4, 0.0), (200, 16, 1024, 0.0)])
+def test_route_permute_bit_exact(B, K, E, skew):
+    ids, _ = gs.route_topk(gs.router_logits(B, E, tag=B, bias_sigma=skew), K)
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(B * K, dtype=torch.int32, device="cuda")
+    status = torch.ones(1, dtype=torch.int32, device="cuda")
+    G.gale_route_permute(to_dev(ids), E, counts, offsets, perm, status)
+    torch.cuda.synchronize()
+    wc, wo, wp = O.route_permute(ids, E)
+    assert int(status.item()) == 0
+    assert np.array_equal(counts.cpu().numpy(), wc)
+    assert np.array_equal(offsets.cpu().numpy(), wo)
+    assert np.array_equal(perm.cpu().numpy(), wp)
+
+
+def test_route_permute_flags_bad_ids():
+    ids = np.array([[0, 1, 2], [3, 3, 4], [5, 300, 6]], np.int32)
+    E = 256
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.full((9,), -7, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    G.gale_route_permute(to_dev(ids), E, counts, offsets, perm, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == G.GALE_ERR_ARG
+    assert int(counts.sum().item()) == 7      # the repeated 3 and the id 300 are dropped
+
+
+# ----------------------------------------------------------------------------
+# MoE layer
+# ----------------------------------------------------------------------------
+
+@pytest.fixture(scope="module")
+def small_layer():
+    return Layer(16, 2048, 1024, layer=1)
+
+
+def _moe(layer, bits, ids, gates, out_dtype=None, flags=0, eps=1e-6):
+    B, K = ids.shape
+    ws = torch.empty(G.gale_moe_workspace_size(layer.desc, B, K), dtype=torch.uint8, device="cuda")
+    out = torch.empty(B, layer.d_model, dtype=out_dtype or torch.float32, device="cuda")
+    G.gale_moe_forward(layer.desc, to_dev(bits, torch.bfloat16), to_dev(ids), to_dev(gates), out, ws,
+                       flags=flags, eps=eps)
+    torch.cuda.synchronize()
+    return out, int(ws[:4].view(torch.int32).item())
+
+
+@pytest.mark.parametrize("B,K", [(1, 6), (5, 6), (33, 4), (2, 1), (70, 6)])
+def test_moe_small(small_layer, B, K):
+    L = small_layer
+    bits, xv = gs.hidden_bf16(B, L.d_model, tag=B)
+    ids, gates = gs.route_topk(gs.router_logits(B, L.E, tag=B), K)
+    out, st = _moe(L, bits, ids, gates)
+    assert st == 0
+    want = O.moe_layer(L.dense, xv, ids, gates)
+    assert rel_l2(out.cpu().numpy(), want) < REL_L2_TOL
+
+
+def test_moe_fused_rmsnorm(small_layer):
+    L = small_layer
+    B = 3
+    bits, xv = gs.hidden_bf16(B, L.d_model, tag=77)
+    ids, gates = gs.route_topk(gs.router_logits(B, L.E, tag=77), 6)
+    out, st = _moe(L, bits, ids, gates, out_dtype=torch.bfloat16, flags=G.GALE_FLAG_RESIDUAL_RMSNORM)
+    assert st == 0
+    want = O.chain_step(L.dense, xv, ids, gates)
+    got = out.float().cpu().numpy()
+    # the output itself is rounded to bf16 (relative 2^-9 per element)
+    assert rel_l2(got, want) < 4e-3
+
+
+def test_moe_bad_ids_status(small_layer):
+    L = small_layer
+    bits, _ = gs.hidden_bf16(2, L.d_model, tag=5)
+    ids = np.array([[0, 1, 2, 3, 4, 99], [1, 1, 2, 3, 4, 5]], np.int32)
+    gates = np.full((2, 6), 1.0 / 6, np.float32)
+    _, st = _moe(L, bits, ids, gates)
+    assert st == G.GALE_ERR_ARG
+
+
+@pytest.fixture(scope="module")
+def full_layer():
+    """256 experts of w1/w3 [2048 x 4096], w2 [4096 x 2048] (about 1.07 GB packed)."""
+    return Layer(256, 4096, 2048, layer=0)
+
+
+@pytest.mark.parametrize("B,skew", [(1, 0.0), (8, 0.0), (64, 0.5)])
+def test_moe_full_size(full_layer, B, skew):
+    L = full_layer
+    bits, xv = gs.hidden_bf16(B, L.d_model, tag=1000 + B)
+    ids, gates = gs.route_topk(gs.router_logits(B, L.E, tag=1000 + B, bias_sigma=skew), 6)
+    out, st = _moe(L, bits, ids, gates)
+    assert st == 0
+    got = out.cpu().numpy()
+    # the oracle evaluates a sample of tokens one by one at B = 64
+    toks = np.arange(B) if B <= 8 else np.array([0, 1, 17, 40, 63])
+    want = O.moe_layer(L.dense, xv[toks], ids[toks], gates[toks])
+    assert rel_l2(got[toks], want) < REL_L2_TOL
+
+
+def test_selftest():
+    scratch = torch.empty(G.gale_selftest_scratch_bytes(), dtype=torch.uint8, device="cuda")
+    assert G.gale_selftest(scratch) == G.GALE_OK
