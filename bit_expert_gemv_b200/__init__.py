@@ -29,8 +29,10 @@ GALE_FLAG_RESIDUAL_RMSNORM = 1
 EXPORTS = (
     "gale_status_string", "gale_pack_layout", "gale_expert_bytes", "gale_pack", "gale_unpack",
     "gale_fwht1024", "gale_expert_gemv", "gale_route_permute", "gale_moe_workspace_size",
-    "gale_moe_forward", "gale_selftest_scratch_bytes", "gale_selftest",
+    "gale_moe_forward", "gale_moe_forward_noalloc", "gale_selftest_scratch_bytes", "gale_selftest",
 )
+
+GALE_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class GaleError(RuntimeError):
@@ -79,6 +81,8 @@ def lib() -> ctypes.CDLL:
             "gale_moe_workspace_size": (sz, [ctypes.POINTER(gale_layer), i32, i32]),
             "gale_moe_forward": (i32, [ctypes.POINTER(gale_layer), vp, vp, vp, i32, i32, vp, i32, i32,
                                        ctypes.c_float, vp, sz, vp]),
+            "gale_moe_forward_noalloc": (i32, [ctypes.POINTER(gale_layer), vp, vp, vp, i32, i32, vp, i32, i32,
+                                               ctypes.c_float, vp, vp]),
             "gale_selftest_scratch_bytes": (sz, []),
             "gale_selftest": (i32, [vp, vp]),
         }
@@ -181,6 +185,16 @@ def gale_moe_forward(layer: gale_layer, x, ids, gates, out, ws, flags: int = 0, 
     _check(lib().gale_moe_forward(ctypes.byref(layer), _ptr(x), _ptr(ids), _ptr(gates), B, K, _ptr(out),
                                   _dtype_code(out), flags, eps, _ptr(ws), ws.numel() * ws.element_size(),
                                   _stream(stream)), "gale_moe_forward")
+
+
+def gale_moe_forward_noalloc(layer: gale_layer, x, ids, gates, out, status=None, flags: int = 0,
+                             eps: float = 1e-6, stream=None):
+    """gale_moe_forward with the library's fixed scratch array instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    B, K = ids.shape
+    _check(lib().gale_moe_forward_noalloc(ctypes.byref(layer), _ptr(x), _ptr(ids), _ptr(gates), B, K,
+                                          _ptr(out), _dtype_code(out), flags, eps, _ptr(status),
+                                          _stream(stream)), "gale_moe_forward_noalloc")
 
 
 def gale_selftest_scratch_bytes() -> int:

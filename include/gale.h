@@ -205,6 +205,37 @@ int gale_moe_forward(const gale_layer* layer, const uint16_t* x, const int32_t* 
                      const float* gates, int B, int K, void* out, int out_dtype, int flags,
                      float eps, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * gale_moe_forward without caller-provided workspace.  This is an interface
+ * addition of this library and has no counterpart on the GALE cards.
+ *
+ * For callers that cannot allocate device memory where they run a layer:
+ * for example a plugin inside a host runtime that owns the device memory pool,
+ * or a process that fixed its device footprint at start-up.  The caller still
+ * owns x, ids, gates, out and status; the scratch comes from one file-scope
+ * device array of GALE_NOALLOC_SCRATCH_BYTES (4 MiB) inside the library,
+ * which every GPU that loads the library holds until the process exits.
+ *
+ * Same computation, arguments and errors as gale_moe_forward, except:
+ *  - no ws / ws_bytes; a call whose workspace (gale_moe_workspace_size)
+ *    exceeds GALE_NOALLOC_SCRATCH_BYTES returns GALE_ERR_WORKSPACE;
+ *  - status: optional device int32; when non-NULL the call ends by copying
+ *    the device status word there (same codes as gale_moe_forward's);
+ *  - the library allocates and frees nothing (no cudaMalloc, no cudaFree);
+ *  - the first call on each device looks up the array's device address with
+ *    that device current and caches it: make that first call before any
+ *    stream capture;
+ *  - all calls on a device share the one array and it keeps the previous
+ *    call's contents (each call clears what must start at zero): calls that
+ *    overlap on the GPU, from any stream or thread, race and give undefined
+ *    results.  Serialise them.
+ * ------------------------------------------------------------------------- */
+#define GALE_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+int gale_moe_forward_noalloc(const gale_layer* layer, const uint16_t* x, const int32_t* ids,
+                             const float* gates, int B, int K, void* out, int out_dtype, int flags,
+                             float eps, int32_t* status, void* stream);
+
 /* Built-in parity self-check on tiny shapes (the card's "optional fast paths
  * verify themselves at startup" -- without any fallback).  Synchronous:
  * allocates nothing itself but needs `scratch` of gale_selftest_scratch_bytes()
