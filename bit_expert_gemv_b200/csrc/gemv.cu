@@ -4,6 +4,7 @@
 // decoded in registers).
 #include "common.cuh"
 #include "gemv_simple.cuh"
+#include "gemv_mma.cuh"
 
 namespace gale {
 
@@ -65,6 +66,8 @@ extern "C" int gale_expert_gemv(const gale_matrix* W, const gale_matrix* W3, con
     cudaStream_t st = as_stream(stream);
     MatView a = make_view(W->packed, W->rows, W->cols);
     MatView b = W3 ? make_view(W3->packed, W3->rows, W3->cols) : a;
+    // decode-sized token counts take the tensor-core path
+    if (gemv_mma_supported(W->cols, ntok)) return launch_gemv_mma(a, b, mode == GALE_MODE_SWIGLU, x_rot, ntok, y, st);
     const int chunk = simple_chunk_tokens(W->cols);
     const size_t smem = size_t(chunk) * W->cols * sizeof(float);
     const int grid = (W->rows + kWarps * kRowsPerWarp - 1) / (kWarps * kRowsPerWarp);

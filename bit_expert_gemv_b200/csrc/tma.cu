@@ -1,0 +1,56 @@
+// Host-side tensor-map encoding (cuTensorMapEncodeTiled through the runtime's
+// driver entry point, so the library does not link libcuda directly).
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "tma.cuh"
+
+namespace gale {
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+}  // namespace
+
+int make_map_3d(CUtensorMap* m, bool u16, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, bool swizzle128) {
+    auto fn = encode_fn();
+    if (!fn) return GALE_ERR_CUDA;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1, stride2};
+    cuuint32_t box[3] = {b0, b1, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = fn(m, u16 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32, 3,
+                    const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GALE_OK : GALE_ERR_CUDA;
+}
+
+// Sign words of one matrix kind across experts: [experts][rows][cols/32] uint32,
+// boxes of 32 words (1024 columns) x 16 rows, 128-byte swizzle.
+int make_sign_map(CUtensorMap* m, const void* first_matrix, int rows, int cols, int experts, int64_t stride) {
+    return make_map_3d(m, false, first_matrix, uint64_t(cols) / 32, uint64_t(rows), uint64_t(experts),
+                       uint64_t(cols) / 8, uint64_t(stride), 32, kTileRows, true);
+}
+
+// Block scales of one matrix kind across experts: [experts][rows][cols/128] fp16,
+// boxes of a full row of scales x 16 rows.
+int make_scale_map(CUtensorMap* m, const void* first_matrix, int rows, int cols, int experts, int64_t stride) {
+    const Layout L = make_layout(rows, cols);
+    const char* p = static_cast<const char*>(first_matrix) + L.off_sblk;
+    return make_map_3d(m, true, p, uint64_t(cols) / 128, uint64_t(rows), uint64_t(experts), uint64_t(cols) / 64,
+                       uint64_t(stride), uint32_t(cols / 128), kTileRows, false);
+}
+
+}  // namespace gale

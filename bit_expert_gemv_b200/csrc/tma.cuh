@@ -1,0 +1,16 @@
+// Tensor maps over packed records (host side).
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace gale {
+
+constexpr int kTileRows = 16;   // rows of one MMA tile (and of one TMA box)
+
+int make_map_3d(CUtensorMap* m, bool u16, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, bool swizzle128);
+int make_sign_map(CUtensorMap* m, const void* first_matrix, int rows, int cols, int experts, int64_t stride);
+int make_scale_map(CUtensorMap* m, const void* first_matrix, int rows, int cols, int experts, int64_t stride);
+
+}  // namespace gale

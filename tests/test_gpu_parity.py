@@ -105,8 +105,10 @@ def _packed_dev(c):
     return dst
 
 
-@pytest.mark.parametrize("rows,cols,ntok", [(2048, 4096, 1), (4096, 2048, 1), (100, 1024, 3), (37, 2048, 8),
-                                             (300, 4096, 5), (64, 3072, 64), (17, 1024, 9)])
+@pytest.mark.parametrize("rows,cols,ntok", [(2048, 4096, 1), (4096, 2048, 1), (4096, 2048, 2), (100, 1024, 1),
+                                             (37, 2048, 2), (300, 4096, 2), (17, 3072, 1), (1, 1024, 1),
+                                             (100, 1024, 3), (37, 2048, 8), (300, 4096, 5), (64, 3072, 64),
+                                             (17, 1024, 9)])
 def test_gemv_plain(rows, cols, ntok):
     c = gs.matrix_canonical(rows, cols, expert=rows, matrix=gs.W2)
     W = _packed_dev(c)
@@ -118,7 +120,8 @@ def test_gemv_plain(rows, cols, ntok):
     assert rel_l2(y.cpu().numpy(), want) < REL_L2_TOL
 
 
-@pytest.mark.parametrize("rows,cols,ntok", [(2048, 4096, 1), (2048, 4096, 8), (200, 2048, 2), (48, 1024, 33)])
+@pytest.mark.parametrize("rows,cols,ntok", [(2048, 4096, 1), (2048, 4096, 2), (2048, 4096, 8), (200, 2048, 2),
+                                             (33, 1024, 1), (48, 1024, 33)])
 def test_gemv_swiglu(rows, cols, ntok):
     c1 = gs.matrix_canonical(rows, cols, expert=7, matrix=gs.W1)
     c3 = gs.matrix_canonical(rows, cols, expert=7, matrix=gs.W3)
@@ -131,20 +134,22 @@ def test_gemv_swiglu(rows, cols, ntok):
     assert rel_l2(y.cpu().numpy(), want) < REL_L2_TOL
 
 
-def test_gemv_unit_scale_integer_exact():
+@pytest.mark.parametrize("rows,cols", [(64, 2048), (50, 4096)])
+def test_gemv_unit_scale_integer_exact(rows, cols):
     """All-unit-scale pack and integer x: the product is an exact integer sum,
-    so the GPU must match the oracle bit for bit."""
-    rows, cols = 64, 2048
+    so the GPU must match the oracle bit for bit (both the tensor-core path,
+    whose e4m3 pieces hold small integers exactly, and the CUDA-core path)."""
     c = gs.matrix_canonical(rows, cols, expert=11)
     c["s_blk"] = np.ones_like(c["s_blk"])
     c["s_row"] = np.ones_like(c["s_row"])
     W = _packed_dev(c)
-    x = np.random.default_rng(3).integers(-8, 9, size=(2, cols)).astype(np.float32)
-    y = torch.empty(2, rows, dtype=torch.float32, device="cuda")
-    G.gale_expert_gemv(W, rows, cols, to_dev(x), y)
-    torch.cuda.synchronize()
-    want = O.gemv(O.dequant(c), x.astype(np.float64))
-    assert np.array_equal(y.cpu().numpy().astype(np.float64), want)
+    for ntok in (1, 2, 4):
+        x = np.random.default_rng(3 + ntok).integers(-8, 9, size=(ntok, cols)).astype(np.float32)
+        y = torch.empty(ntok, rows, dtype=torch.float32, device="cuda")
+        G.gale_expert_gemv(W, rows, cols, to_dev(x), y)
+        torch.cuda.synchronize()
+        want = O.gemv(O.dequant(c), x.astype(np.float64))
+        assert np.array_equal(y.cpu().numpy().astype(np.float64), want), ntok
 
 
 # ----------------------------------------------------------------------------
