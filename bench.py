@@ -257,7 +257,7 @@ def run_gpu(args):
         "b8": {"tokens_per_s": 8 * max(args.steps // 2, 3) * world / t8,
                "hbm_gbs": bytes8 * world / t8 / 1e9, "frac": bytes8 * world / t8 / 1e9 / peak},
         "e2e": {"value": tokens / te, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": 3 * args.steps,
         "clocks": clocks_info,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

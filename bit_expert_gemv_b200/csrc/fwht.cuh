@@ -1,12 +1,16 @@
-// Unnormalised Walsh-Hadamard butterflies over one 1024-block held by a warp:
-// v[i] of lane l is element 32*i + l.  Natural (Sylvester) order.
+// Unnormalised Walsh-Hadamard butterflies over one 1024-block held by a warp.
+// The transform is a product of one butterfly per index bit, so any
+// assignment of the 10 element-index bits to (5 lane bits, 5 register bits)
+// works: stages over lane bits pair lanes, stages over register bits pair
+// registers.  Callers choose the element of (lane, register) they load and
+// read back the same element.  Natural (Sylvester) order.
 #pragma once
 
 namespace gale {
 
 __device__ __forceinline__ void fwht1024_warp(float (&v)[32], int lane) {
-    // strides 1..16: partner lane differs in bit s
-#pragma unroll
+    // partner lane differs in bit s
+#pragma unroll 1
     for (int s = 0; s < 5; ++s) {
         const bool upper = (lane >> s) & 1;
 #pragma unroll
@@ -15,7 +19,7 @@ __device__ __forceinline__ void fwht1024_warp(float (&v)[32], int lane) {
             v[i] = upper ? (o - v[i]) : (v[i] + o);
         }
     }
-    // strides 32..512: partner register differs in bit s
+    // partner register differs in bit s
 #pragma unroll
     for (int s = 0; s < 5; ++s) {
 #pragma unroll

@@ -1,6 +1,6 @@
 // Tensor-core path of gale_expert_gemv for one or two tokens: each warp
 // streams 16-row tiles of the packed matrix (TMA, two stages per warp) and
-// runs the e4m3 AND-mask MMA of mma_tile.cuh on them.
+// runs the int8 AND-mask MMA of mma_tile.cuh on them.
 #include "common.cuh"
 #include "gemv_mma.cuh"
 #include "mma_tile.cuh"
@@ -126,21 +126,21 @@ int launch_gemv_mma(const MatView& a, const MatView& b, bool swiglu, const float
     CUtensorMap sa, ba, sb, bb;
     const Layout La = make_layout(a.rows, a.cols);
     const int64_t stride = align_up(La.total, 256);
-    int rc = make_sign_map(&sa, a.signs, a.rows, a.cols, 1, stride);
-    if (rc == GALE_OK) rc = make_scale_map(&ba, a.signs, a.rows, a.cols, 1, stride);
-    if (rc == GALE_OK) rc = make_sign_map(&sb, b.signs, b.rows, b.cols, 1, stride);
-    if (rc == GALE_OK) rc = make_scale_map(&bb, b.signs, b.rows, b.cols, 1, stride);
+    int rc = cached_map(&sa, false, a.signs, a.rows, a.cols, 1, stride);
+    if (rc == GALE_OK) rc = cached_map(&ba, true, a.signs, a.rows, a.cols, 1, stride);
+    if (rc == GALE_OK) rc = cached_map(&sb, false, b.signs, b.rows, b.cols, 1, stride);
+    if (rc == GALE_OK) rc = cached_map(&bb, true, b.signs, b.rows, b.cols, 1, stride);
     if (rc != GALE_OK) return rc;
     const GemvSmem S = gemv_smem(a.cols, kGemvWarps);
     const int tiles = (a.rows + 15) / 16;
     const int grid = tiles < sm_count() ? tiles : sm_count();
     if (swiglu) {
-        GALE_CUDA_TRY(cudaFuncSetAttribute(gemv_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           S.bytes));
+        rc = ensure_smem(reinterpret_cast<const void*>(gemv_mma_kernel<true>), S.bytes);
+        if (rc != GALE_OK) return rc;
         gemv_mma_kernel<true><<<grid, kGemvWarps * 32, S.bytes, st>>>(sa, ba, sb, bb, a, b, x, ntok, y, S);
     } else {
-        GALE_CUDA_TRY(cudaFuncSetAttribute(gemv_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           S.bytes));
+        rc = ensure_smem(reinterpret_cast<const void*>(gemv_mma_kernel<false>), S.bytes);
+        if (rc != GALE_OK) return rc;
         gemv_mma_kernel<false><<<grid, kGemvWarps * 32, S.bytes, st>>>(sa, ba, sa, ba, a, a, x, ntok, y, S);
     }
     GALE_LAUNCH_CHECK();

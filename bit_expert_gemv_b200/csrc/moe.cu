@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "gemv_simple.cuh"
 #include "moe.cuh"
+#include "moe_decode.cuh"
 #include "route.cuh"
 
 namespace gale {
@@ -153,7 +154,12 @@ int launch_group_gemv(bool swiglu, GroupArgs g, int max_slots, cudaStream_t st) 
 
 extern "C" size_t gale_moe_workspace_size(const gale_layer* layer, int B, int K) {
     if (gale::validate_layer(layer) == GALE_ERR_ARG || B < 0 || K < 1 || K > 16) return 0;
-    return gale::carve_ws(nullptr, *layer, B, K).bytes;
+    size_t n = gale::carve_ws(nullptr, *layer, B, K).bytes;
+    if (gale::decode_supported(*layer, B, K)) {
+        const size_t d = gale::carve_decode_ws(nullptr, *layer, B, K).bytes;
+        n = d > n ? d : n;
+    }
+    return n;
 }
 
 extern "C" int gale_moe_forward(const gale_layer* layer, const uint16_t* x, const int32_t* ids,
@@ -170,7 +176,9 @@ extern "C" int gale_moe_forward(const gale_layer* layer, const uint16_t* x, cons
     if (!ws) return GALE_ERR_WORKSPACE;
     const gale_layer& L = *layer;
     MoeWs w = carve_ws(ws, L, B, K);
-    if (ws_bytes < w.bytes) return GALE_ERR_WORKSPACE;
+    const bool decode = decode_supported(L, B, K);
+    if (ws_bytes < w.bytes || (decode && ws_bytes < carve_decode_ws(nullptr, L, B, K).bytes))
+        return GALE_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return GALE_ERR_ALIGN;
     cudaStream_t st = as_stream(stream);
     GALE_CUDA_TRY(cudaMemsetAsync(w.status, 0, sizeof(int32_t), st));
@@ -179,6 +187,8 @@ extern "C" int gale_moe_forward(const gale_layer* layer, const uint16_t* x, cons
     if (!aligned(x, 4) || !aligned(ids, 4) || !aligned(gates, 4) || !aligned(out, 4)) return GALE_ERR_ALIGN;
     const int64_t BK = int64_t(B) * K;
     if (BK > (1 << 24)) return GALE_ERR_UNSUPPORTED;
+    // decode batches: tensor-core streaming kernels
+    if (decode) return launch_moe_decode(L, x, ids, gates, B, K, out, out_dtype, fuse, eps, ws, st);
 
     GALE_CUDA_TRY(cudaMemsetAsync(w.pos_of_pair, 0xFF, size_t(BK) * 4, st));
     RouteArgs ra{};

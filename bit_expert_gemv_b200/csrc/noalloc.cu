@@ -46,7 +46,8 @@ extern "C" int gale_moe_forward_noalloc(const gale_layer* layer, const uint16_t*
     int rc = gale::validate_layer(layer);
     if (rc != GALE_OK) return rc;
     if (B < 0 || K < 1 || K > 16) return GALE_ERR_ARG;
-    const size_t need = gale::carve_ws(nullptr, *layer, B, K).bytes;
+    const size_t need = gale_moe_workspace_size(layer, B, K);
+    if (need == 0) return GALE_ERR_ARG;
     if (need > size_t(GALE_NOALLOC_SCRATCH_BYTES)) return GALE_ERR_WORKSPACE;
     if (status && !gale::aligned(status, 4)) return GALE_ERR_ALIGN;
     void* ws = nullptr;

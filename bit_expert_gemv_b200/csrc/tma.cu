@@ -53,4 +53,58 @@ int make_scale_map(CUtensorMap* m, const void* first_matrix, int rows, int cols,
                        uint64_t(stride), uint32_t(cols / 128), kTileRows, false);
 }
 
+namespace {
+struct MapEntry {
+    const void* base;
+    int rows, cols, experts;
+    int64_t stride;
+    bool scale;
+    CUtensorMap map;
+};
+constexpr int kMapCache = 128;
+thread_local MapEntry g_maps[kMapCache];
+thread_local int g_map_next = 0;
+}  // namespace
+
+// Tensor maps depend only on (base, shape, stride), so they are encoded once
+// and kept in a small per-thread cache (encoding costs microseconds of host
+// time per map).
+int cached_map(CUtensorMap* out, bool scale, const void* first_matrix, int rows, int cols, int experts,
+               int64_t stride) {
+    for (int i = 0; i < kMapCache; ++i) {
+        const MapEntry& e = g_maps[i];
+        if (e.base == first_matrix && e.rows == rows && e.cols == cols && e.experts == experts &&
+            e.stride == stride && e.scale == scale) {
+            *out = e.map;
+            return GALE_OK;
+        }
+    }
+    MapEntry e{first_matrix, rows, cols, experts, stride, scale, {}};
+    const int rc = scale ? make_scale_map(&e.map, first_matrix, rows, cols, experts, stride)
+                         : make_sign_map(&e.map, first_matrix, rows, cols, experts, stride);
+    if (rc != GALE_OK) return rc;
+    g_maps[g_map_next] = e;
+    g_map_next = (g_map_next + 1) % kMapCache;
+    *out = e.map;
+    return GALE_OK;
+}
+
+int ensure_smem(const void* kernel, int bytes) {
+    constexpr int kMaxDev = 64, kMaxKernels = 32;
+    static const void* kernels[kMaxDev][kMaxKernels] = {};
+    static int set_bytes[kMaxDev][kMaxKernels] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return GALE_ERR_CUDA;
+    int slot = -1;
+    for (int i = 0; i < kMaxKernels; ++i) {
+        if (kernels[dev][i] == kernel) { slot = i; break; }
+        if (!kernels[dev][i]) { slot = i; kernels[dev][i] = kernel; break; }
+    }
+    if (slot >= 0 && set_bytes[dev][slot] >= bytes) return GALE_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return GALE_ERR_CUDA;
+    if (slot >= 0) set_bytes[dev][slot] = bytes;
+    return GALE_OK;
+}
+
 }  // namespace gale

@@ -12,5 +12,9 @@ int make_map_3d(CUtensorMap* m, bool u16, const void* base, uint64_t d0, uint64_
                 uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, bool swizzle128);
 int make_sign_map(CUtensorMap* m, const void* first_matrix, int rows, int cols, int experts, int64_t stride);
 int make_scale_map(CUtensorMap* m, const void* first_matrix, int rows, int cols, int experts, int64_t stride);
+int cached_map(CUtensorMap* out, bool scale, const void* first_matrix, int rows, int cols, int experts,
+               int64_t stride);
+// Raise a kernel's dynamic shared-memory limit once per device.
+int ensure_smem(const void* kernel, int bytes);
 
 }  // namespace gale
