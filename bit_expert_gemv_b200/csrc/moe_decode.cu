@@ -465,31 +465,36 @@ __global__ void __launch_bounds__(kDecThreads + 32, 1) moe_stream_kernel(
     };
 
     if (warp == kDecWarps) {
-        // ---------------- producer: weights only, no dependency on earlier kernels
-        if (lane == 0) {
-            for (int i = 0; i < n_my; ++i) {
-                const int s = i % sh.n_stages;
-                if (i >= sh.n_stages && !mbar_wait(empty + s, ((i / sh.n_stages) - 1) & 1)) {
-                    set_status(A.ws.status, GALE_ERR_TIMEOUT);
-                    break;
-                }
-                const Job Jb = decode_job(R, j0 + i, sh.row_blocks);
-                uint32_t tx = 0;
-                for (int tr = 0; tr < sh.r_tiles; ++tr) {
-                    const int r0 = Jb.tile * sh.job_rows + tr * 16;
-                    if (r0 >= sh.rows) continue;
-                    for (int mt = 0; mt < sh.n_mat; ++mt) tx += tile_tx_bytes(view(Jb.e, mt), r0);
-                }
-                mbar_arrive_expect_tx(full + s, tx);
-                uint8_t* st = smem + S.stages + s * sh.stage_bytes;
-                for (int tr = 0; tr < sh.r_tiles; ++tr) {
-                    const int r0 = Jb.tile * sh.job_rows + tr * 16;
-                    if (r0 >= sh.rows) continue;
-                    for (int mt = 0; mt < sh.n_mat; ++mt)
-                        issue_tile_copies(st + (tr * sh.n_mat + mt) * sh.tile_bytes, full + s, mt ? &sb : &sa,
-                                          mt ? &bb : &ba, view(Jb.e, mt), Jb.e, r0);
-                }
+        // ---------------- producer: weights only, no dependency on earlier kernels.
+        // Lane 0 arms the stage's barrier with the job's byte count, then every
+        // lane issues the copies of one (row tile, matrix) of the job.
+        const int n_tiles = sh.r_tiles * sh.n_mat;
+        for (int i = 0; i < n_my; ++i) {
+            const int s = i % sh.n_stages;
+            int ok_wait = 1;
+            if (lane == 0 && i >= sh.n_stages) ok_wait = mbar_wait(empty + s, ((i / sh.n_stages) - 1) & 1);
+            ok_wait = __shfl_sync(0xffffffffu, ok_wait, 0);
+            if (!ok_wait) {
+                if (lane == 0) set_status(A.ws.status, GALE_ERR_TIMEOUT);
+                break;
             }
+            const Job Jb = decode_job(R, j0 + i, sh.row_blocks);
+            const int tr = lane / sh.n_mat, mt = lane % sh.n_mat;
+            const int r0 = Jb.tile * sh.job_rows + tr * 16;
+            const bool mine = lane < n_tiles && r0 < sh.rows;
+            uint32_t tx = 0;
+            MatView mv{};
+            if (mine) {
+                mv = view(Jb.e, mt);
+                tx = tile_tx_bytes(mv, r0);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) tx += __shfl_xor_sync(0xffffffffu, tx, o);
+            if (lane == 0) mbar_arrive_expect_tx(full + s, tx);
+            __syncwarp();
+            if (mine)
+                issue_tile_copies(smem + S.stages + s * sh.stage_bytes + (tr * sh.n_mat + mt) * sh.tile_bytes,
+                                  full + s, mt ? &sb : &sa, mt ? &bb : &ba, mv, Jb.e, r0);
         }
         return;
     }
