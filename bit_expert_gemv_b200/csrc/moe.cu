@@ -9,6 +9,7 @@
 #include "gemv_simple.cuh"
 #include "moe.cuh"
 #include "moe_decode.cuh"
+#include "moe_prefill.cuh"
 #include "route.cuh"
 
 namespace gale {
@@ -122,6 +123,26 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(CombineArgs c) {
         store_from_f32(c.out, GALE_BF16, int64_t(t) * d + i, c.scratch[int64_t(t) * d + i] * inv);
 }
 
+int launch_moe_combine(const float* o, const int32_t* pos_of_pair, const float* gates, const uint16_t* x, int B,
+                       int K, int d_model, void* out, int out_dtype, bool fuse_norm, float eps, float* scratch,
+                       cudaStream_t st) {
+    CombineArgs c{};
+    c.o = o;
+    c.pos_of_pair = pos_of_pair;
+    c.gates = gates;
+    c.x = x;
+    c.K = K;
+    c.d_model = d_model;
+    c.out = out;
+    c.out_dtype = out_dtype;
+    c.fuse_norm = fuse_norm;
+    c.eps = eps;
+    c.scratch = scratch;
+    moe_combine_kernel<<<B, 256, 32 * sizeof(float), st>>>(c);
+    GALE_LAUNCH_CHECK();
+    return GALE_OK;
+}
+
 int validate_layer(const gale_layer* L) {
     if (!L || !L->base || L->n_experts < 1 || L->n_experts > 1024) return GALE_ERR_ARG;
     if (!valid_cols(L->d_model) || !valid_cols(L->d_ff) || L->d_model > 16384 || L->d_ff > 16384)
@@ -155,11 +176,11 @@ int launch_group_gemv(bool swiglu, GroupArgs g, int max_slots, cudaStream_t st) 
 extern "C" size_t gale_moe_workspace_size(const gale_layer* layer, int B, int K) {
     if (gale::validate_layer(layer) == GALE_ERR_ARG || B < 0 || K < 1 || K > 16) return 0;
     size_t n = gale::carve_ws(nullptr, *layer, B, K).bytes;
-    if (gale::decode_supported(*layer, B, K)) {
-        const size_t d = gale::carve_decode_ws(nullptr, *layer, B, K).bytes;
-        n = d > n ? d : n;
-    }
-    return n;
+    // each batch takes exactly one path; its workspace also holds the status word
+    size_t p = 0;
+    if (gale::decode_supported(*layer, B, K)) p = gale::carve_decode_ws(nullptr, *layer, B, K).bytes;
+    else if (gale::prefill_supported(*layer, B, K)) p = gale::carve_prefill_ws(nullptr, *layer, B, K).bytes;
+    return p > n ? p : n;
 }
 
 extern "C" int gale_moe_forward(const gale_layer* layer, const uint16_t* x, const int32_t* ids,
@@ -177,7 +198,9 @@ extern "C" int gale_moe_forward(const gale_layer* layer, const uint16_t* x, cons
     const gale_layer& L = *layer;
     MoeWs w = carve_ws(ws, L, B, K);
     const bool decode = decode_supported(L, B, K);
-    if (ws_bytes < w.bytes || (decode && ws_bytes < carve_decode_ws(nullptr, L, B, K).bytes))
+    const bool prefill = !decode && prefill_supported(L, B, K);
+    if (ws_bytes < w.bytes || (decode && ws_bytes < carve_decode_ws(nullptr, L, B, K).bytes) ||
+        (prefill && ws_bytes < carve_prefill_ws(nullptr, L, B, K).bytes))
         return GALE_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return GALE_ERR_ALIGN;
     cudaStream_t st = as_stream(stream);
@@ -189,6 +212,8 @@ extern "C" int gale_moe_forward(const gale_layer* layer, const uint16_t* x, cons
     if (BK > (1 << 24)) return GALE_ERR_UNSUPPORTED;
     // decode batches: tensor-core streaming kernels
     if (decode) return launch_moe_decode(L, x, ids, gates, B, K, out, out_dtype, fuse, eps, ws, st);
+    // larger batches: tcgen05 tensor-core tiles
+    if (prefill) return launch_moe_prefill(L, x, ids, gates, B, K, out, out_dtype, fuse, eps, ws, st);
 
     GALE_CUDA_TRY(cudaMemsetAsync(w.pos_of_pair, 0xFF, size_t(BK) * 4, st));
     RouteArgs ra{};
@@ -241,19 +266,6 @@ extern "C" int gale_moe_forward(const gale_layer* layer, const uint16_t* x, cons
     rc = launch_group_gemv(false, g, max_slots, st);
     if (rc != GALE_OK) return rc;
 
-    CombineArgs c{};
-    c.o = w.o;
-    c.pos_of_pair = w.pos_of_pair;
-    c.gates = gates;
-    c.x = x;
-    c.K = K;
-    c.d_model = L.d_model;
-    c.out = out;
-    c.out_dtype = out_dtype;
-    c.fuse_norm = fuse;
-    c.eps = eps;
-    c.scratch = w.x_rot;   // x_rot is dead by now; reused for v = x + y
-    moe_combine_kernel<<<B, 256, 32 * sizeof(float), st>>>(c);
-    GALE_LAUNCH_CHECK();
-    return GALE_OK;
+    // x_rot is dead by now; reused for v = x + y
+    return launch_moe_combine(w.o, w.pos_of_pair, gates, x, B, K, L.d_model, out, out_dtype, fuse, eps, w.x_rot, st);
 }

@@ -42,6 +42,8 @@ def gpu_pack(c: dict, dst, status=None):
 class Layer:
     """A packed MoE layer resident on the GPU plus lazy oracle access."""
 
+    DENSE_CACHE = 48
+
     def __init__(self, n_experts: int, d_model: int, d_ff: int, layer: int = 0):
         import torch
         import bit_expert_gemv_b200 as G
@@ -63,6 +65,8 @@ class Layer:
 
     def dense(self, e: int):
         if e not in self._dense:
+            if len(self._dense) >= self.DENSE_CACHE:   # fp64 experts are large: keep the newest few
+                self._dense.pop(next(iter(self._dense)))
             cs = gs.expert_canonical(self.d_model, self.d_ff, layer=self.layer_id, expert=e)
             self._dense[e] = [O.dequant_packed(O.pack(c), c["rows"], c["cols"]) for c in cs]
         return self._dense[e]

@@ -258,6 +258,72 @@ def test_moe_full_size(full_layer, B, skew):
     assert rel_l2(got[toks], want) < REL_L2_TOL
 
 
+# ----------------------------------------------------------------------------
+# MoE layer, tensor-core (prefill) path: batches past the decode limit
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,K,skew", [(70, 6, 0.0), (200, 6, 0.0), (1000, 6, 0.0), (500, 1, 0.0),
+                                      (300, 4, 2.0)])
+def test_moe_prefill_small(small_layer, B, K, skew):
+    """Several 128-row tiles and K-steps per matrix; experts with more than
+    256 tokens split into chunks with a ragged last chunk (B = 1000, and the
+    skewed routing)."""
+    L = small_layer
+    bits, xv = gs.hidden_bf16(B, L.d_model, tag=2000 + B)
+    ids, gates = gs.route_topk(gs.router_logits(B, L.E, tag=2000 + B, bias_sigma=skew), K)
+    out, st = _moe(L, bits, ids, gates)
+    assert st == 0
+    got = out.cpu().numpy()
+    toks = np.arange(B) if B <= 300 else np.arange(0, B, 7)
+    want = O.moe_layer(L.dense, xv[toks], ids[toks], gates[toks])
+    assert rel_l2(got[toks], want) < REL_L2_TOL
+    # every token, not only the sampled ones, is finite and nonzero
+    assert np.isfinite(got).all() and (np.abs(got).sum(axis=1) > 0).all()
+
+
+def test_moe_prefill_fused_rmsnorm(small_layer):
+    L = small_layer
+    B = 150
+    bits, xv = gs.hidden_bf16(B, L.d_model, tag=78)
+    ids, gates = gs.route_topk(gs.router_logits(B, L.E, tag=78), 6)
+    out, st = _moe(L, bits, ids, gates, out_dtype=torch.bfloat16, flags=G.GALE_FLAG_RESIDUAL_RMSNORM)
+    assert st == 0
+    want = O.chain_step(L.dense, xv, ids, gates)
+    assert rel_l2(out.float().cpu().numpy(), want) < 4e-3
+
+
+def test_moe_prefill_bad_ids(small_layer):
+    """An invalid expert id drops its pair and raises the status; the other
+    tokens are still computed."""
+    L = small_layer
+    B = 100
+    bits, xv = gs.hidden_bf16(B, L.d_model, tag=6)
+    ids, gates = gs.route_topk(gs.router_logits(B, L.E, tag=6), 6)
+    ids = ids.copy()
+    ids[37, 2] = 4000
+    out, st = _moe(L, bits, ids, gates)
+    assert st == G.GALE_ERR_ARG
+    toks = np.array([0, 36, 38, 99])
+    want = O.moe_layer(L.dense, xv[toks], ids[toks], gates[toks])
+    assert rel_l2(out.cpu().numpy()[toks], want) < REL_L2_TOL
+
+
+@pytest.mark.parametrize("skew", [0.0, 1.0])
+def test_moe_prefill_full_size(full_layer, skew):
+    """4096 tokens, top-6 of 256 experts: sampled tokens against the oracle."""
+    L = full_layer
+    B = 4096
+    bits, xv = gs.hidden_bf16(B, L.d_model, tag=4096)
+    ids, gates = gs.route_topk(gs.router_logits(B, L.E, tag=4096, bias_sigma=skew), 6)
+    out, st = _moe(L, bits, ids, gates)
+    assert st == 0
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    toks = np.array([0, 1, 2047, 2048, 4095])
+    want = O.moe_layer(L.dense, xv[toks], ids[toks], gates[toks])
+    assert rel_l2(got[toks], want) < REL_L2_TOL
+
+
 def test_selftest():
     scratch = torch.empty(G.gale_selftest_scratch_bytes(), dtype=torch.uint8, device="cuda")
     assert G.gale_selftest(scratch) == G.GALE_OK
