@@ -3,15 +3,20 @@
 // cores (tcgen05, accumulators in TMEM).
 //
 //   route   : stable counting sort of the (token, slot) pairs by expert
+//   jobs    : every expert's slots cut into chunks (128 tokens for w1/w3,
+//             256 for w2)
 //   gather  : x of every pair, in permuted order, rotated (FWHT-1024) to fp16
-//   w1/w3   : per (expert, 128-row tile, chunk of <= 256 tokens): the packed
-//             signs are expanded to fp16 A tiles +-s_blk (exact) with the
-//             outliers patched in (q * s_row, rounded to fp16), in the K-major
-//             128-byte-swizzled layout the tensor core reads; the tokens come
-//             in by TMA; both products accumulate in TMEM; SwiGLU epilogue
+//   w1/w3   : per (128-row tile, chunk): the packed signs are expanded in
+//             registers to fp16 +-s_blk (exact), the outliers patched in
+//             (q * s_row rounded to fp16), and the A operand is written
+//             straight into TMEM; the tokens come in by TMA as the B operand;
+//             both products accumulate in TMEM; SwiGLU epilogue
 //   rotate  : h -> fp16 FWHT-1024
-//   w2      : same tile kernel with one matrix
+//   w2      : the same tile kernel with one matrix
 //   combine : gate-weighted sum in fixed k order (+ residual, RMSNorm)
+//
+// A in TMEM keeps the shared-memory traffic to the B operand alone: the
+// expansion is paid in instruction issue, the contraction on the tensor pipe.
 #include "common.cuh"
 #include "fwht.cuh"
 #include "moe.cuh"
@@ -24,12 +29,22 @@ namespace gale {
 
 namespace {
 
-constexpr int kTcM = 128;
-constexpr int kTcK = 64;          // K per stage: one 128-byte row of fp16
-constexpr int kTcNRows = 256;     // token rows per chunk
-constexpr int kTcStages = 3;
-constexpr int kTcThreads = 6 * 32;   // producer, MMA, 4 expander/epilogue warps
-constexpr int kPrefetch = 4;      // K-steps of sign words loaded ahead
+constexpr int kTcM = 128;           // weight rows per tile (TMEM lanes)
+constexpr int kTcK = 64;            // K per stage: one 128-byte row of fp16 tokens
+constexpr int kTcStages = 4;
+constexpr int kTcExpWarps = 8;      // expander / epilogue warps: 2 per TMEM lane quarter
+constexpr int kTcThreads = (2 + kTcExpWarps) * 32;
+constexpr int kPrefetch = 4;        // K-steps of sign words loaded ahead
+constexpr int kMaxOutliers = 82;    // per row: round(0.01 * 8192)
+constexpr uint32_t kSentinel = 0xFFFF0000u;
+
+template <int NMAT>
+struct TcCfg {
+    static constexpr int chunk = NMAT == 2 ? 128 : 256;   // tokens per job (MMA N)
+    static constexpr int acc_cols = NMAT * chunk;         // fp32 accumulator columns
+    static constexpr int a_cols = NMAT * 32;              // TMEM columns of one A stage
+    static_assert(acc_cols + kTcStages * a_cols <= 512, "TMEM budget");
+};
 
 struct TcJob {
     int e, n0, n;   // expert, first slot of the chunk, tokens in the chunk
@@ -47,35 +62,87 @@ struct TcArgs {
 };
 
 struct TcSmem {
-    int a0, a1, b, bars, misc, stage_bytes, bytes;
+    int b, idx[2], q[2], srow[2], ent[2], bars, misc, bytes;
 };
 
-__host__ __device__ inline TcSmem tc_smem(int nmat) {
+__host__ __device__ inline int align16(int n) { return (n + 15) & ~15; }
+
+// Shared memory: the token ring, then per matrix the tile's outlier sections
+// (bulk copies) and the outlier lists split by 32-column half.
+__host__ __device__ inline TcSmem tc_smem(int nmat, int chunk, int k) {
     TcSmem s;
-    s.a0 = 0;
-    s.a1 = kTcM * 128;
-    s.b = s.a1 + (nmat == 2 ? kTcM * 128 : 0);
-    s.stage_bytes = s.b + kTcNRows * 128;
-    s.bars = kTcStages * s.stage_bytes;
-    s.misc = s.bars + 8 * (3 * kTcStages + 1);
-    s.bytes = int(align_up(s.misc + 64, 1024)) + 1024;
+    s.b = 0;
+    int o = kTcStages * chunk * 128;
+    for (int mt = 0; mt < 2; ++mt) {
+        s.idx[mt] = s.q[mt] = s.srow[mt] = s.ent[mt] = o;
+        if (mt >= nmat) continue;
+        s.idx[mt] = o;
+        o += align16(kTcM * k * 2);
+        s.q[mt] = o;
+        o += align16(kTcM * k / 2 + 1);
+        s.srow[mt] = o;
+        o += kTcM * 2;
+        s.ent[mt] = o;
+        o += kTcM * (k + 2) * 4;
+    }
+    s.bars = (o + 7) & ~7;
+    s.misc = s.bars + 8 * (3 * kTcStages + 2);
+    s.bytes = s.misc + 16 + 1024;   // + slack to align the base to 1024 bytes
     return s;
 }
 
-// The job list: every expert with tokens, split into chunks of <= 256 slots.
-__global__ void prefill_jobs_kernel(const int32_t* counts, const int32_t* offsets, int E, TcJob* jobs,
-                                    int32_t* n_jobs) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    int n = 0;
-    for (int e = 0; e < E; ++e)
-        for (int t0 = 0; t0 < counts[e]; t0 += kTcNRows) jobs[n++] = TcJob{e, offsets[e] + t0, min(kTcNRows, counts[e] - t0)};
-    *n_jobs = n;
+// Tensor-map encoding of the permuted fp16 activations: boxes of 64 columns
+// x `box_rows` slots, 128-byte swizzle (the K-major SW128 operand layout).
+int act_map(CUtensorMap* m, const void* base, int cols, int64_t rows, int box_rows) {
+    return make_map_3d(m, true, base, uint64_t(cols), uint64_t(rows), 1, uint64_t(cols) * 2,
+                       uint64_t(cols) * 2 * uint64_t(rows), 64, uint32_t(box_rows), true);
 }
 
-// x of every pair in permuted order, rotated, as fp16: one warp per (slot, 1024-block).
-// Slots past the routed pairs (pairs with an invalid expert id are dropped)
-// stay zero.
-__global__ void __launch_bounds__(256) gather_rotate_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
+// Both job lists (chunks of 128 and of 256 slots), one thread per expert.
+__global__ void __launch_bounds__(1024) prefill_jobs_kernel(const int32_t* counts, const int32_t* offsets, int E,
+                                                            TcJob* jobs13, int32_t* n13, TcJob* jobs2,
+                                                            int32_t* n2) {
+    __shared__ int tmp[32];
+    __shared__ int tot[2];
+    const int e = threadIdx.x;
+    const int lane = e & 31, warp = e >> 5;
+    const int n_e = e < E ? counts[e] : 0;
+    for (int which = 0; which < 2; ++which) {
+        const int chunk = which ? 256 : 128;
+        const int c = (n_e + chunk - 1) / chunk;
+        int incl = c;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) tmp[warp] = incl;
+        __syncthreads();
+        if (e == 0) {
+            int run = 0;
+            for (int w = 0; w < int(blockDim.x >> 5); ++w) {
+                const int v = tmp[w];
+                tmp[w] = run;
+                run += v;
+            }
+            tot[which] = run;
+        }
+        __syncthreads();
+        const int first = tmp[warp] + incl - c;
+        TcJob* jobs = which ? jobs2 : jobs13;
+        for (int i = 0; i < c; ++i) jobs[first + i] = TcJob{e, offsets[e] + i * chunk, min(chunk, n_e - i * chunk)};
+        __syncthreads();
+    }
+    if (e == 0) {
+        *n13 = tot[0];
+        *n2 = tot[1];
+    }
+}
+
+// x of every pair in permuted order, rotated, as fp16: one warp per (slot,
+// 1024-block).  Slots past the routed pairs (pairs with an invalid expert id
+// are dropped) are left alone; no job reads them.
+__global__ void __launch_bounds__(256) gather_rotate_kernel(const uint16_t* __restrict__ x,
+                                                            const int32_t* __restrict__ perm,
                                                             const int32_t* __restrict__ n_routed, int K, int d,
                                                             int64_t slots, __half* __restrict__ y) {
     const int lane = threadIdx.x & 31;
@@ -96,35 +163,58 @@ __global__ void __launch_bounds__(256) gather_rotate_kernel(const uint16_t* __re
     for (int i = 0; i < 32; ++i) dst[32 * i + lane] = __float2half_rn(v[i] * (1.0f / 32.0f));
 }
 
-// One (expert, 128-row tile, token chunk) job of w1/w3 (NMAT = 2, SwiGLU
-// epilogue) or w2 (NMAT = 1).
+// The 16 fp16 pairs of 32 weights: sign word w (bit c set = column c negative)
+// and the block scale's fp16 bits sc.  Pair p holds columns 2p (low half) and
+// 2p+1.  Multiplying a byte by 2^(15-2i) + 2^(30-2i) moves its bits 2i and
+// 2i+1 to bit positions 15 and 31; the two shifted copies do not overlap, so
+// no carry disturbs them.
+__device__ __forceinline__ void expand_signs(uint32_t w, uint32_t sc, uint32_t (&v)[16]) {
+    const uint32_t h2 = sc * 0x10001u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t b = __byte_perm(w, 0u, 0x4440u + j);
+        v[4 * j + 0] = ((b * 0x40008000u) & 0x80008000u) ^ h2;
+        v[4 * j + 1] = ((b * 0x10002000u) & 0x80008000u) ^ h2;
+        v[4 * j + 2] = ((b * 0x04000800u) & 0x80008000u) ^ h2;
+        v[4 * j + 3] = ((b * 0x01000200u) & 0x80008000u) ^ h2;
+    }
+}
+
+// One (128-row tile, token chunk) job of w1/w3 (NMAT = 2, SwiGLU epilogue) or
+// w2 (NMAT = 1).  Warp 0 streams token tiles by TMA, warp 1 owns TMEM and
+// issues the MMAs, warps 2..9 expand weights into TMEM and run the epilogue.
 template <int NMAT>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_constant__ CUtensorMap xmap, TcArgs A) {
+    using Cfg = TcCfg<NMAT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
-    const int job_id = blockIdx.x, mtile = blockIdx.y;
+    const int mtile = blockIdx.x, job_id = blockIdx.y;
     if (job_id >= *A.n_jobs) return;
     const TcJob job = A.jobs[job_id];
-    const TcSmem S = tc_smem(NMAT);
+    const int nk = A.cols / kTcK;
+    const int kout = outliers_per_row(A.cols);
+    const TcSmem S = tc_smem(NMAT, Cfg::chunk, kout);
     uint64_t* b_full = reinterpret_cast<uint64_t*>(smem + S.bars);
     uint64_t* a_full = b_full + kTcStages;
     uint64_t* mma_done = a_full + kTcStages;
     uint64_t* acc_full = mma_done + kTcStages;
+    uint64_t* side_full = acc_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S.misc);
     int* fail = reinterpret_cast<int*>(smem + S.misc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nk = A.cols / kTcK;
     const int n_mma = (job.n + 15) & ~15;
-    const int nbox = (job.n + 63) / 64;
     const uint32_t idesc = umma_idesc_f16(kTcM, n_mma);
+    const int r0 = mtile * kTcM;
+    const char* rec = A.base + int64_t(job.e) * A.stride;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kTcStages; ++s) {
             mbar_init(b_full + s, 1);
-            mbar_init(a_full + s, 128);
+            mbar_init(a_full + s, kTcExpWarps * 32);
             mbar_init(mma_done + s, 1);
         }
         mbar_init(acc_full, 1);
+        mbar_init(side_full, 1);
         *fail = 0;
         fence_mbar_init();
     }
@@ -138,8 +228,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------- producer: token tiles by TMA
+        // ---------------- producer: the tile's outlier sections, then token tiles
         if (lane == 0) {
+            const uint32_t idx_bytes = uint32_t(kTcM * kout * 2), q_bytes = uint32_t(kTcM * kout / 2);
+            mbar_arrive_expect_tx(side_full, uint32_t(NMAT) * (idx_bytes + q_bytes + kTcM * 2));
+            for (int mt = 0; mt < NMAT; ++mt) {
+                const MatView mv = make_view(rec + (mt ? A.off_b : A.off_a), A.rows, A.cols);
+                bulk_load(smem + S.idx[mt], mv.idx + int64_t(r0) * kout, idx_bytes, side_full);
+                bulk_load(smem + S.q[mt], mv.q + int64_t(r0) * kout / 2, q_bytes, side_full);
+                bulk_load(smem + S.srow[mt], mv.s_row + r0, kTcM * 2, side_full);
+            }
             int issued = 0;
             for (int ks = 0; ks < nk; ++ks) {
                 const int s = ks % kTcStages;
@@ -147,13 +245,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
                     *fail = 1;
                     break;
                 }
-                uint8_t* bdst = smem + s * S.stage_bytes + S.b;
-                mbar_arrive_expect_tx(b_full + s, uint32_t(nbox * 64 * 128));
-                for (int bx = 0; bx < nbox; ++bx)
-                    tma_load_3d(bdst + bx * 64 * 128, &xmap, b_full + s, ks * kTcK, job.n0 + bx * 64, 0);
+                mbar_arrive_expect_tx(b_full + s, uint32_t(Cfg::chunk * 128));
+                tma_load_3d(smem + S.b + s * Cfg::chunk * 128, &xmap, b_full + s, ks * kTcK, job.n0, 0);
                 issued = ks + 1;
             }
             // no copy may still be landing when the CTA exits
+            if (!mbar_wait(side_full, 0)) *fail = 1;
             for (int ks = issued - kTcStages < 0 ? 0 : issued - kTcStages; ks < issued; ++ks)
                 if (!mbar_wait(b_full + ks % kTcStages, (ks / kTcStages) & 1)) *fail = 1;
         }
@@ -168,47 +265,64 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
                     break;
                 }
                 tc_fence_after();
-                const uint32_t st = smem_u32(smem + s * S.stage_bytes);
+                const uint32_t bst = smem_u32(smem + S.b + s * Cfg::chunk * 128);
+                const uint32_t ast = tmem + uint32_t(Cfg::acc_cols + s * Cfg::a_cols);
 #pragma unroll
                 for (int mt = 0; mt < NMAT; ++mt) {
 #pragma unroll
-                    for (int kk = 0; kk < kTcK / 16; ++kk) {
-                        const uint64_t ad = umma_desc_sw128(st + (mt ? S.a1 : S.a0) + kk * 32);
-                        const uint64_t bd = umma_desc_sw128(st + S.b + kk * 32);
-                        umma_f16(tmem + uint32_t(mt * 256), ad, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < kTcK / 16; ++kk)
+                        umma_f16_ts(tmem + uint32_t(mt * Cfg::chunk), ast + uint32_t(mt * 32 + kk * 8),
+                                    umma_desc_sw128(bst + kk * 32), idesc, (ks > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(mma_done + s);
             }
             umma_commit(acc_full);
         }
     } else {
-        // ---------------- expanders: one weight row per thread
-        const int t = threadIdx.x - 64;
-        const int row = mtile * kTcM + t;
-        const bool valid = row < A.rows;
-        const char* rec = A.base + int64_t(job.e) * A.stride;
+        // ---------------- expanders: thread (row t, half h) covers 32 columns of every K-step
+        const int ew = warp - 2;
+        const int quarter = warp & 3;   // TMEM lane quarter this warp may access
+        const int h = ew >> 2;
+        const int t = 32 * quarter + lane;
+        const int row = r0 + t;
+        const int nb = A.cols / 128;
+        bool ok = mbar_wait(side_full, 0);
+        // this thread's outliers in column order, as (column << 16 | fp16 value)
+        int cur[NMAT];
+        uint32_t ent[NMAT];
+#pragma unroll
+        for (int mt = 0; mt < NMAT; ++mt) {
+            const uint16_t* sidx = reinterpret_cast<const uint16_t*>(smem + S.idx[mt]) + t * kout;
+            const uint8_t* sqv = smem + S.q[mt];
+            const float srow = __half2float(reinterpret_cast<const __half*>(smem + S.srow[mt])[t]);
+            uint32_t* list = reinterpret_cast<uint32_t*>(smem + S.ent[mt]) + t * (kout + 2);
+            int n0 = 0;
+            for (int j = 0; j < kout; ++j) n0 += ((sidx[j] >> 5) & 1) == 0;
+            const int start = h ? n0 + 1 : 0;
+            int o = start;
+            for (int j = 0; j < kout; ++j) {
+                const int c = sidx[j];
+                if (((c >> 5) & 1) != h) continue;
+                const int n = t * kout + j;
+                const int byte = sqv[n >> 1];
+                int qv = (n & 1) ? (byte >> 4) : (byte & 0xF);
+                qv = qv >= 8 ? qv - 16 : qv;
+                list[o++] = (uint32_t(c) << 16) | __half_as_ushort(__float2half_rn(float(qv) * srow));
+            }
+            list[o] = kSentinel;
+            cur[mt] = start;
+            ent[mt] = list[start];
+        }
+        // sign words / block scales of K-steps ks .. ks + kPrefetch - 1
         MatView mv[NMAT];
 #pragma unroll
         for (int mt = 0; mt < NMAT; ++mt) mv[mt] = make_view(rec + (mt ? A.off_b : A.off_a), A.rows, A.cols);
-        const int nb = A.cols / 128;
-        // next outlier of the row per matrix: its position n and column (cols when none is left)
-        int on[NMAT], oc[NMAT];
-        float srow[NMAT];
-#pragma unroll
-        for (int mt = 0; mt < NMAT; ++mt) {
-            on[mt] = 0;
-            oc[mt] = (valid && mv[mt].k > 0) ? int(mv[mt].idx[int64_t(row) * mv[mt].k]) : A.cols;
-            srow[mt] = valid ? __half2float(mv[mt].s_row[row]) : 0.f;
-        }
-        // sign words and block scale of K-steps ks .. ks + kPrefetch - 1, per matrix
-        uint2 wq[NMAT][kPrefetch];
-        uint32_t sq[NMAT][kPrefetch];
-        auto fetch = [&](int mt, int ks, uint2& w, uint32_t& sc) {
-            w = make_uint2(0u, 0u);
+        uint32_t wq[NMAT][kPrefetch], sq[NMAT][kPrefetch];
+        auto fetch = [&](int mt, int ks, uint32_t& w, uint32_t& sc) {
+            w = 0u;
             sc = 0u;
-            if (valid && ks < nk) {
-                w = __ldg(reinterpret_cast<const uint2*>(mv[mt].signs + int64_t(row) * (A.cols / 32)) + ks);
+            if (ks < nk) {
+                w = __ldg(mv[mt].signs + int64_t(row) * (A.cols / 32) + 2 * ks + h);
                 sc = __ldg(reinterpret_cast<const uint16_t*>(mv[mt].s_blk) + int64_t(row) * nb + (ks >> 1));
             }
         };
@@ -216,19 +330,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
         for (int mt = 0; mt < NMAT; ++mt)
 #pragma unroll
             for (int p = 0; p < kPrefetch; ++p) fetch(mt, p, wq[mt][p], sq[mt][p]);
-        bool ok = true;
         for (int ks = 0; ks < nk; ++ks) {
             const int s = ks % kTcStages;
-            if (ok && ks >= kTcStages && !mbar_wait(mma_done + s, ((ks / kTcStages) - 1) & 1)) {
-                ok = false;
-                *fail = 1;
-            }
+            if (ok && ks >= kTcStages && !mbar_wait(mma_done + s, ((ks / kTcStages) - 1) & 1)) ok = false;
+            tc_fence_after();
             const int slot = ks % kPrefetch;
+            const int lo = ks * kTcK + 32 * h, hi = lo + 32;
 #pragma unroll
             for (int mt = 0; mt < NMAT; ++mt) {
-                // this K-step's words, then refill the slot kPrefetch steps ahead
-                uint2 w = make_uint2(0u, 0u);
-                uint32_t sc = 0u;
+                uint32_t w = 0u, sc = 0u;
 #pragma unroll
                 for (int p = 0; p < kPrefetch; ++p)
                     if (p == slot) {
@@ -236,31 +346,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
                         sc = sq[mt][p];
                         fetch(mt, ks + kPrefetch, wq[mt][p], sq[mt][p]);
                     }
-                uint8_t* arow = smem + s * S.stage_bytes + (mt ? S.a1 : S.a0) + t * 128;
-                const uint32_t h2 = sc | (sc << 16);
-                // 16-byte chunk c holds columns 8c .. 8c+7; a set sign bit negates the fp16 scale
+                uint32_t v[16];
+                expand_signs(w, sc, v);
+                // outliers of this range replace their weights
+                int prev_p = -1;
+                uint32_t prev_a = 0u;
+                for (;;) {
+                    const int ecol = int(ent[mt] >> 16);
+                    const bool mine = ecol < hi;
+                    if (!__any_sync(0xffffffffu, mine)) break;
+                    int P = -1;
+                    uint32_t a = 0u;
+                    if (mine) {
+                        const int u = ecol - lo;
+                        P = u >> 1;
+                        const uint32_t val = ent[mt] & 0xFFFFu;
+                        uint32_t other = sc ^ (((w >> (u ^ 1)) & 1u) << 15);
+                        if (P == prev_p) other = (u & 1) ? (prev_a & 0xFFFFu) : (prev_a >> 16);
+                        a = (u & 1) ? (other | (val << 16)) : (val | (other << 16));
+                        prev_p = P;
+                        prev_a = a;
+                        ent[mt] = reinterpret_cast<const uint32_t*>(smem + S.ent[mt])[t * (kout + 2) + ++cur[mt]];
+                    }
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t byte = ((c < 4 ? w.x : w.y) >> (8 * (c & 3))) & 0xFFu;
-                    uint32_t v[4];
-#pragma unroll
-                    for (int p = 0; p < 4; ++p)
-                        v[p] = h2 ^ (((byte >> (2 * p)) & 1u) << 15) ^ (((byte >> (2 * p + 1)) & 1u) << 31);
-                    *reinterpret_cast<uint4*>(arow + ((c ^ (t & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+                    for (int p = 0; p < 16; ++p) v[p] = (P == p) ? a : v[p];
                 }
-                // outliers of this K-step replace their weights by q * s_row
-                const int kend = (ks + 1) * kTcK;
-                while (oc[mt] < kend) {
-                    const int64_t n = int64_t(row) * mv[mt].k + on[mt];
-                    const int c = oc[mt] - ks * kTcK;
-                    const __half val = __float2half_rn(float(load_q(mv[mt].q, n)) * srow[mt]);
-                    if (c >= 0)   // indices are strictly ascending in a valid record
-                        *reinterpret_cast<__half*>(arow + (((c >> 3) ^ (t & 7)) << 4) + (c & 7) * 2) = val;
-                    ++on[mt];
-                    oc[mt] = on[mt] < mv[mt].k ? int(mv[mt].idx[n + 1]) : A.cols;
-                }
+                tmem_st16(tmem + (uint32_t(32 * quarter) << 16) +
+                              uint32_t(Cfg::acc_cols + s * Cfg::a_cols + mt * 32 + 16 * h),
+                          v);
             }
-            fence_proxy_async();
+            tmem_wait_st();
+            tc_fence_before();
             mbar_arrive(a_full + s);
         }
         // ---------------- epilogue: TMEM -> registers -> global
@@ -268,20 +384,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
         ok = __all_sync(0xffffffffu, ok && acc_ok);
         if (!ok) *fail = 1;
         tc_fence_after();
-        const int q = warp & 3;   // TMEM lane quarter this warp may read
-        const int erow = mtile * kTcM + 32 * q + lane;
         if (ok) {
-            for (int col = 0; col < n_mma; col += 16) {
+            constexpr int kHalfCols = Cfg::chunk / 2;
+            for (int col = h * kHalfCols; col < h * kHalfCols + kHalfCols && col < n_mma; col += 16) {
                 float v1[16], v3[16];
-                tmem_ld16(tmem + (uint32_t(32 * q) << 16) + uint32_t(col), v1);
-                if (NMAT == 2) tmem_ld16(tmem + (uint32_t(32 * q) << 16) + uint32_t(256 + col), v3);
-                if (erow < A.rows) {
+                tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(col), v1);
+                if (NMAT == 2) tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(Cfg::chunk + col), v3);
+                if (row < A.rows) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int j = col + i;
                         if (j < job.n) {
                             const float y = NMAT == 2 ? silu(v1[i]) * v3[i] : v1[i];
-                            A.out[int64_t(job.n0 + j) * A.rows + erow] = y;
+                            A.out[int64_t(job.n0 + j) * A.rows + row] = y;
                         }
                     }
                 }
@@ -298,10 +413,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
     }
 }
 
-int act_map(CUtensorMap* m, const void* base, int cols, int64_t rows) {
-    // fp16 [rows][cols], boxes of 64 columns x 64 rows, 128-byte swizzle
-    return make_map_3d(m, true, base, uint64_t(cols), uint64_t(rows), 1, uint64_t(cols) * 2,
-                       uint64_t(cols) * 2 * uint64_t(rows), 64, 64, true);
+template <int NMAT>
+int launch_tc(const CUtensorMap& map, const TcArgs& a, int max_jobs, cudaStream_t st) {
+    const TcSmem S = tc_smem(NMAT, TcCfg<NMAT>::chunk, outliers_per_row(a.cols));
+    int rc = ensure_smem(reinterpret_cast<const void*>(tc_tile_kernel<NMAT>), S.bytes);
+    if (rc != GALE_OK) return rc;
+    dim3 grid(unsigned(a.rows / kTcM), unsigned(max_jobs));
+    tc_tile_kernel<NMAT><<<grid, kTcThreads, S.bytes, st>>>(map, a);
+    GALE_LAUNCH_CHECK();
+    return GALE_OK;
 }
 
 }  // namespace
@@ -321,10 +441,11 @@ PrefillWs carve_prefill_ws(void* ws, const gale_layer& L, int B, int K) {
     w.offsets = reinterpret_cast<int32_t*>(take(4 * (int64_t(L.n_experts) + 1)));
     w.perm = reinterpret_cast<int32_t*>(take(4 * P));
     w.pos_of_pair = reinterpret_cast<int32_t*>(take(4 * P));
-    const int64_t max_jobs = L.n_experts + P / kTcNRows + 1;
-    w.jobs = take(int64_t(sizeof(TcJob)) * max_jobs);
-    w.n_jobs = reinterpret_cast<int32_t*>(take(4));
-    w.max_jobs = int(max_jobs);
+    w.max_jobs13 = int(L.n_experts + P / 128 + 1);
+    w.max_jobs2 = int(L.n_experts + P / 256 + 1);
+    w.jobs13 = take(int64_t(sizeof(TcJob)) * w.max_jobs13);
+    w.jobs2 = take(int64_t(sizeof(TcJob)) * w.max_jobs2);
+    w.n_jobs = reinterpret_cast<int32_t*>(take(8));
     w.x16 = reinterpret_cast<__half*>(take(2 * P * dm));
     w.h = reinterpret_cast<float*>(take(4 * P * df));
     w.h16 = reinterpret_cast<__half*>(take(2 * P * df));
@@ -335,7 +456,11 @@ PrefillWs carve_prefill_ws(void* ws, const gale_layer& L, int B, int K) {
 }
 
 bool prefill_supported(const gale_layer& L, int B, int K) {
-    return int64_t(B) * K <= (int64_t(1) << 24) && L.d_model <= 16384 && L.d_ff <= 16384;
+    if (int64_t(B) * K > (int64_t(1) << 24) || L.n_experts > 1024) return false;
+    // a tile's outlier lists stay in shared memory
+    const int k1 = outliers_per_row(L.d_model), k2 = outliers_per_row(L.d_ff);
+    return k1 <= kMaxOutliers && k2 <= kMaxOutliers && tc_smem(2, TcCfg<2>::chunk, k1).bytes <= 227 * 1024 &&
+           tc_smem(1, TcCfg<1>::chunk, k2).bytes <= 227 * 1024;
 }
 
 int launch_moe_prefill(const gale_layer& L, const uint16_t* x, const int32_t* ids, const float* gates, int B, int K,
@@ -355,60 +480,49 @@ int launch_moe_prefill(const gale_layer& L, const uint16_t* x, const int32_t* id
     ra.status = w.status;
     int rc = launch_route_permute(ra, st);
     if (rc != GALE_OK) return rc;
-    prefill_jobs_kernel<<<1, 32, 0, st>>>(w.counts, w.offsets, L.n_experts, static_cast<TcJob*>(w.jobs), w.n_jobs);
+    prefill_jobs_kernel<<<1, 1024, 0, st>>>(w.counts, w.offsets, L.n_experts, static_cast<TcJob*>(w.jobs13),
+                                            w.n_jobs, static_cast<TcJob*>(w.jobs2), w.n_jobs + 1);
     GALE_LAUNCH_CHECK();
-    // permuted, rotated fp16 activations
-    GALE_CUDA_TRY(cudaMemsetAsync(w.x16, 0, size_t(P) * L.d_model * 2, st));
     {
         const int64_t warps = P * (L.d_model / 1024);
-        gather_rotate_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, st>>>(x, w.perm, w.offsets + L.n_experts, K,
-                                                                               L.d_model, P, w.x16);
+        gather_rotate_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, st>>>(x, w.perm, w.offsets + L.n_experts,
+                                                                                  K, L.d_model, P, w.x16);
         GALE_LAUNCH_CHECK();
     }
     const int64_t l1 = make_layout(L.d_ff, L.d_model).total;
     CUtensorMap xm;
-    rc = act_map(&xm, w.x16, L.d_model, P);
+    rc = act_map(&xm, w.x16, L.d_model, P, TcCfg<2>::chunk);
     if (rc != GALE_OK) return rc;
     TcArgs a{};
     a.base = static_cast<const char*>(L.base);
     a.stride = L.expert_stride;
-    a.jobs = static_cast<const TcJob*>(w.jobs);
-    a.n_jobs = w.n_jobs;
     a.status = w.status;
     // w1 / w3 + SwiGLU
+    a.jobs = static_cast<const TcJob*>(w.jobs13);
+    a.n_jobs = w.n_jobs;
     a.off_a = 0;
     a.off_b = l1;
     a.rows = L.d_ff;
     a.cols = L.d_model;
     a.out = w.h;
-    {
-        const TcSmem S = tc_smem(2);
-        rc = ensure_smem(reinterpret_cast<const void*>(tc_tile_kernel<2>), S.bytes);
-        if (rc != GALE_OK) return rc;
-        dim3 grid(w.max_jobs, (L.d_ff + kTcM - 1) / kTcM);
-        tc_tile_kernel<2><<<grid, kTcThreads, S.bytes, st>>>(xm, a);
-        GALE_LAUNCH_CHECK();
-    }
+    rc = launch_tc<2>(xm, a, w.max_jobs13, st);
+    if (rc != GALE_OK) return rc;
     // rotate h
     rc = gale_fwht1024(w.h, GALE_F32, w.h16, GALE_F16, P, L.d_ff, st);
     if (rc != GALE_OK) return rc;
     CUtensorMap hm;
-    rc = act_map(&hm, w.h16, L.d_ff, P);
+    rc = act_map(&hm, w.h16, L.d_ff, P, TcCfg<1>::chunk);
     if (rc != GALE_OK) return rc;
     // w2
+    a.jobs = static_cast<const TcJob*>(w.jobs2);
+    a.n_jobs = w.n_jobs + 1;
     a.off_a = 2 * l1;
     a.off_b = 2 * l1;
     a.rows = L.d_model;
     a.cols = L.d_ff;
     a.out = w.o;
-    {
-        const TcSmem S = tc_smem(1);
-        rc = ensure_smem(reinterpret_cast<const void*>(tc_tile_kernel<1>), S.bytes);
-        if (rc != GALE_OK) return rc;
-        dim3 grid(w.max_jobs, (L.d_model + kTcM - 1) / kTcM);
-        tc_tile_kernel<1><<<grid, kTcThreads, S.bytes, st>>>(hm, a);
-        GALE_LAUNCH_CHECK();
-    }
+    rc = launch_tc<1>(hm, a, w.max_jobs2, st);
+    if (rc != GALE_OK) return rc;
     return launch_moe_combine(w.o, w.pos_of_pair, gates, x, B, K, L.d_model, out, out_dtype, fuse_norm, eps,
                               w.scratch, st);
 }
