@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_mma_kernel(
     const __grid_constant__ CUtensorMap smap_b, const __grid_constant__ CUtensorMap bmap_b, MatView a, MatView b,
     const float* __restrict__ x, int ntok, float* __restrict__ y, GemvSmem S) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
+    uint8_t* smem = smem_align1024(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int C = a.cols;
     const StageLayout L = stage_layout(C);

@@ -204,7 +204,8 @@ extern "C" int gale_moe_forward(const gale_layer* layer, const uint16_t* x, cons
         return GALE_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return GALE_ERR_ALIGN;
     cudaStream_t st = as_stream(stream);
-    GALE_CUDA_TRY(cudaMemsetAsync(w.status, 0, sizeof(int32_t), st));
+    // the status word and the decode kernel's grid-barrier counters
+    GALE_CUDA_TRY(cudaMemsetAsync(w.status, 0, 8 * sizeof(int32_t), st));
     if (B == 0) return GALE_OK;
     if (!x || !ids || !gates || !out) return GALE_ERR_ARG;
     if (!aligned(x, 4) || !aligned(ids, 4) || !aligned(gates, 4) || !aligned(out, 4)) return GALE_ERR_ALIGN;

@@ -1,19 +1,23 @@
-// Decode path of gale_moe_forward: two streaming kernels chained by
-// programmatic dependent launch.
+// Decode path of gale_moe_forward: one persistent kernel, one CTA per SM,
+// launched cooperatively (all CTAs resident).
 //
-//   w13 : jobs (expert, token pair, row block) of w1 and w3.  Each CTA rotates
-//         (FWHT-1024, warp shuffles) the tokens its jobs need and keeps their
-//         fixed-point int8 digits in shared memory; a producer warp streams the packed
-//         tiles with TMA while 8 consumer warps run the tensor-core tile
-//         routine split by (matrix, 1024-column chunk); SwiGLU; h to global.
-//   w2  : jobs (expert, token pair, row block) of w2.  After waiting for w13,
-//         each CTA rotates the h rows its jobs need; expert outputs go to
-//         global, and the last expert to finish a (token, row block) sums the
-//         K contributions in fixed k order with the gates (deterministic, no
-//         float atomics), optionally adds the residual; the last row block of
-//         a token applies RMSNorm.
-// Both kernels compute the routing themselves from the ids, and w2's producer
-// starts streaming weights before waiting for w13.
+//   routing : every CTA groups the (token, k) pairs by expert from the ids;
+//             a job is (expert, group of <= 2 of its tokens, row block)
+//   stream  : a producer warp copies the packed tiles of the CTA's w1/w3
+//             jobs and then of its w2 jobs into a ring of stages (TMA), with
+//             no dependency on any computation, so the w2 weights arrive
+//             while w1/w3 is still being computed
+//   w1/w3   : 8 consumer warps split each job by (matrix, 1024-column chunk)
+//             on the int8 tensor cores; the outlier corrections of the job
+//             are split by (matrix, row); the last warp to finish a job sums
+//             the pieces and stores h = silu(w1 x) * (w3 x)
+//   barrier : grid-wide (bounded wait): h of every expert is complete
+//   w2      : the same with the rotated h rows; the last warp of a job
+//             stores the expert outputs, and the last expert to finish a
+//             (token, 64-row block) sums the K contributions in fixed k order
+//             with the gates (deterministic, no float atomics), optionally
+//             adding the residual; the last row block of a token applies
+//             RMSNorm.
 #include "common.cuh"
 #include "fwht.cuh"
 #include "moe.cuh"
@@ -24,8 +28,11 @@ namespace gale {
 
 namespace {
 
-constexpr int kDecWarps = 8;
+constexpr int kDecWarps = 8;                   // consumer warps
 constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kDecBlock = kDecThreads + 32;    // + the producer warp
+constexpr int kCapMax = 8;                     // rotated vectors cached per CTA
+constexpr int kMaxStages = 16;
 
 struct DecArgs {
     const char* base;
@@ -45,21 +52,24 @@ struct DecArgs {
 // routing inside a CTA (B*K <= kDecodeMaxPairs, E <= 1024)
 // ----------------------------------------------------------------------------
 
-struct RouteSmem {
-    int cnt[1024];                    // per expert: valid pairs
-    int off[1024];                    // per expert: first slot
-    int aidx[1024];                   // per expert: index among the active experts
-    int pe[kDecodeMaxPairs];          // expert of each pair, -1 if dropped
-    int active[kDecodeMaxPairs];      // active expert ids, increasing
-    int first_slot[kDecodeMaxPairs];
-    int n_tok[kDecodeMaxPairs];
-    int job_start[kDecodeMaxPairs + 1];
-    int grp_base[kDecodeMaxPairs + 1];
-    int slot_tok[kDecodeMaxPairs];    // token of each slot
-    int pos_of_pair[kDecodeMaxPairs]; // slot of each pair (-1: dropped)
-    int tok_valid[kDecodeMaxPairs];   // valid pairs per token
+struct RouteTables {
+    int active[kDecodeMaxPairs];       // active expert ids, increasing
+    int first_slot[kDecodeMaxPairs];   // first slot of each active expert
+    int n_tok[kDecodeMaxPairs];        // valid pairs of each active expert
+    int grp_base[kDecodeMaxPairs + 1]; // first token group of each active expert
+    int slot_tok[kDecodeMaxPairs];     // token of each slot
+    int pos_of_pair[kDecodeMaxPairs];  // slot of each pair (-1: dropped)
+    int tok_valid[kDecodeMaxPairs];    // valid pairs per token
+    int n_active, n_groups, bad;
+};
+
+// Scratch of the block-wide routing; it lives in the ring before any copy starts.
+struct RouteScratch {
+    int cnt[1024];   // per expert: valid pairs
+    int off[1024];   // per expert: first slot
+    int aidx[1024];  // per expert: index among the active experts
+    int pe[kDecodeMaxPairs];
     int scan_tmp[32];
-    int n_active, n_jobs, n_groups, bad;
 };
 
 // Block-wide exclusive scan of a[0..n) (n <= 4 * blockDim.x) in place; returns the total.
@@ -103,178 +113,186 @@ __device__ int block_exclusive_scan(int* a, int n, int* tmp) {
     return total;
 }
 
-// Small batches (B*K <= 32): one warp computes the same tables with
-// shuffles, lane p handling pair p.
-__device__ void build_route_small(const DecArgs& A, RouteSmem& R, int tiles) {
+// Small batches (B*K <= 32): one warp builds the tables.  Lane p holds pair
+// p; a bitonic sort of the keys (expert << 5 | p) leaves the i-th valid pair
+// of the stable expert order in lane i, which is its slot.
+__device__ void build_route_small(const DecArgs& A, RouteTables& R) {
     const int lane = threadIdx.x & 31;
-    const int BK = A.B * A.K, E = A.E;
+    const int BK = A.B * A.K, E = A.E, K = A.K;
     const bool in = lane < BK;
-    int e = in ? A.ids[lane] : -1;
+    const int e = in ? __ldg(A.ids + lane) : -1;
     bool ok = in && e >= 0 && e < E;
-    if (in) {
-        const int t0 = lane - lane % A.K;
-        for (int j = t0; ok && j < lane; ++j) ok = A.ids[j] != e;
-    }
-    if (!ok) e = -1;
-    const unsigned bad = __ballot_sync(0xffffffffu, in && !ok);
-    // slot = rank of (e, p) among the valid pairs; first pair of each expert
-    int rank = 0, same = 0, first_before = 0;
-    bool first = ok;
-    for (int q = 0; q < 32; ++q) {
-        const int eq = __shfl_sync(0xffffffffu, e, q);
-        if (eq < 0) continue;
-        rank += (eq < e) || (eq == e && q < lane);
-        same += (eq == e);
-        if (eq == e && q < lane) first = false;
-    }
-    // active index: number of distinct valid experts below e
-    const unsigned firsts = __ballot_sync(0xffffffffu, first);
-    for (int q = 0; q < 32; ++q) {
-        const int eq = __shfl_sync(0xffffffffu, e, q);
-        if ((firsts >> q) & 1) first_before += (eq < e);
-    }
-    const int n_active = __popc(firsts);
-    if (in) R.pos_of_pair[lane] = ok ? rank : -1;
-    if (ok) R.slot_tok[rank] = lane / A.K;
-    int groups = 0;
-    if (first) {
-        R.active[first_before] = e;
-        R.first_slot[first_before] = rank;
-        R.n_tok[first_before] = same;
-        groups = (same + 1) / 2;
-    }
-    // prefix sums of groups and jobs over the active experts (indexed by first_before)
-    int g_a = 0;
-    for (int q = 0; q < 32; ++q) {
-        const int gq = __shfl_sync(0xffffffffu, groups, q);
-        const int aq = __shfl_sync(0xffffffffu, first_before, q);
-        if (((firsts >> q) & 1) && aq < first_before) g_a += gq;
-    }
-    if (first) {
-        R.grp_base[first_before] = g_a;
-        R.job_start[first_before] = g_a * tiles;
-    }
-    int n_groups = groups;
-    for (int o = 16; o > 0; o >>= 1) n_groups += __shfl_xor_sync(0xffffffffu, n_groups, o);
     {
-        int v = 0;   // valid pairs of token `lane`
-        for (int k = 0; k < A.K; ++k) {
-            const int src = lane * A.K + k;
-            const int okq = __shfl_sync(0xffffffffu, ok ? 1 : 0, src & 31);
-            if (src < BK) v += okq;
+        // an id repeated within a token drops the later pair
+        const int t0 = lane - lane % K;
+#pragma unroll 1
+        for (int j = 0; j < K; ++j) {
+            const int ej = __shfl_sync(0xffffffffu, e, (t0 + j) & 31);
+            if (t0 + j < lane && ej == e) ok = false;
         }
-        if (lane < A.B) R.tok_valid[lane] = v;
     }
+    const unsigned okb = __ballot_sync(0xffffffffu, ok);
+    const unsigned bad = __ballot_sync(0xffffffffu, in && !ok);
+    uint32_t key = ok ? (uint32_t(e) << 5) | uint32_t(lane) : 0xFFFFFFFFu;
+#pragma unroll
+    for (int k2 = 2; k2 <= 32; k2 <<= 1) {
+#pragma unroll
+        for (int j = k2 >> 1; j > 0; j >>= 1) {
+            const uint32_t other = __shfl_xor_sync(0xffffffffu, key, j);
+            const bool keep_min = ((lane & j) == 0) == ((lane & k2) == 0);
+            key = keep_min ? min(key, other) : max(key, other);
+        }
+    }
+    const bool v = key != 0xFFFFFFFFu;
+    const int se = v ? int(key >> 5) : -1, sp = int(key & 31u);
+    const int nvalid = __popc(okb);
+    if (v) {
+        R.slot_tok[lane] = sp / K;
+        R.pos_of_pair[sp] = lane;
+    }
+    if (in && !ok) R.pos_of_pair[lane] = -1;
+    // runs of equal experts in slot order: the active experts
+    const int prev = __shfl_up_sync(0xffffffffu, se, 1);
+    const bool first = v && (lane == 0 || prev != se);
+    const unsigned fb = __ballot_sync(0xffffffffu, first);
+    const unsigned later = lane == 31 ? 0u : fb & (0xFFFFFFFFu << (lane + 1));
+    const int run = (later ? __ffs(later) - 1 : nvalid) - lane;
+    const int groups = first ? (run + 1) / 2 : 0;
+    int incl = groups;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (first) {
+        const int a = __popc(fb & ((1u << lane) - 1u));
+        R.active[a] = se;
+        R.first_slot[a] = lane;
+        R.n_tok[a] = run;
+        R.grp_base[a] = incl - groups;
+    }
+    if (lane < A.B) R.tok_valid[lane] = __popc(okb & (((1u << K) - 1u) << (lane * K)));
+    const int n_groups = __shfl_sync(0xffffffffu, incl, 31);
     if (lane == 0) {
+        const int n_active = __popc(fb);
         R.n_active = n_active;
         R.n_groups = n_groups;
-        R.n_jobs = n_groups * tiles;
-        R.job_start[n_active] = n_groups * tiles;
         R.grp_base[n_active] = n_groups;
         R.bad = bad != 0u;
     }
 }
 
-// Stable grouping of the (token, slot) pairs by expert, and the job table:
-// every active expert has ceil(n_tok / 2) token groups of at most two tokens,
-// and every group has `tiles` row-tile jobs.
-__device__ void build_route(const DecArgs& A, RouteSmem& R, int tiles) {
+// Stable grouping of the (token, k) pairs by expert: every active expert has
+// ceil(n_tok / 2) token groups of at most two tokens.  All threads call it.
+__device__ void build_route(const DecArgs& A, RouteTables& R, RouteScratch& T) {
     const int tid = threadIdx.x;
     const int BK = A.B * A.K, E = A.E;
     if (BK <= 32) {
-        if (tid < 32) build_route_small(A, R, tiles);
+        if (tid < 32) build_route_small(A, R);
         __syncthreads();
         return;
     }
-    for (int e = tid; e < E; e += blockDim.x) R.cnt[e] = 0;
+#pragma unroll 1
+    for (int e = tid; e < E; e += blockDim.x) T.cnt[e] = 0;
+#pragma unroll 1
     for (int t = tid; t < A.B; t += blockDim.x) R.tok_valid[t] = 0;
     if (tid == 0) R.bad = 0;
     __syncthreads();
+#pragma unroll 1
     for (int p = tid; p < BK; p += blockDim.x) {
         const int e = A.ids[p];
         bool ok = e >= 0 && e < E;
         const int t0 = p - p % A.K;
+#pragma unroll 1
         for (int j = t0; ok && j < p; ++j) ok = A.ids[j] != e;
-        R.pe[p] = ok ? e : -1;
+        T.pe[p] = ok ? e : -1;
         if (ok) {
-            atomicAdd(&R.cnt[e], 1);
+            atomicAdd(&T.cnt[e], 1);
             atomicAdd(&R.tok_valid[p / A.K], 1);
         } else {
             R.bad = 1;
         }
     }
     __syncthreads();
+#pragma unroll 1
     for (int e = tid; e < E; e += blockDim.x) {
-        R.off[e] = R.cnt[e];
-        R.aidx[e] = R.cnt[e] > 0;
+        T.off[e] = T.cnt[e];
+        T.aidx[e] = T.cnt[e] > 0;
     }
     __syncthreads();
-    block_exclusive_scan(R.off, E, R.scan_tmp);
-    const int n_active = block_exclusive_scan(R.aidx, E, R.scan_tmp);
+    block_exclusive_scan(T.off, E, T.scan_tmp);
+    const int n_active = block_exclusive_scan(T.aidx, E, T.scan_tmp);
+#pragma unroll 1
     for (int e = tid; e < E; e += blockDim.x) {
-        if (R.cnt[e] > 0) {
-            const int a = R.aidx[e];
+        if (T.cnt[e] > 0) {
+            const int a = T.aidx[e];
             R.active[a] = e;
-            R.first_slot[a] = R.off[e];
-            R.n_tok[a] = R.cnt[e];
-            const int groups = (R.cnt[e] + 1) / 2;
-            R.grp_base[a] = groups;
-            R.job_start[a] = groups * tiles;
+            R.first_slot[a] = T.off[e];
+            R.n_tok[a] = T.cnt[e];
+            R.grp_base[a] = (T.cnt[e] + 1) / 2;
         }
     }
+#pragma unroll 1
     for (int p = tid; p < BK; p += blockDim.x) {
-        const int e = R.pe[p];
+        const int e = T.pe[p];
         int slot = -1;
         if (e >= 0) {
             int rank = 0;
-            for (int q = 0; q < p; ++q) rank += (R.pe[q] == e);
-            slot = R.off[e] + rank;
+#pragma unroll 1
+            for (int q = 0; q < p; ++q) rank += (T.pe[q] == e);
+            slot = T.off[e] + rank;
             R.slot_tok[slot] = p / A.K;
         }
         R.pos_of_pair[p] = slot;
     }
     __syncthreads();
-    const int n_groups = block_exclusive_scan(R.grp_base, n_active, R.scan_tmp);
-    const int n_jobs = block_exclusive_scan(R.job_start, n_active, R.scan_tmp);
+    const int n_groups = block_exclusive_scan(R.grp_base, n_active, T.scan_tmp);
     if (tid == 0) {
         R.n_active = n_active;
-        R.n_jobs = n_jobs;
         R.n_groups = n_groups;
-        R.job_start[n_active] = n_jobs;
         R.grp_base[n_active] = n_groups;
     }
     __syncthreads();
 }
 
 struct Job {
-    int e, a, group, tile, slot0, slot1;
+    int e, tile, slot0, slot1;
 };
 
-__device__ __forceinline__ Job decode_job(const RouteSmem& R, int j, int tiles) {
-    int lo = 0, hi = R.n_active - 1;   // last a with job_start[a] <= j
+// Job j of a phase with `tiles` row blocks per token group.
+__device__ __forceinline__ Job decode_job(const RouteTables& R, int j, int tiles) {
+    const int gi = j / tiles;
+    int lo = 0, hi = R.n_active - 1;   // last a with grp_base[a] <= gi
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (R.job_start[mid] <= j) lo = mid;
+        if (R.grp_base[mid] <= gi) lo = mid;
         else hi = mid - 1;
     }
     Job J;
-    J.a = lo;
     J.e = R.active[lo];
-    const int rem = j - R.job_start[lo];
-    const int gi = rem / tiles;
-    J.tile = rem - gi * tiles;
-    J.group = R.grp_base[lo] + gi;
-    J.slot0 = R.first_slot[lo] + 2 * gi;
-    J.slot1 = (2 * gi + 1 < R.n_tok[lo]) ? J.slot0 + 1 : -1;
+    J.tile = j - gi * tiles;
+    const int g = gi - R.grp_base[lo];
+    J.slot0 = R.first_slot[lo] + 2 * g;
+    J.slot1 = (2 * g + 1 < R.n_tok[lo]) ? J.slot0 + 1 : -1;
+    return J;
+}
+
+// A job packed in 8 bytes: (expert, row block) and the two slots (0xFFFF: none).
+__device__ __forceinline__ uint2 pack_job(const Job& J) {
+    return make_uint2(uint32_t(J.e) | (uint32_t(J.tile) << 16), uint32_t(J.slot0 & 0xFFFF) | (uint32_t(J.slot1 & 0xFFFF) << 16));
+}
+__device__ __forceinline__ Job unpack_job(uint2 v) {
+    Job J;
+    J.e = int(v.x & 0xFFFFu);
+    J.tile = int(v.x >> 16);
+    J.slot0 = int(v.y & 0xFFFFu);
+    J.slot1 = (v.y >> 16) == 0xFFFFu ? -1 : int(v.y >> 16);
     return J;
 }
 
 // ----------------------------------------------------------------------------
-// streaming kernels: one producer warp (TMA ring) + 8 consumer warps that
-// split every job by (row tile, matrix, 1024-column chunk)
+// shapes and shared memory
 // ----------------------------------------------------------------------------
-
-constexpr int kCapMax = 8;
 
 struct Shape {
     int rows, cols;      // rows and columns of the streamed matrices
@@ -285,9 +303,8 @@ struct Shape {
     int row_blocks;      // jobs per token group: ceil(rows / job_rows)
     int tile_bytes;      // stage_layout(cols).bytes
     int stage_bytes;     // r_tiles * n_mat * tile_bytes
-    int n_stages;        // ring depth
-    int tok_cap;         // rotated vectors cached in shared memory
-    int tok_bytes;       // pieces + 128-block sums of one cached vector
+    int tok_bytes;       // digits + 128-block sums + fp16 copy of one rotated vector
+    int pairs;           // (matrix, row) pairs of a job: n_mat * job_rows
 };
 
 __host__ __device__ inline Shape make_shape(int rows, int cols, int n_mat) {
@@ -302,43 +319,7 @@ __host__ __device__ inline Shape make_shape(int rows, int cols, int n_mat) {
     s.tile_bytes = stage_layout(cols).bytes;
     s.stage_bytes = s.r_tiles * n_mat * s.tile_bytes;
     s.tok_bytes = int(align_up(cols * kPieces + (cols / 128) * 4 + cols * 2, 16));
-    return s;
-}
-
-struct CacheSmem {
-    int key[kCapMax];
-    float sigma[kCapMax];
-    int stamp[kCapMax];
-    int plan_slot[2], plan_key[2], n_plan, clock;
-    float red[kDecWarps];
-    int cres[2];       // cache indices of the current job's vectors
-    int flag[8];       // combine / RMSNorm last-arriver flags
-    float wsum[kDecWarps];
-    float inv;
-};
-
-struct StreamSmem {
-    int stages, cache, route, partials, scratch, bars, misc, bytes;
-};
-
-__host__ __device__ inline StreamSmem stream_smem(const Shape& sh) {
-    StreamSmem s;
-    int o = 0;
-    s.stages = o;
-    o += sh.n_stages * sh.stage_bytes;
-    s.cache = o;
-    o += sh.tok_cap * sh.tok_bytes;
-    s.route = o;
-    o += int(align_up(sizeof(RouteSmem), 16));
-    s.partials = o;
-    o += 2 * kDecWarps * 16 * 2 * 4;
-    s.scratch = o;
-    o += kDecWarps * kWarpScratchFloats * 4;
-    s.bars = o;
-    o += 2 * sh.n_stages * 8;
-    s.misc = o;
-    o += int(align_up(sizeof(CacheSmem), 16));
-    s.bytes = int(align_up(o, 1024)) + 1024;
+    s.pairs = n_mat * s.job_rows;
     return s;
 }
 
@@ -348,29 +329,83 @@ __host__ __device__ inline bool shape_ok(int cols, int n_mat) {
     return cols % 1024 == 0 && units >= 1 && units <= kDecWarps && kDecWarps % units == 0;
 }
 
-// Make sure the rotated vectors `key0`, `key1` (tokens for w13, slots for w2;
-// -1 = none) are in the shared-memory cache; returns their cache indices.
-// All 256 consumer threads call it.  A missing vector is loaded (bf16 x or
-// fp32 h), rotated by FWHT-1024 (one warp per 1024-block), and turned into
-// pieces and 128-block sums; the least recently used entry is replaced.
-template <bool W13>
-__device__ void ensure_cached(const DecArgs& A, const Shape& sh, uint8_t* cache, CacheSmem& M, int key0, int key1,
-                              int& c0, int& c1) {
+struct Plan {
+    Shape s13, s2;
+    int n_stages, stage_bytes, cache_bytes, cap13, cap2;
+    int max_jobs;   // jobs of both phases one CTA may get
+};
+
+struct CacheSmem {
+    int key[kCapMax];
+    float sigma[kCapMax];
+    int stamp[kCapMax];
+    int plan_slot[2], plan_key[2], n_plan, clock;
+    float red[kDecWarps];
+    int cres[2];                  // cache indices of the current job's vectors
+    int ecnt[kMaxStages];         // warps done with the job in each stage
+    int gate_ok;
+};
+
+constexpr int kPartFloats = kDecWarps * 32 + 2 * 128;   // per stage: MMA pieces + outlier sums
+
+struct DecSmem {
+    int ring, cache, route, jobs, part, scratch, bars, misc, bytes;
+};
+
+__host__ __device__ inline DecSmem dec_smem(const Plan& P) {
+    DecSmem s;
+    int o = 0;
+    s.ring = o;
+    o += P.n_stages * P.stage_bytes;
+    s.cache = o;
+    o += P.cache_bytes;
+    s.route = o;
+    o += int(align_up(sizeof(RouteTables), 16));
+    s.jobs = o;
+    o += int(align_up(8 * P.max_jobs, 16));
+    s.part = o;
+    o += P.n_stages * kPartFloats * 4;
+    s.scratch = o;
+    o += kDecWarps * kWarpScratchFloats * 4;
+    s.bars = o;
+    o += 2 * P.n_stages * 8;
+    s.misc = o;
+    o += int(align_up(sizeof(CacheSmem), 16));
+    s.bytes = int(align_up(o, 1024)) + 1024;
+    return s;
+}
+
+// ----------------------------------------------------------------------------
+// rotated-vector cache
+// ----------------------------------------------------------------------------
+
+// Make sure the rotated vectors `key0`, `key1` (tokens for w1/w3, slots for
+// w2; -1 = none) are in the shared-memory cache; returns their cache
+// indices.  All consumer threads call it (named barrier 1).  A missing vector
+// is loaded (bf16 x or fp32 h), rotated by FWHT-1024 (one warp per
+// 1024-block), and turned into digits, 128-block sums and an fp16 copy; the
+// least recently used entry is replaced.
+__device__ __forceinline__ void ensure_cached(const DecArgs& A, const Shape& sh, int cap, uint8_t* cache, CacheSmem& M,
+                                          bool W13, int key0, int key1, int& c0, int& c1) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int C = sh.cols, nblk = C / 1024;
     if (tid == 0) {
         const int keys[2] = {key0, key1};
         int found[2] = {-1, -1};
         M.n_plan = 0;
+#pragma unroll 1
         for (int e = 0; e < 2; ++e) {
             if (keys[e] < 0) continue;
-            for (int q = 0; q < sh.tok_cap; ++q)
+#pragma unroll 1
+            for (int q = 0; q < cap; ++q)
                 if (M.key[q] == keys[e]) found[e] = q;
         }
+#pragma unroll 1
         for (int e = 0; e < 2; ++e) {
             if (keys[e] < 0 || found[e] >= 0) continue;
             int victim = -1, best = 0x7fffffff;
-            for (int q = 0; q < sh.tok_cap; ++q) {
+#pragma unroll 1
+            for (int q = 0; q < cap; ++q) {
                 if (q == found[0] || q == found[1]) continue;
                 if (M.stamp[q] < best) {
                     best = M.stamp[q];
@@ -383,6 +418,7 @@ __device__ void ensure_cached(const DecArgs& A, const Shape& sh, uint8_t* cache,
             M.plan_key[M.n_plan] = keys[e];
             ++M.n_plan;
         }
+#pragma unroll 1
         for (int e = 0; e < 2; ++e)
             if (found[e] >= 0) M.stamp[found[e]] = ++M.clock;
         M.cres[0] = found[0];
@@ -393,58 +429,384 @@ __device__ void ensure_cached(const DecArgs& A, const Shape& sh, uint8_t* cache,
     c1 = M.cres[1];
     const int n_plan = M.n_plan;
     if (n_plan == 0) return;
-    // warps [e * nblk, (e + 1) * nblk) rotate entry e, one 1024-block each
+    // warps [e * nblk, (e + 1) * nblk) rotate entry e, one 1024-block each.
+    // Lane l loads elements 32 i + l; butterflies over the register index
+    // (element bits 5..9); a transpose through the entry's own (not yet
+    // written) bytes gives lane l the elements 32 l + i; butterflies over the
+    // register index again (bits 0..4).  Lane l = 4 b + tig then holds the
+    // 32 consecutive columns 128 b + 32 tig + i, which are exactly the four
+    // elements (i = q + 8 i') of each of its digit words (b, tig, q).
     const int e = warp / nblk, blk = warp % nblk;
-    float v[32];
     const bool act = e < n_plan;
+    float v[32];
+    uint8_t* dst = act ? cache + M.plan_slot[e] * sh.tok_bytes : cache;
     if (act) {
         const int key = M.plan_key[e];
         if (W13) {
             const uint16_t* src = A.x + int64_t(key) * C + blk * 1024;
 #pragma unroll
-            for (int r = 0; r < 32; ++r) v[r] = bf16_to_f32(src[piece_elem(lane, r)]);
+            for (int i = 0; i < 32; ++i) v[i] = bf16_to_f32(src[32 * i + lane]);
         } else {
             const float* src = A.ws.h + int64_t(key) * C + blk * 1024;
 #pragma unroll
-            for (int r = 0; r < 32; ++r) v[r] = __ldcg(src + piece_elem(lane, r));
+            for (int i = 0; i < 32; ++i) v[i] = __ldcg(src + 32 * i + lane);
         }
-        fwht1024_warp(v, lane);
+        fwht32_cg(v);
+        float* tb = reinterpret_cast<float*>(dst) + blk * 33 * 32;   // 33-float rows: no bank conflicts
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) tb[i * 33 + lane] = v[i];
+        __syncwarp();
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) v[i] = tb[lane * 33 + i] * (1.0f / 32.0f);
+        fwht32_cg(v);
+        float m = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] *= (1.0f / 32.0f);
-        const float m = block_absmax(v);
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0) M.red[warp] = m;
     }
-    named_bar_sync(1, kDecThreads);
+    named_bar_sync(1, kDecThreads);   // every transpose has been read back; block maxima known
     if (act) {
         float m = 0.f;
         for (int w = e * nblk; w < (e + 1) * nblk; ++w) m = fmaxf(m, M.red[w]);
         const float S = fixed_scale(m);
-        uint8_t* dst = cache + M.plan_slot[e] * sh.tok_bytes;
-        pieces_from_regs(v, S, dst + blk * 8 * kPieceBlockBytes,
-                         reinterpret_cast<float*>(dst + C * kPieces) + blk * 8,
-                         reinterpret_cast<__half*>(dst + C * kPieces + (C / 128) * 4) + blk * 1024);
+        const int b = blk * 8 + (lane >> 2), tig = lane & 3;
+        uint32_t* pieces = reinterpret_cast<uint32_t*>(dst + b * kPieceBlockBytes + tig * 32);
+        // word q takes registers q, q + 8, q + 16, q + 24
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float sc = S * inv_a(q);
+            uint32_t word[kPieces] = {0u, 0u, 0u};
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4) {
+                uint32_t d1, d2, d3;
+                fixed_digits(v[q + 8 * i4] * sc, d1, d2, d3);
+                word[0] |= d1 << (8 * i4);
+                word[1] |= d2 << (8 * i4);
+                word[2] |= d3 << (8 * i4);
+            }
+#pragma unroll
+            for (int j = 0; j < kPieces; ++j) pieces[j * 32 + q] = word[j];
+        }
+        // fp16 copy (for the outliers) and the 128-block sums
+        uint4* x16 = reinterpret_cast<uint4*>(dst + C * kPieces + (C / 128) * 4) + blk * 128 + lane * 4;
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __half2 hh[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                hh[j] = __floats2half2_rn(v[8 * i + 2 * j], v[8 * i + 2 * j + 1]);
+                sum += v[8 * i + 2 * j] + v[8 * i + 2 * j + 1];
+            }
+            x16[i] = *reinterpret_cast<const uint4*>(hh);
+        }
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        if (tig == 0) reinterpret_cast<float*>(dst + C * kPieces)[b] = sum;
         if (blk == 0 && lane == 0) M.sigma[M.plan_slot[e]] = 1.0f / S;
     }
     named_bar_sync(1, kDecThreads);
 }
 
-template <bool W13>
-__global__ void __launch_bounds__(kDecThreads + 32, 1) moe_stream_kernel(
-    const __grid_constant__ CUtensorMap sa, const __grid_constant__ CUtensorMap ba,
-    const __grid_constant__ CUtensorMap sb, const __grid_constant__ CUtensorMap bb, DecArgs A, Shape sh) {
+// ----------------------------------------------------------------------------
+// per-warp pieces of a job
+// ----------------------------------------------------------------------------
+
+// Tensor-core part of one 1024-column chunk `ch` of a staged 16-row tile for
+// up to two tokens: lanes 0..15 return, for row r0 + lane and tokens 0 and 1,
+//   sum_{b in chunk} s_blk[row, b] (X_b - 2 P_b).
+// The chunk's eight 128-column blocks run in two halves of four blocks with
+// one accumulator each, so that consecutive MMAs are independent.
+__device__ __forceinline__ void chunk_mma(const uint8_t* tile, int C, int ch, const TokRef (&tok)[2], float* scratch,
+                                          float (&part)[2]) {
+    const int lane = threadIdx.x & 31;
+    const int nb = C / 128;
+    const StageLayout L = stage_layout(C);
+    const uint8_t* signs = tile + L.signs + ch * 2048;
+    const __half* sblk = reinterpret_cast<const __half*>(tile + L.scales);
+    const int row = lane & 15, half = lane >> 4;
+    const bool has0 = tok[0].pieces != nullptr, has1 = tok[1].pieces != nullptr;
+
+    // block-scale-weighted 128-block sums of x over the chunk (4 blocks per half)
+    float xt0 = 0.f, xt1 = 0.f;
+    {
+        const int b0 = ch * 8 + half * 4;
+        const uint2 sv = *reinterpret_cast<const uint2*>(sblk + row * nb + b0);
+        const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sv.x));
+        const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sv.y));
+        if (has0) {
+            const float4 x = *reinterpret_cast<const float4*>(tok[0].xsum + b0);
+            xt0 = s01.x * x.x + s01.y * x.y + s23.x * x.z + s23.y * x.w;
+        }
+        if (has1) {
+            const float4 x = *reinterpret_cast<const float4*>(tok[1].xsum + b0);
+            xt1 = s01.x * x.x + s01.y * x.y + s23.x * x.z + s23.y * x.w;
+        }
+    }
+
+    const int g = lane >> 2, tig = lane & 3;
+    const bool bsrc = g < 6 && (g < 3 ? has0 : has1);
+    const uint8_t* pieces = (g < 3 ? tok[0].pieces : tok[1].pieces);
+    const uint8_t* bsrc_p = bsrc ? pieces + (g % 3) * 128 + tig * 32 + ch * 8 * kPieceBlockBytes : nullptr;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int hb = 0; hb < 2; ++hb) {
+        uint32_t wg[4], wg8[4];
+        uint4 q0[4], q1[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int bb = 4 * hb + j;
+            const uint8_t* wa = signs + g * 128 + ((bb ^ (g & 7)) << 4) + tig * 4;
+            wg[j] = *reinterpret_cast<const uint32_t*>(wa);
+            wg8[j] = *reinterpret_cast<const uint32_t*>(wa + 1024);
+            if (bsrc) {
+                q0[j] = *reinterpret_cast<const uint4*>(bsrc_p + bb * kPieceBlockBytes);
+                q1[j] = *reinterpret_cast<const uint4*>(bsrc_p + bb * kPieceBlockBytes + 16);
+            } else {
+                q0[j] = make_uint4(0u, 0u, 0u, 0u);
+                q1[j] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        int c[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0;
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t a0, a1, a2, a3;
+                a_regs(wg[j], wg8[j], mm, a0, a1, a2, a3);
+                const uint32_t b0 = mm == 0 ? q0[j].x : mm == 1 ? q0[j].z : mm == 2 ? q1[j].x : q1[j].z;
+                const uint32_t b1 = mm == 0 ? q0[j].y : mm == 1 ? q0[j].w : mm == 2 ? q1[j].y : q1[j].w;
+                mma_s8(c[j], a0, a1, a2, a3, b0, b1);
+            }
+        }
+        const uint2 sg = *reinterpret_cast<const uint2*>(sblk + g * nb + ch * 8 + 4 * hb);
+        const uint2 sg8 = *reinterpret_cast<const uint2*>(sblk + (g + 8) * nb + ch * 8 + 4 * hb);
+        const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
+        const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(&sg.y));
+        const float2 h01 = __half22float2(*reinterpret_cast<const __half2*>(&sg8.x));
+        const float2 h23 = __half22float2(*reinterpret_cast<const __half2*>(&sg8.y));
+        const float sgv[4] = {g01.x, g01.y, g23.x, g23.y}, s8v[4] = {h01.x, h01.y, h23.x, h23.y};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            acc[0] = fmaf(sgv[j], float(c[j][0]), acc[0]);
+            acc[1] = fmaf(sgv[j], float(c[j][1]), acc[1]);
+            acc[2] = fmaf(s8v[j], float(c[j][2]), acc[2]);
+            acc[3] = fmaf(s8v[j], float(c[j][3]), acc[3]);
+        }
+    }
+    // gather the 8 MMA columns of every row through shared memory
+    scratch[g * 8 + 2 * tig] = acc[0];
+    scratch[g * 8 + 2 * tig + 1] = acc[1];
+    scratch[(g + 8) * 8 + 2 * tig] = acc[2];
+    scratch[(g + 8) * 8 + 2 * tig + 1] = acc[3];
+    __syncwarp();
+    xt0 += __shfl_xor_sync(0xffffffffu, xt0, 16);
+    xt1 += __shfl_xor_sync(0xffffffffu, xt1, 16);
+    const float* col = scratch + row * 8;
+    part[0] = has0 ? xt0 - 2.0f * tok[0].sigma * (col[0] * 16384.0f + col[1] * 128.0f + col[2]) : 0.f;
+    part[1] = has1 ? xt1 - 2.0f * tok[1].sigma * (col[3] * 16384.0f + col[4] * 128.0f + col[5]) : 0.f;
+    __syncwarp();
+}
+
+// Outlier corrections  sum_j (q s_row - sign s_blk) x_c  of one row of a
+// staged tile over the outliers j = sub, sub + step, ... (a fixed lane set
+// of the row sums them afterwards in a fixed order); six at a time so that
+// their loads overlap.
+__device__ __forceinline__ void row_outliers(const uint8_t* tile, int C, int k, int q_delta, int row, int sub, int step,
+                                             const TokRef (&tok)[2], float& corr0, float& corr1) {
+    const StageLayout L = stage_layout(C);
+    const int nb = C / 128;
+    const uint16_t* ri = reinterpret_cast<const uint16_t*>(tile + L.idx) + row * k;
+    const uint8_t* qn = tile + L.q + q_delta;
+    const __half* sblk = reinterpret_cast<const __half*>(tile + L.scales) + row * nb;
+    const uint8_t* signs = tile + L.signs + row * 128;
+    const float srow = __half2float(reinterpret_cast<const __half*>(tile + L.srow)[row]);
+    const bool has0 = tok[0].pieces != nullptr, has1 = tok[1].pieces != nullptr;
+    const __half* x0 = tok[0].x16;
+    const __half* x1 = tok[1].x16;
+    for (int jb = sub; jb < k; jb += 6 * step) {
+        int c[6];
+        bool use[6];
+#pragma unroll
+        for (int u = 0; u < 6; ++u) {
+            const int j = jb + u * step;
+            c[u] = j < k ? int(ri[j]) : C;
+            use[u] = c[u] < C;   // past the row's outliers, or a record that failed validation
+            if (!use[u]) c[u] = 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 6; ++u) {
+            const int n = row * k + (use[u] ? jb + u * step : 0);
+            const int qb = int(qn[n >> 1]) >> ((n & 1) * 4);
+            const int qv = (qb & 15) - ((qb & 8) << 1);
+            const int w = (c[u] >> 5) & 31;
+            const uint32_t word = *reinterpret_cast<const uint32_t*>(
+                signs + (c[u] >> 10) * 2048 + (((w >> 2) ^ (row & 7)) << 4) + (w & 3) * 4);
+            const float sb = __half2float(sblk[c[u] >> 7]);
+            float wq = fmaf(float(qv), srow, ((word >> (c[u] & 31)) & 1u) ? sb : -sb);
+            wq = use[u] ? wq : 0.f;
+            if (has0) corr0 = fmaf(wq, __half2float(x0[c[u]]), corr0);
+            if (has1) corr1 = fmaf(wq, __half2float(x1[c[u]]), corr1);
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------
+// the kernel
+// ----------------------------------------------------------------------------
+
+// The epilogue of a job, run by the last warp to finish it: w1/w3 stores
+// h = silu(w1 x) * (w3 x); w2 stores the expert outputs and runs the
+// (token, 64-row block) combine and the RMSNorm of finished tokens.
+__device__ __forceinline__ void job_epilogue(const DecArgs& A, const RouteTables& R, const Shape& sh, bool W13,
+                                          const Job& Jb, const float* pb, int lane, int* ecnt) {
+    const int d = A.d_model;
+    const int comb_blocks = (d + 63) / 64;
+    __threadfence_block();
+    if (lane == 0) *ecnt = 0;
+    const float* pc = pb + kDecWarps * 32;
+    if (W13) {
+#pragma unroll 1
+        for (int v = lane; v < sh.r_tiles * 32; v += 32) {
+            const int t_r = v >> 5, row = v & 15, t = (v >> 4) & 1;
+            const int slot = t ? Jb.slot1 : Jb.slot0;
+            const int r = Jb.tile * sh.job_rows + t_r * 16 + row;
+            float y1 = pc[(t_r * 16 + row) * 2 + t], y3 = pc[(sh.job_rows + t_r * 16 + row) * 2 + t];
+#pragma unroll 1
+            for (int c2 = 0; c2 < sh.n_chunk; ++c2) {
+                y1 += pb[((t_r * 2 + 0) * sh.n_chunk + c2) * 32 + row * 2 + t];
+                y3 += pb[((t_r * 2 + 1) * sh.n_chunk + c2) * 32 + row * 2 + t];
+            }
+            if (slot >= 0 && r < sh.rows) A.ws.h[int64_t(slot) * sh.rows + r] = silu(y1) * y3;
+        }
+    } else {
+#pragma unroll 1
+        for (int v = lane; v < sh.r_tiles * 32; v += 32) {
+            const int t_r = v >> 5, row = v & 15, t = (v >> 4) & 1;
+            const int slot = t ? Jb.slot1 : Jb.slot0;
+            const int r = Jb.tile * sh.job_rows + t_r * 16 + row;
+            float y = pc[(t_r * 16 + row) * 2 + t];
+#pragma unroll 1
+            for (int c2 = 0; c2 < sh.n_chunk; ++c2) y += pb[(t_r * sh.n_chunk + c2) * 32 + row * 2 + t];
+            if (slot >= 0 && r < d) A.ws.o[int64_t(slot) * d + r] = y;
+        }
+        __threadfence();
+        __syncwarp();
+        // the (token, 64-row block) combine: the last expert to finish sums the K outputs
+        const int nsub = sh.job_rows / 64;
+        int flags = 0;
+        if (lane < 2 * nsub) {
+            const int sl = lane & 1, sb = lane >> 1;
+            const int slot = sl ? Jb.slot1 : Jb.slot0;
+            const int rb = Jb.tile * nsub + sb;
+            if (slot >= 0 && rb < comb_blocks) {
+                const int t = R.slot_tok[slot];
+                flags = atomicAdd(A.ws.comb_cnt + t * comb_blocks + rb, 1) == R.tok_valid[t] - 1;
+            }
+        }
+        const unsigned fl = __ballot_sync(0xffffffffu, flags);
+#pragma unroll 1
+        for (int f = 0; f < 2 * nsub; ++f) {
+            if (!((fl >> f) & 1)) continue;
+            __threadfence();
+            const int sl = f & 1, sb = f >> 1;
+            const int t = R.slot_tok[sl ? Jb.slot1 : Jb.slot0];
+            const int rb = Jb.tile * nsub + sb;
+            float ss = 0.f;
+#pragma unroll 1
+            for (int rr = lane; rr < 64; rr += 32) {
+                const int r = rb * 64 + rr;
+                if (r >= d) continue;
+                float y = 0.f;
+#pragma unroll 1
+                for (int kk = 0; kk < A.K; ++kk) {
+                    const int pos = R.pos_of_pair[t * A.K + kk];
+                    if (pos >= 0) y = fmaf(A.gates[t * A.K + kk], __ldcg(A.ws.o + int64_t(pos) * d + r), y);
+                }
+                if (!A.fuse_norm) {
+                    store_from_f32(A.out, A.out_dtype, int64_t(t) * d + r, y);
+                } else {
+                    const float v = bf16_to_f32(A.x[int64_t(t) * d + r]) + y;
+                    A.ws.v[int64_t(t) * d + r] = v;
+                    ss = fmaf(v, v, ss);
+                }
+            }
+            if (!A.fuse_norm) continue;
+            // sum of squares of this 64-row block (fixed order), then the
+            // last block of the token normalises the whole row
+            ss = warp_sum(ss);
+            int lastblk = 0;
+            if (lane == 0) {
+                A.ws.ssq[t * comb_blocks + rb] = ss;
+                __threadfence();
+                lastblk = atomicAdd(A.ws.tok_cnt + t, 1) == comb_blocks - 1;
+            }
+            __syncwarp();
+            lastblk = __shfl_sync(0xffffffffu, lastblk, 0);
+            if (!lastblk) continue;
+            __threadfence();
+            float tot = 0.f;
+#pragma unroll 1
+            for (int q = lane; q < comb_blocks; q += 32) tot += __ldcg(A.ws.ssq + t * comb_blocks + q);
+            tot = warp_sum(tot);
+            const float inv = rsqrtf(tot / float(d) + A.eps);
+#pragma unroll 1
+            for (int c = lane; c < d; c += 32)
+                store_from_f32(A.out, GALE_BF16, int64_t(t) * d + c,
+                               __ldcg(A.ws.v + int64_t(t) * d + c) * inv);
+        }
+    }
+}
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Grid-wide barrier of the cooperative launch, one thread per CTA; the
+// counters start at zero every call.  False if the wait ran out (2 s).
+__device__ bool grid_barrier(int32_t* cnt, int32_t* flag, int G) {
+    __threadfence();
+    if (atomicAdd(cnt, 1) == G - 1) {
+        __threadfence();
+        atomicExch(flag, 1);
+        return true;
+    }
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire(flag) == 0) {
+        if (globaltimer_ns() - t0 > 2000000000ull) return false;
+        __nanosleep(64);
+    }
+    __threadfence();
+    return true;
+}
+
+struct Maps {
+    CUtensorMap s1, b1, s3, b3, s2, b2;
+};
+
+__global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_constant__ Maps maps, DecArgs A,
+                                                                  Plan P) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
-    const StreamSmem S = stream_smem(sh);
-    RouteSmem& R = *reinterpret_cast<RouteSmem*>(smem + S.route);
+    uint8_t* smem = smem_align1024(smem_raw);
+    const DecSmem S = dec_smem(P);
+    RouteTables& R = *reinterpret_cast<RouteTables*>(smem + S.route);
     CacheSmem& M = *reinterpret_cast<CacheSmem*>(smem + S.misc);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + S.bars);
-    uint64_t* empty = full + sh.n_stages;
+    uint64_t* empty = full + P.n_stages;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = gridDim.x;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < sh.n_stages; ++s) {
+        for (int s = 0; s < P.n_stages; ++s) {
             mbar_init(full + s, 1);
             mbar_init(empty + s, kDecWarps);
+            M.ecnt[s] = 0;
         }
         fence_mbar_init();
         for (int q = 0; q < kCapMax; ++q) {
@@ -453,48 +815,56 @@ __global__ void __launch_bounds__(kDecThreads + 32, 1) moe_stream_kernel(
         }
         M.clock = 0;
     }
-    build_route(A, R, sh.row_blocks);   // contains __syncthreads
-    // contiguous job range of this CTA
-    const int J = R.n_jobs, G = gridDim.x;
-    const int j0 = int((int64_t(J) * blockIdx.x) / G), j1 = int((int64_t(J) * (blockIdx.x + 1)) / G);
-    const int n_my = j1 - j0;
-    const int64_t off_a = W13 ? A.off_w1 : A.off_w2;
-    const int64_t off_b = W13 ? A.off_w3 : A.off_w2;
-    auto view = [&](int e, int mat) {
-        return make_view(A.base + int64_t(e) * A.stride + (mat ? off_b : off_a), sh.rows, sh.cols);
-    };
+    build_route(A, R, *reinterpret_cast<RouteScratch*>(smem + S.ring));   // contains __syncthreads
+    // contiguous job ranges of this CTA in both phases
+    const int J13 = R.n_groups * P.s13.row_blocks, J2 = R.n_groups * P.s2.row_blocks;
+    const int a0 = int((int64_t(J13) * blockIdx.x) / G), n13 = int((int64_t(J13) * (blockIdx.x + 1)) / G) - a0;
+    const int b0 = int((int64_t(J2) * blockIdx.x) / G), n2 = int((int64_t(J2) * (blockIdx.x + 1)) / G) - b0;
+    uint2* jobs = reinterpret_cast<uint2*>(smem + S.jobs);
+    for (int i = threadIdx.x; i < n13 + n2; i += blockDim.x)
+        jobs[i] = pack_job(i < n13 ? decode_job(R, a0 + i, P.s13.row_blocks) : decode_job(R, b0 + (i - n13), P.s2.row_blocks));
+    __syncthreads();
 
     if (warp == kDecWarps) {
-        // ---------------- producer: weights only, no dependency on earlier kernels.
-        // Lane 0 arms the stage's barrier with the job's byte count, then every
-        // lane issues the copies of one (row tile, matrix) of the job.
-        const int n_tiles = sh.r_tiles * sh.n_mat;
-        for (int i = 0; i < n_my; ++i) {
-            const int s = i % sh.n_stages;
+        // ---------------- producer: weights only.  Lane 0 arms the stage's
+        // barrier with the job's byte count, then every lane issues the
+        // copies of one (row tile, matrix) of the job.
+        int s = 0, ph = 0;
+        for (int i = 0; i < n13 + n2; ++i) {
             int ok_wait = 1;
-            if (lane == 0 && i >= sh.n_stages) ok_wait = mbar_wait(empty + s, ((i / sh.n_stages) - 1) & 1);
+            if (lane == 0 && i >= P.n_stages) ok_wait = mbar_wait(empty + s, uint32_t(ph ^ 1));
             ok_wait = __shfl_sync(0xffffffffu, ok_wait, 0);
             if (!ok_wait) {
                 if (lane == 0) set_status(A.ws.status, GALE_ERR_TIMEOUT);
                 break;
             }
-            const Job Jb = decode_job(R, j0 + i, sh.row_blocks);
+            const bool w13 = i < n13;
+            const Shape& sh = w13 ? P.s13 : P.s2;
+            const Job Jb = unpack_job(jobs[i]);
             const int tr = lane / sh.n_mat, mt = lane % sh.n_mat;
             const int r0 = Jb.tile * sh.job_rows + tr * 16;
-            const bool mine = lane < n_tiles && r0 < sh.rows;
+            const bool mine = lane < sh.r_tiles * sh.n_mat && r0 < sh.rows;
             uint32_t tx = 0;
             MatView mv{};
+            const int64_t off = w13 ? (mt ? A.off_w3 : A.off_w1) : A.off_w2;
             if (mine) {
-                mv = view(Jb.e, mt);
+                mv = make_view(A.base + int64_t(Jb.e) * A.stride + off, sh.rows, sh.cols);
                 tx = tile_tx_bytes(mv, r0);
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) tx += __shfl_xor_sync(0xffffffffu, tx, o);
             if (lane == 0) mbar_arrive_expect_tx(full + s, tx);
             __syncwarp();
-            if (mine)
-                issue_tile_copies(smem + S.stages + s * sh.stage_bytes + (tr * sh.n_mat + mt) * sh.tile_bytes,
-                                  full + s, mt ? &sb : &sa, mt ? &bb : &ba, mv, Jb.e, r0);
+            if (mine) {
+                const CUtensorMap* smap = w13 ? (mt ? &maps.s3 : &maps.s1) : &maps.s2;
+                const CUtensorMap* bmap = w13 ? (mt ? &maps.b3 : &maps.b1) : &maps.b2;
+                issue_tile_copies(smem + S.ring + s * P.stage_bytes + (tr * sh.n_mat + mt) * sh.tile_bytes,
+                                  full + s, smap, bmap, mv, Jb.e, r0);
+            }
+            if (++s == P.n_stages) {
+                s = 0;
+                ph ^= 1;
+            }
         }
         return;
     }
@@ -502,189 +872,147 @@ __global__ void __launch_bounds__(kDecThreads + 32, 1) moe_stream_kernel(
     // ---------------- consumers
     const int tid = threadIdx.x;   // 0..255
     const int d = A.d_model;
-    const int comb_blocks = (d + 63) / 64;   // w2 row blocks (64 rows)
-    if (W13) {
-        // w2's counters start at zero; w2 touches them only after waiting for this grid
-        if (blockIdx.x == 0) {
-            for (int i = tid; i < A.B * comb_blocks; i += kDecThreads) A.ws.comb_cnt[i] = 0;
-            for (int i = tid; i < A.B; i += kDecThreads) A.ws.tok_cnt[i] = 0;
-            if (tid == 0 && R.bad) set_status(A.ws.status, GALE_ERR_ARG);
-        }
-        pdl_launch_dependents();
-    } else {
-        pdl_wait();   // h of every expert and the zeroed counters
+    const int comb_blocks = (d + 63) / 64;
+    if (blockIdx.x == 0) {
+        // the combine counters start at zero; they are used only after the grid barrier
+        for (int i = tid; i < A.B * comb_blocks; i += kDecThreads) A.ws.comb_cnt[i] = 0;
+        for (int i = tid; i < A.B; i += kDecThreads) A.ws.tok_cnt[i] = 0;
+        if (tid == 0 && R.bad) set_status(A.ws.status, GALE_ERR_ARG);
     }
     uint8_t* cache = smem + S.cache;
-    const int tr = warp / (sh.n_mat * sh.n_chunk);
-    const int mat = (warp / sh.n_chunk) % sh.n_mat;
-    const int ch = warp % sh.n_chunk;
     float* scratch = reinterpret_cast<float*>(smem + S.scratch) + warp * kWarpScratchFloats;
-    float* partials = reinterpret_cast<float*>(smem + S.partials);
-    const int C = sh.cols;
     bool ok = true;
-    int pk0 = -2, pk1 = -2, c0 = -1, c1 = -1;
+    int st = 0, ph = 0;   // ring position of the next job
 
-    for (int i = 0; i < n_my; ++i) {
-        const Job Jb = decode_job(R, j0 + i, sh.row_blocks);
-        const int key0 = Jb.slot0 < 0 ? -1 : (W13 ? R.slot_tok[Jb.slot0] : Jb.slot0);
-        const int key1 = Jb.slot1 < 0 ? -1 : (W13 ? R.slot_tok[Jb.slot1] : Jb.slot1);
-        if (key0 != pk0 || key1 != pk1) {   // uniform over the CTA
-            ensure_cached<W13>(A, sh, cache, M, key0, key1, c0, c1);
-            pk0 = key0;
-            pk1 = key1;
-        }
-        TokRef tok[2];
-        for (int e = 0; e < 2; ++e) {
-            const int cs = e ? c1 : c0;
-            if (cs < 0) {
-                tok[e] = TokRef{nullptr, nullptr, nullptr, 1.f, nullptr};
-                continue;
+#pragma unroll 1
+    for (int phase = 0; phase < 2; ++phase) {
+        const bool W13 = phase == 0;
+        const Shape& sh = W13 ? P.s13 : P.s2;
+        const int cap = W13 ? P.cap13 : P.cap2;
+        const int n_my = W13 ? n13 : n2, ibase = W13 ? 0 : n13;
+        const int C = sh.cols, k = outliers_per_row(C);
+        // this warp's MMA piece of every job ...
+        const int tr = warp / (sh.n_mat * sh.n_chunk);
+        const int mat = (warp / sh.n_chunk) % sh.n_mat;
+        const int ch = warp % sh.n_chunk;
+        // ... and its (matrix, row) pairs of outlier corrections
+        const int ppw = sh.pairs / kDecWarps, lpp = 32 / ppw;
+        const int pair = warp * ppw + lane / lpp, sub = lane % lpp;
+        const int o_mat = pair / sh.job_rows, o_tr = (pair % sh.job_rows) / 16, o_row = pair % 16;
+        int pk0 = -2, pk1 = -2, c0 = -1, c1 = -1;
+
+        for (int i = 0; i < n_my; ++i) {
+            const Job Jb = unpack_job(jobs[ibase + i]);
+            const int key0 = Jb.slot0 < 0 ? -1 : (W13 ? R.slot_tok[Jb.slot0] : Jb.slot0);
+            const int key1 = Jb.slot1 < 0 ? -1 : (W13 ? R.slot_tok[Jb.slot1] : Jb.slot1);
+            if (key0 != pk0 || key1 != pk1) {   // uniform over the consumers
+                ensure_cached(A, sh, cap, cache, M, W13, key0, key1, c0, c1);
+                pk0 = key0;
+                pk1 = key1;
             }
-            const uint8_t* base = cache + cs * sh.tok_bytes;
-            tok[e] = TokRef{base, reinterpret_cast<const float*>(base + C * kPieces), nullptr, M.sigma[cs],
-                            reinterpret_cast<const __half*>(base + C * kPieces + (C / 128) * 4)};
-        }
-        const int s = i % sh.n_stages;
-        if (ok && !mbar_wait(full + s, (i / sh.n_stages) & 1)) {
-            ok = false;
-            if (lane == 0) set_status(A.ws.status, GALE_ERR_TIMEOUT);
-        }
-        const int r0 = Jb.tile * sh.job_rows + tr * 16;
-        float part[2] = {0.f, 0.f};
-        if (ok && r0 < sh.rows) {
-            uint8_t* tile = smem + S.stages + s * sh.stage_bytes + (tr * sh.n_mat + mat) * sh.tile_bytes;
-            chunk_compute(tile, view(Jb.e, mat), r0, ch, tok, scratch, part);
-        }
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty + s);
-        float* pb = partials + (i & 1) * (kDecWarps * 32);
-        if (lane < 16) {
-            pb[warp * 32 + lane * 2] = part[0];
-            pb[warp * 32 + lane * 2 + 1] = part[1];
-        }
-        named_bar_sync(1, kDecThreads);
-        if (W13) {
-            // h = silu(w1 x) * (w3 x) for the job's rows and tokens
-            if (tid < sh.r_tiles * 32) {
-                const int t_r = tid >> 5, row = tid & 15, t = (tid >> 4) & 1;
-                const int slot = t ? Jb.slot1 : Jb.slot0;
-                const int r = Jb.tile * sh.job_rows + t_r * 16 + row;
-                float y1 = 0.f, y3 = 0.f;
-                for (int c2 = 0; c2 < sh.n_chunk; ++c2) {
-                    y1 += pb[((t_r * 2 + 0) * sh.n_chunk + c2) * 32 + row * 2 + t];
-                    y3 += pb[((t_r * 2 + 1) * sh.n_chunk + c2) * 32 + row * 2 + t];
+            TokRef tok[2];
+            for (int e = 0; e < 2; ++e) {
+                const int cs = e ? c1 : c0;
+                if (cs < 0) {
+                    tok[e] = TokRef{nullptr, nullptr, nullptr, 1.f, nullptr};
+                    continue;
                 }
-                if (slot >= 0 && r < sh.rows) A.ws.h[int64_t(slot) * sh.rows + r] = silu(y1) * y3;
+                const uint8_t* base = cache + cs * sh.tok_bytes;
+                tok[e] = TokRef{base, reinterpret_cast<const float*>(base + C * kPieces), nullptr, M.sigma[cs],
+                                reinterpret_cast<const __half*>(base + C * kPieces + (C / 128) * 4)};
             }
-            continue;
-        }
-        // ---- w2: expert outputs of the job's rows, then the (token, row block) combine
-        if (tid < sh.r_tiles * 32) {
-            const int t_r = tid >> 5, row = tid & 15, t = (tid >> 4) & 1;
-            const int slot = t ? Jb.slot1 : Jb.slot0;
-            const int r = Jb.tile * sh.job_rows + t_r * 16 + row;
-            float y = 0.f;
-            for (int c2 = 0; c2 < sh.n_chunk; ++c2) y += pb[(t_r * sh.n_chunk + c2) * 32 + row * 2 + t];
-            if (slot >= 0 && r < d) A.ws.o[int64_t(slot) * d + r] = y;
-            __threadfence();
-        }
-        named_bar_sync(1, kDecThreads);
-        // combine granularity: 64-row blocks of d_model (a job covers job_rows >= 64 rows)
-        const int nsub = sh.job_rows / 64;
-        if (tid < 2 * nsub) {
-            const int sl = tid & 1, sub = tid >> 1;
-            const int slot = sl ? Jb.slot1 : Jb.slot0;
+            const int s = st;
+            if (ok && !mbar_wait(full + s, uint32_t(ph))) {
+                ok = false;
+                if (lane == 0) set_status(A.ws.status, GALE_ERR_TIMEOUT);
+            }
+            uint8_t* stage = smem + S.ring + s * P.stage_bytes;
+            float* pb = reinterpret_cast<float*>(smem + S.part) + s * kPartFloats;
+            float part[2] = {0.f, 0.f};
+            const int r0 = Jb.tile * sh.job_rows + tr * 16;
+            if (ok && r0 < sh.rows)
+                chunk_mma(stage + (tr * sh.n_mat + mat) * sh.tile_bytes, C, ch, tok, scratch, part);
+            float corr0 = 0.f, corr1 = 0.f;
+            const int or0 = Jb.tile * sh.job_rows + o_tr * 16;
+            if (ok && or0 + o_row < sh.rows && k) {
+                const MatView ov = make_view(A.base + int64_t(Jb.e) * A.stride +
+                                                 (W13 ? (o_mat ? A.off_w3 : A.off_w1) : A.off_w2),
+                                             sh.rows, C);
+                const int q_delta =
+                    int(reinterpret_cast<uintptr_t>(reinterpret_cast<const char*>(ov.q) + int64_t(or0) * k / 2) & 15);
+                row_outliers(stage + (o_tr * sh.n_mat + o_mat) * sh.tile_bytes, C, k, q_delta, o_row, sub, lpp, tok,
+                             corr0, corr1);
+            }
+            for (int o = 1; o < lpp; o <<= 1) {
+                corr0 += __shfl_xor_sync(0xffffffffu, corr0, o);
+                corr1 += __shfl_xor_sync(0xffffffffu, corr1, o);
+            }
+            if (lane < 16) {
+                pb[warp * 32 + lane * 2] = part[0];
+                pb[warp * 32 + lane * 2 + 1] = part[1];
+            }
+            if (sub == 0) {
+                pb[kDecWarps * 32 + pair * 2] = corr0;
+                pb[kDecWarps * 32 + pair * 2 + 1] = corr1;
+            }
+            __threadfence_block();
             int last = 0;
-            const int rb = Jb.tile * nsub + sub;
-            if (slot >= 0 && rb < comb_blocks) {
-                const int t = R.slot_tok[slot];
-                last = atomicAdd(A.ws.comb_cnt + t * comb_blocks + rb, 1) == R.tok_valid[t] - 1;
+            if (lane == 0) last = atomicAdd(&M.ecnt[s], 1) == kDecWarps - 1;
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (last) job_epilogue(A, R, sh, W13, Jb, pb, lane, &M.ecnt[s]);
+            // the stage (and its partial sums) may be refilled once all warps are past here
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + s);
+            if (++st == P.n_stages) {
+                st = 0;
+                ph ^= 1;
             }
-            M.flag[tid] = last;   // flag index = 2 * sub + sl (nsub <= 2)
         }
-        named_bar_sync(1, kDecThreads);
-        for (int f = 0; f < 2 * nsub; ++f) {
-            if (!M.flag[f]) continue;
-            const int sl = f & 1, sub = f >> 1;
-            const int slot = sl ? Jb.slot1 : Jb.slot0;
-            const int t = R.slot_tok[slot];
-            const int rb = Jb.tile * nsub + sub;
+
+        if (phase == 0) {
+            // ---------------- grid barrier: h of every expert is in global memory
             __threadfence();
-            float v = 0.f;
-            const int r = rb * 64 + tid;
-            const bool mine = tid < 64 && r < d;
-            if (mine) {
-                float y = 0.f;
-                for (int k = 0; k < A.K; ++k) {
-                    const int pos = R.pos_of_pair[t * A.K + k];
-                    if (pos >= 0) y = fmaf(A.gates[t * A.K + k], __ldcg(A.ws.o + int64_t(pos) * d + r), y);
-                }
-                if (!A.fuse_norm) store_from_f32(A.out, A.out_dtype, int64_t(t) * d + r, y);
-                else {
-                    v = bf16_to_f32(A.x[int64_t(t) * d + r]) + y;
-                    A.ws.v[int64_t(t) * d + r] = v;
-                }
-            }
-            if (!A.fuse_norm) continue;
-            // sum of squares of this 64-row block, fixed order
-            const float ss = warp_sum(mine ? v * v : 0.f);
-            if (lane == 0 && warp < 2) M.wsum[warp] = ss;
-            if (mine) __threadfence();
             named_bar_sync(1, kDecThreads);
             if (tid == 0) {
-                A.ws.ssq[t * comb_blocks + rb] = M.wsum[0] + M.wsum[1];
-                __threadfence();
-                M.flag[2 * nsub] = atomicAdd(A.ws.tok_cnt + t, 1) == comb_blocks - 1;
+                M.gate_ok = grid_barrier(A.ws.gbar, A.ws.gbar + 1, G);
+                if (!M.gate_ok) set_status(A.ws.status, GALE_ERR_TIMEOUT);
+                for (int q = 0; q < kCapMax; ++q) {   // the cache now holds slots of h
+                    M.key[q] = -1;
+                    M.stamp[q] = 0;
+                }
             }
             named_bar_sync(1, kDecThreads);
-            if (!M.flag[2 * nsub]) continue;
-            // every row block of token t is done: RMSNorm over d_model
-            __threadfence();
-            if (warp == 0) {
-                float tot = 0.f;
-                for (int q = lane; q < comb_blocks; q += 32) tot += __ldcg(A.ws.ssq + t * comb_blocks + q);
-                tot = warp_sum(tot);
-                if (lane == 0) M.inv = rsqrtf(tot / float(d) + A.eps);
-            }
-            named_bar_sync(1, kDecThreads);
-            const float inv = M.inv;
-            for (int c = tid; c < d; c += kDecThreads)
-                store_from_f32(A.out, GALE_BF16, int64_t(t) * d + c, __ldcg(A.ws.v + int64_t(t) * d + c) * inv);
-            named_bar_sync(1, kDecThreads);
+            if (!M.gate_ok) ok = false;
         }
     }
 }
 
-template <typename Kern, typename... Args>
-int launch_pdl(Kern kernel, int grid, int block, int smem, cudaStream_t st, bool pdl, Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = size_t(smem);
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? GALE_OK : GALE_ERR_CUDA;
-}
-
-// Deepest ring (up to 6 stages) with at least `min_cap` cached vectors that
-// fits the shared-memory budget.
-Shape fit_shape(Shape sh, int min_cap, int max_cap) {
+// Deepest ring that fits the shared-memory budget with at least two cached
+// vectors per phase; what is left over goes to the cache.
+bool make_plan(const gale_layer& L, int B, int K, Plan& P) {
     constexpr int kBudget = 226 * 1024;
-    for (int cap = max_cap; cap >= min_cap; --cap) {
-        for (int st = 6; st >= 3; --st) {
-            sh.n_stages = st;
-            sh.tok_cap = cap;
-            if (stream_smem(sh).bytes <= kBudget) return sh;
-        }
+    P.s13 = make_shape(L.d_ff, L.d_model, 2);
+    P.s2 = make_shape(L.d_model, L.d_ff, 1);
+    // at most B*K token groups; a CTA gets its share of both phases' jobs, rounded up
+    const int64_t groups = int64_t(B) * K, G = sm_count();
+    P.max_jobs = int((groups * P.s13.row_blocks + G - 1) / G + (groups * P.s2.row_blocks + G - 1) / G);
+    P.stage_bytes = P.s13.stage_bytes > P.s2.stage_bytes ? P.s13.stage_bytes : P.s2.stage_bytes;
+    const int min_cache = 2 * (P.s13.tok_bytes > P.s2.tok_bytes ? P.s13.tok_bytes : P.s2.tok_bytes);
+    for (int st = kMaxStages; st >= 3; --st) {
+        P.n_stages = st;
+        P.cache_bytes = min_cache;
+        const int room = kBudget - dec_smem(P).bytes;
+        if (room < 0) continue;
+        // the space left grows the cache, up to kCapMax entries of the larger phase
+        const int big = P.s13.tok_bytes > P.s2.tok_bytes ? P.s13.tok_bytes : P.s2.tok_bytes;
+        const int cap_big = 2 + room / big > kCapMax ? kCapMax : 2 + room / big;
+        P.cache_bytes = cap_big * big;
+        P.cap13 = P.cache_bytes / P.s13.tok_bytes > kCapMax ? kCapMax : P.cache_bytes / P.s13.tok_bytes;
+        P.cap2 = P.cache_bytes / P.s2.tok_bytes > kCapMax ? kCapMax : P.cache_bytes / P.s2.tok_bytes;
+        if (dec_smem(P).bytes <= kBudget) return true;
     }
-    sh.n_stages = 2;
-    sh.tok_cap = min_cap;
-    return sh;
+    return false;
 }
 
 }  // namespace
@@ -701,6 +1029,7 @@ DecodeWs carve_decode_ws(void* ws, const gale_layer& L, int B, int K) {
     const int64_t P = int64_t(B) * K, dm = L.d_model, df = L.d_ff;
     const int64_t blocks = (dm + 63) / 64;
     w.status = reinterpret_cast<int32_t*>(take(256));
+    w.gbar = w.status + 4;   // two counters inside the status block, zeroed every call
     w.comb_cnt = reinterpret_cast<int32_t*>(take(4 * B * blocks));
     w.tok_cnt = reinterpret_cast<int32_t*>(take(4 * int64_t(B)));
     w.ssq = reinterpret_cast<float*>(take(4 * B * blocks));
@@ -716,7 +1045,10 @@ bool decode_supported(const gale_layer& L, int B, int K) {
         L.n_experts > 1024 || !shape_ok(L.d_model, 2) || !shape_ok(L.d_ff, 1))
         return false;
     // the w2 jobs must cover whole 64-row combine blocks
-    return make_shape(L.d_model, L.d_ff, 1).job_rows % 64 == 0 && make_shape(L.d_model, L.d_ff, 1).job_rows <= 128;
+    const Shape s2 = make_shape(L.d_model, L.d_ff, 1);
+    if (s2.job_rows % 64 != 0 || s2.job_rows > 128) return false;
+    Plan P;
+    return make_plan(L, B, K, P);
 }
 
 int launch_moe_decode(const gale_layer& L, const uint16_t* x, const int32_t* ids, const float* gates, int B, int K,
@@ -741,31 +1073,34 @@ int launch_moe_decode(const gale_layer& L, const uint16_t* x, const int32_t* ids
     A.fuse_norm = fuse_norm;
     A.eps = eps;
     A.ws = carve_decode_ws(ws, L, B, K);
+    Plan P;
+    if (!make_plan(L, B, K, P)) return GALE_ERR_UNSUPPORTED;
 
-    CUtensorMap s1, b1, s3, b3, s2, b2;
+    Maps m;
     const char* base = static_cast<const char*>(L.base);
-    int rc = cached_map(&s1, false, base, L.d_ff, L.d_model, L.n_experts, L.expert_stride);
-    if (rc == GALE_OK) rc = cached_map(&b1, true, base, L.d_ff, L.d_model, L.n_experts, L.expert_stride);
-    if (rc == GALE_OK) rc = cached_map(&s3, false, base + l1, L.d_ff, L.d_model, L.n_experts, L.expert_stride);
-    if (rc == GALE_OK) rc = cached_map(&b3, true, base + l1, L.d_ff, L.d_model, L.n_experts, L.expert_stride);
-    if (rc == GALE_OK) rc = cached_map(&s2, false, base + 2 * l1, L.d_model, L.d_ff, L.n_experts, L.expert_stride);
-    if (rc == GALE_OK) rc = cached_map(&b2, true, base + 2 * l1, L.d_model, L.d_ff, L.n_experts, L.expert_stride);
+    int rc = cached_map(&m.s1, false, base, L.d_ff, L.d_model, L.n_experts, L.expert_stride);
+    if (rc == GALE_OK) rc = cached_map(&m.b1, true, base, L.d_ff, L.d_model, L.n_experts, L.expert_stride);
+    if (rc == GALE_OK) rc = cached_map(&m.s3, false, base + l1, L.d_ff, L.d_model, L.n_experts, L.expert_stride);
+    if (rc == GALE_OK) rc = cached_map(&m.b3, true, base + l1, L.d_ff, L.d_model, L.n_experts, L.expert_stride);
+    if (rc == GALE_OK) rc = cached_map(&m.s2, false, base + 2 * l1, L.d_model, L.d_ff, L.n_experts, L.expert_stride);
+    if (rc == GALE_OK) rc = cached_map(&m.b2, true, base + 2 * l1, L.d_model, L.d_ff, L.n_experts, L.expert_stride);
     if (rc != GALE_OK) return rc;
 
-    const int grid = sm_count();
-    // w1/w3: an ordinary launch, so that it follows all earlier work on the stream
-    const Shape s13 = fit_shape(make_shape(L.d_ff, L.d_model, 2), 2, 4);
-    StreamSmem S = stream_smem(s13);
-    rc = ensure_smem(reinterpret_cast<const void*>(moe_stream_kernel<true>), S.bytes);
+    const DecSmem S = dec_smem(P);
+    rc = ensure_smem(reinterpret_cast<const void*>(moe_decode_kernel), S.bytes);
     if (rc != GALE_OK) return rc;
-    rc = launch_pdl(moe_stream_kernel<true>, grid, kDecThreads + 32, S.bytes, st, false, s1, b1, s3, b3, A, s13);
-    if (rc != GALE_OK) return rc;
-    // w2: programmatic dependent launch after w1/w3
-    const Shape s2sh = fit_shape(make_shape(L.d_model, L.d_ff, 1), 2, 8);
-    S = stream_smem(s2sh);
-    rc = ensure_smem(reinterpret_cast<const void*>(moe_stream_kernel<false>), S.bytes);
-    if (rc != GALE_OK) return rc;
-    return launch_pdl(moe_stream_kernel<false>, grid, kDecThreads + 32, S.bytes, st, true, s2, b2, s2, b2, A, s2sh);
+    // all CTAs resident at once (the grid barrier), one per SM
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(sm_count()));
+    cfg.blockDim = dim3(kDecBlock);
+    cfg.dynamicSmemBytes = size_t(S.bytes);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, moe_decode_kernel, m, A, P) == cudaSuccess ? GALE_OK : GALE_ERR_CUDA;
 }
 
 }  // namespace gale

@@ -187,7 +187,7 @@ template <int NMAT>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_constant__ CUtensorMap xmap, TcArgs A) {
     using Cfg = TcCfg<NMAT>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
+    uint8_t* smem = smem_align1024(smem_raw);
     const int mtile = blockIdx.x, job_id = blockIdx.y;
     if (job_id >= *A.n_jobs) return;
     const TcJob job = A.jobs[job_id];

@@ -10,6 +10,13 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte aligned byte of a dynamic shared-memory array.  Pointer
+// arithmetic on the array itself keeps the shared state space known to the
+// compiler (shared loads and stores instead of generic ones).
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* raw) {
+    return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
@@ -95,11 +102,12 @@ __device__ __forceinline__ void smem_and(uint32_t addr, uint32_t v) {
     asm volatile("atom.shared.and.b32 _, [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-// Bounded wait on an mbarrier phase: false once `limit_ns` has passed.
+// Bounded wait on an mbarrier phase: false once `limit_ns` has passed.  Plain
+// try_wait polling (each try already waits a short, hardware-chosen time).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait_sleep(bar, parity))
+    while (!mbar_try_wait(bar, parity))
         if (globaltimer_ns() - t0 > limit_ns) return false;
     return true;
 }
@@ -128,7 +136,7 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // D += A(16x32, s8, row) * B(32x8, s8, col), exact int32 accumulate.
 __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
