@@ -33,17 +33,25 @@ import gale_synth as gs  # noqa: E402
 METRIC = "MoE expert-layer tokens/s and packed-expert HBM GB/s (% of B200 roofline)"
 UNIT = "tokens/s"
 D_MODEL, D_FF, N_EXPERTS, TOP_K = 4096, 2048, 256, 6
+PREFILL_B = 4096
+# kernels of this library launched per decode step (the cooperative layer kernel)
+DECODE_LAUNCHES = 1
+# dram read + write bytes of one decode launch at this workload, from the ncu
+# capture summarised in profiles/moe_decode_kernel_b1.md (None once the
+# kernel has changed since that capture)
+DECODE_TRAFFIC = 25_176_320
 WORKLOAD = ("moe_layer_decode: 256 GALE-1bit experts (w1/w3 [2048x4096], w2 [4096x2048]), "
             "top-6 softmax routing, bf16 hidden [B x 4096]")
 
 
 def peaks():
+    """HBM GB/s and dense 16-bit tensor TFLOP/s (burst) of this machine's B200s."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
 
 
 def dist_env():
@@ -130,12 +138,15 @@ def build_layer(torch, G, layer_id: int = 0):
     return buf, stride
 
 
-def routing_pool(n: int, B: int, tag0: int):
+def routing_pool(n: int, B: int, tag0: int, bias_sigma: float = 0.0, n_x: int = 0):
+    """n seeded (hidden, ids, gates, distinct experts) steps; n_x > 0 reuses
+    that many hidden-state draws (large batches: the routing is what varies)."""
     pool = []
+    xs = [gs.hidden_bf16(B, D_MODEL, tag=tag0 + i)[0] for i in range(n_x)] if n_x else None
     for i in range(n):
-        lg = gs.router_logits(B, N_EXPERTS, tag=tag0 + i)
+        lg = gs.router_logits(B, N_EXPERTS, tag=tag0 + i, bias_sigma=bias_sigma)
         ids, gates = gs.route_topk(lg, TOP_K)
-        bits, _ = gs.hidden_bf16(B, D_MODEL, tag=tag0 + i)
+        bits = xs[i % n_x] if n_x else gs.hidden_bf16(B, D_MODEL, tag=tag0 + i)[0]
         pool.append((bits, ids, gates, len(np.unique(ids))))
     return pool
 
@@ -158,8 +169,8 @@ def run_gpu(args):
     flush = torch.empty(max(2 * l2, 256 * 2 ** 20), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def measure(B, steps, warmup, tag0):
-        pool = routing_pool(steps + warmup, B, tag0 + 7919 * rank)
+    def measure(B, steps, warmup, tag0, bias_sigma=0.0, n_x=0):
+        pool = routing_pool(steps + warmup, B, tag0 + 7919 * rank, bias_sigma, n_x)
         dev = [(torch.from_numpy(b).view(torch.bfloat16).cuda(), torch.from_numpy(i).cuda(),
                 torch.from_numpy(g).cuda(), nd) for b, i, g, nd in pool]
         ws = torch.empty(G.gale_moe_workspace_size(layer, B, TOP_K), dtype=torch.uint8, device="cuda")
@@ -230,16 +241,20 @@ def run_gpu(args):
     clocks_info = clocks.stop()
     t8, bytes8, _ = measure(8, max(args.steps // 2, 3), args.warmup, 20_000)
     te, h2d, d2h = measure_e2e(1, args.steps, args.warmup, 30_000)
+    # prefill: 4096 tokens, skewed routing (tensor-core tile path)
+    pf_steps = max(3, min(args.steps // 5, 10))
+    tp, _, _ = measure(PREFILL_B, pf_steps, 3, 40_000, bias_sigma=0.5, n_x=2)
 
     # max over ranks of the device time
-    tt = torch.tensor([t1, t8, te], dtype=torch.float64, device="cuda")
+    tt = torch.tensor([t1, t8, te, tp], dtype=torch.float64, device="cuda")
     if world > 1:
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    t1, t8, te = [float(v) for v in tt.tolist()]
+    t1, t8, te, tp = [float(v) for v in tt.tolist()]
     tokens = 1 * args.steps * world
     value = tokens / t1
     gbs = bytes1 * world / t1 / 1e9
-    peak, peak_kind = peaks()
+    peak, tpeak, peak_kind = peaks()
+    pf_flops = 2.0 * PREFILL_B * TOP_K * 3 * D_FF * D_MODEL   # dense-equivalent, per layer
     avg_launch = t1 / args.steps
     achieved = bytes1 / args.steps / avg_launch / 1e9
     result = {
@@ -252,12 +267,18 @@ def run_gpu(args):
                    "routing": "fresh seeded routing every step", "parallelism": f"replicas{world}"},
         "hbm_gbs": gbs,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
-                     "kernel": "gale_moe_forward (whole layer)"},
+                     "frac": achieved / peak, "traffic": DECODE_TRAFFIC, "peak_kind": peak_kind,
+                     "kernel": "moe_decode_kernel (the whole layer is this one launch)",
+                     "algorithmic_bytes_per_launch": bytes1 / args.steps},
         "b8": {"tokens_per_s": 8 * max(args.steps // 2, 3) * world / t8,
                "hbm_gbs": bytes8 * world / t8 / 1e9, "frac": bytes8 * world / t8 / 1e9 / peak},
+        "prefill": {"workload": "4096 tokens, top-6 with per-expert bias N(0, 0.5) (skewed), same 256 experts",
+                    "tokens_per_s": PREFILL_B * pf_steps * world / tp, "ms_per_step": 1e3 * tp / pf_steps,
+                    "tflops": pf_flops * pf_steps / tp / 1e12, "peak_tflops": tpeak,
+                    "frac": pf_flops * pf_steps / tp / 1e12 / tpeak, "bound": "tensor",
+                    "flops_per_step": pf_flops, "steps": pf_steps},
         "e2e": {"value": tokens / te, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": DECODE_LAUNCHES * args.steps,
         "clocks": clocks_info,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -267,6 +288,35 @@ def run_gpu(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def run_profile(args):
+    """A short fixed sequence for ncu captures: build the layer, run
+    --warmup calls, flush L2, run --steps calls (decode: unbiased routing;
+    prefill: per-expert bias N(0, 0.5)), print the device status."""
+    import torch
+    import bit_expert_gemv_b200 as G
+    G.lib()
+    buf, stride = build_layer(torch, G)
+    layer = G.make_layer(buf, stride, N_EXPERTS, D_MODEL, D_FF)
+    B = args.batch
+    pool = routing_pool(args.steps + args.warmup, B, 80_000, 0.5 if args.only == "prefill" else 0.0,
+                        n_x=2 if B > 64 else 0)
+    dev = [(torch.from_numpy(b).view(torch.bfloat16).cuda(), torch.from_numpy(i).cuda(),
+            torch.from_numpy(g).cuda()) for b, i, g, _ in pool]
+    ws = torch.empty(G.gale_moe_workspace_size(layer, B, TOP_K), dtype=torch.uint8, device="cuda")
+    out = torch.empty(B, D_MODEL, dtype=torch.float32, device="cuda")
+    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device="cuda")
+    for s in range(args.warmup):
+        G.gale_moe_forward(layer, *dev[s], out, ws)
+    torch.cuda.synchronize()
+    flush.zero_()
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        G.gale_moe_forward(layer, *dev[args.warmup + s], out, ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": args.only, "batch": B, "steps": args.steps,
+                      "status": int(ws[:4].view(torch.int32).item())}), flush=True)
 
 
 # ----------------------------------------------------------------------------
@@ -343,11 +393,16 @@ def main():
     ap.add_argument("--impl", default="gale", choices=["gale", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["decode", "prefill"], default=None,
+                    help="profiling driver: warm-up, an L2 flush, then --steps layer calls of one path")
+    ap.add_argument("--batch", type=int, default=1, help="tokens per step with --only")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.only:
+        run_profile(args)
     else:
         run_gpu(args)
 

@@ -929,12 +929,12 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_c
             uint8_t* stage = smem + S.ring + s * P.stage_bytes;
             float* pb = reinterpret_cast<float*>(smem + S.part) + s * kPartFloats;
             float part[2] = {0.f, 0.f};
-            const int r0 = Jb.tile * sh.job_rows + tr * 16;
-            if (ok && r0 < sh.rows)
-                chunk_mma(stage + (tr * sh.n_mat + mat) * sh.tile_bytes, C, ch, tok, scratch, part);
             float corr0 = 0.f, corr1 = 0.f;
+            const int r0 = Jb.tile * sh.job_rows + tr * 16;
             const int or0 = Jb.tile * sh.job_rows + o_tr * 16;
-            if (ok && or0 + o_row < sh.rows && k) {
+            const bool do_mma = ok && r0 < sh.rows, do_out = ok && or0 + o_row < sh.rows && k;
+            if (do_mma) chunk_mma(stage + (tr * sh.n_mat + mat) * sh.tile_bytes, C, ch, tok, scratch, part);
+            if (do_out) {
                 const MatView ov = make_view(A.base + int64_t(Jb.e) * A.stride +
                                                  (W13 ? (o_mat ? A.off_w3 : A.off_w1) : A.off_w2),
                                              sh.rows, C);
@@ -960,8 +960,9 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_c
             if (lane == 0) last = atomicAdd(&M.ecnt[s], 1) == kDecWarps - 1;
             last = __shfl_sync(0xffffffffu, last, 0);
             if (last) job_epilogue(A, R, sh, W13, Jb, pb, lane, &M.ecnt[s]);
-            // the stage (and its partial sums) may be refilled once all warps are past here
-            fence_proxy_async();
+            // the stage (and its partial sums) may be refilled once all warps
+            // are past here; the stage was only read, so the barrier alone
+            // orders the reads before the next copy
             __syncwarp();
             if (lane == 0) mbar_arrive(empty + s);
             if (++st == P.n_stages) {
