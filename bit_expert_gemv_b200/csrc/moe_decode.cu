@@ -294,6 +294,36 @@ __device__ __forceinline__ Job unpack_job(uint2 v) {
 // shapes and shared memory
 // ----------------------------------------------------------------------------
 
+// One matrix's part of a staged job of R consecutive rows.  In a packed record
+// the R rows of every section are contiguous, so each section arrives in one
+// bulk copy (large copies keep the copy engines near full bandwidth; 16-row
+// boxes of 2 KB reached about a third of it).  Signs stay in record order:
+// row r at r * C / 8 bytes.
+struct JobTile {
+    int signs, scales, idx, q, srow, bytes;
+};
+
+__host__ __device__ inline JobTile job_tile(int C, int R) {
+    const int k = outliers_per_row(C);
+    JobTile t;
+    int o = 0;
+    t.signs = o;
+    o += R * (C / 8);
+    t.scales = o;
+    o += R * (C / 64);
+    t.idx = o;
+    o += (R * k * 2 + 15) & ~15;
+    t.q = o;
+    o += ((R * k + 1) / 2 + 31) & ~15;   // plus the source's offset from a 16-byte boundary
+    t.srow = o;
+    o += (R * 2 + 15) & ~15;
+    t.bytes = (o + 127) & ~127;
+    return t;
+}
+
+// ----------------------------------------------------------------------------
+// ----------------------------------------------------------------------------
+
 struct Shape {
     int rows, cols;      // rows and columns of the streamed matrices
     int n_mat;           // 2 (w1, w3) or 1 (w2)
@@ -301,8 +331,8 @@ struct Shape {
     int r_tiles;         // 16-row tiles per job: 8 / (n_mat * n_chunk)
     int job_rows;        // 16 * r_tiles
     int row_blocks;      // jobs per token group: ceil(rows / job_rows)
-    int tile_bytes;      // stage_layout(cols).bytes
-    int stage_bytes;     // r_tiles * n_mat * tile_bytes
+    int mat_bytes;       // job_tile(cols, job_rows).bytes
+    int stage_bytes;     // n_mat * mat_bytes
     int tok_bytes;       // digits + 128-block sums + fp16 copy of one rotated vector
     int pairs;           // (matrix, row) pairs of a job: n_mat * job_rows
 };
@@ -316,8 +346,8 @@ __host__ __device__ inline Shape make_shape(int rows, int cols, int n_mat) {
     s.r_tiles = kDecWarps / (n_mat * s.n_chunk);
     s.job_rows = 16 * s.r_tiles;
     s.row_blocks = (rows + s.job_rows - 1) / s.job_rows;
-    s.tile_bytes = stage_layout(cols).bytes;
-    s.stage_bytes = s.r_tiles * n_mat * s.tile_bytes;
+    s.mat_bytes = job_tile(cols, s.job_rows).bytes;
+    s.stage_bytes = n_mat * s.mat_bytes;
     s.tok_bytes = int(align_up(cols * kPieces + (cols / 128) * 4 + cols * 2, 16));
     s.pairs = n_mat * s.job_rows;
     return s;
@@ -514,18 +544,17 @@ __device__ __forceinline__ void ensure_cached(const DecArgs& A, const Shape& sh,
 // per-warp pieces of a job
 // ----------------------------------------------------------------------------
 
-// Tensor-core part of one 1024-column chunk `ch` of a staged 16-row tile for
+// Tensor-core part of one 1024-column chunk `ch` of 16 staged rows (signs in
+// record order from `signs16`, block scales from `sblk`) for
 // up to two tokens: lanes 0..15 return, for row r0 + lane and tokens 0 and 1,
 //   sum_{b in chunk} s_blk[row, b] (X_b - 2 P_b).
 // The chunk's eight 128-column blocks run in two halves of four blocks with
 // one accumulator each, so that consecutive MMAs are independent.
-__device__ __forceinline__ void chunk_mma(const uint8_t* tile, int C, int ch, const TokRef (&tok)[2], float* scratch,
-                                          float (&part)[2]) {
+__device__ __forceinline__ void chunk_mma(const uint8_t* signs16, const __half* sblk, int C, int ch,
+                                          const TokRef (&tok)[2], float* scratch, float (&part)[2]) {
     const int lane = threadIdx.x & 31;
-    const int nb = C / 128;
-    const StageLayout L = stage_layout(C);
-    const uint8_t* signs = tile + L.signs + ch * 2048;
-    const __half* sblk = reinterpret_cast<const __half*>(tile + L.scales);
+    const int nb = C / 128, rowb = C / 8;
+    const uint8_t* signs = signs16 + ch * 128;
     const int row = lane & 15, half = lane >> 4;
     const bool has0 = tok[0].pieces != nullptr, has1 = tok[1].pieces != nullptr;
 
@@ -558,9 +587,9 @@ __device__ __forceinline__ void chunk_mma(const uint8_t* tile, int C, int ch, co
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int bb = 4 * hb + j;
-            const uint8_t* wa = signs + g * 128 + ((bb ^ (g & 7)) << 4) + tig * 4;
+            const uint8_t* wa = signs + g * rowb + bb * 16 + tig * 4;
             wg[j] = *reinterpret_cast<const uint32_t*>(wa);
-            wg8[j] = *reinterpret_cast<const uint32_t*>(wa + 1024);
+            wg8[j] = *reinterpret_cast<const uint32_t*>(wa + 8 * rowb);
             if (bsrc) {
                 q0[j] = *reinterpret_cast<const uint4*>(bsrc_p + bb * kPieceBlockBytes);
                 q1[j] = *reinterpret_cast<const uint4*>(bsrc_p + bb * kPieceBlockBytes + 16);
@@ -616,14 +645,13 @@ __device__ __forceinline__ void chunk_mma(const uint8_t* tile, int C, int ch, co
 // staged tile over the outliers j = sub, sub + step, ... (a fixed lane set
 // of the row sums them afterwards in a fixed order); six at a time so that
 // their loads overlap.
-__device__ __forceinline__ void row_outliers(const uint8_t* tile, int C, int k, int q_delta, int row, int sub, int step,
-                                             const TokRef (&tok)[2], float& corr0, float& corr1) {
-    const StageLayout L = stage_layout(C);
+__device__ __forceinline__ void row_outliers(const uint8_t* tile, const JobTile& L, int C, int k, int q_delta, int row,
+                                             int sub, int step, const TokRef (&tok)[2], float& corr0, float& corr1) {
     const int nb = C / 128;
     const uint16_t* ri = reinterpret_cast<const uint16_t*>(tile + L.idx) + row * k;
     const uint8_t* qn = tile + L.q + q_delta;
     const __half* sblk = reinterpret_cast<const __half*>(tile + L.scales) + row * nb;
-    const uint8_t* signs = tile + L.signs + row * 128;
+    const uint8_t* signs = tile + L.signs + row * (C / 8);
     const float srow = __half2float(reinterpret_cast<const __half*>(tile + L.srow)[row]);
     const bool has0 = tok[0].pieces != nullptr, has1 = tok[1].pieces != nullptr;
     const __half* x0 = tok[0].x16;
@@ -643,9 +671,7 @@ __device__ __forceinline__ void row_outliers(const uint8_t* tile, int C, int k, 
             const int n = row * k + (use[u] ? jb + u * step : 0);
             const int qb = int(qn[n >> 1]) >> ((n & 1) * 4);
             const int qv = (qb & 15) - ((qb & 8) << 1);
-            const int w = (c[u] >> 5) & 31;
-            const uint32_t word = *reinterpret_cast<const uint32_t*>(
-                signs + (c[u] >> 10) * 2048 + (((w >> 2) ^ (row & 7)) << 4) + (w & 3) * 4);
+            const uint32_t word = *reinterpret_cast<const uint32_t*>(signs + (c[u] >> 5) * 4);
             const float sb = __half2float(sblk[c[u] >> 7]);
             float wq = fmaf(float(qv), srow, ((word >> (c[u] & 31)) & 1u) ? sb : -sb);
             wq = use[u] ? wq : 0.f;
@@ -659,108 +685,136 @@ __device__ __forceinline__ void row_outliers(const uint8_t* tile, int C, int k, 
 // the kernel
 // ----------------------------------------------------------------------------
 
-// The epilogue of a job, run by the last warp to finish it: w1/w3 stores
-// h = silu(w1 x) * (w3 x); w2 stores the expert outputs and runs the
-// (token, 64-row block) combine and the RMSNorm of finished tokens.
-__device__ __forceinline__ void job_epilogue(const DecArgs& A, const RouteTables& R, const Shape& sh, bool W13,
-                                          const Job& Jb, const float* pb, int lane, int* ecnt) {
-    const int d = A.d_model;
-    const int comb_blocks = (d + 63) / 64;
-    __threadfence_block();
-    if (lane == 0) *ecnt = 0;
+// The epilogue of a job, run by the last warp to finish it, in two parts:
+// epi_gather reads the job's partial sums (shared memory of the job's stage)
+// into registers, after which the stage can be refilled; epi_finish does the
+// global-memory work: w1/w3 stores h = silu(w1 x) * (w3 x); w2 stores the
+// expert outputs and runs the (token, 64-row block) combine and the RMSNorm of
+// finished tokens.  Lane l holds value i for row block tile i, row l & 15,
+// token l >> 4.
+constexpr int kMaxRT = 8;   // row tiles per job (job_rows <= 128)
+
+__device__ __forceinline__ void epi_gather(const Shape& sh, bool W13, const float* pb, int lane, float (&ya)[kMaxRT],
+                                           float (&yb)[kMaxRT]) {
     const float* pc = pb + kDecWarps * 32;
-    if (W13) {
-#pragma unroll 1
-        for (int v = lane; v < sh.r_tiles * 32; v += 32) {
-            const int t_r = v >> 5, row = v & 15, t = (v >> 4) & 1;
-            const int slot = t ? Jb.slot1 : Jb.slot0;
-            const int r = Jb.tile * sh.job_rows + t_r * 16 + row;
-            float y1 = pc[(t_r * 16 + row) * 2 + t], y3 = pc[(sh.job_rows + t_r * 16 + row) * 2 + t];
-#pragma unroll 1
+    const int row = lane & 15, t = lane >> 4;
+#pragma unroll
+    for (int i = 0; i < kMaxRT; ++i) {
+        ya[i] = 0.f;
+        yb[i] = 0.f;
+        if (i >= sh.r_tiles) continue;
+        if (W13) {
+            float y1 = pc[(i * 16 + row) * 2 + t], y3 = pc[(sh.job_rows + i * 16 + row) * 2 + t];
             for (int c2 = 0; c2 < sh.n_chunk; ++c2) {
-                y1 += pb[((t_r * 2 + 0) * sh.n_chunk + c2) * 32 + row * 2 + t];
-                y3 += pb[((t_r * 2 + 1) * sh.n_chunk + c2) * 32 + row * 2 + t];
+                y1 += pb[((i * 2 + 0) * sh.n_chunk + c2) * 32 + row * 2 + t];
+                y3 += pb[((i * 2 + 1) * sh.n_chunk + c2) * 32 + row * 2 + t];
             }
-            if (slot >= 0 && r < sh.rows) A.ws.h[int64_t(slot) * sh.rows + r] = silu(y1) * y3;
-        }
-    } else {
-#pragma unroll 1
-        for (int v = lane; v < sh.r_tiles * 32; v += 32) {
-            const int t_r = v >> 5, row = v & 15, t = (v >> 4) & 1;
-            const int slot = t ? Jb.slot1 : Jb.slot0;
-            const int r = Jb.tile * sh.job_rows + t_r * 16 + row;
-            float y = pc[(t_r * 16 + row) * 2 + t];
-#pragma unroll 1
-            for (int c2 = 0; c2 < sh.n_chunk; ++c2) y += pb[(t_r * sh.n_chunk + c2) * 32 + row * 2 + t];
-            if (slot >= 0 && r < d) A.ws.o[int64_t(slot) * d + r] = y;
-        }
-        __threadfence();
-        __syncwarp();
-        // the (token, 64-row block) combine: the last expert to finish sums the K outputs
-        const int nsub = sh.job_rows / 64;
-        int flags = 0;
-        if (lane < 2 * nsub) {
-            const int sl = lane & 1, sb = lane >> 1;
-            const int slot = sl ? Jb.slot1 : Jb.slot0;
-            const int rb = Jb.tile * nsub + sb;
-            if (slot >= 0 && rb < comb_blocks) {
-                const int t = R.slot_tok[slot];
-                flags = atomicAdd(A.ws.comb_cnt + t * comb_blocks + rb, 1) == R.tok_valid[t] - 1;
-            }
-        }
-        const unsigned fl = __ballot_sync(0xffffffffu, flags);
-#pragma unroll 1
-        for (int f = 0; f < 2 * nsub; ++f) {
-            if (!((fl >> f) & 1)) continue;
-            __threadfence();
-            const int sl = f & 1, sb = f >> 1;
-            const int t = R.slot_tok[sl ? Jb.slot1 : Jb.slot0];
-            const int rb = Jb.tile * nsub + sb;
-            float ss = 0.f;
-#pragma unroll 1
-            for (int rr = lane; rr < 64; rr += 32) {
-                const int r = rb * 64 + rr;
-                if (r >= d) continue;
-                float y = 0.f;
-#pragma unroll 1
-                for (int kk = 0; kk < A.K; ++kk) {
-                    const int pos = R.pos_of_pair[t * A.K + kk];
-                    if (pos >= 0) y = fmaf(A.gates[t * A.K + kk], __ldcg(A.ws.o + int64_t(pos) * d + r), y);
-                }
-                if (!A.fuse_norm) {
-                    store_from_f32(A.out, A.out_dtype, int64_t(t) * d + r, y);
-                } else {
-                    const float v = bf16_to_f32(A.x[int64_t(t) * d + r]) + y;
-                    A.ws.v[int64_t(t) * d + r] = v;
-                    ss = fmaf(v, v, ss);
-                }
-            }
-            if (!A.fuse_norm) continue;
-            // sum of squares of this 64-row block (fixed order), then the
-            // last block of the token normalises the whole row
-            ss = warp_sum(ss);
-            int lastblk = 0;
-            if (lane == 0) {
-                A.ws.ssq[t * comb_blocks + rb] = ss;
-                __threadfence();
-                lastblk = atomicAdd(A.ws.tok_cnt + t, 1) == comb_blocks - 1;
-            }
-            __syncwarp();
-            lastblk = __shfl_sync(0xffffffffu, lastblk, 0);
-            if (!lastblk) continue;
-            __threadfence();
-            float tot = 0.f;
-#pragma unroll 1
-            for (int q = lane; q < comb_blocks; q += 32) tot += __ldcg(A.ws.ssq + t * comb_blocks + q);
-            tot = warp_sum(tot);
-            const float inv = rsqrtf(tot / float(d) + A.eps);
-#pragma unroll 1
-            for (int c = lane; c < d; c += 32)
-                store_from_f32(A.out, GALE_BF16, int64_t(t) * d + c,
-                               __ldcg(A.ws.v + int64_t(t) * d + c) * inv);
+            ya[i] = y1;
+            yb[i] = y3;
+        } else {
+            float y = pc[(i * 16 + row) * 2 + t];
+            for (int c2 = 0; c2 < sh.n_chunk; ++c2) y += pb[(i * sh.n_chunk + c2) * 32 + row * 2 + t];
+            ya[i] = y;
         }
     }
 }
+
+__device__ __forceinline__ void epi_finish(const DecArgs& A, const RouteTables& R, const Shape& sh, bool W13,
+                                           const Job& Jb, int lane, const float (&ya)[kMaxRT],
+                                           const float (&yb)[kMaxRT]) {
+    const int d = A.d_model;
+    const int comb_blocks = (d + 63) / 64;
+    const int row = lane & 15, t_l = lane >> 4;
+    const int slot_l = t_l ? Jb.slot1 : Jb.slot0;
+    if (W13) {
+#pragma unroll
+        for (int i = 0; i < kMaxRT; ++i) {
+            const int r = Jb.tile * sh.job_rows + i * 16 + row;
+            if (i < sh.r_tiles && slot_l >= 0 && r < sh.rows) A.ws.h[int64_t(slot_l) * sh.rows + r] = silu(ya[i]) * yb[i];
+        }
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxRT; ++i) {
+        const int r = Jb.tile * sh.job_rows + i * 16 + row;
+        if (i < sh.r_tiles && slot_l >= 0 && r < d) A.ws.o[int64_t(slot_l) * d + r] = ya[i];
+    }
+    __threadfence();
+    __syncwarp();
+    // the (token, 64-row block) combine: the last expert to finish sums the K outputs
+    const int nsub = sh.job_rows / 64;
+    int flags = 0;
+    if (lane < 2 * nsub) {
+        const int sl = lane & 1, sb = lane >> 1;
+        const int slot = sl ? Jb.slot1 : Jb.slot0;
+        const int rb = Jb.tile * nsub + sb;
+        if (slot >= 0 && rb < comb_blocks) {
+            const int t = R.slot_tok[slot];
+            flags = atomicAdd(A.ws.comb_cnt + t * comb_blocks + rb, 1) == R.tok_valid[t] - 1;
+        }
+    }
+    const unsigned fl = __ballot_sync(0xffffffffu, flags);
+    for (int f = 0; f < 2 * nsub; ++f) {
+        if (!((fl >> f) & 1)) continue;
+        __threadfence();
+        const int sl = f & 1, sb = f >> 1;
+        const int t = R.slot_tok[sl ? Jb.slot1 : Jb.slot0];
+        const int rb = Jb.tile * nsub + sb;
+        float ss = 0.f;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int r = rb * 64 + lane + 32 * h2;
+            if (r >= d) continue;
+            // all K loads first, then the sum in fixed k order
+            float ov[16], gv[16];
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk) {
+                ov[kk] = 0.f;
+                gv[kk] = 0.f;
+                if (kk < A.K) {
+                    const int pos = R.pos_of_pair[t * A.K + kk];
+                    if (pos >= 0) {
+                        ov[kk] = __ldcg(A.ws.o + int64_t(pos) * d + r);
+                        gv[kk] = A.gates[t * A.K + kk];
+                    }
+                }
+            }
+            float y = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk)
+                if (kk < A.K) y = fmaf(gv[kk], ov[kk], y);
+            if (!A.fuse_norm) {
+                store_from_f32(A.out, A.out_dtype, int64_t(t) * d + r, y);
+            } else {
+                const float v = bf16_to_f32(A.x[int64_t(t) * d + r]) + y;
+                A.ws.v[int64_t(t) * d + r] = v;
+                ss = fmaf(v, v, ss);
+            }
+        }
+        if (!A.fuse_norm) continue;
+        // sum of squares of this 64-row block (fixed order), then the last
+        // block of the token normalises the whole row
+        ss = warp_sum(ss);
+        int lastblk = 0;
+        if (lane == 0) {
+            A.ws.ssq[t * comb_blocks + rb] = ss;
+            __threadfence();
+            lastblk = atomicAdd(A.ws.tok_cnt + t, 1) == comb_blocks - 1;
+        }
+        __syncwarp();
+        lastblk = __shfl_sync(0xffffffffu, lastblk, 0);
+        if (!lastblk) continue;
+        __threadfence();
+        float tot = 0.f;
+        for (int q = lane; q < comb_blocks; q += 32) tot += __ldcg(A.ws.ssq + t * comb_blocks + q);
+        tot = warp_sum(tot);
+        const float inv = rsqrtf(tot / float(d) + A.eps);
+#pragma unroll 4
+        for (int c = lane; c < d; c += 32)
+            store_from_f32(A.out, GALE_BF16, int64_t(t) * d + c, __ldcg(A.ws.v + int64_t(t) * d + c) * inv);
+    }
+}
+
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
     int v;
@@ -786,12 +840,8 @@ __device__ bool grid_barrier(int32_t* cnt, int32_t* flag, int G) {
     return true;
 }
 
-struct Maps {
-    CUtensorMap s1, b1, s3, b3, s2, b2;
-};
 
-__global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_constant__ Maps maps, DecArgs A,
-                                                                  Plan P) {
+__global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Plan P) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_align1024(smem_raw);
     const DecSmem S = dec_smem(P);
@@ -826,9 +876,10 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_c
     __syncthreads();
 
     if (warp == kDecWarps) {
-        // ---------------- producer: weights only.  Lane 0 arms the stage's
-        // barrier with the job's byte count, then every lane issues the
-        // copies of one (row tile, matrix) of the job.
+        // ---------------- producer: weights only.  Lane mt copies matrix mt of
+        // the job (five bulk copies: signs, block scales, outlier columns,
+        // outlier values, row scales of all the job's rows); lane 0 arms the
+        // stage's barrier with the job's byte count first.
         int s = 0, ph = 0;
         for (int i = 0; i < n13 + n2; ++i) {
             int ok_wait = 1;
@@ -841,25 +892,40 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_c
             const bool w13 = i < n13;
             const Shape& sh = w13 ? P.s13 : P.s2;
             const Job Jb = unpack_job(jobs[i]);
-            const int tr = lane / sh.n_mat, mt = lane % sh.n_mat;
-            const int r0 = Jb.tile * sh.job_rows + tr * 16;
-            const bool mine = lane < sh.r_tiles * sh.n_mat && r0 < sh.rows;
-            uint32_t tx = 0;
-            MatView mv{};
-            const int64_t off = w13 ? (mt ? A.off_w3 : A.off_w1) : A.off_w2;
+            const int C = sh.cols, nb = C / 128, k = outliers_per_row(C);
+            const int r0 = Jb.tile * sh.job_rows;
+            const int R = min(sh.job_rows, sh.rows - r0);
+            const bool mine = lane < sh.n_mat;
+            const JobTile L = job_tile(C, sh.job_rows);
+            uint32_t sz[5] = {0u, 0u, 0u, 0u, 0u};
+            const char* src[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
             if (mine) {
-                mv = make_view(A.base + int64_t(Jb.e) * A.stride + off, sh.rows, sh.cols);
-                tx = tile_tx_bytes(mv, r0);
+                const int64_t off = w13 ? (lane ? A.off_w3 : A.off_w1) : A.off_w2;
+                const MatView mv = make_view(A.base + int64_t(Jb.e) * A.stride + off, sh.rows, C);
+                const char* qs = reinterpret_cast<const char*>(mv.q) + int64_t(r0) * k / 2;   // r0 is even
+                const int qd = int(reinterpret_cast<uintptr_t>(qs) & 15);
+                src[0] = reinterpret_cast<const char*>(mv.signs + int64_t(r0) * (C / 32));
+                sz[0] = uint32_t(R * (C / 8));
+                src[1] = reinterpret_cast<const char*>(mv.s_blk + int64_t(r0) * nb);
+                sz[1] = uint32_t(R * (C / 64));
+                src[2] = reinterpret_cast<const char*>(mv.idx + int64_t(r0) * k);
+                sz[2] = k ? uint32_t(R * k * 2) : 0u;
+                src[3] = qs - qd;
+                sz[3] = k ? uint32_t((qd + (R * k + 1) / 2 + 15) & ~15) : 0u;
+                src[4] = reinterpret_cast<const char*>(mv.s_row + r0);
+                sz[4] = uint32_t(R * 2);
             }
+            uint32_t tx = sz[0] + sz[1] + sz[2] + sz[3] + sz[4];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) tx += __shfl_xor_sync(0xffffffffu, tx, o);
             if (lane == 0) mbar_arrive_expect_tx(full + s, tx);
             __syncwarp();
             if (mine) {
-                const CUtensorMap* smap = w13 ? (mt ? &maps.s3 : &maps.s1) : &maps.s2;
-                const CUtensorMap* bmap = w13 ? (mt ? &maps.b3 : &maps.b1) : &maps.b2;
-                issue_tile_copies(smem + S.ring + s * P.stage_bytes + (tr * sh.n_mat + mt) * sh.tile_bytes,
-                                  full + s, smap, bmap, mv, Jb.e, r0);
+                uint8_t* dst = smem + S.ring + s * P.stage_bytes + lane * sh.mat_bytes;
+                const int dsto[5] = {L.signs, L.scales, L.idx, L.q, L.srow};
+#pragma unroll
+                for (int c = 0; c < 5; ++c)
+                    if (sz[c]) bulk_load(dst + dsto[c], src[c], sz[c], full + s);
             }
             if (++s == P.n_stages) {
                 s = 0;
@@ -933,15 +999,22 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_c
             const int r0 = Jb.tile * sh.job_rows + tr * 16;
             const int or0 = Jb.tile * sh.job_rows + o_tr * 16;
             const bool do_mma = ok && r0 < sh.rows, do_out = ok && or0 + o_row < sh.rows && k;
-            if (do_mma) chunk_mma(stage + (tr * sh.n_mat + mat) * sh.tile_bytes, C, ch, tok, scratch, part);
+            const JobTile L = job_tile(C, sh.job_rows);
+            if (do_mma) {
+                const uint8_t* mt_tile = stage + mat * sh.mat_bytes;
+                chunk_mma(mt_tile + L.signs + tr * 16 * (C / 8),
+                          reinterpret_cast<const __half*>(mt_tile + L.scales) + tr * 16 * (C / 128), C, ch, tok,
+                          scratch, part);
+            }
             if (do_out) {
                 const MatView ov = make_view(A.base + int64_t(Jb.e) * A.stride +
                                                  (W13 ? (o_mat ? A.off_w3 : A.off_w1) : A.off_w2),
                                              sh.rows, C);
-                const int q_delta =
-                    int(reinterpret_cast<uintptr_t>(reinterpret_cast<const char*>(ov.q) + int64_t(or0) * k / 2) & 15);
-                row_outliers(stage + (o_tr * sh.n_mat + o_mat) * sh.tile_bytes, C, k, q_delta, o_row, sub, lpp, tok,
-                             corr0, corr1);
+                const int q_delta = int(
+                    reinterpret_cast<uintptr_t>(reinterpret_cast<const char*>(ov.q) + int64_t(Jb.tile * sh.job_rows) * k / 2) &
+                    15);
+                row_outliers(stage + o_mat * sh.mat_bytes, L, C, k, q_delta, o_tr * 16 + o_row, sub, lpp, tok, corr0,
+                             corr1);
             }
             for (int o = 1; o < lpp; o <<= 1) {
                 corr0 += __shfl_xor_sync(0xffffffffu, corr0, o);
@@ -959,12 +1032,21 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_c
             int last = 0;
             if (lane == 0) last = atomicAdd(&M.ecnt[s], 1) == kDecWarps - 1;
             last = __shfl_sync(0xffffffffu, last, 0);
-            if (last) job_epilogue(A, R, sh, W13, Jb, pb, lane, &M.ecnt[s]);
-            // the stage (and its partial sums) may be refilled once all warps
-            // are past here; the stage was only read, so the barrier alone
-            // orders the reads before the next copy
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty + s);
+            // the stage (and its partial sums) may be refilled once every warp
+            // has read what it needs; the stage was only read, so the barrier
+            // alone orders those reads before the next copy
+            if (last) {
+                __threadfence_block();
+                if (lane == 0) M.ecnt[s] = 0;
+                float ya[kMaxRT], yb[kMaxRT];
+                epi_gather(sh, W13, pb, lane, ya, yb);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty + s);
+                epi_finish(A, R, sh, W13, Jb, lane, ya, yb);
+            } else {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty + s);
+            }
             if (++st == P.n_stages) {
                 st = 0;
                 ph ^= 1;
@@ -1077,16 +1159,7 @@ int launch_moe_decode(const gale_layer& L, const uint16_t* x, const int32_t* ids
     Plan P;
     if (!make_plan(L, B, K, P)) return GALE_ERR_UNSUPPORTED;
 
-    Maps m;
-    const char* base = static_cast<const char*>(L.base);
-    int rc = cached_map(&m.s1, false, base, L.d_ff, L.d_model, L.n_experts, L.expert_stride);
-    if (rc == GALE_OK) rc = cached_map(&m.b1, true, base, L.d_ff, L.d_model, L.n_experts, L.expert_stride);
-    if (rc == GALE_OK) rc = cached_map(&m.s3, false, base + l1, L.d_ff, L.d_model, L.n_experts, L.expert_stride);
-    if (rc == GALE_OK) rc = cached_map(&m.b3, true, base + l1, L.d_ff, L.d_model, L.n_experts, L.expert_stride);
-    if (rc == GALE_OK) rc = cached_map(&m.s2, false, base + 2 * l1, L.d_model, L.d_ff, L.n_experts, L.expert_stride);
-    if (rc == GALE_OK) rc = cached_map(&m.b2, true, base + 2 * l1, L.d_model, L.d_ff, L.n_experts, L.expert_stride);
-    if (rc != GALE_OK) return rc;
-
+    int rc = GALE_OK;
     const DecSmem S = dec_smem(P);
     rc = ensure_smem(reinterpret_cast<const void*>(moe_decode_kernel), S.bytes);
     if (rc != GALE_OK) return rc;
@@ -1101,7 +1174,7 @@ int launch_moe_decode(const gale_layer& L, const uint16_t* x, const int32_t* ids
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, moe_decode_kernel, m, A, P) == cudaSuccess ? GALE_OK : GALE_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, moe_decode_kernel, A, P) == cudaSuccess ? GALE_OK : GALE_ERR_CUDA;
 }
 
 }  // namespace gale

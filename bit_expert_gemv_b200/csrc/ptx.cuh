@@ -96,6 +96,11 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Arrive on a named barrier without waiting (the waiting side uses
+// named_bar_sync with the same total count).
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 // atom.shared.and on a shared-memory byte address.
 __device__ __forceinline__ void smem_and(uint32_t addr, uint32_t v) {
