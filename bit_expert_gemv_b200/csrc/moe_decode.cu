@@ -372,7 +372,6 @@ struct CacheSmem {
     int plan_slot[2], plan_key[2], n_plan, clock;
     float red[kDecWarps];
     int cres[2];                  // cache indices of the current job's vectors
-    int ecnt[kMaxStages];         // warps done with the job in each stage
     int gate_ok;
 };
 
@@ -398,7 +397,7 @@ __host__ __device__ inline DecSmem dec_smem(const Plan& P) {
     s.scratch = o;
     o += kDecWarps * kWarpScratchFloats * 4;
     s.bars = o;
-    o += 2 * P.n_stages * 8;
+    o += 3 * P.n_stages * 8;
     s.misc = o;
     o += int(align_up(sizeof(CacheSmem), 16));
     s.bytes = int(align_up(o, 1024)) + 1024;
@@ -849,6 +848,7 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
     CacheSmem& M = *reinterpret_cast<CacheSmem*>(smem + S.misc);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + S.bars);
     uint64_t* empty = full + P.n_stages;
+    uint64_t* done = empty + P.n_stages;   // the 8 pieces of the stage's job are in its partial sums
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x;
 
@@ -856,7 +856,7 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
         for (int s = 0; s < P.n_stages; ++s) {
             mbar_init(full + s, 1);
             mbar_init(empty + s, kDecWarps);
-            M.ecnt[s] = 0;
+            mbar_init(done + s, kDecWarps);
         }
         fence_mbar_init();
         for (int q = 0; q < kCapMax; ++q) {
@@ -1028,23 +1028,25 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
                 pb[kDecWarps * 32 + pair * 2] = corr0;
                 pb[kDecWarps * 32 + pair * 2 + 1] = corr1;
             }
-            __threadfence_block();
-            int last = 0;
-            if (lane == 0) last = atomicAdd(&M.ecnt[s], 1) == kDecWarps - 1;
-            last = __shfl_sync(0xffffffffu, last, 0);
-            // the stage (and its partial sums) may be refilled once every warp
-            // has read what it needs; the stage was only read, so the barrier
-            // alone orders those reads before the next copy
-            if (last) {
-                __threadfence_block();
-                if (lane == 0) M.ecnt[s] = 0;
+            // warp (job index mod 8) finishes the job: the epilogues (with their
+            // global-memory round trips) rotate over the warps instead of
+            // landing on whichever warp happens to be last
+            __syncwarp();
+            if (lane == 0) mbar_arrive(done + s);
+            if (((ibase + i) & (kDecWarps - 1)) == warp) {
+                if (ok && !mbar_wait(done + s, uint32_t(ph))) {
+                    ok = false;
+                    if (lane == 0) set_status(A.ws.status, GALE_ERR_TIMEOUT);
+                }
                 float ya[kMaxRT], yb[kMaxRT];
                 epi_gather(sh, W13, pb, lane, ya, yb);
+                // the stage (and its partial sums) may be refilled once every
+                // warp has read what it needs; the stage was only read, so the
+                // barrier alone orders those reads before the next copy
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty + s);
                 epi_finish(A, R, sh, W13, Jb, lane, ya, yb);
             } else {
-                __syncwarp();
                 if (lane == 0) mbar_arrive(empty + s);
             }
             if (++st == P.n_stages) {
