@@ -34,6 +34,7 @@ METRIC = "MoE expert-layer tokens/s and packed-expert HBM GB/s (% of B200 roofli
 UNIT = "tokens/s"
 D_MODEL, D_FF, N_EXPERTS, TOP_K = 4096, 2048, 256, 6
 PREFILL_B = 4096
+CHAIN_LAYERS = 43
 # kernels of this library launched per decode step (the cooperative layer kernel)
 DECODE_LAUNCHES = 1
 # dram read + write bytes of one decode launch at this workload, from the ncu
@@ -118,20 +119,24 @@ class Clocks:
 # the layer on the device
 # ----------------------------------------------------------------------------
 
-def build_layer(torch, G, layer_id: int = 0):
-    """Pack 256 seeded experts into one resident device buffer (gale_pack)."""
+def build_layer(torch, G, layer_id: int = 0, dst=None):
+    """Pack 256 seeded experts into one resident device buffer: the seeded
+    canonical matrices are drawn on the device (torch port of the generator)
+    and packed by gale_pack."""
     stride = G.gale_expert_bytes(D_MODEL, D_FF)
-    buf = torch.empty(N_EXPERTS * stride, dtype=torch.uint8, device="cuda")
+    buf = dst if dst is not None else torch.empty(N_EXPERTS * stride, dtype=torch.uint8, device="cuda")
     l1 = G.gale_pack_layout(D_FF, D_MODEL)["total"]
     offs = [0, l1, 2 * l1]
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    for e in range(N_EXPERTS):
-        for m, c in enumerate(gs.expert_canonical(D_MODEL, D_FF, layer=layer_id, expert=e)):
-            dev = {k: torch.from_numpy(np.ascontiguousarray(v)).cuda()
-                   for k, v in (("signs", c["signs"]), ("s_blk", c["s_blk"].view(np.uint16)),
-                                ("s_row", c["s_row"].view(np.uint16)), ("idx", c["idx"]), ("q", c["q"]))}
-            G.gale_pack(dev["signs"], dev["s_blk"], dev["s_row"], dev["idx"], dev["q"], c["rows"], c["cols"],
-                        buf[e * stride + offs[m]:], status)
+    shapes = [(D_FF, D_MODEL, gs.W1), (D_FF, D_MODEL, gs.W3), (D_MODEL, D_FF, gs.W2)]
+    chunk = 16
+    for m, (rows, cols, mat) in enumerate(shapes):
+        for e0 in range(0, N_EXPERTS, chunk):
+            es = list(range(e0, min(N_EXPERTS, e0 + chunk)))
+            c = gs.matrices_canonical_torch(rows, cols, layer_id, es, mat, device="cuda")
+            for i, e in enumerate(es):
+                G.gale_pack(c["signs"][i], c["s_blk"][i], c["s_row"][i], c["idx"][i], c["q"][i], rows, cols,
+                            buf[e * stride + offs[m]:], status)
     torch.cuda.synchronize()
     if int(status.item()) != 0:
         raise RuntimeError("gale_pack reported invalid outliers")
@@ -235,6 +240,73 @@ def run_gpu(args):
         d2h = B * D_MODEL * 4
         return total, h2d, d2h
 
+    def measure_chain(steps, warmup, n_layers=CHAIN_LAYERS):
+        """Decode batch 1 through n_layers layers of 256 resident experts each:
+        x_{l+1} = bf16(RMSNorm(x_l + MoE_l(x_l))), fresh seeded routing per
+        layer and step.  46 GB of packs are far larger than L2, so every layer
+        reads its experts from HBM.  Returns (seconds, packed bytes read, used graph)."""
+        lb = N_EXPERTS * expert_bytes
+        big = torch.empty(n_layers * lb, dtype=torch.uint8, device="cuda")
+        layers = []
+        for l in range(n_layers):
+            build_layer(torch, G, layer_id=l, dst=big[l * lb:(l + 1) * lb])
+            layers.append(G.make_layer(big[l * lb:], expert_bytes, N_EXPERTS, D_MODEL, D_FF))
+        n = steps + warmup
+        ids = torch.empty(n, n_layers, 1, TOP_K, dtype=torch.int32, device="cuda")
+        gts = torch.empty(n, n_layers, 1, TOP_K, dtype=torch.float32, device="cuda")
+        distinct = 0
+        for s in range(n):
+            for l in range(n_layers):
+                i_, g_ = gs.route_topk(gs.router_logits(1, N_EXPERTS, tag=90_000 + 1000 * s + l), TOP_K)
+                ids[s, l] = torch.from_numpy(i_)
+                gts[s, l] = torch.from_numpy(g_)
+                if s >= warmup:
+                    distinct += len(np.unique(i_))
+        x0 = torch.from_numpy(gs.hidden_bf16(1, D_MODEL, tag=91_000)[0]).view(torch.bfloat16).cuda()
+        ws = torch.empty(G.gale_moe_workspace_size(layers[0], 1, TOP_K), dtype=torch.uint8, device="cuda")
+        xb = [torch.empty(1, D_MODEL, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+        cur_ids = torch.empty(n_layers, 1, TOP_K, dtype=torch.int32, device="cuda")
+        cur_g = torch.empty(n_layers, 1, TOP_K, dtype=torch.float32, device="cuda")
+
+        def token():
+            x = x0
+            for l in range(n_layers):
+                G.gale_moe_forward(layers[l], x, cur_ids[l], cur_g[l], xb[l % 2], ws,
+                                   flags=G.GALE_FLAG_RESIDUAL_RMSNORM, eps=1e-6)
+                x = xb[l % 2]
+
+        for s in range(warmup):
+            cur_ids.copy_(ids[s])
+            cur_g.copy_(gts[s])
+            token()
+        torch.cuda.synchronize()
+        if int(ws[:4].view(torch.int32).item()) != 0:
+            raise RuntimeError("device status after chain warm-up")
+        graph = None
+        try:   # the 43 launches of a token as one CUDA graph
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                token()
+            graph = g
+        except Exception:
+            graph = None
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for s in range(steps):
+            cur_ids.copy_(ids[warmup + s])
+            cur_g.copy_(gts[warmup + s])
+            ev[s][0].record(stream)
+            if graph is not None:
+                graph.replay()
+            else:
+                token()
+            ev[s][1].record(stream)
+        torch.cuda.synchronize()
+        t = sum(a.elapsed_time(b) * 1e-3 for a, b in ev)
+        del big
+        torch.cuda.empty_cache()
+        return t, distinct * expert_bytes, graph is not None
+
     clocks = Clocks(local)
     clocks.start()
     t1, bytes1, times1 = measure(1, args.steps, args.warmup, 10_000)
@@ -244,12 +316,14 @@ def run_gpu(args):
     # prefill: 4096 tokens, skewed routing (tensor-core tile path)
     pf_steps = max(3, min(args.steps // 5, 10))
     tp, _, _ = measure(PREFILL_B, pf_steps, 3, 40_000, bias_sigma=0.5, n_x=2)
+    ch_steps = max(3, min(args.steps // 5, 10))
+    tc, bytes_c, ch_graph = measure_chain(ch_steps, 3) if not args.no_chain else (float("nan"), 0, False)
 
     # max over ranks of the device time
-    tt = torch.tensor([t1, t8, te, tp], dtype=torch.float64, device="cuda")
+    tt = torch.tensor([t1, t8, te, tp, tc], dtype=torch.float64, device="cuda")
     if world > 1:
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    t1, t8, te, tp = [float(v) for v in tt.tolist()]
+    t1, t8, te, tp, tc = [float(v) for v in tt.tolist()]
     tokens = 1 * args.steps * world
     value = tokens / t1
     gbs = bytes1 * world / t1 / 1e9
@@ -272,6 +346,11 @@ def run_gpu(args):
                      "algorithmic_bytes_per_launch": bytes1 / args.steps},
         "b8": {"tokens_per_s": 8 * max(args.steps // 2, 3) * world / t8,
                "hbm_gbs": bytes8 * world / t8 / 1e9, "frac": bytes8 * world / t8 / 1e9 / peak},
+        "chain43": {"workload": f"decode batch 1 through {CHAIN_LAYERS} layers x 256 resident experts "
+                                f"(46 GB), residual + RMSNorm between layers, bf16 hidden state",
+                    "tokens_per_s": ch_steps * world / tc, "ms_per_token": 1e3 * tc / ch_steps,
+                    "hbm_gbs": bytes_c * world / tc / 1e9, "frac": bytes_c * world / tc / 1e9 / peak,
+                    "cuda_graph": ch_graph, "steps": ch_steps},
         "prefill": {"workload": "4096 tokens, top-6 with per-expert bias N(0, 0.5) (skewed), same 256 experts",
                     "tokens_per_s": PREFILL_B * pf_steps * world / tp, "ms_per_step": 1e3 * tp / pf_steps,
                     "tflops": pf_flops * pf_steps / tp / 1e12, "peak_tflops": tpeak,
@@ -393,6 +472,7 @@ def main():
     ap.add_argument("--impl", default="gale", choices=["gale", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-chain", action="store_true", help="skip the 43-layer chain measurement")
     ap.add_argument("--only", choices=["decode", "prefill"], default=None,
                     help="profiling driver: warm-up, an L2 flush, then --steps layer calls of one path")
     ap.add_argument("--batch", type=int, default=1, help="tokens per step with --only")

@@ -204,3 +204,91 @@ def route_topk(logits: np.ndarray, k: int):
     e = np.exp(sel - sel.max(axis=1, keepdims=True))
     gates = (e / e.sum(axis=1, keepdims=True)).astype(np.float32)
     return order.astype(np.int32), gates
+
+
+# ----------------------------------------------------------------------------
+# the same matrix generator on a torch device (for large resident workloads)
+# ----------------------------------------------------------------------------
+
+def _t_mix64(z):
+    """SplitMix64 output function on an int64 torch tensor holding uint64 bit
+    patterns (wrapping multiply; logical right shifts by masking)."""
+    import torch
+    m30 = (1 << 34) - 1
+    m27 = (1 << 37) - 1
+    m31 = (1 << 33) - 1
+    c1 = 0xBF58476D1CE4E5B9 - (1 << 64)
+    c2 = 0x94D049BB133111EB - (1 << 64)
+    z = (z ^ ((z >> 30) & m30)) * c1
+    z = (z ^ ((z >> 27) & m27)) * c2
+    return z ^ ((z >> 31) & m31)
+
+
+def _t_u64(keys, idx):
+    """Elements idx (int64 tensor, broadcast against keys) of the streams keys."""
+    g = GOLDEN - (1 << 64)
+    return _t_mix64(keys + (idx + 1) * g)
+
+
+def _t_uniform(keys, idx):
+    import torch
+    u = _t_u64(keys, idx)
+    hi = (u >> 11) & ((1 << 53) - 1)
+    return (hi.to(torch.float64) + 0.5) * (2.0 ** -53)
+
+
+def _t_normal(keys, n):
+    import torch
+    i = torch.arange(n, dtype=torch.int64, device=keys.device)
+    u1 = _t_uniform(keys, 2 * i)
+    u2 = _t_uniform(keys, 2 * i + 1)
+    return torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(2.0 * torch.pi * u2)
+
+
+def _t_keys(fields_list, device):
+    import torch
+    ks = [stream_key(*f) for f in fields_list]
+    return torch.tensor([k - (1 << 64) if k >= (1 << 63) else k for k in ks], dtype=torch.int64, device=device)
+
+
+def matrices_canonical_torch(rows: int, cols: int, layer: int, experts, matrix: int, device="cuda",
+                             frac: float = 0.01) -> dict:
+    """``matrix_canonical`` for several experts at once on a torch device.
+
+    Integer draws (signs, outlier columns, outlier values) are bit-identical to
+    the numpy version; the scales go through the device's fp64 log, cos and
+    exp, which may round a rare value to a neighbouring fp16.  Tensors carry a
+    leading expert dimension.
+    """
+    import torch
+    E = len(experts)
+    base = [(KIND_MATRIX, layer, e, matrix) for e in experts]
+    col = lambda t: t.view(E, 1)
+    # signs: bit (c % 64) of draw r*(cols/64) + c/64
+    kw = col(_t_keys([b + (SEC_SIGNS,) for b in base], device))
+    nw = rows * (cols // 64)
+    words = _t_u64(kw, torch.arange(nw, dtype=torch.int64, device=device).view(1, nw))
+    bits = torch.arange(64, dtype=torch.int64, device=device)
+    signs = ((words.view(E, nw, 1) >> bits) & 1).to(torch.uint8).view(E, rows, cols)
+    nb = cols // 128
+    z = _t_normal(col(_t_keys([b + (SEC_SBLK,) for b in base], device)), rows * nb)
+    s_blk = torch.exp(BLK_MU + BLK_SIGMA * z).to(torch.float16).view(E, rows, nb)
+    z = _t_normal(col(_t_keys([b + (SEC_SROW,) for b in base], device)), rows)
+    s_row = torch.exp(ROW_MU + ROW_SIGMA * z).to(torch.float16).view(E, rows)
+    k = outlier_count(cols, frac)
+    ki = col(_t_keys([b + (SEC_IDX,) for b in base], device)).view(E, 1, 1)
+    r_ids = torch.arange(rows, dtype=torch.int64, device=device).view(1, rows, 1)
+    sel = torch.zeros((E, rows, k), dtype=torch.int64, device=device)
+    for step in range(k):
+        j = cols - k + step
+        u = _t_u64(ki, r_ids * k + step).view(E, rows)
+        t = (((u >> 32) & 0xFFFFFFFF) * (j + 1)) >> 32
+        if step:
+            dup = (sel[:, :, :step] == t.unsqueeze(-1)).any(dim=-1)
+            t = torch.where(dup, torch.full_like(t, j), t)
+        sel[:, :, step] = t
+    idx = torch.sort(sel, dim=-1).values.to(torch.int32).to(torch.int16)
+    kq = col(_t_keys([b + (SEC_Q,) for b in base], device))
+    n = torch.arange(rows * k, dtype=torch.int64, device=device).view(1, rows * k)
+    q = (((_t_u64(kq, n) >> 60) & 0xF) - 8).to(torch.int8).view(E, rows, k)
+    return {"rows": rows, "cols": cols, "signs": signs, "s_blk": s_blk, "s_row": s_row, "idx": idx, "q": q}
