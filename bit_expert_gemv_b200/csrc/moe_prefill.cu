@@ -34,7 +34,6 @@ constexpr int kTcK = 64;            // K per stage: one 128-byte row of fp16 tok
 constexpr int kTcStages = 4;
 constexpr int kTcExpWarps = 8;      // expander / epilogue warps: 2 per TMEM lane quarter
 constexpr int kTcThreads = (2 + kTcExpWarps) * 32;
-constexpr int kPrefetch = 4;        // K-steps of sign words loaded ahead
 constexpr int kMaxOutliers = 82;    // per row: round(0.01 * 8192)
 constexpr uint32_t kSentinel = 0xFFFF0000u;
 
@@ -83,7 +82,7 @@ __host__ __device__ inline TcSmem tc_smem(int nmat, int chunk, int k) {
         s.srow[mt] = o;
         o += kTcM * 2;
         s.ent[mt] = o;
-        o += kTcM * (k + 2) * 4;
+        o += kTcM * (k + 4) * 4;
     }
     s.bars = (o + 7) & ~7;
     s.misc = s.bars + 8 * (3 * kTcStages + 2);
@@ -289,16 +288,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
         bool ok = mbar_wait(side_full, 0);
         // this thread's outliers in column order, as (column << 16 | fp16 value)
         int cur[NMAT];
-        uint32_t ent[NMAT];
+        uint32_t ent[NMAT], nxt[NMAT];
 #pragma unroll
         for (int mt = 0; mt < NMAT; ++mt) {
             const uint16_t* sidx = reinterpret_cast<const uint16_t*>(smem + S.idx[mt]) + t * kout;
             const uint8_t* sqv = smem + S.q[mt];
             const float srow = __half2float(reinterpret_cast<const __half*>(smem + S.srow[mt])[t]);
-            uint32_t* list = reinterpret_cast<uint32_t*>(smem + S.ent[mt]) + t * (kout + 2);
+            uint32_t* list = reinterpret_cast<uint32_t*>(smem + S.ent[mt]) + t * (kout + 4);
             int n0 = 0;
             for (int j = 0; j < kout; ++j) n0 += ((sidx[j] >> 5) & 1) == 0;
-            const int start = h ? n0 + 1 : 0;
+            const int start = h ? n0 + 2 : 0;   // each half ends in two sentinels
             int o = start;
             for (int j = 0; j < kout; ++j) {
                 const int c = sidx[j];
@@ -310,74 +309,91 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
                 list[o++] = (uint32_t(c) << 16) | __half_as_ushort(__float2half_rn(float(qv) * srow));
             }
             list[o] = kSentinel;
+            list[o + 1] = kSentinel;
             cur[mt] = start;
             ent[mt] = list[start];
+            nxt[mt] = list[start + 1];
         }
-        // sign words / block scales of K-steps ks .. ks + kPrefetch - 1
-        MatView mv[NMAT];
+        // Sign words and block scales arrive a group of kTcStages K-steps ahead:
+        // two 16-byte loads hold the group's words of both halves, one 4-byte
+        // load its two block scales.
+        const uint4* wsrc[NMAT];
+        const uint32_t* ssrc[NMAT];
 #pragma unroll
-        for (int mt = 0; mt < NMAT; ++mt) mv[mt] = make_view(rec + (mt ? A.off_b : A.off_a), A.rows, A.cols);
-        uint32_t wq[NMAT][kPrefetch], sq[NMAT][kPrefetch];
-        auto fetch = [&](int mt, int ks, uint32_t& w, uint32_t& sc) {
-            w = 0u;
-            sc = 0u;
-            if (ks < nk) {
-                w = __ldg(mv[mt].signs + int64_t(row) * (A.cols / 32) + 2 * ks + h);
-                sc = __ldg(reinterpret_cast<const uint16_t*>(mv[mt].s_blk) + int64_t(row) * nb + (ks >> 1));
-            }
-        };
+        for (int mt = 0; mt < NMAT; ++mt) {
+            const MatView mv = make_view(rec + (mt ? A.off_b : A.off_a), A.rows, A.cols);
+            wsrc[mt] = reinterpret_cast<const uint4*>(mv.signs + int64_t(row) * (A.cols / 32));
+            ssrc[mt] = reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint16_t*>(mv.s_blk) + int64_t(row) * nb);
+        }
+        uint4 wa[NMAT], wb[NMAT];
+        uint32_t sp[NMAT];
 #pragma unroll
-        for (int mt = 0; mt < NMAT; ++mt)
-#pragma unroll
-            for (int p = 0; p < kPrefetch; ++p) fetch(mt, p, wq[mt][p], sq[mt][p]);
-        for (int ks = 0; ks < nk; ++ks) {
-            const int s = ks % kTcStages;
-            if (ok && ks >= kTcStages && !mbar_wait(mma_done + s, ((ks / kTcStages) - 1) & 1)) ok = false;
-            tc_fence_after();
-            const int slot = ks % kPrefetch;
-            const int lo = ks * kTcK + 32 * h, hi = lo + 32;
+        for (int mt = 0; mt < NMAT; ++mt) {
+            wa[mt] = __ldg(wsrc[mt]);
+            wb[mt] = __ldg(wsrc[mt] + 1);
+            sp[mt] = __ldg(ssrc[mt]);
+        }
+        const int ng = nk / kTcStages;
+        for (int g = 0; g < ng; ++g) {
+            uint32_t wg[NMAT][kTcStages], sg[NMAT][2];
 #pragma unroll
             for (int mt = 0; mt < NMAT; ++mt) {
-                uint32_t w = 0u, sc = 0u;
-#pragma unroll
-                for (int p = 0; p < kPrefetch; ++p)
-                    if (p == slot) {
-                        w = wq[mt][p];
-                        sc = sq[mt][p];
-                        fetch(mt, ks + kPrefetch, wq[mt][p], sq[mt][p]);
-                    }
-                uint32_t v[16];
-                expand_signs(w, sc, v);
-                // outliers of this range replace their weights
-                int prev_p = -1;
-                uint32_t prev_a = 0u;
-                for (;;) {
-                    const int ecol = int(ent[mt] >> 16);
-                    const bool mine = ecol < hi;
-                    if (!__any_sync(0xffffffffu, mine)) break;
-                    int P = -1;
-                    uint32_t a = 0u;
-                    if (mine) {
-                        const int u = ecol - lo;
-                        P = u >> 1;
-                        const uint32_t val = ent[mt] & 0xFFFFu;
-                        uint32_t other = sc ^ (((w >> (u ^ 1)) & 1u) << 15);
-                        if (P == prev_p) other = (u & 1) ? (prev_a & 0xFFFFu) : (prev_a >> 16);
-                        a = (u & 1) ? (other | (val << 16)) : (val | (other << 16));
-                        prev_p = P;
-                        prev_a = a;
-                        ent[mt] = reinterpret_cast<const uint32_t*>(smem + S.ent[mt])[t * (kout + 2) + ++cur[mt]];
-                    }
-#pragma unroll
-                    for (int p = 0; p < 16; ++p) v[p] = (P == p) ? a : v[p];
+                wg[mt][0] = h ? wa[mt].y : wa[mt].x;
+                wg[mt][1] = h ? wa[mt].w : wa[mt].z;
+                wg[mt][2] = h ? wb[mt].y : wb[mt].x;
+                wg[mt][3] = h ? wb[mt].w : wb[mt].z;
+                sg[mt][0] = sp[mt] & 0xFFFFu;
+                sg[mt][1] = sp[mt] >> 16;
+                if (g + 1 < ng) {
+                    wa[mt] = __ldg(wsrc[mt] + 2 * (g + 1));
+                    wb[mt] = __ldg(wsrc[mt] + 2 * (g + 1) + 1);
+                    sp[mt] = __ldg(ssrc[mt] + g + 1);
                 }
-                tmem_st16(tmem + (uint32_t(32 * quarter) << 16) +
-                              uint32_t(Cfg::acc_cols + s * Cfg::a_cols + mt * 32 + 16 * h),
-                          v);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(a_full + s);
+#pragma unroll
+            for (int s = 0; s < kTcStages; ++s) {
+                if (ok && g > 0 && !mbar_wait(mma_done + s, (g - 1) & 1)) ok = false;
+                tc_fence_after();
+                const int lo = (g * kTcStages + s) * kTcK + 32 * h, hi = lo + 32;
+#pragma unroll
+                for (int mt = 0; mt < NMAT; ++mt) {
+                    const uint32_t w = wg[mt][s], sc = sg[mt][s >> 1];
+                    uint32_t v[16];
+                    expand_signs(w, sc, v);
+                    // outliers of this range replace their weights; the entry
+                    // after the current one is already loaded
+                    const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + S.ent[mt]) + t * (kout + 4);
+                    int prev_p = -1;
+                    uint32_t prev_a = 0u;
+                    for (;;) {
+                        const int ecol = int(ent[mt] >> 16);
+                        const bool mine = ecol < hi;
+                        if (!__any_sync(0xffffffffu, mine)) break;
+                        int P = -1;
+                        uint32_t a = 0u;
+                        if (mine) {
+                            const int u = ecol - lo;
+                            P = u >> 1;
+                            const uint32_t val = ent[mt] & 0xFFFFu;
+                            uint32_t other = sc ^ (((w >> (u ^ 1)) & 1u) << 15);
+                            if (P == prev_p) other = (u & 1) ? (prev_a & 0xFFFFu) : (prev_a >> 16);
+                            a = (u & 1) ? (other | (val << 16)) : (val | (other << 16));
+                            prev_p = P;
+                            prev_a = a;
+                            ent[mt] = nxt[mt];
+                            nxt[mt] = list[++cur[mt] + 1];
+                        }
+#pragma unroll
+                        for (int p = 0; p < 16; ++p) v[p] = (P == p) ? a : v[p];
+                    }
+                    tmem_st16(tmem + (uint32_t(32 * quarter) << 16) +
+                                  uint32_t(Cfg::acc_cols + s * Cfg::a_cols + mt * 32 + 16 * h),
+                              v);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(a_full + s);
+            }
         }
         // ---------------- epilogue: TMEM -> registers -> global
         const bool acc_ok = mbar_wait(acc_full, 0);
@@ -457,6 +473,8 @@ PrefillWs carve_prefill_ws(void* ws, const gale_layer& L, int B, int K) {
 
 bool prefill_supported(const gale_layer& L, int B, int K) {
     if (int64_t(B) * K > (int64_t(1) << 24) || L.n_experts > 1024) return false;
+    // the expanders walk K in groups of one pass over the stage ring
+    if (L.d_model % (kTcK * kTcStages) != 0 || L.d_ff % (kTcK * kTcStages) != 0) return false;
     // a tile's outlier lists stay in shared memory
     const int k1 = outliers_per_row(L.d_model), k2 = outliers_per_row(L.d_ff);
     return k1 <= kMaxOutliers && k2 <= kMaxOutliers && tc_smem(2, TcCfg<2>::chunk, k1).bytes <= 227 * 1024 &&
