@@ -47,7 +47,9 @@ __device__ __forceinline__ float fixed_scale(float m) {
 
 // The three int8 digits of round(u), |u| <= 2^20, each in the low byte.
 __device__ __forceinline__ void fixed_digits(float u, uint32_t& d1, uint32_t& d2, uint32_t& d3) {
-    const int X = __float2int_rn(u);
+    // round(u) through the 1.5 * 2^23 addition: exact for |u| < 2^22 and
+    // ties to even, the same as a round-to-nearest conversion
+    const int X = __float_as_int(__fadd_rn(u, 12582912.0f)) - 0x4B400000;
     const int p1 = (X + 8192) >> 14;
     const int r = X - (p1 << 14);
     const int p2 = (r + 64) >> 7;

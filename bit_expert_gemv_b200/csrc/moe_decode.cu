@@ -30,7 +30,8 @@ namespace {
 
 constexpr int kDecWarps = 8;                   // consumer warps
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecBlock = kDecThreads + 32;    // + the producer warp
+constexpr int kDecBlock = kDecThreads + 64;    // + the producer warp and the epilogue warp
+constexpr int kPhaseBar = kDecThreads + 32;     // consumers and the epilogue warp
 constexpr int kCapMax = 8;                     // rotated vectors cached per CTA
 constexpr int kMaxStages = 16;
 
@@ -418,40 +419,61 @@ __device__ __forceinline__ void ensure_cached(const DecArgs& A, const Shape& sh,
                                           bool W13, int key0, int key1, int& c0, int& c1) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int C = sh.cols, nblk = C / 1024;
-    if (tid == 0) {
-        const int keys[2] = {key0, key1};
-        int found[2] = {-1, -1};
-        M.n_plan = 0;
-#pragma unroll 1
-        for (int e = 0; e < 2; ++e) {
-            if (keys[e] < 0) continue;
-#pragma unroll 1
-            for (int q = 0; q < cap; ++q)
-                if (M.key[q] == keys[e]) found[e] = q;
-        }
-#pragma unroll 1
-        for (int e = 0; e < 2; ++e) {
-            if (keys[e] < 0 || found[e] >= 0) continue;
-            int victim = -1, best = 0x7fffffff;
-#pragma unroll 1
-            for (int q = 0; q < cap; ++q) {
-                if (q == found[0] || q == found[1]) continue;
-                if (M.stamp[q] < best) {
-                    best = M.stamp[q];
-                    victim = q;
+    if (warp == 0) {
+        // lane q < cap looks after cache entry q; hits by ballot, victims by a
+        // warp-wide argmin of (stamp, entry)
+        const int kq = lane < cap ? M.key[lane] : -2;
+        int stq = lane < cap ? M.stamp[lane] : 0x7fffffff;
+        const unsigned m0 = __ballot_sync(0xffffffffu, key0 >= 0 && kq == key0);
+        const unsigned m1 = __ballot_sync(0xffffffffu, key1 >= 0 && kq == key1);
+        int f0 = m0 ? __ffs(m0) - 1 : -1, f1 = m1 ? __ffs(m1) - 1 : -1;
+        int nk = kq, n_plan = 0;
+        auto victim = [&](int other) {
+            int best = (lane < cap && lane != other) ? stq : 0x7fffffff, bl = lane;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const int ob = __shfl_xor_sync(0xffffffffu, best, o), ol = __shfl_xor_sync(0xffffffffu, bl, o);
+                if (ob < best || (ob == best && ol < bl)) {
+                    best = ob;
+                    bl = ol;
                 }
             }
-            found[e] = victim;
-            M.key[victim] = keys[e];
-            M.plan_slot[M.n_plan] = victim;
-            M.plan_key[M.n_plan] = keys[e];
-            ++M.n_plan;
+            return bl;
+        };
+        if (key0 >= 0 && f0 < 0) {
+            f0 = victim(f1);
+            if (lane == f0) nk = key0;
+            if (lane == 0) {
+                M.plan_slot[n_plan] = f0;
+                M.plan_key[n_plan] = key0;
+            }
+            ++n_plan;
         }
-#pragma unroll 1
-        for (int e = 0; e < 2; ++e)
-            if (found[e] >= 0) M.stamp[found[e]] = ++M.clock;
-        M.cres[0] = found[0];
-        M.cres[1] = found[1];
+        if (key1 >= 0 && f1 < 0) {
+            f1 = victim(f0);
+            if (lane == f1) nk = key1;
+            if (lane == 0) {
+                M.plan_slot[n_plan] = f1;
+                M.plan_key[n_plan] = key1;
+            }
+            ++n_plan;
+        }
+        int clk = M.clock;
+        if (f0 >= 0 && lane == f0) stq = clk + 1;
+        if (f0 >= 0) ++clk;
+        if (f1 >= 0 && lane == f1) stq = clk + 1;
+        if (f1 >= 0) ++clk;
+        __syncwarp();
+        if (lane < cap) {
+            M.key[lane] = nk;
+            M.stamp[lane] = stq;
+        }
+        if (lane == 0) {
+            M.clock = clk;
+            M.n_plan = n_plan;
+            M.cres[0] = f0;
+            M.cres[1] = f1;
+        }
     }
     named_bar_sync(1, kDecThreads);
     c0 = M.cres[0];
@@ -808,9 +830,29 @@ __device__ __forceinline__ void epi_finish(const DecArgs& A, const RouteTables& 
         for (int q = lane; q < comb_blocks; q += 32) tot += __ldcg(A.ws.ssq + t * comb_blocks + q);
         tot = warp_sum(tot);
         const float inv = rsqrtf(tot / float(d) + A.eps);
-#pragma unroll 4
-        for (int c = lane; c < d; c += 32)
-            store_from_f32(A.out, GALE_BF16, int64_t(t) * d + c, __ldcg(A.ws.v + int64_t(t) * d + c) * inv);
+        // sixteen 16-byte loads in flight per lane, then the stores
+        const float4* vrow = reinterpret_cast<const float4*>(A.ws.v + int64_t(t) * d);
+        const int n4 = d / 4;
+#pragma unroll 1
+        for (int c0 = 0; c0 < n4; c0 += 32 * 16) {
+            float4 vv[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int c = c0 + 32 * j + lane;
+                vv[j] = c < n4 ? __ldcg(vrow + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int c = c0 + 32 * j + lane;
+                if (c < n4) {
+                    const int64_t o = int64_t(t) * d + 4 * c;
+                    store_from_f32(A.out, GALE_BF16, o, vv[j].x * inv);
+                    store_from_f32(A.out, GALE_BF16, o + 1, vv[j].y * inv);
+                    store_from_f32(A.out, GALE_BF16, o + 2, vv[j].z * inv);
+                    store_from_f32(A.out, GALE_BF16, o + 3, vv[j].w * inv);
+                }
+            }
+        }
     }
 }
 
@@ -855,7 +897,7 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
     if (threadIdx.x == 0) {
         for (int s = 0; s < P.n_stages; ++s) {
             mbar_init(full + s, 1);
-            mbar_init(empty + s, kDecWarps);
+            mbar_init(empty + s, 1);           // the epilogue warp, once it has gathered the job
             mbar_init(done + s, kDecWarps);
         }
         fence_mbar_init();
@@ -864,6 +906,12 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
             M.stamp[q] = 0;
         }
         M.clock = 0;
+    }
+    {
+        // the first tokens' rows of x head for L2 while the routing is built
+        const int64_t xb = int64_t(A.B < 8 ? A.B : 8) * A.d_model * 2;
+        for (int64_t o = int64_t(threadIdx.x) * 128; o < xb; o += int64_t(blockDim.x) * 128)
+            prefetch_l2(reinterpret_cast<const char*>(A.x) + o);
     }
     build_route(A, R, *reinterpret_cast<RouteScratch*>(smem + S.ring));   // contains __syncthreads
     // contiguous job ranges of this CTA in both phases
@@ -930,6 +978,48 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
             if (++s == P.n_stages) {
                 s = 0;
                 ph ^= 1;
+            }
+        }
+        return;
+    }
+
+    if (warp == kDecWarps + 1) {
+        // ---------------- epilogue warp: once the 8 pieces of a job are in its
+        // stage's partial sums, gather them, release the stage and finish the
+        // job (h rows in phase 1; o rows and the combine in phase 2), so that
+        // the consumers go straight on to the next job
+        bool eok = true;
+        int s = 0, ph = 0;
+#pragma unroll 1
+        for (int phase = 0; phase < 2; ++phase) {
+            const bool W13 = phase == 0;
+            const Shape& sh = W13 ? P.s13 : P.s2;
+            const int n_my = W13 ? n13 : n2, ibase = W13 ? 0 : n13;
+#pragma unroll 1
+            for (int i = 0; i < n_my; ++i) {
+                const Job Jb = unpack_job(jobs[ibase + i]);
+                if (eok && !mbar_wait(done + s, uint32_t(ph))) {
+                    eok = false;
+                    if (lane == 0) set_status(A.ws.status, GALE_ERR_TIMEOUT);
+                }
+                const float* pb = reinterpret_cast<const float*>(smem + S.part) + s * kPartFloats;
+                float ya[kMaxRT], yb[kMaxRT];
+                epi_gather(sh, W13, pb, lane, ya, yb);
+                // the consumers only read the stage, so the barrier alone orders
+                // their reads (and this gather) before the next copy into it
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty + s);
+                if (eok) epi_finish(A, R, sh, W13, Jb, lane, ya, yb);
+                if (++s == P.n_stages) {
+                    s = 0;
+                    ph ^= 1;
+                }
+            }
+            if (phase == 0) {
+                __threadfence();
+                named_bar_sync(2, kPhaseBar);   // this CTA's h rows are written
+                named_bar_sync(2, kPhaseBar);   // the grid barrier has been passed
+                if (!M.gate_ok) eok = false;
             }
         }
         return;
@@ -1028,27 +1118,8 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
                 pb[kDecWarps * 32 + pair * 2] = corr0;
                 pb[kDecWarps * 32 + pair * 2 + 1] = corr1;
             }
-            // warp (job index mod 8) finishes the job: the epilogues (with their
-            // global-memory round trips) rotate over the warps instead of
-            // landing on whichever warp happens to be last
             __syncwarp();
             if (lane == 0) mbar_arrive(done + s);
-            if (((ibase + i) & (kDecWarps - 1)) == warp) {
-                if (ok && !mbar_wait(done + s, uint32_t(ph))) {
-                    ok = false;
-                    if (lane == 0) set_status(A.ws.status, GALE_ERR_TIMEOUT);
-                }
-                float ya[kMaxRT], yb[kMaxRT];
-                epi_gather(sh, W13, pb, lane, ya, yb);
-                // the stage (and its partial sums) may be refilled once every
-                // warp has read what it needs; the stage was only read, so the
-                // barrier alone orders those reads before the next copy
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty + s);
-                epi_finish(A, R, sh, W13, Jb, lane, ya, yb);
-            } else {
-                if (lane == 0) mbar_arrive(empty + s);
-            }
             if (++st == P.n_stages) {
                 st = 0;
                 ph ^= 1;
@@ -1058,7 +1129,7 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
         if (phase == 0) {
             // ---------------- grid barrier: h of every expert is in global memory
             __threadfence();
-            named_bar_sync(1, kDecThreads);
+            named_bar_sync(2, kPhaseBar);   // with the epilogue warp: this CTA's phase-1 work is done
             if (tid == 0) {
                 M.gate_ok = grid_barrier(A.ws.gbar, A.ws.gbar + 1, G);
                 if (!M.gate_ok) set_status(A.ws.status, GALE_ERR_TIMEOUT);
@@ -1067,7 +1138,7 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
                     M.stamp[q] = 0;
                 }
             }
-            named_bar_sync(1, kDecThreads);
+            named_bar_sync(2, kPhaseBar);
             if (!M.gate_ok) ok = false;
         }
     }

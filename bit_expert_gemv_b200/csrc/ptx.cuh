@@ -93,6 +93,8 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
 }
 
 // Named barrier over `count` threads (a multiple of 32).
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
