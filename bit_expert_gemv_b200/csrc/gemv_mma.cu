@@ -78,7 +78,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_mma_kernel(
     float* xr = reinterpret_cast<float*>(smem + S.xr);
     float* red = reinterpret_cast<float*>(smem + S.red);
     TokRef tok[2];
-    for (int t = 0; t < 2; ++t) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {   // unrolled: tok stays in registers
         tok[t] = TokRef{nullptr, nullptr, nullptr, 1.f};
         if (t >= ntok) continue;
         for (int c = threadIdx.x; c < C; c += blockDim.x) xr[c] = x[int64_t(t) * C + c];
@@ -107,7 +108,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_mma_kernel(
             continue;
         }
         if (lane < 16 && r < a.rows) {
-            for (int t = 0; t < ntok; ++t) {
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {   // static indices keep y1 / yv in registers
+                if (t >= ntok) break;
                 const float v = SWIGLU ? silu(y1[t]) * yv[t] : yv[t];
                 y[int64_t(t) * a.rows + r] = v;
             }

@@ -220,7 +220,10 @@ __device__ __forceinline__ void tile_compute(uint8_t* stage, const MatView& m, i
     // 3. tensor-core loop over the 128-column blocks
     const int g = lane >> 2, tig = lane & 3;
     const uint8_t* src = nullptr;
-    if (g < 6 && tok[g / 3].pieces) src = tok[g / 3].pieces + (g % 3) * 128 + tig * 32;
+    {
+        const uint8_t* pc = g < 3 ? tok[0].pieces : tok[1].pieces;   // a select: no local-memory copy of tok
+        if (g < 6 && pc) src = pc + (g % 3) * 128 + tig * 32;
+    }
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int b = 0; b < nb; ++b) {
         uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
@@ -411,7 +414,7 @@ __device__ __forceinline__ void chunk_compute(uint8_t* tile, const MatView& m, i
     // 3. tensor-core loop over the chunk's eight 128-column blocks
     const int g = lane >> 2, tig = lane & 3;
     const bool bsrc = g < 6 && (g < 3 ? has0 : has1);
-    const uint32_t src = bsrc ? smem_u32(tok[g / 3].pieces) + (g % 3) * 128 + tig * 32 : 0u;
+    const uint32_t src = bsrc ? smem_u32(g < 3 ? tok[0].pieces : tok[1].pieces) + (g % 3) * 128 + tig * 32 : 0u;
     const uint32_t w_base = signs_s + ch * 2048 + g * 128 + tig * 4;
     const uint32_t sc_base = sblk_s + 2 * (ch * 8);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};

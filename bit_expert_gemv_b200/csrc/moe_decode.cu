@@ -23,6 +23,7 @@
 #include "moe.cuh"
 #include "moe_decode.cuh"
 #include "mma_tile.cuh"
+#include "tma.cuh"
 
 namespace gale {
 
@@ -318,7 +319,7 @@ __host__ __device__ inline JobTile job_tile(int C, int R) {
     o += ((R * k + 1) / 2 + 31) & ~15;   // plus the source's offset from a 16-byte boundary
     t.srow = o;
     o += (R * 2 + 15) & ~15;
-    t.bytes = (o + 127) & ~127;
+    t.bytes = (o + 1023) & ~1023;   // the signs of every tile start on a 1024-byte swizzle atom
     return t;
 }
 
@@ -504,14 +505,14 @@ __device__ __forceinline__ void ensure_cached(const DecArgs& A, const Shape& sh,
         }
         fwht32_cg(v);
         float* tb = reinterpret_cast<float*>(dst) + blk * 33 * 32;   // 33-float rows: no bank conflicts
-#pragma unroll 8
+#pragma unroll
         for (int i = 0; i < 32; ++i) tb[i * 33 + lane] = v[i];
         __syncwarp();
-#pragma unroll 8
+#pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = tb[lane * 33 + i] * (1.0f / 32.0f);
         fwht32_cg(v);
         float m = 0.f;
-#pragma unroll 8
+#pragma unroll
         for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -571,11 +572,12 @@ __device__ __forceinline__ void ensure_cached(const DecArgs& A, const Shape& sh,
 //   sum_{b in chunk} s_blk[row, b] (X_b - 2 P_b).
 // The chunk's eight 128-column blocks run in two halves of four blocks with
 // one accumulator each, so that consecutive MMAs are independent.
-__device__ __forceinline__ void chunk_mma(const uint8_t* signs16, const __half* sblk, int C, int ch,
+__device__ __forceinline__ void chunk_mma(const uint8_t* signs, const __half* sblk, int C, int ch,
                                           const TokRef (&tok)[2], float* scratch, float (&part)[2]) {
+    // signs: this chunk's 128-byte piece of the tile's first row, swizzled
+    // (16-byte chunk bb of row r at position bb ^ (r & 7)); rows 128 bytes apart
     const int lane = threadIdx.x & 31;
-    const int nb = C / 128, rowb = C / 8;
-    const uint8_t* signs = signs16 + ch * 128;
+    const int nb = C / 128;
     const int row = lane & 15, half = lane >> 4;
     const bool has0 = tok[0].pieces != nullptr, has1 = tok[1].pieces != nullptr;
 
@@ -608,9 +610,9 @@ __device__ __forceinline__ void chunk_mma(const uint8_t* signs16, const __half* 
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int bb = 4 * hb + j;
-            const uint8_t* wa = signs + g * rowb + bb * 16 + tig * 4;
+            const uint8_t* wa = signs + g * 128 + ((bb ^ g) << 4) + tig * 4;   // rows g and g + 8 share g & 7
             wg[j] = *reinterpret_cast<const uint32_t*>(wa);
-            wg8[j] = *reinterpret_cast<const uint32_t*>(wa + 8 * rowb);
+            wg8[j] = *reinterpret_cast<const uint32_t*>(wa + 8 * 128);
             if (bsrc) {
                 q0[j] = *reinterpret_cast<const uint4*>(bsrc_p + bb * kPieceBlockBytes);
                 q1[j] = *reinterpret_cast<const uint4*>(bsrc_p + bb * kPieceBlockBytes + 16);
@@ -666,13 +668,16 @@ __device__ __forceinline__ void chunk_mma(const uint8_t* signs16, const __half* 
 // staged tile over the outliers j = sub, sub + step, ... (a fixed lane set
 // of the row sums them afterwards in a fixed order); six at a time so that
 // their loads overlap.
-__device__ __forceinline__ void row_outliers(const uint8_t* tile, const JobTile& L, int C, int k, int q_delta, int row,
-                                             int sub, int step, const TokRef (&tok)[2], float& corr0, float& corr1) {
+__device__ __forceinline__ void row_outliers(const uint8_t* tile, const JobTile& L, int C, int job_rows, int k,
+                                             int q_delta, int row, int sub, int step, const TokRef (&tok)[2],
+                                             float& corr0, float& corr1) {
     const int nb = C / 128;
     const uint16_t* ri = reinterpret_cast<const uint16_t*>(tile + L.idx) + row * k;
     const uint8_t* qn = tile + L.q + q_delta;
     const __half* sblk = reinterpret_cast<const __half*>(tile + L.scales) + row * nb;
-    const uint8_t* signs = tile + L.signs + row * (C / 8);
+    // the row in the swizzled sign layout: [piece][row][128 bytes]
+    const uint8_t* signs = tile + L.signs + row * 128;
+    const int piece_bytes = job_rows * 128, sw = row & 7;
     const float srow = __half2float(reinterpret_cast<const __half*>(tile + L.srow)[row]);
     const bool has0 = tok[0].pieces != nullptr, has1 = tok[1].pieces != nullptr;
     const __half* x0 = tok[0].x16;
@@ -692,7 +697,9 @@ __device__ __forceinline__ void row_outliers(const uint8_t* tile, const JobTile&
             const int n = row * k + (use[u] ? jb + u * step : 0);
             const int qb = int(qn[n >> 1]) >> ((n & 1) * 4);
             const int qv = (qb & 15) - ((qb & 8) << 1);
-            const uint32_t word = *reinterpret_cast<const uint32_t*>(signs + (c[u] >> 5) * 4);
+            const int wd = (c[u] >> 5) & 31;   // word within the 1024-column piece
+            const uint32_t word = *reinterpret_cast<const uint32_t*>(signs + (c[u] >> 10) * piece_bytes +
+                                                                     (((wd >> 2) ^ sw) << 4) + (wd & 3) * 4);
             const float sb = __half2float(sblk[c[u] >> 7]);
             float wq = fmaf(float(qv), srow, ((word >> (c[u] & 31)) & 1u) ? sb : -sb);
             wq = use[u] ? wq : 0.f;
@@ -882,7 +889,9 @@ __device__ bool grid_barrier(int32_t* cnt, int32_t* flag, int G) {
 }
 
 
-__global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Plan P) {
+__global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_constant__ CUtensorMap map13,
+                                                                   const __grid_constant__ CUtensorMap map2, DecArgs A,
+                                                                   Plan P) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_align1024(smem_raw);
     const DecSmem S = dec_smem(P);
@@ -925,9 +934,10 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
 
     if (warp == kDecWarps) {
         // ---------------- producer: weights only.  Lane mt copies matrix mt of
-        // the job (five bulk copies: signs, block scales, outlier columns,
-        // outlier values, row scales of all the job's rows); lane 0 arms the
-        // stage's barrier with the job's byte count first.
+        // the job: the signs of all the job's rows as one swizzled tensor box,
+        // then four bulk copies (block scales, outlier columns, outlier values,
+        // row scales); lane 0 arms the stage's barrier with the job's byte
+        // count first (a tensor box always delivers its full size).
         int s = 0, ph = 0;
         for (int i = 0; i < n13 + n2; ++i) {
             int ok_wait = 1;
@@ -952,8 +962,7 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
                 const MatView mv = make_view(A.base + int64_t(Jb.e) * A.stride + off, sh.rows, C);
                 const char* qs = reinterpret_cast<const char*>(mv.q) + int64_t(r0) * k / 2;   // r0 is even
                 const int qd = int(reinterpret_cast<uintptr_t>(qs) & 15);
-                src[0] = reinterpret_cast<const char*>(mv.signs + int64_t(r0) * (C / 32));
-                sz[0] = uint32_t(R * (C / 8));
+                sz[0] = uint32_t(sh.job_rows * (C / 8));
                 src[1] = reinterpret_cast<const char*>(mv.s_blk + int64_t(r0) * nb);
                 sz[1] = uint32_t(R * (C / 64));
                 src[2] = reinterpret_cast<const char*>(mv.idx + int64_t(r0) * k);
@@ -970,9 +979,10 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
             __syncwarp();
             if (mine) {
                 uint8_t* dst = smem + S.ring + s * P.stage_bytes + lane * sh.mat_bytes;
+                tma_load_5d(dst + L.signs, w13 ? &map13 : &map2, full + s, 0, r0, 0, w13 ? lane : 0, Jb.e);
                 const int dsto[5] = {L.signs, L.scales, L.idx, L.q, L.srow};
 #pragma unroll
-                for (int c = 0; c < 5; ++c)
+                for (int c = 1; c < 5; ++c)
                     if (sz[c]) bulk_load(dst + dsto[c], src[c], sz[c], full + s);
             }
             if (++s == P.n_stages) {
@@ -1092,7 +1102,7 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
             const JobTile L = job_tile(C, sh.job_rows);
             if (do_mma) {
                 const uint8_t* mt_tile = stage + mat * sh.mat_bytes;
-                chunk_mma(mt_tile + L.signs + tr * 16 * (C / 8),
+                chunk_mma(mt_tile + L.signs + ch * sh.job_rows * 128 + tr * 16 * 128,
                           reinterpret_cast<const __half*>(mt_tile + L.scales) + tr * 16 * (C / 128), C, ch, tok,
                           scratch, part);
             }
@@ -1103,8 +1113,8 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(DecArgs A, Pla
                 const int q_delta = int(
                     reinterpret_cast<uintptr_t>(reinterpret_cast<const char*>(ov.q) + int64_t(Jb.tile * sh.job_rows) * k / 2) &
                     15);
-                row_outliers(stage + o_mat * sh.mat_bytes, L, C, k, q_delta, o_tr * 16 + o_row, sub, lpp, tok, corr0,
-                             corr1);
+                row_outliers(stage + o_mat * sh.mat_bytes, L, C, sh.job_rows, k, q_delta, o_tr * 16 + o_row, sub, lpp,
+                             tok, corr0, corr1);
             }
             for (int o = 1; o < lpp; o <<= 1) {
                 corr0 += __shfl_xor_sync(0xffffffffu, corr0, o);
@@ -1233,6 +1243,13 @@ int launch_moe_decode(const gale_layer& L, const uint16_t* x, const int32_t* ids
     if (!make_plan(L, B, K, P)) return GALE_ERR_UNSUPPORTED;
 
     int rc = GALE_OK;
+    CUtensorMap map13, map2;
+    rc = cached_sign_map5(&map13, A.base + A.off_w1, L.d_ff, L.d_model, 2, A.off_w3 - A.off_w1, L.n_experts,
+                          L.expert_stride, P.s13.job_rows);
+    if (rc == GALE_OK)
+        rc = cached_sign_map5(&map2, A.base + A.off_w2, L.d_model, L.d_ff, 1, A.off_w3 - A.off_w1, L.n_experts,
+                              L.expert_stride, P.s2.job_rows);
+    if (rc != GALE_OK) return rc;
     const DecSmem S = dec_smem(P);
     rc = ensure_smem(reinterpret_cast<const void*>(moe_decode_kernel), S.bytes);
     if (rc != GALE_OK) return rc;
@@ -1247,7 +1264,7 @@ int launch_moe_decode(const gale_layer& L, const uint16_t* x, const int32_t* ids
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, moe_decode_kernel, A, P) == cudaSuccess ? GALE_OK : GALE_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, moe_decode_kernel, map13, map2, A, P) == cudaSuccess ? GALE_OK : GALE_ERR_CUDA;
 }
 
 }  // namespace gale

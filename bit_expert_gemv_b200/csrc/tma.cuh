@@ -14,6 +14,10 @@ int make_sign_map(CUtensorMap* m, const void* first_matrix, int rows, int cols, 
 int make_scale_map(CUtensorMap* m, const void* first_matrix, int rows, int cols, int experts, int64_t stride);
 int cached_map(CUtensorMap* out, bool scale, const void* first_matrix, int rows, int cols, int experts,
                int64_t stride);
+int make_sign_map5(CUtensorMap* m, const void* first_matrix, int rows, int cols, int n_mat, int64_t mat_stride,
+                   int experts, int64_t stride, int box_rows);
+int cached_sign_map5(CUtensorMap* out, const void* first_matrix, int rows, int cols, int n_mat, int64_t mat_stride,
+                     int experts, int64_t stride, int box_rows);
 // Raise a kernel's dynamic shared-memory limit once per device.
 int ensure_smem(const void* kernel, int bytes);
 
