@@ -870,20 +870,17 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
     return v;
 }
 
-// Grid-wide barrier of the cooperative launch, one thread per CTA; the
-// counters start at zero every call.  False if the wait ran out (2 s).
-__device__ bool grid_barrier(int32_t* cnt, int32_t* flag, int G) {
+// Grid-wide barrier of the cooperative launch, one thread per CTA (whose
+// threads have fenced their writes before the CTA barrier that precedes it);
+// the counter starts at zero every call.  Every CTA adds one and polls the
+// counter itself until all G have arrived: the release is the last arrival,
+// with no separate flag.  False if the wait ran out (2 s).
+__device__ bool grid_barrier(int32_t* cnt, int G) {
     __threadfence();
-    if (atomicAdd(cnt, 1) == G - 1) {
-        __threadfence();
-        atomicExch(flag, 1);
-        return true;
-    }
+    atomicAdd(cnt, 1);
     const uint64_t t0 = globaltimer_ns();
-    while (ld_acquire(flag) == 0) {
+    while (ld_acquire(cnt) < G)
         if (globaltimer_ns() - t0 > 2000000000ull) return false;
-        __nanosleep(64);
-    }
     __threadfence();
     return true;
 }
@@ -1141,7 +1138,7 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_c
             __threadfence();
             named_bar_sync(2, kPhaseBar);   // with the epilogue warp: this CTA's phase-1 work is done
             if (tid == 0) {
-                M.gate_ok = grid_barrier(A.ws.gbar, A.ws.gbar + 1, G);
+                M.gate_ok = grid_barrier(A.ws.gbar, G);
                 if (!M.gate_ok) set_status(A.ws.status, GALE_ERR_TIMEOUT);
                 for (int q = 0; q < kCapMax; ++q) {   // the cache now holds slots of h
                     M.key[q] = -1;
@@ -1195,7 +1192,7 @@ DecodeWs carve_decode_ws(void* ws, const gale_layer& L, int B, int K) {
     const int64_t P = int64_t(B) * K, dm = L.d_model, df = L.d_ff;
     const int64_t blocks = (dm + 63) / 64;
     w.status = reinterpret_cast<int32_t*>(take(256));
-    w.gbar = w.status + 4;   // two counters inside the status block, zeroed every call
+    w.gbar = w.status + 4;   // a counter inside the status block, zeroed every call
     w.comb_cnt = reinterpret_cast<int32_t*>(take(4 * B * blocks));
     w.tok_cnt = reinterpret_cast<int32_t*>(take(4 * int64_t(B)));
     w.ssq = reinterpret_cast<float*>(take(4 * B * blocks));

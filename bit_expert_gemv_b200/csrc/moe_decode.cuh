@@ -11,7 +11,7 @@ constexpr int kDecodeMaxDff = 4096;
 
 struct DecodeWs {
     int32_t* status;
-    int32_t* gbar;         // [2] grid-barrier arrivals and release flag (in the status block)
+    int32_t* gbar;         // grid-barrier arrivals (in the status block)
     int32_t* comb_cnt;     // [B][d_model/64] experts finished per (token, 64-row block)
     int32_t* tok_cnt;      // [B]            row blocks finished per token (RMSNorm)
     float* ssq;            // [B][d_model/64] partial sums of squares (RMSNorm)
