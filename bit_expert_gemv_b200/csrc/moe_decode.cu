@@ -18,6 +18,8 @@
 //             with the gates (deterministic, no float atomics), optionally
 //             adding the residual; the last row block of a token applies
 //             RMSNorm.
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "fwht.cuh"
 #include "moe.cuh"
@@ -726,24 +728,24 @@ __device__ __forceinline__ void epi_gather(const Shape& sh, bool W13, const floa
                                            float (&yb)[kMaxRT]) {
     const float* pc = pb + kDecWarps * 32;
     const int row = lane & 15, t = lane >> 4;
+    const int m1 = W13 ? 2 : 1;
+#pragma unroll
+    for (int i = 0; i < kMaxRT; ++i) ya[i] = yb[i] = 0.f;
 #pragma unroll
     for (int i = 0; i < kMaxRT; ++i) {
-        ya[i] = 0.f;
-        yb[i] = 0.f;
-        if (i >= sh.r_tiles) continue;
-        if (W13) {
-            float y1 = pc[(i * 16 + row) * 2 + t], y3 = pc[(sh.job_rows + i * 16 + row) * 2 + t];
-            for (int c2 = 0; c2 < sh.n_chunk; ++c2) {
-                y1 += pb[((i * 2 + 0) * sh.n_chunk + c2) * 32 + row * 2 + t];
-                y3 += pb[((i * 2 + 1) * sh.n_chunk + c2) * 32 + row * 2 + t];
-            }
-            ya[i] = y1;
-            yb[i] = y3;
-        } else {
-            float y = pc[(i * 16 + row) * 2 + t];
-            for (int c2 = 0; c2 < sh.n_chunk; ++c2) y += pb[(i * sh.n_chunk + c2) * 32 + row * 2 + t];
-            ya[i] = y;
+        if (i >= sh.r_tiles) break;
+        // outlier sums first, then the MMA pieces in chunk order
+        float y1 = pc[(i * 16 + row) * 2 + t];
+        float y3 = W13 ? pc[(sh.job_rows + i * 16 + row) * 2 + t] : 0.f;
+        const float* p1 = pb + i * m1 * sh.n_chunk * 32 + row * 2 + t;
+        const float* p3 = p1 + sh.n_chunk * 32;
+#pragma unroll 4
+        for (int c2 = 0; c2 < sh.n_chunk; ++c2) {
+            y1 += p1[c2 * 32];
+            if (W13) y3 += p3[c2 * 32];
         }
+        ya[i] = y1;
+        yb[i] = y3;
     }
 }
 
@@ -758,7 +760,8 @@ __device__ __forceinline__ void epi_finish(const DecArgs& A, const RouteTables& 
 #pragma unroll
         for (int i = 0; i < kMaxRT; ++i) {
             const int r = Jb.tile * sh.job_rows + i * 16 + row;
-            if (i < sh.r_tiles && slot_l >= 0 && r < sh.rows) A.ws.h[int64_t(slot_l) * sh.rows + r] = silu(ya[i]) * yb[i];
+            if (i < sh.r_tiles && slot_l >= 0 && r < sh.rows)
+                A.ws.h[int64_t(slot_l) * sh.rows + r] = __fdividef(ya[i], 1.0f + __expf(-ya[i])) * yb[i];
         }
         return;
     }
@@ -782,44 +785,63 @@ __device__ __forceinline__ void epi_finish(const DecArgs& A, const RouteTables& 
         }
     }
     const unsigned fl = __ballot_sync(0xffffffffu, flags);
+#pragma unroll 1
     for (int f = 0; f < 2 * nsub; ++f) {
         if (!((fl >> f) & 1)) continue;
         __threadfence();
         const int sl = f & 1, sb = f >> 1;
         const int t = R.slot_tok[sl ? Jb.slot1 : Jb.slot0];
         const int rb = Jb.tile * nsub + sb;
-        float ss = 0.f;
+        // lane k holds the token's (k0 + k)-th (slot, gate); eight experts'
+        // loads in flight at a time; the sum runs in fixed k order
+        const int r0 = rb * 64 + lane, r1 = r0 + 32;
+        float y0 = 0.f, y1 = 0.f;
+#pragma unroll 1
+        for (int k0 = 0; k0 < A.K; k0 += 32) {
+            int pos_l = -1;
+            float g_l = 0.f;
+            if (k0 + lane < A.K) {
+                pos_l = R.pos_of_pair[t * A.K + k0 + lane];
+                g_l = A.gates[t * A.K + k0 + lane];
+            }
+            const int kn = A.K - k0 < 32 ? A.K - k0 : 32;
+#pragma unroll 1
+            for (int k8 = 0; k8 < kn; k8 += 8) {
+                float o0[8], o1[8], gg[8];
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            const int r = rb * 64 + lane + 32 * h2;
-            if (r >= d) continue;
-            // all K loads first, then the sum in fixed k order
-            float ov[16], gv[16];
-#pragma unroll
-            for (int kk = 0; kk < 16; ++kk) {
-                ov[kk] = 0.f;
-                gv[kk] = 0.f;
-                if (kk < A.K) {
-                    const int pos = R.pos_of_pair[t * A.K + kk];
-                    if (pos >= 0) {
-                        ov[kk] = __ldcg(A.ws.o + int64_t(pos) * d + r);
-                        gv[kk] = A.gates[t * A.K + kk];
+                for (int j = 0; j < 8; ++j) {
+                    const int pos = __shfl_sync(0xffffffffu, pos_l, (k8 + j) & 31);
+                    gg[j] = __shfl_sync(0xffffffffu, g_l, (k8 + j) & 31);
+                    o0[j] = o1[j] = 0.f;
+                    if (k8 + j < kn && pos >= 0) {
+                        const float* orow = A.ws.o + int64_t(pos) * d;
+                        if (r0 < d) o0[j] = __ldcg(orow + r0);
+                        if (r1 < d) o1[j] = __ldcg(orow + r1);
                     }
                 }
-            }
-            float y = 0.f;
 #pragma unroll
-            for (int kk = 0; kk < 16; ++kk)
-                if (kk < A.K) y = fmaf(gv[kk], ov[kk], y);
-            if (!A.fuse_norm) {
-                store_from_f32(A.out, A.out_dtype, int64_t(t) * d + r, y);
-            } else {
-                const float v = bf16_to_f32(A.x[int64_t(t) * d + r]) + y;
-                A.ws.v[int64_t(t) * d + r] = v;
-                ss = fmaf(v, v, ss);
+                for (int j = 0; j < 8; ++j) {
+                    y0 = fmaf(gg[j], o0[j], y0);
+                    y1 = fmaf(gg[j], o1[j], y1);
+                }
             }
         }
-        if (!A.fuse_norm) continue;
+        if (!A.fuse_norm) {
+            if (r0 < d) store_from_f32(A.out, A.out_dtype, int64_t(t) * d + r0, y0);
+            if (r1 < d) store_from_f32(A.out, A.out_dtype, int64_t(t) * d + r1, y1);
+            continue;
+        }
+        float ss = 0.f;
+        if (r0 < d) {
+            const float v = bf16_to_f32(A.x[int64_t(t) * d + r0]) + y0;
+            A.ws.v[int64_t(t) * d + r0] = v;
+            ss = v * v;
+        }
+        if (r1 < d) {
+            const float v = bf16_to_f32(A.x[int64_t(t) * d + r1]) + y1;
+            A.ws.v[int64_t(t) * d + r1] = v;
+            ss = fmaf(v, v, ss);
+        }
         // sum of squares of this 64-row block (fixed order), then the last
         // block of the token normalises the whole row
         ss = warp_sum(ss);
@@ -837,8 +859,9 @@ __device__ __forceinline__ void epi_finish(const DecArgs& A, const RouteTables& 
         for (int q = lane; q < comb_blocks; q += 32) tot += __ldcg(A.ws.ssq + t * comb_blocks + q);
         tot = warp_sum(tot);
         const float inv = rsqrtf(tot / float(d) + A.eps);
-        // sixteen 16-byte loads in flight per lane, then the stores
+        // sixteen 16-byte loads in flight per lane, then bf16 pairs out
         const float4* vrow = reinterpret_cast<const float4*>(A.ws.v + int64_t(t) * d);
+        __nv_bfloat162* orow = reinterpret_cast<__nv_bfloat162*>(static_cast<uint16_t*>(A.out) + int64_t(t) * d);
         const int n4 = d / 4;
 #pragma unroll 1
         for (int c0 = 0; c0 < n4; c0 += 32 * 16) {
@@ -852,11 +875,8 @@ __device__ __forceinline__ void epi_finish(const DecArgs& A, const RouteTables& 
             for (int j = 0; j < 16; ++j) {
                 const int c = c0 + 32 * j + lane;
                 if (c < n4) {
-                    const int64_t o = int64_t(t) * d + 4 * c;
-                    store_from_f32(A.out, GALE_BF16, o, vv[j].x * inv);
-                    store_from_f32(A.out, GALE_BF16, o + 1, vv[j].y * inv);
-                    store_from_f32(A.out, GALE_BF16, o + 2, vv[j].z * inv);
-                    store_from_f32(A.out, GALE_BF16, o + 3, vv[j].w * inv);
+                    orow[2 * c] = __floats2bfloat162_rn(vv[j].x * inv, vv[j].y * inv);
+                    orow[2 * c + 1] = __floats2bfloat162_rn(vv[j].z * inv, vv[j].w * inv);
                 }
             }
         }
