@@ -526,39 +526,44 @@ __device__ __forceinline__ void ensure_cached(const DecArgs& A, const Shape& sh,
         for (int w = e * nblk; w < (e + 1) * nblk; ++w) m = fmaxf(m, M.red[w]);
         const float S = fixed_scale(m);
         const int b = blk * 8 + (lane >> 2), tig = lane & 3;
-        uint32_t* pieces = reinterpret_cast<uint32_t*>(dst + b * kPieceBlockBytes + tig * 32);
-        // word q takes registers q, q + 8, q + 16, q + 24
+        // fp16 copy (for the outliers) and the 128-block sums
+        uint4* x16 = reinterpret_cast<uint4*>(dst + C * kPieces + (C / 128) * 4) + blk * 128 + lane * 4;
+        float sum = 0.f;
 #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t hw[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const __half2 h2 = __floats2half2_rn(v[8 * i + 2 * j], v[8 * i + 2 * j + 1]);
+                hw[j] = *reinterpret_cast<const uint32_t*>(&h2);
+                sum += v[8 * i + 2 * j] + v[8 * i + 2 * j + 1];
+            }
+            x16[i] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        }
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        if (tig == 0) reinterpret_cast<float*>(dst + C * kPieces)[b] = sum;
+        // digit word q takes registers q, q + 8, q + 16, q + 24: a rolled loop
+        // over q that shifts the registers down by one each time (small code
+        // for a step that runs once per vector)
+        uint32_t* pieces = reinterpret_cast<uint32_t*>(dst + b * kPieceBlockBytes + tig * 32);
+#pragma unroll 1
         for (int q = 0; q < 8; ++q) {
             const float sc = S * inv_a(q);
             uint32_t word[kPieces] = {0u, 0u, 0u};
 #pragma unroll
             for (int i4 = 0; i4 < 4; ++i4) {
                 uint32_t d1, d2, d3;
-                fixed_digits(v[q + 8 * i4] * sc, d1, d2, d3);
+                fixed_digits(v[8 * i4] * sc, d1, d2, d3);
                 word[0] |= d1 << (8 * i4);
                 word[1] |= d2 << (8 * i4);
                 word[2] |= d3 << (8 * i4);
             }
 #pragma unroll
             for (int j = 0; j < kPieces; ++j) pieces[j * 32 + q] = word[j];
-        }
-        // fp16 copy (for the outliers) and the 128-block sums
-        uint4* x16 = reinterpret_cast<uint4*>(dst + C * kPieces + (C / 128) * 4) + blk * 128 + lane * 4;
-        float sum = 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            __half2 hh[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                hh[j] = __floats2half2_rn(v[8 * i + 2 * j], v[8 * i + 2 * j + 1]);
-                sum += v[8 * i + 2 * j] + v[8 * i + 2 * j + 1];
-            }
-            x16[i] = *reinterpret_cast<const uint4*>(hh);
+            for (int i = 0; i < 31; ++i) v[i] = v[i + 1];
         }
-        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-        if (tig == 0) reinterpret_cast<float*>(dst + C * kPieces)[b] = sum;
         if (blk == 0 && lane == 0) M.sigma[M.plan_slot[e]] = 1.0f / S;
     }
     named_bar_sync(1, kDecThreads);
@@ -715,25 +720,21 @@ __device__ __forceinline__ void row_outliers(const uint8_t* tile, const JobTile&
 // the kernel
 // ----------------------------------------------------------------------------
 
-// The epilogue of a job, run by the last warp to finish it, in two parts:
-// epi_gather reads the job's partial sums (shared memory of the job's stage)
-// into registers, after which the stage can be refilled; epi_finish does the
-// global-memory work: w1/w3 stores h = silu(w1 x) * (w3 x); w2 stores the
-// expert outputs and runs the (token, 64-row block) combine and the RMSNorm of
-// finished tokens.  Lane l holds value i for row block tile i, row l & 15,
-// token l >> 4.
-constexpr int kMaxRT = 8;   // row tiles per job (job_rows <= 128)
-
-__device__ __forceinline__ void epi_gather(const Shape& sh, bool W13, const float* pb, int lane, float (&ya)[kMaxRT],
-                                           float (&yb)[kMaxRT]) {
+// The epilogue of a job, run by the epilogue warp, in two parts.  epi_rows
+// sums the job's partial sums (shared memory of the job's stage) row tile by
+// row tile and stores the rows: h = silu(w1 x) * (w3 x) for w1/w3, the expert
+// outputs o for w2; after it the stage can be refilled.  epi_combine (w2
+// only) runs the (token, 64-row block) combine and the RMSNorm of finished
+// tokens.  Lane l covers row l & 15 of every row tile and token slot l >> 4.
+__device__ __forceinline__ void epi_rows(const DecArgs& A, const Shape& sh, bool W13, const Job& Jb,
+                                         const float* pb, int lane) {
     const float* pc = pb + kDecWarps * 32;
     const int row = lane & 15, t = lane >> 4;
     const int m1 = W13 ? 2 : 1;
-#pragma unroll
-    for (int i = 0; i < kMaxRT; ++i) ya[i] = yb[i] = 0.f;
-#pragma unroll
-    for (int i = 0; i < kMaxRT; ++i) {
-        if (i >= sh.r_tiles) break;
+    const int slot = t ? Jb.slot1 : Jb.slot0;
+    const int d = A.d_model;
+#pragma unroll 1
+    for (int i = 0; i < sh.r_tiles; ++i) {
         // outlier sums first, then the MMA pieces in chunk order
         float y1 = pc[(i * 16 + row) * 2 + t];
         float y3 = W13 ? pc[(sh.job_rows + i * 16 + row) * 2 + t] : 0.f;
@@ -744,32 +745,17 @@ __device__ __forceinline__ void epi_gather(const Shape& sh, bool W13, const floa
             y1 += p1[c2 * 32];
             if (W13) y3 += p3[c2 * 32];
         }
-        ya[i] = y1;
-        yb[i] = y3;
+        const int r = Jb.tile * sh.job_rows + i * 16 + row;
+        if (slot < 0 || r >= sh.rows) continue;
+        if (W13) A.ws.h[int64_t(slot) * sh.rows + r] = __fdividef(y1, 1.0f + __expf(-y1)) * y3;
+        else A.ws.o[int64_t(slot) * d + r] = y1;
     }
 }
 
-__device__ __forceinline__ void epi_finish(const DecArgs& A, const RouteTables& R, const Shape& sh, bool W13,
-                                           const Job& Jb, int lane, const float (&ya)[kMaxRT],
-                                           const float (&yb)[kMaxRT]) {
+__device__ __forceinline__ void epi_combine(const DecArgs& A, const RouteTables& R, const Shape& sh, const Job& Jb,
+                                            int lane) {
     const int d = A.d_model;
     const int comb_blocks = (d + 63) / 64;
-    const int row = lane & 15, t_l = lane >> 4;
-    const int slot_l = t_l ? Jb.slot1 : Jb.slot0;
-    if (W13) {
-#pragma unroll
-        for (int i = 0; i < kMaxRT; ++i) {
-            const int r = Jb.tile * sh.job_rows + i * 16 + row;
-            if (i < sh.r_tiles && slot_l >= 0 && r < sh.rows)
-                A.ws.h[int64_t(slot_l) * sh.rows + r] = __fdividef(ya[i], 1.0f + __expf(-ya[i])) * yb[i];
-        }
-        return;
-    }
-#pragma unroll
-    for (int i = 0; i < kMaxRT; ++i) {
-        const int r = Jb.tile * sh.job_rows + i * 16 + row;
-        if (i < sh.r_tiles && slot_l >= 0 && r < d) A.ws.o[int64_t(slot_l) * d + r] = ya[i];
-    }
     __threadfence();
     __syncwarp();
     // the (token, 64-row block) combine: the last expert to finish sums the K outputs
@@ -1030,13 +1016,12 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_c
                     if (lane == 0) set_status(A.ws.status, GALE_ERR_TIMEOUT);
                 }
                 const float* pb = reinterpret_cast<const float*>(smem + S.part) + s * kPartFloats;
-                float ya[kMaxRT], yb[kMaxRT];
-                epi_gather(sh, W13, pb, lane, ya, yb);
+                if (eok) epi_rows(A, sh, W13, Jb, pb, lane);
                 // the consumers only read the stage, so the barrier alone orders
-                // their reads (and this gather) before the next copy into it
+                // their reads (and these sums) before the next copy into it
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty + s);
-                if (eok) epi_finish(A, R, sh, W13, Jb, lane, ya, yb);
+                if (eok && !W13) epi_combine(A, R, sh, Jb, lane);
                 if (++s == P.n_stages) {
                     s = 0;
                     ph ^= 1;
