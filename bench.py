@@ -37,10 +37,9 @@ PREFILL_B = 4096
 CHAIN_LAYERS = 43
 # kernels of this library launched per decode step (the cooperative layer kernel)
 DECODE_LAUNCHES = 1
-# dram read + write bytes of one decode launch at this workload, from the ncu
-# capture summarised in profiles/moe_decode_kernel_b1.md (None once the
-# kernel has changed since that capture)
-DECODE_TRAFFIC = 25_176_320
+# dram read + write bytes of one decode launch at this workload, from an ncu
+# capture of the current kernel (None once the kernel has changed since)
+DECODE_TRAFFIC = 25_177_600
 WORKLOAD = ("moe_layer_decode: 256 GALE-1bit experts (w1/w3 [2048x4096], w2 [4096x2048]), "
             "top-6 softmax routing, bf16 hidden [B x 4096]")
 
@@ -81,10 +80,18 @@ class Clocks:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader",
-                                          "-i", str(self.index), "-lms", "200"], stdout=self.fh,
+                                          "-i", str(self.index), "-lms", "50"], stdout=self.fh,
                                          stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        # the sampler takes a moment to start: the timed region begins after its first line
+        t0 = time.time()
+        while time.time() - t0 < 10.0 and self.proc.poll() is None:
+            self.fh.flush()
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.05)
 
     def stop(self):
         if self.proc is None:
@@ -307,10 +314,10 @@ def run_gpu(args):
         torch.cuda.empty_cache()
         return t, distinct * expert_bytes, graph is not None
 
+    # nvidia-smi samples the clocks through every timed measurement below
     clocks = Clocks(local)
     clocks.start()
     t1, bytes1, times1 = measure(1, args.steps, args.warmup, 10_000)
-    clocks_info = clocks.stop()
     t8, bytes8, _ = measure(8, max(args.steps // 2, 3), args.warmup, 20_000)
     te, h2d, d2h = measure_e2e(1, args.steps, args.warmup, 30_000)
     # prefill: 4096 tokens, skewed routing (tensor-core tile path)
@@ -318,6 +325,7 @@ def run_gpu(args):
     tp, _, _ = measure(PREFILL_B, pf_steps, 3, 40_000, bias_sigma=0.5, n_x=2)
     ch_steps = max(3, min(args.steps // 5, 10))
     tc, bytes_c, ch_graph = measure_chain(ch_steps, 3) if not args.no_chain else (float("nan"), 0, False)
+    clocks_info = clocks.stop()
 
     # max over ranks of the device time
     tt = torch.tensor([t1, t8, te, tp, tc], dtype=torch.float64, device="cuda")
