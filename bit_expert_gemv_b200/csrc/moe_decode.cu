@@ -925,15 +925,45 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_c
         for (int64_t o = int64_t(threadIdx.x) * 128; o < xb; o += int64_t(blockDim.x) * 128)
             prefetch_l2(reinterpret_cast<const char*>(A.x) + o);
     }
-    build_route(A, R, *reinterpret_cast<RouteScratch*>(smem + S.ring));   // contains __syncthreads
-    // contiguous job ranges of this CTA in both phases
+    const bool small = A.B * A.K <= 32;
+    if (small) {
+        // small batches: the epilogue warp routes the pairs and releases the
+        // producer at once; meanwhile, for one or two tokens, the consumers
+        // rotate x (its tokens are known without the routing) into cache
+        // entries that the jobs then find
+        __syncthreads();   // the cache bookkeeping is initialised
+        if (warp == kDecWarps + 1) {
+            build_route_small(A, R);
+            __syncwarp();
+            named_bar_arrive(3, 64);          // with the producer
+            named_bar_arrive(4, kPhaseBar);   // with the consumers
+        } else if (warp == kDecWarps) {
+            named_bar_sync(3, 64);
+        } else {
+            if (A.B <= 2) {
+                int c0, c1;
+                ensure_cached(A, P.s13, P.cap13, smem + S.cache, M, true, 0, A.B > 1 ? 1 : -1, c0, c1);
+            }
+            named_bar_sync(4, kPhaseBar);
+        }
+    } else {
+        build_route(A, R, *reinterpret_cast<RouteScratch*>(smem + S.ring));   // contains __syncthreads
+    }
+    // contiguous job ranges of this CTA in both phases; the producer decodes
+    // its jobs as it goes, the other warps read them from a table
     const int J13 = R.n_groups * P.s13.row_blocks, J2 = R.n_groups * P.s2.row_blocks;
     const int a0 = int((int64_t(J13) * blockIdx.x) / G), n13 = int((int64_t(J13) * (blockIdx.x + 1)) / G) - a0;
     const int b0 = int((int64_t(J2) * blockIdx.x) / G), n2 = int((int64_t(J2) * (blockIdx.x + 1)) / G) - b0;
     uint2* jobs = reinterpret_cast<uint2*>(smem + S.jobs);
-    for (int i = threadIdx.x; i < n13 + n2; i += blockDim.x)
-        jobs[i] = pack_job(i < n13 ? decode_job(R, a0 + i, P.s13.row_blocks) : decode_job(R, b0 + (i - n13), P.s2.row_blocks));
-    __syncthreads();
+    if (warp < kDecWarps)
+        for (int i = threadIdx.x; i < n13 + n2; i += kDecThreads)
+            jobs[i] = pack_job(i < n13 ? decode_job(R, a0 + i, P.s13.row_blocks)
+                                       : decode_job(R, b0 + (i - n13), P.s2.row_blocks));
+    if (small) {
+        if (warp != kDecWarps) named_bar_sync(2, kPhaseBar);   // the table is written
+    } else {
+        __syncthreads();
+    }
 
     if (warp == kDecWarps) {
         // ---------------- producer: weights only.  Lane mt copies matrix mt of
@@ -952,7 +982,7 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_c
             }
             const bool w13 = i < n13;
             const Shape& sh = w13 ? P.s13 : P.s2;
-            const Job Jb = unpack_job(jobs[i]);
+            const Job Jb = w13 ? decode_job(R, a0 + i, P.s13.row_blocks) : decode_job(R, b0 + (i - n13), P.s2.row_blocks);
             const int C = sh.cols, nb = C / 128, k = outliers_per_row(C);
             const int r0 = Jb.tile * sh.job_rows;
             const int R = min(sh.job_rows, sh.rows - r0);
