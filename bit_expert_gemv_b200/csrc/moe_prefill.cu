@@ -61,7 +61,7 @@ struct TcArgs {
 };
 
 struct TcSmem {
-    int b, idx[2], q[2], srow[2], ent[2], bars, misc, bytes;
+    int b, idx[2], q[2], srow[2], ent[2], patch, bars, misc, bytes;
 };
 
 __host__ __device__ inline int align16(int n) { return (n + 15) & ~15; }
@@ -84,6 +84,9 @@ __host__ __device__ inline TcSmem tc_smem(int nmat, int chunk, int k) {
         s.ent[mt] = o;
         o += kTcM * (k + 4) * 4;
     }
+    // per expander warp, 16 words x 32 lanes of patched (outlier) words
+    s.patch = o;
+    o += kTcExpWarps * 16 * 32 * 4;
     s.bars = (o + 7) & ~7;
     s.misc = s.bars + 8 * (3 * kTcStages + 2);
     s.bytes = s.misc + 16 + 1024;   // + slack to align the base to 1024 bytes
@@ -333,6 +336,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
             wb[mt] = __ldg(wsrc[mt] + 1);
             sp[mt] = __ldg(ssrc[mt]);
         }
+        uint32_t* pw = reinterpret_cast<uint32_t*>(smem + S.patch) + ew * 512 + lane;   // this lane's column
         const int ng = nk / kTcStages;
         for (int g = 0; g < ng; ++g) {
             uint32_t wg[NMAT][kTcStages], sg[NMAT][2];
@@ -360,32 +364,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
                     const uint32_t w = wg[mt][s], sc = sg[mt][s >> 1];
                     uint32_t v[16];
                     expand_signs(w, sc, v);
-                    // outliers of this range replace their weights; the entry
-                    // after the current one is already loaded
+                    // outliers of this range replace their weights: each lane
+                    // walks its own entries (the next one already loaded),
+                    // parks the patched words in its column of the warp's
+                    // patch area and marks them; a predicated load per word
+                    // then takes them in, with no per-outlier select over the
+                    // sixteen words
                     const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + S.ent[mt]) + t * (kout + 4);
+                    uint32_t m = 0u;
                     int prev_p = -1;
                     uint32_t prev_a = 0u;
-                    for (;;) {
-                        const int ecol = int(ent[mt] >> 16);
-                        const bool mine = ecol < hi;
-                        if (!__any_sync(0xffffffffu, mine)) break;
-                        int P = -1;
-                        uint32_t a = 0u;
-                        if (mine) {
-                            const int u = ecol - lo;
-                            P = u >> 1;
-                            const uint32_t val = ent[mt] & 0xFFFFu;
-                            uint32_t other = sc ^ (((w >> (u ^ 1)) & 1u) << 15);
-                            if (P == prev_p) other = (u & 1) ? (prev_a & 0xFFFFu) : (prev_a >> 16);
-                            a = (u & 1) ? (other | (val << 16)) : (val | (other << 16));
-                            prev_p = P;
-                            prev_a = a;
-                            ent[mt] = nxt[mt];
-                            nxt[mt] = list[++cur[mt] + 1];
-                        }
-#pragma unroll
-                        for (int p = 0; p < 16; ++p) v[p] = (P == p) ? a : v[p];
+                    while (int(ent[mt] >> 16) < hi) {
+                        const int u = int(ent[mt] >> 16) - lo;
+                        const int P = u >> 1;
+                        const uint32_t val = ent[mt] & 0xFFFFu;
+                        uint32_t other = sc ^ (((w >> (u ^ 1)) & 1u) << 15);
+                        if (P == prev_p) other = (u & 1) ? (prev_a & 0xFFFFu) : (prev_a >> 16);
+                        const uint32_t a = (u & 1) ? (other | (val << 16)) : (val | (other << 16));
+                        prev_p = P;
+                        prev_a = a;
+                        pw[P * 32] = a;
+                        m |= 1u << P;
+                        ent[mt] = nxt[mt];
+                        nxt[mt] = list[++cur[mt] + 1];
                     }
+#pragma unroll
+                    for (int p = 0; p < 16; ++p)
+                        if ((m >> p) & 1u) v[p] = pw[p * 32];
+                    __syncwarp();
                     tmem_st16(tmem + (uint32_t(32 * quarter) << 16) +
                                   uint32_t(Cfg::acc_cols + s * Cfg::a_cols + mt * 32 + 16 * h),
                               v);
