@@ -140,29 +140,34 @@ __global__ void __launch_bounds__(1024) prefill_jobs_kernel(const int32_t* count
     }
 }
 
-// x of every pair in permuted order, rotated, as fp16: one warp per (slot,
-// 1024-block).  Slots past the routed pairs (pairs with an invalid expert id
-// are dropped) are left alone; no job reads them.
+// x of every pair in permuted order, rotated, as fp16: one warp per (token,
+// 1024-block) rotates the block once and writes it to the slot of each of the
+// token's routed pairs (pairs with an invalid expert id have no slot).
 __global__ void __launch_bounds__(256) gather_rotate_kernel(const uint16_t* __restrict__ x,
-                                                            const int32_t* __restrict__ perm,
-                                                            const int32_t* __restrict__ n_routed, int K, int d,
-                                                            int64_t slots, __half* __restrict__ y) {
+                                                            const int32_t* __restrict__ pos_of_pair, int B, int K,
+                                                            int d, __half* __restrict__ y) {
     const int lane = threadIdx.x & 31;
     const int64_t wid = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
     const int nb = d / 1024;
-    if (wid >= slots * nb) return;
-    const int64_t s = wid / nb;
-    if (s >= *n_routed) return;
-    const int blk = int(wid - s * nb);
-    const int t = perm[s] / K;
-    const uint16_t* src = x + int64_t(t) * d + blk * 1024;
+    if (wid >= int64_t(B) * nb) return;
+    const int64_t t = wid / nb;
+    const int blk = int(wid - t * nb);
+    const uint16_t* src = x + t * d + blk * 1024;
     float v[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = bf16_to_f32(src[32 * i + lane]);
     fwht1024_warp(v, lane);
-    __half* dst = y + s * d + blk * 1024;
+    __half hv[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) dst[32 * i + lane] = __float2half_rn(v[i] * (1.0f / 32.0f));
+    for (int i = 0; i < 32; ++i) hv[i] = __float2half_rn(v[i] * (1.0f / 32.0f));
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+        const int64_t s = pos_of_pair[t * K + k];
+        if (s < 0) continue;
+        __half* dst = y + s * d + blk * 1024;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dst[32 * i + lane] = hv[i];
+    }
 }
 
 // The 16 fp16 pairs of 32 weights: sign word w (bit c set = column c negative)
@@ -508,9 +513,9 @@ int launch_moe_prefill(const gale_layer& L, const uint16_t* x, const int32_t* id
                                             w.n_jobs, static_cast<TcJob*>(w.jobs2), w.n_jobs + 1);
     GALE_LAUNCH_CHECK();
     {
-        const int64_t warps = P * (L.d_model / 1024);
-        gather_rotate_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, st>>>(x, w.perm, w.offsets + L.n_experts,
-                                                                                  K, L.d_model, P, w.x16);
+        const int64_t warps = int64_t(B) * (L.d_model / 1024);
+        gather_rotate_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, st>>>(x, w.pos_of_pair, B, K, L.d_model,
+                                                                                  w.x16);
         GALE_LAUNCH_CHECK();
     }
     const int64_t l1 = make_layout(L.d_ff, L.d_model).total;

@@ -1,107 +1,109 @@
 // Routing permute: stable counting sort of the (token, slot) pairs by expert.
 //
-// One CTA of 1024 threads.  Pairs are placed in rounds of 1024 in pair order;
-// within a round a pair's rank among equal experts is its rank inside its
-// warp (match_any) plus the counts of that expert in the earlier warps, so the
-// result is the stable order, independent of scheduling.
+// One CTA of 1024 threads.  Warp w owns the contiguous pair range
+// [w * chunk, (w + 1) * chunk) and walks it 32 pairs at a time, in order:
+// pass 1 counts each expert's pairs per warp (match_any groups, the group's
+// leader adds); a scan in (expert, warp) order gives every warp the first
+// position of each of its experts; pass 2 walks the range again and places
+// each pair at that base + its running rank.  The order is the stable one
+// (pair order within an expert), independent of scheduling.
 #include "common.cuh"
 #include "route.cuh"
 
 namespace gale {
 
+namespace {
+// Expert of pair p, or -1 when out of range or repeated earlier in its token.
+__device__ __forceinline__ int valid_expert(const RouteArgs& a, int p) {
+    const int e = a.ids[p];
+    if (e < 0 || e >= a.E) return -1;
+    const int t0 = p - p % a.K;
+    for (int j = t0; j < p; ++j)
+        if (a.ids[j] == e) return -1;
+    return e;
+}
+}  // namespace
+
 __global__ void __launch_bounds__(1024) route_permute_kernel(RouteArgs a) {
     extern __shared__ int smem[];
     const int E = a.E;
-    int* cnt = smem;                 // [E]
-    int* cur = cnt + E;              // [E]
-    int* wcnt = cur + E;             // [32][E]
+    int* wcnt = smem;                // [32][E]: pairs of expert e in warp w's range, then w's base
+    int* scan = wcnt + 32 * E;       // [2 * 1024] scan scratch
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int BK = a.B * a.K;
+    const int chunk = (BK + 31) / 32;
+    const int p0 = warp * chunk, p1 = min(BK, p0 + chunk);
 
-    for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+    for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
-    // histogram + validation (out-of-range or repeated within a token)
-    for (int p = tid; p < BK; p += blockDim.x) {
-        int e = a.ids[p];
-        bool ok = e >= 0 && e < E;
-        if (ok) {
-            int t0 = p - p % a.K;
-            for (int j = t0; j < p; ++j)
-                if (a.ids[j] == e) ok = false;
-        }
-        if (ok) atomicAdd(&cnt[e], 1);
-        else set_status(a.status, GALE_ERR_ARG);
-    }
-    __syncthreads();
-    // exclusive scan of counts (E <= 1024: one element per thread), plus the
-    // list of experts with at least one pair, in increasing id order
-    {
-        int c = tid < E ? cnt[tid] : 0;
-        int nz = c > 0;
-        // block-wide inclusive scans through shared memory (two arrays in wcnt)
-        int* s1 = wcnt;
-        int* s2 = wcnt + 1024;
-        s1[tid] = c;
-        s2[tid] = nz;
-        __syncthreads();
-        for (int off = 1; off < 1024; off <<= 1) {
-            int v1 = tid >= off ? s1[tid - off] : 0;
-            int v2 = tid >= off ? s2[tid - off] : 0;
-            __syncthreads();
-            s1[tid] += v1;
-            s2[tid] += v2;
-            __syncthreads();
-        }
-        if (tid < E) {
-            int excl = s1[tid] - c;
-            cur[tid] = excl;
-            if (a.counts) a.counts[tid] = c;
-            if (a.offsets) a.offsets[tid] = excl;
-            if (tid == E - 1 && a.offsets) a.offsets[E] = s1[tid];
-            if (nz && a.active) a.active[s2[tid] - 1] = tid;
-            if (tid == E - 1 && a.n_active) *a.n_active = s2[tid];
-        }
-        __syncthreads();
-    }
-    // stable placement, 1024 pairs per round
-    for (int base = 0; base < BK; base += blockDim.x) {
-        for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
-        __syncthreads();
-        const int p = base + tid;
+    // pass 1: per-warp counts (and validation)
+    for (int base = p0; base < p1; base += 32) {
+        const int p = base + lane;
         int e = -1;
-        if (p < BK) {
-            e = a.ids[p];
-            bool ok = e >= 0 && e < E;
-            if (ok) {
-                int t0 = p - p % a.K;
-                for (int j = t0; j < p; ++j)
-                    if (a.ids[j] == e) ok = false;
-            }
-            if (!ok) e = -1;
+        if (p < p1) {
+            e = valid_expert(a, p);
+            if (e < 0) set_status(a.status, GALE_ERR_ARG);
         }
         const unsigned grp = __match_any_sync(0xffffffffu, e);
-        const int rank = __popc(grp & ((1u << lane) - 1u));
-        if (e >= 0 && rank == 0) wcnt[warp * E + e] = __popc(grp);
+        if (e >= 0 && lane == __ffs(grp) - 1) wcnt[warp * E + e] += __popc(grp);
+        __syncwarp();
+    }
+    __syncthreads();
+    // totals per expert (thread e sums its column in warp order), exclusive
+    // scans of the totals and of the non-empty flags
+    const int c = tid < E ? [&] {
+        int t = 0;
+        for (int w = 0; w < 32; ++w) t += wcnt[w * E + tid];
+        return t;
+    }() : 0;
+    const int nz = c > 0;
+    int* s1 = scan;
+    int* s2 = scan + 1024;
+    s1[tid] = c;
+    s2[tid] = nz;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {
+        const int v1 = tid >= off ? s1[tid - off] : 0;
+        const int v2 = tid >= off ? s2[tid - off] : 0;
         __syncthreads();
+        s1[tid] += v1;
+        s2[tid] += v2;
+        __syncthreads();
+    }
+    if (tid < E) {
+        const int excl = s1[tid] - c;
+        if (a.counts) a.counts[tid] = c;
+        if (a.offsets) a.offsets[tid] = excl;
+        if (tid == E - 1 && a.offsets) a.offsets[E] = s1[tid];
+        if (nz && a.active) a.active[s2[tid] - 1] = tid;
+        if (tid == E - 1 && a.n_active) *a.n_active = s2[tid];
+        // first position of expert tid in each warp's range
+        int run = excl;
+        for (int w = 0; w < 32; ++w) {
+            const int n = wcnt[w * E + tid];
+            wcnt[w * E + tid] = run;
+            run += n;
+        }
+    }
+    __syncthreads();
+    // pass 2: placement in pair order
+    for (int base = p0; base < p1; base += 32) {
+        const int p = base + lane;
+        const int e = p < p1 ? valid_expert(a, p) : -1;
+        const unsigned grp = __match_any_sync(0xffffffffu, e);
         if (e >= 0) {
-            int pos = cur[e] + rank;
-            for (int w = 0; w < warp; ++w) pos += wcnt[w * E + e];
+            const int pos = wcnt[warp * E + e] + __popc(grp & ((1u << lane) - 1u));
             a.perm[pos] = p;
             if (a.pos_of_pair) a.pos_of_pair[p] = pos;
         }
-        __syncthreads();
-        for (int ee = tid; ee < E; ee += blockDim.x) {
-            int s = 0;
-            for (int w = 0; w < 32; ++w) s += wcnt[w * E + ee];
-            cur[ee] += s;
-        }
-        __syncthreads();
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(grp) - 1) wcnt[warp * E + e] += __popc(grp);
+        __syncwarp();
     }
 }
 
 int launch_route_permute(const RouteArgs& a, cudaStream_t st) {
-    size_t smem = size_t(34) * a.E * sizeof(int);
-    if (smem < 2048 * sizeof(int) + 2 * a.E * sizeof(int)) smem = 2048 * sizeof(int) + 2 * a.E * sizeof(int);
+    const size_t smem = (size_t(32) * a.E + 2048) * sizeof(int);
     if (smem > 48 * 1024)
         GALE_CUDA_TRY(cudaFuncSetAttribute(route_permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            int(smem)));
