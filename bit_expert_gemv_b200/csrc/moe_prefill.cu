@@ -32,7 +32,7 @@ namespace {
 constexpr int kTcM = 128;           // weight rows per tile (TMEM lanes)
 constexpr int kTcK = 64;            // K per stage: one 128-byte row of fp16 tokens
 constexpr int kTcStages = 4;
-constexpr int kTcExpWarps = 8;      // expander / epilogue warps: 2 per TMEM lane quarter
+constexpr int kTcExpWarps = 16;     // expander / epilogue warps: two groups of 8, 2 per TMEM lane quarter each
 constexpr int kTcThreads = (2 + kTcExpWarps) * 32;
 constexpr int kMaxOutliers = 82;    // per row: round(0.01 * 8192)
 constexpr uint32_t kSentinel = 0xFFFF0000u;
@@ -82,7 +82,7 @@ __host__ __device__ inline TcSmem tc_smem(int nmat, int chunk, int k) {
         s.srow[mt] = o;
         o += kTcM * 2;
         s.ent[mt] = o;
-        o += kTcM * (k + 4) * 4;
+        o += kTcM * (k + 2 * (nmat == 2 ? 2 : 4)) * 4;   // sub-lists of a row, each closed by two sentinels
     }
     // per expander warp, 16 words x 32 lanes of patched (outlier) words
     s.patch = o;
@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
     if (threadIdx.x == 0) {
         for (int s = 0; s < kTcStages; ++s) {
             mbar_init(b_full + s, 1);
-            mbar_init(a_full + s, kTcExpWarps * 32);
+            mbar_init(a_full + s, (NMAT == 2 ? kTcExpWarps : kTcExpWarps / 2) * 32);
             mbar_init(mma_done + s, 1);
         }
         mbar_init(acc_full, 1);
@@ -286,30 +286,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
             umma_commit(acc_full);
         }
     } else {
-        // ---------------- expanders: thread (row t, half h) covers 32 columns of every K-step
+        // ---------------- expanders: two groups of 8 warps; thread (row t, half h)
+        // of group G covers 32 columns of its K-steps.  For w1/w3 group G expands
+        // matrix G at every K-step; for w2 both groups expand the one matrix,
+        // group G at the K-steps of parity G.
         const int ew = warp - 2;
+        const int G = ew >> 3;
         const int quarter = warp & 3;   // TMEM lane quarter this warp may access
-        const int h = ew >> 2;
+        const int h = (ew >> 2) & 1;
         const int t = 32 * quarter + lane;
         const int row = r0 + t;
         const int nb = A.cols / 128;
+        const int mt = NMAT == 2 ? G : 0;
+        constexpr int NS = NMAT == 2 ? 2 : 4;   // outlier sub-lists per (row, matrix)
+        const int key = NMAT == 2 ? h : (h | (G << 1));
+        auto key_of = [](int c) { return NMAT == 2 ? ((c >> 5) & 1) : (((c >> 5) & 1) | (((c >> 6) & 1) << 1)); };
         bool ok = mbar_wait(side_full, 0);
-        // this thread's outliers in column order, as (column << 16 | fp16 value)
-        int cur[NMAT];
-        uint32_t ent[NMAT], nxt[NMAT];
-#pragma unroll
-        for (int mt = 0; mt < NMAT; ++mt) {
-            const uint16_t* sidx = reinterpret_cast<const uint16_t*>(smem + S.idx[mt]) + t * kout;
-            const uint8_t* sqv = smem + S.q[mt];
-            const float srow = __half2float(reinterpret_cast<const __half*>(smem + S.srow[mt])[t]);
-            uint32_t* list = reinterpret_cast<uint32_t*>(smem + S.ent[mt]) + t * (kout + 4);
-            int n0 = 0;
-            for (int j = 0; j < kout; ++j) n0 += ((sidx[j] >> 5) & 1) == 0;
-            const int start = h ? n0 + 2 : 0;   // each half ends in two sentinels
+        // this thread's outliers in column order, as (column << 16 | fp16 value):
+        // the row's sub-lists in key order, each closed by two sentinels
+        const uint16_t* sidx = reinterpret_cast<const uint16_t*>(smem + (mt ? S.idx[1] : S.idx[0])) + t * kout;
+        const uint8_t* sqv = smem + (mt ? S.q[1] : S.q[0]);
+        const float srow = __half2float(reinterpret_cast<const __half*>(smem + (mt ? S.srow[1] : S.srow[0]))[t]);
+        uint32_t* list = reinterpret_cast<uint32_t*>(smem + (mt ? S.ent[1] : S.ent[0])) + t * (kout + 2 * NS);
+        int start = 2 * key;
+        for (int j = 0; j < kout; ++j) start += key_of(sidx[j]) < key;
+        {
             int o = start;
             for (int j = 0; j < kout; ++j) {
                 const int c = sidx[j];
-                if (((c >> 5) & 1) != h) continue;
+                if (key_of(c) != key) continue;
                 const int n = t * kout + j;
                 const int byte = sqv[n >> 1];
                 int qv = (n & 1) ? (byte >> 4) : (byte & 0xF);
@@ -318,89 +323,67 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
             }
             list[o] = kSentinel;
             list[o + 1] = kSentinel;
-            cur[mt] = start;
-            ent[mt] = list[start];
-            nxt[mt] = list[start + 1];
         }
+        int cur = start;
+        uint32_t ent = list[start], nxt = list[start + 1];
         // Sign words and block scales arrive a group of kTcStages K-steps ahead:
         // two 16-byte loads hold the group's words of both halves, one 4-byte
         // load its two block scales.
-        const uint4* wsrc[NMAT];
-        const uint32_t* ssrc[NMAT];
-#pragma unroll
-        for (int mt = 0; mt < NMAT; ++mt) {
-            const MatView mv = make_view(rec + (mt ? A.off_b : A.off_a), A.rows, A.cols);
-            wsrc[mt] = reinterpret_cast<const uint4*>(mv.signs + int64_t(row) * (A.cols / 32));
-            ssrc[mt] = reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint16_t*>(mv.s_blk) + int64_t(row) * nb);
-        }
-        uint4 wa[NMAT], wb[NMAT];
-        uint32_t sp[NMAT];
-#pragma unroll
-        for (int mt = 0; mt < NMAT; ++mt) {
-            wa[mt] = __ldg(wsrc[mt]);
-            wb[mt] = __ldg(wsrc[mt] + 1);
-            sp[mt] = __ldg(ssrc[mt]);
-        }
+        const MatView mv = make_view(rec + (mt ? A.off_b : A.off_a), A.rows, A.cols);
+        const uint4* wsrc = reinterpret_cast<const uint4*>(mv.signs + int64_t(row) * (A.cols / 32));
+        const uint32_t* ssrc =
+            reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint16_t*>(mv.s_blk) + int64_t(row) * nb);
+        uint4 wa = __ldg(wsrc), wb = __ldg(wsrc + 1);
+        uint32_t sp = __ldg(ssrc);
         uint32_t* pw = reinterpret_cast<uint32_t*>(smem + S.patch) + ew * 512 + lane;   // this lane's column
         const int ng = nk / kTcStages;
         for (int g = 0; g < ng; ++g) {
-            uint32_t wg[NMAT][kTcStages], sg[NMAT][2];
-#pragma unroll
-            for (int mt = 0; mt < NMAT; ++mt) {
-                wg[mt][0] = h ? wa[mt].y : wa[mt].x;
-                wg[mt][1] = h ? wa[mt].w : wa[mt].z;
-                wg[mt][2] = h ? wb[mt].y : wb[mt].x;
-                wg[mt][3] = h ? wb[mt].w : wb[mt].z;
-                sg[mt][0] = sp[mt] & 0xFFFFu;
-                sg[mt][1] = sp[mt] >> 16;
-                if (g + 1 < ng) {
-                    wa[mt] = __ldg(wsrc[mt] + 2 * (g + 1));
-                    wb[mt] = __ldg(wsrc[mt] + 2 * (g + 1) + 1);
-                    sp[mt] = __ldg(ssrc[mt] + g + 1);
-                }
+            const uint32_t wg[kTcStages] = {h ? wa.y : wa.x, h ? wa.w : wa.z, h ? wb.y : wb.x, h ? wb.w : wb.z};
+            const uint32_t sg[2] = {sp & 0xFFFFu, sp >> 16};
+            if (g + 1 < ng) {
+                wa = __ldg(wsrc + 2 * (g + 1));
+                wb = __ldg(wsrc + 2 * (g + 1) + 1);
+                sp = __ldg(ssrc + g + 1);
             }
 #pragma unroll
             for (int s = 0; s < kTcStages; ++s) {
+                if (NMAT == 1 && (s & 1) != G) continue;
                 if (ok && g > 0 && !mbar_wait(mma_done + s, (g - 1) & 1)) ok = false;
                 tc_fence_after();
                 const int lo = (g * kTcStages + s) * kTcK + 32 * h, hi = lo + 32;
-#pragma unroll
-                for (int mt = 0; mt < NMAT; ++mt) {
-                    const uint32_t w = wg[mt][s], sc = sg[mt][s >> 1];
-                    uint32_t v[16];
-                    expand_signs(w, sc, v);
-                    // outliers of this range replace their weights: each lane
-                    // walks its own entries (the next one already loaded),
-                    // parks the patched words in its column of the warp's
-                    // patch area and marks them; a predicated load per word
-                    // then takes them in, with no per-outlier select over the
-                    // sixteen words
-                    const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + S.ent[mt]) + t * (kout + 4);
-                    uint32_t m = 0u;
-                    int prev_p = -1;
-                    uint32_t prev_a = 0u;
-                    while (int(ent[mt] >> 16) < hi) {
-                        const int u = int(ent[mt] >> 16) - lo;
-                        const int P = u >> 1;
-                        const uint32_t val = ent[mt] & 0xFFFFu;
-                        uint32_t other = sc ^ (((w >> (u ^ 1)) & 1u) << 15);
-                        if (P == prev_p) other = (u & 1) ? (prev_a & 0xFFFFu) : (prev_a >> 16);
-                        const uint32_t a = (u & 1) ? (other | (val << 16)) : (val | (other << 16));
-                        prev_p = P;
-                        prev_a = a;
-                        pw[P * 32] = a;
-                        m |= 1u << P;
-                        ent[mt] = nxt[mt];
-                        nxt[mt] = list[++cur[mt] + 1];
-                    }
-#pragma unroll
-                    for (int p = 0; p < 16; ++p)
-                        if ((m >> p) & 1u) v[p] = pw[p * 32];
-                    __syncwarp();
-                    tmem_st16(tmem + (uint32_t(32 * quarter) << 16) +
-                                  uint32_t(Cfg::acc_cols + s * Cfg::a_cols + mt * 32 + 16 * h),
-                              v);
+                const uint32_t w = wg[s], sc = sg[s >> 1];
+                uint32_t v[16];
+                expand_signs(w, sc, v);
+                // outliers of this range replace their weights: each lane
+                // walks its own entries (the next one already loaded),
+                // parks the patched words in its column of the warp's
+                // patch area and marks them; a predicated load per word
+                // then takes them in, with no per-outlier select over the
+                // sixteen words
+                uint32_t m = 0u;
+                int prev_p = -1;
+                uint32_t prev_a = 0u;
+                while (int(ent >> 16) < hi) {
+                    const int u = int(ent >> 16) - lo;
+                    const int P = u >> 1;
+                    const uint32_t val = ent & 0xFFFFu;
+                    uint32_t other = sc ^ (((w >> (u ^ 1)) & 1u) << 15);
+                    if (P == prev_p) other = (u & 1) ? (prev_a & 0xFFFFu) : (prev_a >> 16);
+                    const uint32_t a = (u & 1) ? (other | (val << 16)) : (val | (other << 16));
+                    prev_p = P;
+                    prev_a = a;
+                    pw[P * 32] = a;
+                    m |= 1u << P;
+                    ent = nxt;
+                    nxt = list[++cur + 1];
                 }
+#pragma unroll
+                for (int p = 0; p < 16; ++p)
+                    if ((m >> p) & 1u) v[p] = pw[p * 32];
+                __syncwarp();
+                tmem_st16(tmem + (uint32_t(32 * quarter) << 16) +
+                              uint32_t(Cfg::acc_cols + s * Cfg::a_cols + mt * 32 + 16 * h),
+                          v);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(a_full + s);
@@ -412,8 +395,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
         if (!ok) *fail = 1;
         tc_fence_after();
         if (ok) {
-            constexpr int kHalfCols = Cfg::chunk / 2;
-            for (int col = h * kHalfCols; col < h * kHalfCols + kHalfCols && col < n_mma; col += 16) {
+            constexpr int kQCols = Cfg::chunk / 4;   // each (group, half) takes a quarter of the tokens
+            const int q4 = h + 2 * G;
+            for (int col = q4 * kQCols; col < q4 * kQCols + kQCols && col < n_mma; col += 16) {
                 float v1[16], v3[16];
                 tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(col), v1);
                 if (NMAT == 2) tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(Cfg::chunk + col), v3);
