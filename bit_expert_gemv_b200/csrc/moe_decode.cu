@@ -906,6 +906,10 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_c
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x;
 
+    if (warp == kDecWarps && lane == 0) {   // the producer's descriptors, before the routing is known
+        prefetch_tensormap(&map13);
+        prefetch_tensormap(&map2);
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < P.n_stages; ++s) {
             mbar_init(full + s, 1);

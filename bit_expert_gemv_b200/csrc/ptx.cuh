@@ -94,6 +94,10 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
 
 // Named barrier over `count` threads (a multiple of 32).
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+// Bring a tensor map (a __grid_constant__ kernel parameter) into the TMA unit's descriptor cache.
+__device__ __forceinline__ void prefetch_tensormap(const void* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
 
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
