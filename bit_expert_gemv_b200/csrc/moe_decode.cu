@@ -610,7 +610,7 @@ __device__ __forceinline__ void chunk_mma(const uint8_t* signs, const __half* sb
     const uint8_t* pieces = (g < 3 ? tok[0].pieces : tok[1].pieces);
     const uint8_t* bsrc_p = bsrc ? pieces + (g % 3) * 128 + tig * 32 + ch * 8 * kPieceBlockBytes : nullptr;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
+#pragma unroll
     for (int hb = 0; hb < 2; ++hb) {
         uint32_t wg[4], wg8[4];
         uint4 q0[4], q1[4];
