@@ -781,6 +781,12 @@ __device__ __forceinline__ void epi_combine(const DecArgs& A, const RouteTables&
         // lane k holds the token's (k0 + k)-th (slot, gate); eight experts'
         // loads in flight at a time; the sum runs in fixed k order
         const int r0 = rb * 64 + lane, r1 = r0 + 32;
+        // the residual rows are loaded first, alongside the expert outputs
+        float x0 = 0.f, x1 = 0.f;
+        if (A.fuse_norm) {
+            if (r0 < d) x0 = bf16_to_f32(A.x[int64_t(t) * d + r0]);
+            if (r1 < d) x1 = bf16_to_f32(A.x[int64_t(t) * d + r1]);
+        }
         float y0 = 0.f, y1 = 0.f;
 #pragma unroll 1
         for (int k0 = 0; k0 < A.K; k0 += 32) {
@@ -819,12 +825,12 @@ __device__ __forceinline__ void epi_combine(const DecArgs& A, const RouteTables&
         }
         float ss = 0.f;
         if (r0 < d) {
-            const float v = bf16_to_f32(A.x[int64_t(t) * d + r0]) + y0;
+            const float v = x0 + y0;
             A.ws.v[int64_t(t) * d + r0] = v;
             ss = v * v;
         }
         if (r1 < d) {
-            const float v = bf16_to_f32(A.x[int64_t(t) * d + r1]) + y1;
+            const float v = x1 + y1;
             A.ws.v[int64_t(t) * d + r1] = v;
             ss = fmaf(v, v, ss);
         }
@@ -841,14 +847,12 @@ __device__ __forceinline__ void epi_combine(const DecArgs& A, const RouteTables&
         lastblk = __shfl_sync(0xffffffffu, lastblk, 0);
         if (!lastblk) continue;
         __threadfence();
-        float tot = 0.f;
-        for (int q = lane; q < comb_blocks; q += 32) tot += __ldcg(A.ws.ssq + t * comb_blocks + q);
-        tot = warp_sum(tot);
-        const float inv = rsqrtf(tot / float(d) + A.eps);
-        // sixteen 16-byte loads in flight per lane, then bf16 pairs out
+        // sixteen 16-byte loads of the row in flight per lane (the first
+        // batch together with the block sums of squares), then bf16 pairs out
         const float4* vrow = reinterpret_cast<const float4*>(A.ws.v + int64_t(t) * d);
         __nv_bfloat162* orow = reinterpret_cast<__nv_bfloat162*>(static_cast<uint16_t*>(A.out) + int64_t(t) * d);
         const int n4 = d / 4;
+        float inv = 0.f;
 #pragma unroll 1
         for (int c0 = 0; c0 < n4; c0 += 32 * 16) {
             float4 vv[16];
@@ -856,6 +860,12 @@ __device__ __forceinline__ void epi_combine(const DecArgs& A, const RouteTables&
             for (int j = 0; j < 16; ++j) {
                 const int c = c0 + 32 * j + lane;
                 vv[j] = c < n4 ? __ldcg(vrow + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            if (c0 == 0) {
+                float tot = 0.f;
+                for (int q = lane; q < comb_blocks; q += 32) tot += __ldcg(A.ws.ssq + t * comb_blocks + q);
+                tot = warp_sum(tot);
+                inv = rsqrtf(tot / float(d) + A.eps);
             }
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
