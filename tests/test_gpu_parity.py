@@ -205,8 +205,12 @@ def _moe(layer, bits, ids, gates, out_dtype=None, flags=0, eps=1e-6):
     return out, int(ws[:4].view(torch.int32).item())
 
 
-@pytest.mark.parametrize("B,K", [(1, 6), (5, 6), (33, 4), (2, 1), (70, 6)])
+@pytest.mark.parametrize("B,K", [(1, 6), (5, 6), (33, 4), (2, 1), (70, 6), (1, 16), (2, 16), (3, 10)])
 def test_moe_small(small_layer, B, K):
+    """Decode and prefill paths on a 16-expert layer: batch 1-2 (x rotated
+    while the routing runs), one-warp routing up to 32 pairs, block routing
+    above, and combines over K = 10 and 16 experts (more than one batch of
+    eight expert loads)."""
     L = small_layer
     bits, xv = gs.hidden_bf16(B, L.d_model, tag=B)
     ids, gates = gs.route_topk(gs.router_logits(B, L.E, tag=B), K)
@@ -227,6 +231,29 @@ def test_moe_fused_rmsnorm(small_layer):
     got = out.float().cpu().numpy()
     # the output itself is rounded to bf16 (relative 2^-9 per element)
     assert rel_l2(got, want) < 4e-3
+
+
+@pytest.mark.parametrize("B,K", [(1, 6), (2, 16)])
+def test_moe_fused_rmsnorm_small_batch(small_layer, B, K):
+    """Residual + RMSNorm through the decode kernel at batch 1-2 (the last
+    64-row block of a token normalises the row)."""
+    L = small_layer
+    bits, xv = gs.hidden_bf16(B, L.d_model, tag=88 + B)
+    ids, gates = gs.route_topk(gs.router_logits(B, L.E, tag=88 + B), K)
+    out, st = _moe(L, bits, ids, gates, out_dtype=torch.bfloat16, flags=G.GALE_FLAG_RESIDUAL_RMSNORM)
+    assert st == 0
+    want = O.chain_step(L.dense, xv, ids, gates)
+    assert rel_l2(out.float().cpu().numpy(), want) < 4e-3
+
+
+def test_moe_empty_batch(small_layer):
+    """B = 0: nothing to do, status 0."""
+    L = small_layer
+    bits = np.zeros((0, L.d_model), np.uint16)
+    ids = np.zeros((0, 6), np.int32)
+    gates = np.zeros((0, 6), np.float32)
+    out, st = _moe(L, bits, ids, gates)
+    assert st == 0 and out.shape == (0, L.d_model)
 
 
 def test_moe_bad_ids_status(small_layer):
