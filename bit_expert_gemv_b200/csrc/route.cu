@@ -13,13 +13,20 @@
 namespace gale {
 
 namespace {
-// Expert of pair p, or -1 when out of range or repeated earlier in its token.
-__device__ __forceinline__ int valid_expert(const RouteArgs& a, int p) {
-    const int e = a.ids[p];
-    if (e < 0 || e >= a.E) return -1;
+// Experts of the 32 pairs base .. base + 31 of a warp step (lane = pair), or
+// -1 past the range end, out of range, or repeated earlier in the token.  The
+// earlier pairs of a token (K <= 16) are in this step or the previous one:
+// `prev` holds the previous step's ids (its lane l = pair base - 32 + l).
+__device__ __forceinline__ int step_experts(const RouteArgs& a, int base, int end, int id, int prev) {
+    const int lane = threadIdx.x & 31, p = base + lane;
+    int e = (p < end && id >= 0 && id < a.E) ? id : -1;
     const int t0 = p - p % a.K;
-    for (int j = t0; j < p; ++j)
-        if (a.ids[j] == e) return -1;
+    for (int j = 1; j < a.K; ++j) {   // uniform trip count: every lane shuffles
+        const int q = p - j, src = q - base;
+        const int vc = __shfl_sync(0xffffffffu, id, src & 31), vp = __shfl_sync(0xffffffffu, prev, src & 31);
+        const int v = src >= 0 ? vc : vp;
+        if (q >= t0 && v == e) e = -1;
+    }
     return e;
 }
 }  // namespace
@@ -36,14 +43,22 @@ __global__ void __launch_bounds__(1024) route_permute_kernel(RouteArgs a) {
 
     for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
-    // pass 1: per-warp counts (and validation)
+    // pass 1: per-warp counts (and validation); the ids of the next step are
+    // loaded while this one is counted
+    int prev, id = p0 + lane < p1 ? a.ids[p0 + lane] : -1;
+    {
+        // the token of the range's first pair may start in the previous range
+        const int q = p0 - 32 + lane;
+        prev = (q >= 0 && q < BK && p0 < p1) ? a.ids[q] : -1;
+    }
+    const int prev0 = prev;
     for (int base = p0; base < p1; base += 32) {
         const int p = base + lane;
-        int e = -1;
-        if (p < p1) {
-            e = valid_expert(a, p);
-            if (e < 0) set_status(a.status, GALE_ERR_ARG);
-        }
+        const int nid = p + 32 < p1 ? a.ids[p + 32] : -1;
+        const int e = step_experts(a, base, p1, id, prev);
+        if (p < p1 && e < 0) set_status(a.status, GALE_ERR_ARG);
+        prev = id;
+        id = nid;
         const unsigned grp = __match_any_sync(0xffffffffu, e);
         if (e >= 0 && lane == __ffs(grp) - 1) wcnt[warp * E + e] += __popc(grp);
         __syncwarp();
@@ -87,9 +102,14 @@ __global__ void __launch_bounds__(1024) route_permute_kernel(RouteArgs a) {
     }
     __syncthreads();
     // pass 2: placement in pair order
+    prev = prev0;
+    id = p0 + lane < p1 ? a.ids[p0 + lane] : -1;
     for (int base = p0; base < p1; base += 32) {
         const int p = base + lane;
-        const int e = p < p1 ? valid_expert(a, p) : -1;
+        const int nid = p + 32 < p1 ? a.ids[p + 32] : -1;
+        const int e = step_experts(a, base, p1, id, prev);
+        prev = id;
+        id = nid;
         const unsigned grp = __match_any_sync(0xffffffffu, e);
         if (e >= 0) {
             const int pos = wcnt[warp * E + e] + __popc(grp & ((1u << lane) - 1u));
