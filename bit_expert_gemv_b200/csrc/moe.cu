@@ -89,23 +89,54 @@ __global__ void __launch_bounds__(256) moe_group_gemv_kernel(GroupArgs g) {
 
 // One CTA per token: y = sum_k gates[t,k] * o[pos(t,k)] in fixed k order,
 // then either stored, or v = x + y normalised (RMSNorm, unit weight) to bf16.
+// The token's slots and gates are read once into shared memory; each thread
+// takes four consecutive columns at a time with all K loads in flight.
 __global__ void __launch_bounds__(256) moe_combine_kernel(CombineArgs c) {
-    extern __shared__ float red[];
+    __shared__ int spos[16];
+    __shared__ float sg[16];
+    __shared__ float red[32];
     const int t = blockIdx.x;
-    const int d = c.d_model;
+    const int d = c.d_model, n4 = d / 4;
+    if (threadIdx.x < c.K) {
+        spos[threadIdx.x] = c.pos_of_pair[t * c.K + threadIdx.x];
+        sg[threadIdx.x] = c.gates[t * c.K + threadIdx.x];
+    }
+    __syncthreads();
     float ss = 0.f;
-    for (int i = threadIdx.x; i < d; i += blockDim.x) {
-        float y = 0.f;
-        for (int k = 0; k < c.K; ++k) {
-            const int pos = c.pos_of_pair[t * c.K + k];
-            if (pos >= 0) y = fmaf(c.gates[t * c.K + k], c.o[int64_t(pos) * d + i], y);
+    for (int i4 = threadIdx.x; i4 < n4; i4 += blockDim.x) {
+        float4 ov[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            ov[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (k < c.K && spos[k] >= 0) ov[k] = __ldcs(reinterpret_cast<const float4*>(c.o + int64_t(spos[k]) * d) + i4);
         }
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            if (k >= c.K) break;
+            const float g = spos[k] >= 0 ? sg[k] : 0.f;
+            y.x = fmaf(g, ov[k].x, y.x);
+            y.y = fmaf(g, ov[k].y, y.y);
+            y.z = fmaf(g, ov[k].z, y.z);
+            y.w = fmaf(g, ov[k].w, y.w);
+        }
+        const int64_t e = int64_t(t) * d + 4 * i4;
         if (c.fuse_norm) {
-            const float v = bf16_to_f32(c.x[int64_t(t) * d + i]) + y;
-            c.scratch[int64_t(t) * d + i] = v;
-            ss = fmaf(v, v, ss);
+            // x is only known to be 4-byte aligned: two 32-bit loads
+            const uint32_t x01 = *reinterpret_cast<const uint32_t*>(c.x + e);
+            const uint32_t x23 = *reinterpret_cast<const uint32_t*>(c.x + e + 2);
+            const float4 v = make_float4(bf16_to_f32(uint16_t(x01)) + y.x, bf16_to_f32(uint16_t(x01 >> 16)) + y.y,
+                                         bf16_to_f32(uint16_t(x23)) + y.z, bf16_to_f32(uint16_t(x23 >> 16)) + y.w);
+            reinterpret_cast<float4*>(c.scratch + int64_t(t) * d)[i4] = v;
+            ss = fmaf(v.x, v.x, ss);
+            ss = fmaf(v.y, v.y, ss);
+            ss = fmaf(v.z, v.z, ss);
+            ss = fmaf(v.w, v.w, ss);
         } else {
-            store_from_f32(c.out, c.out_dtype, int64_t(t) * d + i, y);
+            store_from_f32(c.out, c.out_dtype, e, y.x);
+            store_from_f32(c.out, c.out_dtype, e + 1, y.y);
+            store_from_f32(c.out, c.out_dtype, e + 2, y.z);
+            store_from_f32(c.out, c.out_dtype, e + 3, y.w);
         }
     }
     if (!c.fuse_norm) return;
@@ -119,8 +150,15 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(CombineArgs c) {
     }
     __syncthreads();
     const float inv = rsqrtf(red[0] / float(d) + c.eps);
-    for (int i = threadIdx.x; i < d; i += blockDim.x)
-        store_from_f32(c.out, GALE_BF16, int64_t(t) * d + i, c.scratch[int64_t(t) * d + i] * inv);
+    uint16_t* out = static_cast<uint16_t*>(c.out);
+    for (int i4 = threadIdx.x; i4 < n4; i4 += blockDim.x) {
+        const float4 v = reinterpret_cast<const float4*>(c.scratch + int64_t(t) * d)[i4];
+        const int64_t e = int64_t(t) * d + 4 * i4;
+        out[e] = f32_to_bf16(v.x * inv);
+        out[e + 1] = f32_to_bf16(v.y * inv);
+        out[e + 2] = f32_to_bf16(v.z * inv);
+        out[e + 3] = f32_to_bf16(v.w * inv);
+    }
 }
 
 int launch_moe_combine(const float* o, const int32_t* pos_of_pair, const float* gates, const uint16_t* x, int B,
@@ -138,7 +176,8 @@ int launch_moe_combine(const float* o, const int32_t* pos_of_pair, const float* 
     c.fuse_norm = fuse_norm;
     c.eps = eps;
     c.scratch = scratch;
-    moe_combine_kernel<<<B, 256, 32 * sizeof(float), st>>>(c);
+    if (K > 16 || d_model % 4 != 0) return GALE_ERR_UNSUPPORTED;
+    moe_combine_kernel<<<B, 256, 0, st>>>(c);
     GALE_LAUNCH_CHECK();
     return GALE_OK;
 }
