@@ -30,6 +30,7 @@ EXPORTS = (
     "gale_status_string", "gale_pack_layout", "gale_expert_bytes", "gale_pack", "gale_unpack",
     "gale_fwht1024", "gale_expert_gemv", "gale_route_permute", "gale_moe_workspace_size",
     "gale_moe_forward", "gale_moe_forward_noalloc", "gale_selftest_scratch_bytes", "gale_selftest",
+    "gale_moe_host_staging_bytes", "gale_moe_host_workspace_size", "gale_moe_forward_host",
 )
 
 GALE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -83,6 +84,10 @@ def lib() -> ctypes.CDLL:
                                        ctypes.c_float, vp, sz, vp]),
             "gale_moe_forward_noalloc": (i32, [ctypes.POINTER(gale_layer), vp, vp, vp, i32, i32, vp, i32, i32,
                                                ctypes.c_float, vp, vp]),
+            "gale_moe_host_staging_bytes": (sz, [i32, i32, i32]),
+            "gale_moe_host_workspace_size": (sz, [ctypes.POINTER(gale_layer), i32, i32]),
+            "gale_moe_forward_host": (i32, [ctypes.POINTER(gale_layer), vp, vp, vp, i32, i32, vp, i32, i32,
+                                            ctypes.c_float, vp, sz, vp, sz, vp]),
             "gale_selftest_scratch_bytes": (sz, []),
             "gale_selftest": (i32, [vp, vp]),
         }
@@ -195,6 +200,28 @@ def gale_moe_forward_noalloc(layer: gale_layer, x, ids, gates, out, status=None,
     _check(lib().gale_moe_forward_noalloc(ctypes.byref(layer), _ptr(x), _ptr(ids), _ptr(gates), B, K,
                                           _ptr(out), _dtype_code(out), flags, eps, _ptr(status),
                                           _stream(stream)), "gale_moe_forward_noalloc")
+
+
+def gale_moe_host_staging_bytes(B: int, K: int, d_model: int) -> int:
+    return int(lib().gale_moe_host_staging_bytes(B, K, d_model))
+
+
+def gale_moe_host_workspace_size(layer: gale_layer, B: int, K: int) -> int:
+    return int(lib().gale_moe_host_workspace_size(ctypes.byref(layer), B, K))
+
+
+def gale_moe_forward_host(layer: gale_layer, x, ids, gates, out, ws, staging, flags: int = 0,
+                          eps: float = 1e-6, stream=None):
+    """gale_moe_forward with x, ids, gates in host memory and out in pinned
+    host memory; `staging` is a pinned host byte tensor of at least
+    gale_moe_host_staging_bytes() bytes, `ws` a device workspace of at least
+    gale_moe_host_workspace_size() bytes.  Asynchronous: synchronise the
+    stream before reading `out` or refilling `staging`."""
+    B, K = ids.shape
+    _check(lib().gale_moe_forward_host(ctypes.byref(layer), _ptr(x), _ptr(ids), _ptr(gates), B, K, _ptr(out),
+                                       _dtype_code(out), flags, eps, _ptr(ws), ws.numel() * ws.element_size(),
+                                       _ptr(staging), staging.numel() * staging.element_size(), _stream(stream)),
+           "gale_moe_forward_host")
 
 
 def gale_selftest_scratch_bytes() -> int:

@@ -236,6 +236,34 @@ int gale_moe_forward_noalloc(const gale_layer* layer, const uint16_t* x, const i
                              const float* gates, int B, int K, void* out, int out_dtype, int flags,
                              float eps, int32_t* status, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * gale_moe_forward with the inputs and the result in host memory.  An
+ * interface addition of this library, with no counterpart on the GALE cards:
+ * a decode step moves a few kilobytes but pays a fixed cost per transfer, so
+ * the inputs cross in one copy and a small result is written in place.
+ *
+ * Same computation, flags and errors as gale_moe_forward, except:
+ *  - x, ids, gates: host memory of any kind (the call copies them, with the
+ *    CPU, into `staging`, then moves `staging` to the device in one copy);
+ *  - staging: pinned host memory (cudaHostAlloc / cudaMallocHost), 16-byte
+ *    aligned, at least gale_moe_host_staging_bytes(B, K, d_model) bytes,
+ *    owned by the caller; it must not be written again until the stream has
+ *    passed this call;
+ *  - out: pinned host memory (or device memory) of out_dtype [B][d_model].
+ *    A result of up to 1 MiB is written there by the layer's kernels; a
+ *    larger one goes through the workspace and one device-to-host copy.  The
+ *    result is complete once the stream has passed this call;
+ *  - ws: device workspace of at least gale_moe_host_workspace_size() bytes
+ *    (the status word is its first int32, as for gale_moe_forward).
+ * Pageable staging or out returns GALE_ERR_ARG.  Asynchronous on `stream`.
+ * ------------------------------------------------------------------------- */
+size_t gale_moe_host_staging_bytes(int B, int K, int d_model);
+size_t gale_moe_host_workspace_size(const gale_layer* layer, int B, int K);
+int gale_moe_forward_host(const gale_layer* layer, const uint16_t* x, const int32_t* ids,
+                          const float* gates, int B, int K, void* out, int out_dtype, int flags,
+                          float eps, void* ws, size_t ws_bytes, void* staging, size_t staging_bytes,
+                          void* stream);
+
 /* Built-in parity self-check on tiny shapes (the card's "optional fast paths
  * verify themselves at startup" -- without any fallback).  Synchronous:
  * allocates nothing itself but needs `scratch` of gale_selftest_scratch_bytes()

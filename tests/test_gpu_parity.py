@@ -256,6 +256,41 @@ def test_moe_empty_batch(small_layer):
     assert st == 0 and out.shape == (0, L.d_model)
 
 
+@pytest.mark.parametrize("B,K,fused", [(1, 6, False), (2, 16, True), (200, 6, False)])
+def test_moe_forward_host_matches_device(small_layer, B, K, fused):
+    """Host-buffer entry point: one packed input copy, the result written into
+    pinned host memory (or copied back when over 1 MiB, B = 200); bit-identical
+    to the device-buffer call."""
+    L = small_layer
+    bits, _ = gs.hidden_bf16(B, L.d_model, tag=300 + B)
+    ids, gates = gs.route_topk(gs.router_logits(B, L.E, tag=300 + B), K)
+    flags = G.GALE_FLAG_RESIDUAL_RMSNORM if fused else 0
+    dt = torch.bfloat16 if fused else torch.float32
+    want, st = _moe(L, bits, ids, gates, out_dtype=dt, flags=flags)
+    assert st == 0
+    x_h = torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16)
+    ids_h, gates_h = torch.from_numpy(ids), torch.from_numpy(gates)
+    staging = torch.empty(G.gale_moe_host_staging_bytes(B, K, L.d_model), dtype=torch.uint8).pin_memory()
+    ws = torch.empty(G.gale_moe_host_workspace_size(L.desc, B, K), dtype=torch.uint8, device="cuda")
+    out_h = torch.empty(B, L.d_model, dtype=dt).pin_memory()
+    G.gale_moe_forward_host(L.desc, x_h, ids_h, gates_h, out_h, ws, staging, flags=flags)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    assert torch.equal(out_h, want.cpu())
+
+
+def test_moe_forward_host_rejects_pageable_output(small_layer):
+    L = small_layer
+    bits, _ = gs.hidden_bf16(1, L.d_model, tag=5)
+    ids, gates = gs.route_topk(gs.router_logits(1, L.E, tag=5), 6)
+    staging = torch.empty(G.gale_moe_host_staging_bytes(1, 6, L.d_model), dtype=torch.uint8).pin_memory()
+    ws = torch.empty(G.gale_moe_host_workspace_size(L.desc, 1, 6), dtype=torch.uint8, device="cuda")
+    out_pageable = torch.empty(1, L.d_model, dtype=torch.float32)
+    with pytest.raises(G.GaleError):
+        G.gale_moe_forward_host(L.desc, torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16),
+                                torch.from_numpy(ids), torch.from_numpy(gates), out_pageable, ws, staging)
+
+
 def test_moe_bad_ids_status(small_layer):
     L = small_layer
     bits, _ = gs.hidden_bf16(2, L.d_model, tag=5)
