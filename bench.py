@@ -61,6 +61,25 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(values, world, device):
+    """Per-rank device times -> their maximum over all ranks (every rank gets
+    it).  One all-reduce, the same on every rank, whatever the backend."""
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return [float(v) for v in tt.tolist()]
+
+
+def job_throughput(batch, steps, world, t_max):
+    """Whole-job tokens and tokens/s: every rank is an independent replica
+    running `steps` steps of `batch` tokens; the job takes the slowest
+    rank's time."""
+    tokens = batch * steps * world
+    return tokens, tokens / t_max
+
+
 # ----------------------------------------------------------------------------
 # clocks sampling (nvidia-smi during the timed region)
 # ----------------------------------------------------------------------------
@@ -322,12 +341,8 @@ def run_gpu(args):
     clocks_info = clocks.stop()
 
     # max over ranks of the device time
-    tt = torch.tensor([t1, t8, te, tp, tc], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    t1, t8, te, tp, tc = [float(v) for v in tt.tolist()]
-    tokens = 1 * args.steps * world
-    value = tokens / t1
+    t1, t8, te, tp, tc = max_over_ranks([t1, t8, te, tp, tc], world, "cuda")
+    tokens, value = job_throughput(1, args.steps, world, t1)
     gbs = bytes1 * world / t1 / 1e9
     peak, tpeak, peak_kind = peaks()
     pf_flops = 2.0 * PREFILL_B * TOP_K * 3 * D_FF * D_MODEL   # dense-equivalent, per layer
