@@ -966,8 +966,10 @@ __global__ void __launch_bounds__(kDecBlock, 1) moe_decode_kernel(const __grid_c
     // contiguous job ranges of this CTA in both phases; the producer decodes
     // its jobs as it goes, the other warps read them from a table
     const int J13 = R.n_groups * P.s13.row_blocks, J2 = R.n_groups * P.s2.row_blocks;
-    const int a0 = int((int64_t(J13) * blockIdx.x) / G), n13 = int((int64_t(J13) * (blockIdx.x + 1)) / G) - a0;
-    const int b0 = int((int64_t(J2) * blockIdx.x) / G), n2 = int((int64_t(J2) * (blockIdx.x + 1)) / G) - b0;
+    // (J * G < 2^32: at most 384 groups x 256 row blocks x the SM count; 32-bit divisions)
+    const unsigned g = unsigned(G), bx = blockIdx.x;
+    const int a0 = int(unsigned(J13) * bx / g), n13 = int(unsigned(J13) * (bx + 1) / g) - a0;
+    const int b0 = int(unsigned(J2) * bx / g), n2 = int(unsigned(J2) * (bx + 1) / g) - b0;
     uint2* jobs = reinterpret_cast<uint2*>(smem + S.jobs);
     if (warp < kDecWarps)
         for (int i = threadIdx.x; i < n13 + n2; i += kDecThreads)
