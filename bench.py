@@ -39,7 +39,7 @@ CHAIN_LAYERS = 43
 DECODE_LAUNCHES = 1
 # dram read + write bytes of one decode launch at this workload, from an ncu
 # capture of the current kernel (None once the kernel has changed since)
-DECODE_TRAFFIC = 25_196_544
+DECODE_TRAFFIC = 25_196_800
 WORKLOAD = ("moe_layer_decode: 256 GALE-1bit experts (w1/w3 [2048x4096], w2 [4096x2048]), "
             "top-6 softmax routing, bf16 hidden [B x 4096]")
 
