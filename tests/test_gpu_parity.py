@@ -291,6 +291,20 @@ def test_moe_forward_host_rejects_pageable_output(small_layer):
                                 torch.from_numpy(ids), torch.from_numpy(gates), out_pageable, ws, staging)
 
 
+def test_moe_general_path_wide_ff():
+    """d_ff = 16384: more outliers per w2 row (164) than the tile path stages
+    and wider than the decode kernel takes, so the layer runs on the general
+    kernels (routing permute, FWHT, grouped GEMVs, combine)."""
+    L = Layer(2, 1024, 16384, layer=2)
+    for B, K in [(1, 2), (3, 1)]:
+        bits, xv = gs.hidden_bf16(B, L.d_model, tag=500 + B)
+        ids, gates = gs.route_topk(gs.router_logits(B, L.E, tag=500 + B), K)
+        out, st = _moe(L, bits, ids, gates)
+        assert st == 0
+        want = O.moe_layer(L.dense, xv, ids, gates)
+        assert rel_l2(out.cpu().numpy(), want) < REL_L2_TOL
+
+
 def test_moe_bad_ids_status(small_layer):
     L = small_layer
     bits, _ = gs.hidden_bf16(2, L.d_model, tag=5)
