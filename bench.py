@@ -21,6 +21,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -92,7 +93,8 @@ class Clocks:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = os.path.join(os.environ.get("GALE_CLOCKS_DIR", tempfile.gettempdir()),
+                                 f"gale_clocks_rank{index}.csv")
 
     def start(self):
         try:
