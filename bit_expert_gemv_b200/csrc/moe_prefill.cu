@@ -301,6 +301,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
         constexpr int NS = NMAT == 2 ? 2 : 4;   // outlier sub-lists per (row, matrix)
         const int key = NMAT == 2 ? h : (h | (G << 1));
         auto key_of = [](int c) { return NMAT == 2 ? ((c >> 5) & 1) : (((c >> 5) & 1) | (((c >> 6) & 1) << 1)); };
+        // Sign words and block scales arrive a group of kTcStages K-steps ahead:
+        // two 16-byte loads hold the group's words of both halves, one 4-byte
+        // load its two block scales.  The first group is requested before the
+        // outlier sections have landed.
+        const MatView mv = make_view(rec + (mt ? A.off_b : A.off_a), A.rows, A.cols);
+        const uint4* wsrc = reinterpret_cast<const uint4*>(mv.signs + int64_t(row) * (A.cols / 32));
+        const uint32_t* ssrc =
+            reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint16_t*>(mv.s_blk) + int64_t(row) * nb);
+        uint4 wa = __ldg(wsrc), wb = __ldg(wsrc + 1);
+        uint32_t sp = __ldg(ssrc);
         bool ok = mbar_wait(side_full, 0);
         // this thread's outliers in column order, as (column << 16 | fp16 value):
         // the row's sub-lists in key order, each closed by two sentinels
@@ -326,15 +336,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
         }
         int cur = start;
         uint32_t ent = list[start], nxt = list[start + 1];
-        // Sign words and block scales arrive a group of kTcStages K-steps ahead:
-        // two 16-byte loads hold the group's words of both halves, one 4-byte
-        // load its two block scales.
-        const MatView mv = make_view(rec + (mt ? A.off_b : A.off_a), A.rows, A.cols);
-        const uint4* wsrc = reinterpret_cast<const uint4*>(mv.signs + int64_t(row) * (A.cols / 32));
-        const uint32_t* ssrc =
-            reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint16_t*>(mv.s_blk) + int64_t(row) * nb);
-        uint4 wa = __ldg(wsrc), wb = __ldg(wsrc + 1);
-        uint32_t sp = __ldg(ssrc);
         uint32_t* pw = reinterpret_cast<uint32_t*>(smem + S.patch) + ew * 512 + lane;   // this lane's column
         const int ng = nk / kTcStages;
         for (int g = 0; g < ng; ++g) {
@@ -406,7 +407,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
                     for (int i = 0; i < 16; ++i) {
                         const int j = col + i;
                         if (j < job.n) {
-                            const float y = NMAT == 2 ? silu(v1[i]) * v3[i] : v1[i];
+                            const float y = NMAT == 2 ? __fdividef(v1[i], 1.0f + __expf(-v1[i])) * v3[i] : v1[i];
                             A.out[int64_t(job.n0 + j) * A.rows + row] = y;
                         }
                     }
