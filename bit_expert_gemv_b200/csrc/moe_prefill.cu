@@ -37,13 +37,12 @@ constexpr int kTcThreads = (2 + kTcExpWarps) * 32;
 constexpr int kMaxOutliers = 82;    // per row: round(0.01 * 8192)
 constexpr uint32_t kSentinel = 0xFFFF0000u;
 
-template <int NMAT>
-struct TcCfg {
-    static constexpr int chunk = NMAT == 2 ? 128 : 256;   // tokens per job (MMA N)
-    static constexpr int acc_cols = NMAT * chunk;         // fp32 accumulator columns
-    static constexpr int a_cols = NMAT * 32;              // TMEM columns of one A stage
-    static_assert(acc_cols + kTcStages * a_cols <= 512, "TMEM budget");
-};
+// Every job multiplies two A operands by one token chunk: w1 and w3 over the
+// same 128 rows (SwiGLU epilogue), or two consecutive 128-row tiles of w2.
+constexpr int kTcChunk = 128;                  // tokens per job (MMA N)
+constexpr int kTcAccCols = 2 * kTcChunk;       // fp32 accumulator columns, one block per operand
+constexpr int kTcACols = 2 * 32;               // TMEM columns of one A stage (both operands)
+static_assert(kTcAccCols + kTcStages * kTcACols <= 512, "TMEM budget");
 
 struct TcJob {
     int e, n0, n;   // expert, first slot of the chunk, tokens in the chunk
@@ -66,15 +65,13 @@ struct TcSmem {
 
 __host__ __device__ inline int align16(int n) { return (n + 15) & ~15; }
 
-// Shared memory: the token ring, then per matrix the tile's outlier sections
+// Shared memory: the token ring, then per operand the tile's outlier sections
 // (bulk copies) and the outlier lists split by 32-column half.
-__host__ __device__ inline TcSmem tc_smem(int nmat, int chunk, int k) {
+__host__ __device__ inline TcSmem tc_smem(int k) {
     TcSmem s;
     s.b = 0;
-    int o = kTcStages * chunk * 128;
+    int o = kTcStages * kTcChunk * 128;
     for (int mt = 0; mt < 2; ++mt) {
-        s.idx[mt] = s.q[mt] = s.srow[mt] = s.ent[mt] = o;
-        if (mt >= nmat) continue;
         s.idx[mt] = o;
         o += align16(kTcM * k * 2);
         s.q[mt] = o;
@@ -82,7 +79,7 @@ __host__ __device__ inline TcSmem tc_smem(int nmat, int chunk, int k) {
         s.srow[mt] = o;
         o += kTcM * 2;
         s.ent[mt] = o;
-        o += kTcM * (k + 2 * (nmat == 2 ? 2 : 4)) * 4;   // sub-lists of a row, each closed by two sentinels
+        o += kTcM * (k + 2 * 2) * 4;   // the two sub-lists of a row, each closed by two sentinels
     }
     // per expander warp, 16 words x 32 lanes of patched (outlier) words
     s.patch = o;
@@ -100,44 +97,34 @@ int act_map(CUtensorMap* m, const void* base, int cols, int64_t rows, int box_ro
                        uint64_t(cols) * 2 * uint64_t(rows), 64, uint32_t(box_rows), true);
 }
 
-// Both job lists (chunks of 128 and of 256 slots), one thread per expert.
+// The job list: every expert's slots in chunks of kTcChunk, one thread per expert.
 __global__ void __launch_bounds__(1024) prefill_jobs_kernel(const int32_t* counts, const int32_t* offsets, int E,
-                                                            TcJob* jobs13, int32_t* n13, TcJob* jobs2,
-                                                            int32_t* n2) {
+                                                            TcJob* jobs, int32_t* n_jobs) {
     __shared__ int tmp[32];
-    __shared__ int tot[2];
     const int e = threadIdx.x;
     const int lane = e & 31, warp = e >> 5;
     const int n_e = e < E ? counts[e] : 0;
-    for (int which = 0; which < 2; ++which) {
-        const int chunk = which ? 256 : 128;
-        const int c = (n_e + chunk - 1) / chunk;
-        int incl = c;
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        if (lane == 31) tmp[warp] = incl;
-        __syncthreads();
-        if (e == 0) {
-            int run = 0;
-            for (int w = 0; w < int(blockDim.x >> 5); ++w) {
-                const int v = tmp[w];
-                tmp[w] = run;
-                run += v;
-            }
-            tot[which] = run;
-        }
-        __syncthreads();
-        const int first = tmp[warp] + incl - c;
-        TcJob* jobs = which ? jobs2 : jobs13;
-        for (int i = 0; i < c; ++i) jobs[first + i] = TcJob{e, offsets[e] + i * chunk, min(chunk, n_e - i * chunk)};
-        __syncthreads();
+    const int c = (n_e + kTcChunk - 1) / kTcChunk;
+    int incl = c;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
     }
+    if (lane == 31) tmp[warp] = incl;
+    __syncthreads();
     if (e == 0) {
-        *n13 = tot[0];
-        *n2 = tot[1];
+        int run = 0;
+        for (int w = 0; w < int(blockDim.x >> 5); ++w) {
+            const int v = tmp[w];
+            tmp[w] = run;
+            run += v;
+        }
+        *n_jobs = run;
     }
+    __syncthreads();
+    const int first = tmp[warp] + incl - c;
+    for (int i = 0; i < c; ++i)
+        jobs[first + i] = TcJob{e, offsets[e] + i * kTcChunk, min(kTcChunk, n_e - i * kTcChunk)};
 }
 
 // x of every pair in permuted order, rotated, as fp16: one warp per (token,
@@ -187,12 +174,13 @@ __device__ __forceinline__ void expand_signs(uint32_t w, uint32_t sc, uint32_t (
     }
 }
 
-// One (128-row tile, token chunk) job of w1/w3 (NMAT = 2, SwiGLU epilogue) or
-// w2 (NMAT = 1).  Warp 0 streams token tiles by TMA, warp 1 owns TMEM and
-// issues the MMAs, warps 2..9 expand weights into TMEM and run the epilogue.
-template <int NMAT>
+// One (rows, token chunk) job: w1 and w3 over one 128-row tile with the
+// SwiGLU epilogue (GLU), or two consecutive 128-row tiles of w2.  Warp 0
+// streams token tiles by TMA, warp 1 owns TMEM and issues the MMAs, warps
+// 2..17 expand weights into TMEM and run the epilogue.
+template <bool GLU>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_constant__ CUtensorMap xmap, TcArgs A) {
-    using Cfg = TcCfg<NMAT>;
+    constexpr int kRowsPerCta = GLU ? kTcM : 2 * kTcM;   // rows of the streamed matrix per CTA
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_align1024(smem_raw);
     const int mtile = blockIdx.x, job_id = blockIdx.y;
@@ -200,7 +188,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
     const TcJob job = A.jobs[job_id];
     const int nk = A.cols / kTcK;
     const int kout = outliers_per_row(A.cols);
-    const TcSmem S = tc_smem(NMAT, Cfg::chunk, kout);
+    const TcSmem S = tc_smem(kout);
     uint64_t* b_full = reinterpret_cast<uint64_t*>(smem + S.bars);
     uint64_t* a_full = b_full + kTcStages;
     uint64_t* mma_done = a_full + kTcStages;
@@ -211,13 +199,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_mma = (job.n + 15) & ~15;
     const uint32_t idesc = umma_idesc_f16(kTcM, n_mma);
-    const int r0 = mtile * kTcM;
+    const int r0 = mtile * kRowsPerCta;
     const char* rec = A.base + int64_t(job.e) * A.stride;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kTcStages; ++s) {
             mbar_init(b_full + s, 1);
-            mbar_init(a_full + s, (NMAT == 2 ? kTcExpWarps : kTcExpWarps / 2) * 32);
+            mbar_init(a_full + s, kTcExpWarps * 32);
             mbar_init(mma_done + s, 1);
         }
         mbar_init(acc_full, 1);
@@ -238,12 +226,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
         // ---------------- producer: the tile's outlier sections, then token tiles
         if (lane == 0) {
             const uint32_t idx_bytes = uint32_t(kTcM * kout * 2), q_bytes = uint32_t(kTcM * kout / 2);
-            mbar_arrive_expect_tx(side_full, uint32_t(NMAT) * (idx_bytes + q_bytes + kTcM * 2));
-            for (int mt = 0; mt < NMAT; ++mt) {
+            mbar_arrive_expect_tx(side_full, 2u * (idx_bytes + q_bytes + kTcM * 2));
+            for (int mt = 0; mt < 2; ++mt) {
                 const MatView mv = make_view(rec + (mt ? A.off_b : A.off_a), A.rows, A.cols);
-                bulk_load(smem + S.idx[mt], mv.idx + int64_t(r0) * kout, idx_bytes, side_full);
-                bulk_load(smem + S.q[mt], mv.q + int64_t(r0) * kout / 2, q_bytes, side_full);
-                bulk_load(smem + S.srow[mt], mv.s_row + r0, kTcM * 2, side_full);
+                const int rm = r0 + (GLU ? 0 : mt * kTcM);   // first row of operand mt
+                bulk_load(smem + S.idx[mt], mv.idx + int64_t(rm) * kout, idx_bytes, side_full);
+                bulk_load(smem + S.q[mt], mv.q + int64_t(rm) * kout / 2, q_bytes, side_full);
+                bulk_load(smem + S.srow[mt], mv.s_row + rm, kTcM * 2, side_full);
             }
             int issued = 0;
             for (int ks = 0; ks < nk; ++ks) {
@@ -252,8 +241,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
                     *fail = 1;
                     break;
                 }
-                mbar_arrive_expect_tx(b_full + s, uint32_t(Cfg::chunk * 128));
-                tma_load_3d(smem + S.b + s * Cfg::chunk * 128, &xmap, b_full + s, ks * kTcK, job.n0, 0);
+                mbar_arrive_expect_tx(b_full + s, uint32_t(kTcChunk * 128));
+                tma_load_3d(smem + S.b + s * kTcChunk * 128, &xmap, b_full + s, ks * kTcK, job.n0, 0);
                 issued = ks + 1;
             }
             // no copy may still be landing when the CTA exits
@@ -272,13 +261,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
                     break;
                 }
                 tc_fence_after();
-                const uint32_t bst = smem_u32(smem + S.b + s * Cfg::chunk * 128);
-                const uint32_t ast = tmem + uint32_t(Cfg::acc_cols + s * Cfg::a_cols);
+                const uint32_t bst = smem_u32(smem + S.b + s * kTcChunk * 128);
+                const uint32_t ast = tmem + uint32_t(kTcAccCols + s * kTcACols);
 #pragma unroll
-                for (int mt = 0; mt < NMAT; ++mt) {
+                for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
                     for (int kk = 0; kk < kTcK / 16; ++kk)
-                        umma_f16_ts(tmem + uint32_t(mt * Cfg::chunk), ast + uint32_t(mt * 32 + kk * 8),
+                        umma_f16_ts(tmem + uint32_t(mt * kTcChunk), ast + uint32_t(mt * 32 + kk * 8),
                                     umma_desc_sw128(bst + kk * 32), idesc, (ks > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(mma_done + s);
@@ -286,21 +275,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
             umma_commit(acc_full);
         }
     } else {
-        // ---------------- expanders: two groups of 8 warps; thread (row t, half h)
-        // of group G covers 32 columns of its K-steps.  For w1/w3 group G expands
-        // matrix G at every K-step; for w2 both groups expand the one matrix,
-        // group G at the K-steps of parity G.
+        // ---------------- expanders: two groups of 8 warps; group G expands
+        // operand G (w1 / w3, or the first / second 128-row tile of w2) and
+        // its thread (row t, half h) the 32 columns of half h of every K-step.
         const int ew = warp - 2;
         const int G = ew >> 3;
         const int quarter = warp & 3;   // TMEM lane quarter this warp may access
         const int h = (ew >> 2) & 1;
         const int t = 32 * quarter + lane;
-        const int row = r0 + t;
+        const int mt = G;
+        const int row = r0 + (GLU ? 0 : mt * kTcM) + t;
         const int nb = A.cols / 128;
-        const int mt = NMAT == 2 ? G : 0;
-        constexpr int NS = NMAT == 2 ? 2 : 4;   // outlier sub-lists per (row, matrix)
-        const int key = NMAT == 2 ? h : (h | (G << 1));
-        auto key_of = [](int c) { return NMAT == 2 ? ((c >> 5) & 1) : (((c >> 5) & 1) | (((c >> 6) & 1) << 1)); };
+        const int key = h;   // outlier sub-list of this thread: columns of half h of a K-step
+        auto key_of = [](int c) { return (c >> 5) & 1; };
         // Sign words and block scales arrive a group of kTcStages K-steps ahead:
         // two 16-byte loads hold the group's words of both halves, one 4-byte
         // load its two block scales.  The first group is requested before the
@@ -317,7 +304,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
         const uint16_t* sidx = reinterpret_cast<const uint16_t*>(smem + (mt ? S.idx[1] : S.idx[0])) + t * kout;
         const uint8_t* sqv = smem + (mt ? S.q[1] : S.q[0]);
         const float srow = __half2float(reinterpret_cast<const __half*>(smem + (mt ? S.srow[1] : S.srow[0]))[t]);
-        uint32_t* list = reinterpret_cast<uint32_t*>(smem + (mt ? S.ent[1] : S.ent[0])) + t * (kout + 2 * NS);
+        uint32_t* list = reinterpret_cast<uint32_t*>(smem + (mt ? S.ent[1] : S.ent[0])) + t * (kout + 4);
         int start = 2 * key;
         for (int j = 0; j < kout; ++j) start += key_of(sidx[j]) < key;
         {
@@ -348,7 +335,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
             }
 #pragma unroll
             for (int s = 0; s < kTcStages; ++s) {
-                if (NMAT == 1 && (s & 1) != G) continue;
                 if (ok && g > 0 && !mbar_wait(mma_done + s, (g - 1) & 1)) ok = false;
                 tc_fence_after();
                 const int lo = (g * kTcStages + s) * kTcK + 32 * h, hi = lo + 32;
@@ -383,7 +369,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
                     if ((m >> p) & 1u) v[p] = pw[p * 32];
                 __syncwarp();
                 tmem_st16(tmem + (uint32_t(32 * quarter) << 16) +
-                              uint32_t(Cfg::acc_cols + s * Cfg::a_cols + mt * 32 + 16 * h),
+                              uint32_t(kTcAccCols + s * kTcACols + mt * 32 + 16 * h),
                           v);
                 tmem_wait_st();
                 tc_fence_before();
@@ -396,19 +382,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
         if (!ok) *fail = 1;
         tc_fence_after();
         if (ok) {
-            constexpr int kQCols = Cfg::chunk / 4;   // each (group, half) takes a quarter of the tokens
+            constexpr int kQCols = kTcChunk / 4;   // each (group, half) takes a quarter of the tokens
             const int q4 = h + 2 * G;
             for (int col = q4 * kQCols; col < q4 * kQCols + kQCols && col < n_mma; col += 16) {
                 float v1[16], v3[16];
                 tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(col), v1);
-                if (NMAT == 2) tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(Cfg::chunk + col), v3);
-                if (row < A.rows) {
+                tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(kTcChunk + col), v3);
+                const int ra = r0 + t, rb = r0 + kTcM + t;   // rows of the two accumulators (two w2 tiles)
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int j = col + i;
-                        if (j < job.n) {
-                            const float y = NMAT == 2 ? __fdividef(v1[i], 1.0f + __expf(-v1[i])) * v3[i] : v1[i];
-                            A.out[int64_t(job.n0 + j) * A.rows + row] = y;
+                for (int i = 0; i < 16; ++i) {
+                    const int j = col + i;
+                    if (j < job.n) {
+                        float* o = A.out + int64_t(job.n0 + j) * A.rows;
+                        if (GLU) {
+                            o[ra] = __fdividef(v1[i], 1.0f + __expf(-v1[i])) * v3[i];
+                        } else {
+                            o[ra] = v1[i];
+                            o[rb] = v3[i];
                         }
                     }
                 }
@@ -425,13 +415,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
     }
 }
 
-template <int NMAT>
+template <bool GLU>
 int launch_tc(const CUtensorMap& map, const TcArgs& a, int max_jobs, cudaStream_t st) {
-    const TcSmem S = tc_smem(NMAT, TcCfg<NMAT>::chunk, outliers_per_row(a.cols));
-    int rc = ensure_smem(reinterpret_cast<const void*>(tc_tile_kernel<NMAT>), S.bytes);
+    const TcSmem S = tc_smem(outliers_per_row(a.cols));
+    int rc = ensure_smem(reinterpret_cast<const void*>(tc_tile_kernel<GLU>), S.bytes);
     if (rc != GALE_OK) return rc;
-    dim3 grid(unsigned(a.rows / kTcM), unsigned(max_jobs));
-    tc_tile_kernel<NMAT><<<grid, kTcThreads, S.bytes, st>>>(map, a);
+    const int rows_per_cta = GLU ? kTcM : 2 * kTcM;
+    dim3 grid(unsigned(a.rows / rows_per_cta), unsigned(max_jobs));
+    tc_tile_kernel<GLU><<<grid, kTcThreads, S.bytes, st>>>(map, a);
     GALE_LAUNCH_CHECK();
     return GALE_OK;
 }
@@ -453,10 +444,8 @@ PrefillWs carve_prefill_ws(void* ws, const gale_layer& L, int B, int K) {
     w.offsets = reinterpret_cast<int32_t*>(take(4 * (int64_t(L.n_experts) + 1)));
     w.perm = reinterpret_cast<int32_t*>(take(4 * P));
     w.pos_of_pair = reinterpret_cast<int32_t*>(take(4 * P));
-    w.max_jobs13 = int(L.n_experts + P / 128 + 1);
-    w.max_jobs2 = int(L.n_experts + P / 256 + 1);
-    w.jobs13 = take(int64_t(sizeof(TcJob)) * w.max_jobs13);
-    w.jobs2 = take(int64_t(sizeof(TcJob)) * w.max_jobs2);
+    w.max_jobs = int(L.n_experts + P / kTcChunk + 1);
+    w.jobs = take(int64_t(sizeof(TcJob)) * w.max_jobs);
     w.n_jobs = reinterpret_cast<int32_t*>(take(8));
     w.x16 = reinterpret_cast<__half*>(take(2 * P * dm));
     w.h = reinterpret_cast<float*>(take(4 * P * df));
@@ -473,8 +462,9 @@ bool prefill_supported(const gale_layer& L, int B, int K) {
     if (L.d_model % (kTcK * kTcStages) != 0 || L.d_ff % (kTcK * kTcStages) != 0) return false;
     // a tile's outlier lists stay in shared memory
     const int k1 = outliers_per_row(L.d_model), k2 = outliers_per_row(L.d_ff);
-    return k1 <= kMaxOutliers && k2 <= kMaxOutliers && tc_smem(2, TcCfg<2>::chunk, k1).bytes <= 227 * 1024 &&
-           tc_smem(1, TcCfg<1>::chunk, k2).bytes <= 227 * 1024;
+    // w2 goes by pairs of 128-row tiles
+    return k1 <= kMaxOutliers && k2 <= kMaxOutliers && tc_smem(k1).bytes <= 227 * 1024 &&
+           tc_smem(k2).bytes <= 227 * 1024 && L.d_model % (2 * kTcM) == 0;
 }
 
 int launch_moe_prefill(const gale_layer& L, const uint16_t* x, const int32_t* ids, const float* gates, int B, int K,
@@ -494,8 +484,7 @@ int launch_moe_prefill(const gale_layer& L, const uint16_t* x, const int32_t* id
     ra.status = w.status;
     int rc = launch_route_permute(ra, st);
     if (rc != GALE_OK) return rc;
-    prefill_jobs_kernel<<<1, 1024, 0, st>>>(w.counts, w.offsets, L.n_experts, static_cast<TcJob*>(w.jobs13),
-                                            w.n_jobs, static_cast<TcJob*>(w.jobs2), w.n_jobs + 1);
+    prefill_jobs_kernel<<<1, 1024, 0, st>>>(w.counts, w.offsets, L.n_experts, static_cast<TcJob*>(w.jobs), w.n_jobs);
     GALE_LAUNCH_CHECK();
     {
         const int64_t warps = int64_t(B) * (L.d_model / 1024);
@@ -505,37 +494,35 @@ int launch_moe_prefill(const gale_layer& L, const uint16_t* x, const int32_t* id
     }
     const int64_t l1 = make_layout(L.d_ff, L.d_model).total;
     CUtensorMap xm;
-    rc = act_map(&xm, w.x16, L.d_model, P, TcCfg<2>::chunk);
+    rc = act_map(&xm, w.x16, L.d_model, P, kTcChunk);
     if (rc != GALE_OK) return rc;
     TcArgs a{};
     a.base = static_cast<const char*>(L.base);
     a.stride = L.expert_stride;
     a.status = w.status;
     // w1 / w3 + SwiGLU
-    a.jobs = static_cast<const TcJob*>(w.jobs13);
+    a.jobs = static_cast<const TcJob*>(w.jobs);
     a.n_jobs = w.n_jobs;
     a.off_a = 0;
     a.off_b = l1;
     a.rows = L.d_ff;
     a.cols = L.d_model;
     a.out = w.h;
-    rc = launch_tc<2>(xm, a, w.max_jobs13, st);
+    rc = launch_tc<true>(xm, a, w.max_jobs, st);
     if (rc != GALE_OK) return rc;
     // rotate h
     rc = gale_fwht1024(w.h, GALE_F32, w.h16, GALE_F16, P, L.d_ff, st);
     if (rc != GALE_OK) return rc;
     CUtensorMap hm;
-    rc = act_map(&hm, w.h16, L.d_ff, P, TcCfg<1>::chunk);
+    rc = act_map(&hm, w.h16, L.d_ff, P, kTcChunk);
     if (rc != GALE_OK) return rc;
-    // w2
-    a.jobs = static_cast<const TcJob*>(w.jobs2);
-    a.n_jobs = w.n_jobs + 1;
+    // w2: two 128-row tiles per CTA, the same 128-slot chunks as w1/w3
     a.off_a = 2 * l1;
     a.off_b = 2 * l1;
     a.rows = L.d_model;
     a.cols = L.d_ff;
     a.out = w.o;
-    rc = launch_tc<1>(hm, a, w.max_jobs2, st);
+    rc = launch_tc<false>(hm, a, w.max_jobs, st);
     if (rc != GALE_OK) return rc;
     return launch_moe_combine(w.o, w.pos_of_pair, gates, x, B, K, L.d_model, out, out_dtype, fuse_norm, eps,
                               w.scratch, st);

@@ -13,10 +13,9 @@ struct PrefillWs {
     int32_t* offsets;       // [E+1]
     int32_t* perm;          // [B*K]
     int32_t* pos_of_pair;   // [B*K]
-    void* jobs13;           // [max_jobs13] (expert, first slot, tokens), chunks of 128 slots
-    void* jobs2;            // [max_jobs2], chunks of 256 slots
-    int32_t* n_jobs;        // [2]
-    int max_jobs13, max_jobs2;
+    void* jobs;             // [max_jobs] (expert, first slot, tokens), chunks of 128 slots
+    int32_t* n_jobs;        // [1]
+    int max_jobs;
     __half* x16;            // [B*K][d_model] rotated x of each pair, permuted order
     float* h;               // [B*K][d_ff]
     __half* h16;            // [B*K][d_ff] rotated h

@@ -341,9 +341,10 @@ def test_moe_full_size(full_layer, B, skew):
 @pytest.mark.parametrize("B,K,skew", [(70, 6, 0.0), (200, 6, 0.0), (1000, 6, 0.0), (500, 1, 0.0),
                                       (300, 4, 2.0)])
 def test_moe_prefill_small(small_layer, B, K, skew):
-    """Several 128-row tiles and K-steps per matrix; experts with more than
-    256 tokens split into chunks with a ragged last chunk (B = 1000, and the
-    skewed routing)."""
+    """Several 128-row tiles (w2: several pairs of them) and K-steps per
+    matrix; experts with more than 128 tokens split into chunks of 128 with a
+    ragged last chunk (B = 1000: ~375 tokens per expert, and the skewed
+    routing)."""
     L = small_layer
     bits, xv = gs.hidden_bf16(B, L.d_model, tag=2000 + B)
     ids, gates = gs.route_topk(gs.router_logits(B, L.E, tag=2000 + B, bias_sigma=skew), K)
