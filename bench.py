@@ -334,6 +334,8 @@ def run_gpu(args):
     clocks.start()
     t1, bytes1, times1 = measure(1, args.steps, args.warmup, 10_000)
     t8, bytes8, _ = measure(8, max(args.steps // 2, 3), args.warmup, 20_000)
+    # decode batch 64 with per-expert popularity bias N(0, 0.5) (skewed tokens per expert)
+    t64, bytes64, _ = measure(64, max(args.steps // 2, 3), args.warmup, 25_000, bias_sigma=0.5)
     te, h2d, d2h = measure_e2e(1, args.steps, args.warmup, 30_000)
     # prefill: 4096 tokens, skewed routing (tensor-core tile path)
     pf_steps = max(3, min(args.steps // 5, 10))
@@ -343,7 +345,7 @@ def run_gpu(args):
     clocks_info = clocks.stop()
 
     # max over ranks of the device time
-    t1, t8, te, tp, tc = max_over_ranks([t1, t8, te, tp, tc], world, "cuda")
+    t1, t8, t64, te, tp, tc = max_over_ranks([t1, t8, t64, te, tp, tc], world, "cuda")
     tokens, value = job_throughput(1, args.steps, world, t1)
     gbs = bytes1 * world / t1 / 1e9
     peak, tpeak, peak_kind = peaks()
@@ -365,6 +367,10 @@ def run_gpu(args):
                      "algorithmic_bytes_per_launch": bytes1 / args.steps},
         "b8": {"tokens_per_s": 8 * max(args.steps // 2, 3) * world / t8,
                "hbm_gbs": bytes8 * world / t8 / 1e9, "frac": bytes8 * world / t8 / 1e9 / peak},
+        "b64": {"tokens_per_s": 64 * max(args.steps // 2, 3) * world / t64,
+                "ms_per_step": 1e3 * t64 / max(args.steps // 2, 3),
+                "hbm_gbs": bytes64 * world / t64 / 1e9, "frac": bytes64 * world / t64 / 1e9 / peak,
+                "routing": "top-6 with per-expert bias N(0, 0.5) (skewed)"},
         "chain43": {"workload": f"decode batch 1 through {CHAIN_LAYERS} layers x 256 resident experts "
                                 f"(46 GB), residual + RMSNorm between layers, bf16 hidden state",
                     "tokens_per_s": ch_steps * world / tc, "ms_per_token": 1e3 * tc / ch_steps,

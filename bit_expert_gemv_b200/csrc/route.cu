@@ -29,6 +29,19 @@ __device__ __forceinline__ int step_experts(const RouteArgs& a, int base, int en
     }
     return e;
 }
+
+// Steps a warp walks per batch of id loads.
+constexpr int kBlockSteps = 8;
+
+// The ids of the kBlockSteps steps from base0 (lane = pair), -1 past `end`.
+__device__ __forceinline__ void load_block(const RouteArgs& a, int base0, int end, int (&idb)[kBlockSteps]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < kBlockSteps; ++j) {
+        const int p = base0 + 32 * j + lane;
+        idb[j] = p < end ? __ldg(a.ids + p) : -1;
+    }
+}
 }  // namespace
 
 __global__ void __launch_bounds__(1024) route_permute_kernel(RouteArgs a) {
@@ -43,25 +56,30 @@ __global__ void __launch_bounds__(1024) route_permute_kernel(RouteArgs a) {
 
     for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
-    // pass 1: per-warp counts (and validation); the ids of the next step are
-    // loaded while this one is counted
-    int prev, id = p0 + lane < p1 ? a.ids[p0 + lane] : -1;
+    // pass 1: per-warp counts (and validation); the ids of kBlockSteps steps
+    // are loaded at once, so that their latencies overlap
+    int prev;
     {
         // the token of the range's first pair may start in the previous range
         const int q = p0 - 32 + lane;
         prev = (q >= 0 && q < BK && p0 < p1) ? a.ids[q] : -1;
     }
     const int prev0 = prev;
-    for (int base = p0; base < p1; base += 32) {
-        const int p = base + lane;
-        const int nid = p + 32 < p1 ? a.ids[p + 32] : -1;
-        const int e = step_experts(a, base, p1, id, prev);
-        if (p < p1 && e < 0) set_status(a.status, GALE_ERR_ARG);
-        prev = id;
-        id = nid;
-        const unsigned grp = __match_any_sync(0xffffffffu, e);
-        if (e >= 0 && lane == __ffs(grp) - 1) wcnt[warp * E + e] += __popc(grp);
-        __syncwarp();
+    for (int base0 = p0; base0 < p1; base0 += 32 * kBlockSteps) {
+        int idb[kBlockSteps];
+        load_block(a, base0, p1, idb);
+#pragma unroll
+        for (int j = 0; j < kBlockSteps; ++j) {
+            const int base = base0 + 32 * j;
+            if (base >= p1) break;
+            const int p = base + lane;
+            const int e = step_experts(a, base, p1, idb[j], prev);
+            if (p < p1 && e < 0) set_status(a.status, GALE_ERR_ARG);
+            prev = idb[j];
+            const unsigned grp = __match_any_sync(0xffffffffu, e);
+            if (e >= 0 && lane == __ffs(grp) - 1) wcnt[warp * E + e] += __popc(grp);
+            __syncwarp();
+        }
     }
     __syncthreads();
     // totals per expert (thread e sums its column in warp order), exclusive
@@ -103,22 +121,26 @@ __global__ void __launch_bounds__(1024) route_permute_kernel(RouteArgs a) {
     __syncthreads();
     // pass 2: placement in pair order
     prev = prev0;
-    id = p0 + lane < p1 ? a.ids[p0 + lane] : -1;
-    for (int base = p0; base < p1; base += 32) {
-        const int p = base + lane;
-        const int nid = p + 32 < p1 ? a.ids[p + 32] : -1;
-        const int e = step_experts(a, base, p1, id, prev);
-        prev = id;
-        id = nid;
-        const unsigned grp = __match_any_sync(0xffffffffu, e);
-        if (e >= 0) {
-            const int pos = wcnt[warp * E + e] + __popc(grp & ((1u << lane) - 1u));
-            a.perm[pos] = p;
-            if (a.pos_of_pair) a.pos_of_pair[p] = pos;
+    for (int base0 = p0; base0 < p1; base0 += 32 * kBlockSteps) {
+        int idb[kBlockSteps];
+        load_block(a, base0, p1, idb);
+#pragma unroll
+        for (int j = 0; j < kBlockSteps; ++j) {
+            const int base = base0 + 32 * j;
+            if (base >= p1) break;
+            const int p = base + lane;
+            const int e = step_experts(a, base, p1, idb[j], prev);
+            prev = idb[j];
+            const unsigned grp = __match_any_sync(0xffffffffu, e);
+            if (e >= 0) {
+                const int pos = wcnt[warp * E + e] + __popc(grp & ((1u << lane) - 1u));
+                a.perm[pos] = p;
+                if (a.pos_of_pair) a.pos_of_pair[p] = pos;
+            }
+            __syncwarp();
+            if (e >= 0 && lane == __ffs(grp) - 1) wcnt[warp * E + e] += __popc(grp);
+            __syncwarp();
         }
-        __syncwarp();
-        if (e >= 0 && lane == __ffs(grp) - 1) wcnt[warp * E + e] += __popc(grp);
-        __syncwarp();
     }
 }
 

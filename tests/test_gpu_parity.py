@@ -186,6 +186,37 @@ def test_route_permute_flags_bad_ids():
     assert int(counts.sum().item()) == 7      # the repeated 3 and the id 300 are dropped
 
 
+def test_route_permute_drops_repeats_at_walk_boundaries():
+    """Repeated ids planted where a token's pairs straddle the boundaries of
+    the kernel's walk: B = 4001, K = 6 gives 32 warp ranges of 751 pairs,
+    walked 32 pairs a step and eight steps per batch of loads.  Token 125
+    straddles warp ranges 0 / 1 (pair 751), token 5 a step boundary (pair 32),
+    token 167 the batch boundary of range 1 (pair 751 + 256 = 1007).  The
+    later pair of each repeat is dropped; the rest is the stable sort by
+    (expert, pair), checked against a plain sort of the valid pairs."""
+    B, K, E = 4001, 6, 256
+    ids, _ = gs.route_topk(gs.router_logits(B, E, tag=4001, bias_sigma=0.5), K)
+    ids = ids.copy()
+    ids[125, 1] = ids[125, 0]   # pairs 750 | 751
+    ids[5, 3] = ids[5, 0]       # pairs 30 | 33
+    ids[167, 5] = ids[167, 1]   # pairs 1003 | 1007
+    flat = ids.reshape(-1)
+    valid = [p for p in range(B * K) if flat[p] not in flat[p - p % K:p]]
+    assert len(valid) == B * K - 3
+    want_counts = np.bincount(flat[valid], minlength=E).astype(np.int32)
+    want_perm = np.array(sorted(valid, key=lambda p: (flat[p], p)), np.int32)
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.full((B * K,), -7, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    G.gale_route_permute(to_dev(ids), E, counts, offsets, perm, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == G.GALE_ERR_ARG
+    assert np.array_equal(counts.cpu().numpy(), want_counts)
+    assert np.array_equal(offsets.cpu().numpy(), np.concatenate([[0], np.cumsum(want_counts)]).astype(np.int32))
+    assert np.array_equal(perm.cpu().numpy()[:len(valid)], want_perm)
+
+
 # ----------------------------------------------------------------------------
 # MoE layer
 # ----------------------------------------------------------------------------
