@@ -32,8 +32,9 @@ namespace {
 constexpr int kTcM = 128;           // weight rows per tile (TMEM lanes)
 constexpr int kTcK = 64;            // K per stage: one 128-byte row of fp16 tokens
 constexpr int kTcStages = 4;
-constexpr int kTcExpWarps = 16;     // expander / epilogue warps: two groups of 8, 2 per TMEM lane quarter each
-constexpr int kTcThreads = (2 + kTcExpWarps) * 32;
+constexpr int kTcExpWarps = 16;     // expander warps: two groups of 8, 2 per TMEM lane quarter each
+constexpr int kTcAuxWarps = 4;      // outlier lists of the next job, epilogue of the last one
+constexpr int kTcThreads = (2 + kTcExpWarps + kTcAuxWarps) * 32;
 constexpr int kMaxOutliers = 82;    // per row: round(0.01 * 8192)
 constexpr uint32_t kSentinel = 0xFFFF0000u;
 
@@ -60,13 +61,30 @@ struct TcArgs {
 };
 
 struct TcSmem {
-    int b, idx[2], q[2], srow[2], ent[2], patch, bars, misc, bytes;
+    int b, idx[2], q[2], srow[2], ent[2][2], start1[2], patch, bars, misc, bytes;
+};
+
+// Barriers of the tile kernel, in their shared-memory order.
+enum TcBar {
+    kBarBFull = 0,                        // [kTcStages] token tile landed
+    kBarAFull = kTcStages,                // [kTcStages] A stage expanded (16 warps)
+    kBarMmaDone = 2 * kTcStages,          // [kTcStages] the stage's MMAs completed
+    kBarAccFull = 3 * kTcStages,          // the job's accumulators are final
+    kBarAccEmpty,                         // the epilogue has read them (aux threads)
+    kBarSideFull,                         // the job's outlier sections landed
+    kBarSideFree,                         // the lists have been built from them (aux threads)
+    kBarListReady,                        // [2] lists of a job in buffer b (aux threads)
+    kBarListFree = kBarListReady + 2,     // [2] the expanders are done with buffer b
+    kTcBars = kBarListFree + 2
 };
 
 __host__ __device__ inline int align16(int n) { return (n + 15) & ~15; }
 
-// Shared memory: the token ring, then per operand the tile's outlier sections
-// (bulk copies) and the outlier lists split by 32-column half.
+// Shared memory: the token ring; per operand the job's outlier sections (bulk
+// copies, one buffer); two buffers of outlier lists (per operand and row: the
+// columns of the first and of the second 32-column half of every K-step, each
+// list closed by two sentinels, and where the second list starts); the
+// expanders' patch areas; barriers.
 __host__ __device__ inline TcSmem tc_smem(int k) {
     TcSmem s;
     s.b = 0;
@@ -78,14 +96,20 @@ __host__ __device__ inline TcSmem tc_smem(int k) {
         o += align16(kTcM * k / 2 + 1);
         s.srow[mt] = o;
         o += kTcM * 2;
-        s.ent[mt] = o;
-        o += kTcM * (k + 2 * 2) * 4;   // the two sub-lists of a row, each closed by two sentinels
+    }
+    for (int b = 0; b < 2; ++b) {
+        for (int mt = 0; mt < 2; ++mt) {
+            s.ent[b][mt] = o;
+            o += kTcM * (k + 4) * 4;
+        }
+        s.start1[b] = o;
+        o += 2 * kTcM * 4;
     }
     // per expander warp, 16 words x 32 lanes of patched (outlier) words
     s.patch = o;
     o += kTcExpWarps * 16 * 32 * 4;
     s.bars = (o + 7) & ~7;
-    s.misc = s.bars + 8 * (3 * kTcStages + 2);
+    s.misc = s.bars + 8 * kTcBars;
     s.bytes = s.misc + 16 + 1024;   // + slack to align the base to 1024 bytes
     return s;
 }
@@ -174,42 +198,66 @@ __device__ __forceinline__ void expand_signs(uint32_t w, uint32_t sc, uint32_t (
     }
 }
 
-// One (rows, token chunk) job: w1 and w3 over one 128-row tile with the
-// SwiGLU epilogue (GLU), or two consecutive 128-row tiles of w2.  Warp 0
-// streams token tiles by TMA, warp 1 owns TMEM and issues the MMAs, warps
-// 2..17 expand weights into TMEM and run the epilogue.
+// Persistent tile kernel: CTA c takes the (row tile, job) items c, c + grid,
+// ... in order, where a row tile is 128 rows of w1 and w3 (SwiGLU epilogue,
+// GLU) or two consecutive 128-row tiles of w2.  Warp 0 streams the outlier
+// sections and the token tiles, warp 1 owns TMEM and issues the MMAs, warps
+// 2..17 expand weights into TMEM, and warps 18..21 build the outlier lists of
+// the next item and write out the accumulators of the last one, so that
+// neither sits between two items' K loops.
 template <bool GLU>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_constant__ CUtensorMap xmap, TcArgs A) {
-    constexpr int kRowsPerCta = GLU ? kTcM : 2 * kTcM;   // rows of the streamed matrix per CTA
+    constexpr int kRowsPerCta = GLU ? kTcM : 2 * kTcM;   // rows of the streamed matrix per item
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_align1024(smem_raw);
-    const int mtile = blockIdx.x, job_id = blockIdx.y;
-    if (job_id >= *A.n_jobs) return;
-    const TcJob job = A.jobs[job_id];
+    const int n_mtiles = A.rows / kRowsPerCta;
+    const int n_items = n_mtiles * *A.n_jobs;
+    if (int(blockIdx.x) >= n_items) return;
+    const int n_my = (n_items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1;   // items of this CTA
     const int nk = A.cols / kTcK;
     const int kout = outliers_per_row(A.cols);
     const TcSmem S = tc_smem(kout);
-    uint64_t* b_full = reinterpret_cast<uint64_t*>(smem + S.bars);
-    uint64_t* a_full = b_full + kTcStages;
-    uint64_t* mma_done = a_full + kTcStages;
-    uint64_t* acc_full = mma_done + kTcStages;
-    uint64_t* side_full = acc_full + 1;
+    // offsets by operand / buffer as selects (an indexed TcSmem would live in local memory)
+    auto off_idx = [&](int mt) { return mt ? S.idx[1] : S.idx[0]; };
+    auto off_q = [&](int mt) { return mt ? S.q[1] : S.q[0]; };
+    auto off_srow = [&](int mt) { return mt ? S.srow[1] : S.srow[0]; };
+    auto off_ent = [&](int b, int mt) { return b ? (mt ? S.ent[1][1] : S.ent[1][0]) : (mt ? S.ent[0][1] : S.ent[0][0]); };
+    auto off_start1 = [&](int b) { return b ? S.start1[1] : S.start1[0]; };
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + S.bars);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S.misc);
-    int* fail = reinterpret_cast<int*>(smem + S.misc + 4);
+    volatile int* fail = reinterpret_cast<volatile int*>(smem + S.misc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_mma = (job.n + 15) & ~15;
-    const uint32_t idesc = umma_idesc_f16(kTcM, n_mma);
-    const int r0 = mtile * kRowsPerCta;
-    const char* rec = A.base + int64_t(job.e) * A.stride;
+    // item i of this CTA: its row tile and job
+    auto item = [&](int i, int& r0, TcJob& job) {
+        const int w = int(blockIdx.x) + i * int(gridDim.x);
+        const int jid = w / n_mtiles;
+        r0 = (w - jid * n_mtiles) * kRowsPerCta;
+        job = A.jobs[jid];
+    };
+    // a bounded wait that gives up at once after any earlier one ran out
+    // (the flag is read only when the phase is not complete yet)
+    auto wait = [&](int b, uint32_t parity) -> bool {
+        if (mbar_try_wait(bar + b, parity)) return true;
+        if (*fail) return false;
+        if (mbar_wait(bar + b, parity)) return true;
+        *fail = 1;
+        return false;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kTcStages; ++s) {
-            mbar_init(b_full + s, 1);
-            mbar_init(a_full + s, kTcExpWarps * 32);
-            mbar_init(mma_done + s, 1);
+            mbar_init(bar + kBarBFull + s, 1);
+            mbar_init(bar + kBarAFull + s, kTcExpWarps * 32);
+            mbar_init(bar + kBarMmaDone + s, 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(side_full, 1);
+        mbar_init(bar + kBarAccFull, 1);
+        mbar_init(bar + kBarAccEmpty, kTcAuxWarps * 32);
+        mbar_init(bar + kBarSideFull, 1);
+        mbar_init(bar + kBarSideFree, kTcAuxWarps * 32);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar + kBarListReady + b, kTcAuxWarps * 32);
+            mbar_init(bar + kBarListFree + b, kTcExpWarps * 32);
+        }
         *fail = 0;
         fence_mbar_init();
     }
@@ -223,58 +271,90 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------- producer: the tile's outlier sections, then token tiles
+        // ---------------- producer: the outlier sections of item i + 1 once
+        // the lists of item i are built, then the token tiles of item i
         if (lane == 0) {
             const uint32_t idx_bytes = uint32_t(kTcM * kout * 2), q_bytes = uint32_t(kTcM * kout / 2);
-            mbar_arrive_expect_tx(side_full, 2u * (idx_bytes + q_bytes + kTcM * 2));
-            for (int mt = 0; mt < 2; ++mt) {
-                const MatView mv = make_view(rec + (mt ? A.off_b : A.off_a), A.rows, A.cols);
-                const int rm = r0 + (GLU ? 0 : mt * kTcM);   // first row of operand mt
-                bulk_load(smem + S.idx[mt], mv.idx + int64_t(rm) * kout, idx_bytes, side_full);
-                bulk_load(smem + S.q[mt], mv.q + int64_t(rm) * kout / 2, q_bytes, side_full);
-                bulk_load(smem + S.srow[mt], mv.s_row + rm, kTcM * 2, side_full);
-            }
-            int issued = 0;
-            for (int ks = 0; ks < nk; ++ks) {
-                const int s = ks % kTcStages;
-                if (ks >= kTcStages && !mbar_wait(mma_done + s, ((ks / kTcStages) - 1) & 1)) {
-                    *fail = 1;
-                    break;
+            auto load_side = [&](int i) {
+                int r0;
+                TcJob job;
+                item(i, r0, job);
+                const char* rec = A.base + int64_t(job.e) * A.stride;
+                mbar_arrive_expect_tx(bar + kBarSideFull, 2u * (idx_bytes + q_bytes + kTcM * 2));
+                for (int mt = 0; mt < 2; ++mt) {
+                    const MatView mv = make_view(rec + (mt ? A.off_b : A.off_a), A.rows, A.cols);
+                    const int rm = r0 + (GLU ? 0 : mt * kTcM);   // first row of operand mt
+                    bulk_load(smem + off_idx(mt), mv.idx + int64_t(rm) * kout, idx_bytes, bar + kBarSideFull);
+                    bulk_load(smem + off_q(mt), mv.q + int64_t(rm) * kout / 2, q_bytes, bar + kBarSideFull);
+                    bulk_load(smem + off_srow(mt), mv.s_row + rm, kTcM * 2, bar + kBarSideFull);
                 }
-                mbar_arrive_expect_tx(b_full + s, uint32_t(kTcChunk * 128));
-                tma_load_3d(smem + S.b + s * kTcChunk * 128, &xmap, b_full + s, ks * kTcK, job.n0, 0);
-                issued = ks + 1;
+            };
+            load_side(0);
+            int sides = 1, gs = 0;
+            for (int i = 0; i < n_my; ++i) {
+                int r0;
+                TcJob job;
+                item(i, r0, job);
+                if (i + 1 < n_my) {
+                    if (!wait(kBarSideFree, uint32_t(i & 1))) break;
+                    load_side(i + 1);
+                    ++sides;
+                }
+                bool ok = true;
+                for (int ks = 0; ks < nk; ++ks, ++gs) {
+                    const int s = gs % kTcStages;
+                    if (gs >= kTcStages && !wait(kBarMmaDone + s, uint32_t(((gs / kTcStages) - 1) & 1))) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bar + kBarBFull + s, uint32_t(kTcChunk * 128));
+                    tma_load_3d(smem + S.b + s * kTcChunk * 128, &xmap, bar + kBarBFull + s, ks * kTcK, job.n0, 0);
+                }
+                if (!ok) break;
             }
-            // no copy may still be landing when the CTA exits
-            if (!mbar_wait(side_full, 0)) *fail = 1;
-            for (int ks = issued - kTcStages < 0 ? 0 : issued - kTcStages; ks < issued; ++ks)
-                if (!mbar_wait(b_full + ks % kTcStages, (ks / kTcStages) & 1)) *fail = 1;
+            // no copy may still be landing when the CTA exits (bounded waits,
+            // also after a failure)
+            mbar_wait(bar + kBarSideFull, uint32_t((sides - 1) & 1));
+            for (int g = gs - kTcStages < 0 ? 0 : gs - kTcStages; g < gs; ++g)
+                mbar_wait(bar + kBarBFull + g % kTcStages, uint32_t((g / kTcStages) & 1));
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer: item i starts once the epilogue has read
+        // the accumulators of item i - 1
         if (lane == 0) {
-            for (int ks = 0; ks < nk; ++ks) {
-                const int s = ks % kTcStages;
-                const uint32_t par = (ks / kTcStages) & 1;
-                if (!mbar_wait(a_full + s, par) || !mbar_wait(b_full + s, par)) {
-                    *fail = 1;
-                    break;
-                }
+            int gs = 0;
+            for (int i = 0; i < n_my; ++i) {
+                int r0;
+                TcJob job;
+                item(i, r0, job);
+                const uint32_t idesc = umma_idesc_f16(kTcM, (job.n + 15) & ~15);
+                if (i > 0 && !wait(kBarAccEmpty, uint32_t((i - 1) & 1))) break;
                 tc_fence_after();
-                const uint32_t bst = smem_u32(smem + S.b + s * kTcChunk * 128);
-                const uint32_t ast = tmem + uint32_t(kTcAccCols + s * kTcACols);
+                bool ok = true;
+                for (int ks = 0; ks < nk; ++ks, ++gs) {
+                    const int s = gs % kTcStages;
+                    const uint32_t par = (gs / kTcStages) & 1;
+                    if (!wait(kBarAFull + s, par) || !wait(kBarBFull + s, par)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t bst = smem_u32(smem + S.b + s * kTcChunk * 128);
+                    const uint32_t ast = tmem + uint32_t(kTcAccCols + s * kTcACols);
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
+                    for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-                    for (int kk = 0; kk < kTcK / 16; ++kk)
-                        umma_f16_ts(tmem + uint32_t(mt * kTcChunk), ast + uint32_t(mt * 32 + kk * 8),
-                                    umma_desc_sw128(bst + kk * 32), idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kTcK / 16; ++kk)
+                            umma_f16_ts(tmem + uint32_t(mt * kTcChunk), ast + uint32_t(mt * 32 + kk * 8),
+                                        umma_desc_sw128(bst + kk * 32), idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar + kBarMmaDone + s);
                 }
-                umma_commit(mma_done + s);
+                if (!ok) break;
+                umma_commit(bar + kBarAccFull);
             }
-            umma_commit(acc_full);
         }
-    } else {
+    } else if (warp < 2 + kTcExpWarps) {
         // ---------------- expanders: two groups of 8 warps; group G expands
         // operand G (w1 / w3, or the first / second 128-row tile of w2) and
         // its thread (row t, half h) the 32 columns of half h of every K-step.
@@ -284,124 +364,176 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
         const int h = (ew >> 2) & 1;
         const int t = 32 * quarter + lane;
         const int mt = G;
-        const int row = r0 + (GLU ? 0 : mt * kTcM) + t;
         const int nb = A.cols / 128;
-        const int key = h;   // outlier sub-list of this thread: columns of half h of a K-step
-        auto key_of = [](int c) { return (c >> 5) & 1; };
+        const int ng = nk / kTcStages;
+        uint32_t* pw = reinterpret_cast<uint32_t*>(smem + S.patch) + ew * 512 + lane;   // this lane's column
         // Sign words and block scales arrive a group of kTcStages K-steps ahead:
         // two 16-byte loads hold the group's words of both halves, one 4-byte
-        // load its two block scales.  The first group is requested before the
-        // outlier sections have landed.
-        const MatView mv = make_view(rec + (mt ? A.off_b : A.off_a), A.rows, A.cols);
-        const uint4* wsrc = reinterpret_cast<const uint4*>(mv.signs + int64_t(row) * (A.cols / 32));
-        const uint32_t* ssrc =
-            reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint16_t*>(mv.s_blk) + int64_t(row) * nb);
+        // load its two block scales; the next item's first group is requested
+        // during the last group of the current one.
+        auto row_src = [&](int r0, const TcJob& job, const uint4*& wsrc, const uint32_t*& ssrc) {
+            const int row = r0 + (GLU ? 0 : mt * kTcM) + t;
+            const MatView mv = make_view(A.base + int64_t(job.e) * A.stride + (mt ? A.off_b : A.off_a), A.rows, A.cols);
+            wsrc = reinterpret_cast<const uint4*>(mv.signs + int64_t(row) * (A.cols / 32));
+            ssrc = reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint16_t*>(mv.s_blk) + int64_t(row) * nb);
+        };
+        const uint4* wsrc;
+        const uint32_t* ssrc;
+        {
+            int r0;
+            TcJob job;
+            item(0, r0, job);
+            row_src(r0, job, wsrc, ssrc);
+        }
         uint4 wa = __ldg(wsrc), wb = __ldg(wsrc + 1);
         uint32_t sp = __ldg(ssrc);
-        bool ok = mbar_wait(side_full, 0);
-        // this thread's outliers in column order, as (column << 16 | fp16 value):
-        // the row's sub-lists in key order, each closed by two sentinels
-        const uint16_t* sidx = reinterpret_cast<const uint16_t*>(smem + (mt ? S.idx[1] : S.idx[0])) + t * kout;
-        const uint8_t* sqv = smem + (mt ? S.q[1] : S.q[0]);
-        const float srow = __half2float(reinterpret_cast<const __half*>(smem + (mt ? S.srow[1] : S.srow[0]))[t]);
-        uint32_t* list = reinterpret_cast<uint32_t*>(smem + (mt ? S.ent[1] : S.ent[0])) + t * (kout + 4);
-        int start = 2 * key;
-        for (int j = 0; j < kout; ++j) start += key_of(sidx[j]) < key;
-        {
-            int o = start;
-            for (int j = 0; j < kout; ++j) {
-                const int c = sidx[j];
-                if (key_of(c) != key) continue;
-                const int n = t * kout + j;
-                const int byte = sqv[n >> 1];
-                int qv = (n & 1) ? (byte >> 4) : (byte & 0xF);
-                qv = qv >= 8 ? qv - 16 : qv;
-                list[o++] = (uint32_t(c) << 16) | __half_as_ushort(__float2half_rn(float(qv) * srow));
-            }
-            list[o] = kSentinel;
-            list[o + 1] = kSentinel;
-        }
-        int cur = start;
-        uint32_t ent = list[start], nxt = list[start + 1];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(smem + S.patch) + ew * 512 + lane;   // this lane's column
-        const int ng = nk / kTcStages;
-        for (int g = 0; g < ng; ++g) {
-            const uint32_t wg[kTcStages] = {h ? wa.y : wa.x, h ? wa.w : wa.z, h ? wb.y : wb.x, h ? wb.w : wb.z};
-            const uint32_t sg[2] = {sp & 0xFFFFu, sp >> 16};
-            if (g + 1 < ng) {
-                wa = __ldg(wsrc + 2 * (g + 1));
-                wb = __ldg(wsrc + 2 * (g + 1) + 1);
-                sp = __ldg(ssrc + g + 1);
-            }
-#pragma unroll
-            for (int s = 0; s < kTcStages; ++s) {
-                if (ok && g > 0 && !mbar_wait(mma_done + s, (g - 1) & 1)) ok = false;
-                tc_fence_after();
-                const int lo = (g * kTcStages + s) * kTcK + 32 * h, hi = lo + 32;
-                const uint32_t w = wg[s], sc = sg[s >> 1];
-                uint32_t v[16];
-                expand_signs(w, sc, v);
-                // outliers of this range replace their weights: each lane
-                // walks its own entries (the next one already loaded),
-                // parks the patched words in its column of the warp's
-                // patch area and marks them; a predicated load per word
-                // then takes them in, with no per-outlier select over the
-                // sixteen words
-                uint32_t m = 0u;
-                int prev_p = -1;
-                uint32_t prev_a = 0u;
-                while (int(ent >> 16) < hi) {
-                    const int u = int(ent >> 16) - lo;
-                    const int P = u >> 1;
-                    const uint32_t val = ent & 0xFFFFu;
-                    uint32_t other = sc ^ (((w >> (u ^ 1)) & 1u) << 15);
-                    if (P == prev_p) other = (u & 1) ? (prev_a & 0xFFFFu) : (prev_a >> 16);
-                    const uint32_t a = (u & 1) ? (other | (val << 16)) : (val | (other << 16));
-                    prev_p = P;
-                    prev_a = a;
-                    pw[P * 32] = a;
-                    m |= 1u << P;
-                    ent = nxt;
-                    nxt = list[++cur + 1];
+        bool ok = true;
+        int gg = 0;   // groups expanded so far (all items)
+        for (int i = 0; i < n_my; ++i) {
+            const int buf = i & 1;
+            if (ok && !wait(kBarListReady + buf, uint32_t((i >> 1) & 1))) ok = false;
+            // this thread's outliers in column order, as (column << 16 | fp16 value)
+            const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + off_ent(buf, mt)) + t * (kout + 4);
+            int cur = h ? reinterpret_cast<const int*>(smem + off_start1(buf))[mt * kTcM + t] : 0;
+            uint32_t ent = list[cur], nxt = list[cur + 1];
+            // the next item's job is read now and used in the last group
+            int r0n = 0;
+            TcJob jn{};
+            if (i + 1 < n_my) item(i + 1, r0n, jn);
+            const uint4* wsrc_n = wsrc;
+            const uint32_t* ssrc_n = ssrc;
+            for (int g = 0; g < ng; ++g, ++gg) {
+                const uint32_t wg[kTcStages] = {h ? wa.y : wa.x, h ? wa.w : wa.z, h ? wb.y : wb.x, h ? wb.w : wb.z};
+                const uint32_t sg[2] = {sp & 0xFFFFu, sp >> 16};
+                if (g + 1 < ng) {
+                    wa = __ldg(wsrc + 2 * (g + 1));
+                    wb = __ldg(wsrc + 2 * (g + 1) + 1);
+                    sp = __ldg(ssrc + g + 1);
+                } else if (i + 1 < n_my) {
+                    row_src(r0n, jn, wsrc_n, ssrc_n);
+                    wa = __ldg(wsrc_n);
+                    wb = __ldg(wsrc_n + 1);
+                    sp = __ldg(ssrc_n);
                 }
 #pragma unroll
-                for (int p = 0; p < 16; ++p)
-                    if ((m >> p) & 1u) v[p] = pw[p * 32];
-                __syncwarp();
-                tmem_st16(tmem + (uint32_t(32 * quarter) << 16) +
-                              uint32_t(kTcAccCols + s * kTcACols + mt * 32 + 16 * h),
-                          v);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(a_full + s);
-            }
-        }
-        // ---------------- epilogue: TMEM -> registers -> global
-        const bool acc_ok = mbar_wait(acc_full, 0);
-        ok = __all_sync(0xffffffffu, ok && acc_ok);
-        if (!ok) *fail = 1;
-        tc_fence_after();
-        if (ok) {
-            constexpr int kQCols = kTcChunk / 4;   // each (group, half) takes a quarter of the tokens
-            const int q4 = h + 2 * G;
-            for (int col = q4 * kQCols; col < q4 * kQCols + kQCols && col < n_mma; col += 16) {
-                float v1[16], v3[16];
-                tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(col), v1);
-                tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(kTcChunk + col), v3);
-                const int ra = r0 + t, rb = r0 + kTcM + t;   // rows of the two accumulators (two w2 tiles)
+                for (int s = 0; s < kTcStages; ++s) {
+                    if (ok && gg > 0 && !wait(kBarMmaDone + s, uint32_t((gg - 1) & 1))) ok = false;
+                    tc_fence_after();
+                    const int lo = (g * kTcStages + s) * kTcK + 32 * h, hi = lo + 32;
+                    const uint32_t w = wg[s], sc = sg[s >> 1];
+                    uint32_t v[16];
+                    expand_signs(w, sc, v);
+                    // outliers of this range replace their weights: each lane
+                    // walks its own entries (the next one already loaded),
+                    // parks the patched words in its column of the warp's
+                    // patch area and marks them; a predicated load per word
+                    // then takes them in, with no per-outlier select over the
+                    // sixteen words
+                    uint32_t m = 0u;
+                    int prev_p = -1;
+                    uint32_t prev_a = 0u;
+                    while (int(ent >> 16) < hi) {
+                        const int u = int(ent >> 16) - lo;
+                        const int P = u >> 1;
+                        const uint32_t val = ent & 0xFFFFu;
+                        uint32_t other = sc ^ (((w >> (u ^ 1)) & 1u) << 15);
+                        if (P == prev_p) other = (u & 1) ? (prev_a & 0xFFFFu) : (prev_a >> 16);
+                        const uint32_t a = (u & 1) ? (other | (val << 16)) : (val | (other << 16));
+                        prev_p = P;
+                        prev_a = a;
+                        pw[P * 32] = a;
+                        m |= 1u << P;
+                        ent = nxt;
+                        nxt = list[++cur + 1];
+                    }
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int j = col + i;
-                    if (j < job.n) {
-                        float* o = A.out + int64_t(job.n0 + j) * A.rows;
-                        if (GLU) {
-                            o[ra] = __fdividef(v1[i], 1.0f + __expf(-v1[i])) * v3[i];
-                        } else {
-                            o[ra] = v1[i];
-                            o[rb] = v3[i];
+                    for (int p = 0; p < 16; ++p)
+                        if ((m >> p) & 1u) v[p] = pw[p * 32];
+                    __syncwarp();
+                    tmem_st16(tmem + (uint32_t(32 * quarter) << 16) +
+                                  uint32_t(kTcAccCols + s * kTcACols + mt * 32 + 16 * h),
+                              v);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar + kBarAFull + s);
+                }
+            }
+            mbar_arrive(bar + kBarListFree + buf);   // the lists of item i are no longer read
+            wsrc = wsrc_n;
+            ssrc = ssrc_n;
+        }
+    } else {
+        // ---------------- aux warps: thread t owns row t of both operands.
+        // Step i builds the outlier lists of item i, then writes out the
+        // accumulators of item i - 1.
+        const int quarter = warp & 3;   // TMEM lane quarter this warp may access
+        const int t = 32 * quarter + lane;
+        for (int i = 0; i <= n_my; ++i) {
+            if (i < n_my) {
+                const int buf = i & 1;
+                bool ok = wait(kBarSideFull, uint32_t(i & 1));
+                if (ok && i >= 2) ok = wait(kBarListFree + buf, uint32_t(((i >> 1) - 1) & 1));
+                if (ok) {
+                    for (int mt = 0; mt < 2; ++mt) {
+                        // the columns of the first 32-column half of every K-step
+                        // (bit 5 clear), then those of the second half
+                        const uint16_t* sidx = reinterpret_cast<const uint16_t*>(smem + off_idx(mt)) + t * kout;
+                        const uint8_t* sqv = smem + off_q(mt);
+                        const float srow = __half2float(reinterpret_cast<const __half*>(smem + off_srow(mt))[t]);
+                        uint32_t* list = reinterpret_cast<uint32_t*>(smem + off_ent(buf, mt)) + t * (kout + 4);
+                        int n0 = 0;
+                        for (int j = 0; j < kout; ++j) n0 += ((sidx[j] >> 5) & 1) == 0;
+                        int o0 = 0, o1 = n0 + 2;
+                        for (int j = 0; j < kout; ++j) {
+                            const int c = sidx[j];
+                            const int n = t * kout + j;
+                            const int byte = sqv[n >> 1];
+                            int qv = (n & 1) ? (byte >> 4) : (byte & 0xF);
+                            qv = qv >= 8 ? qv - 16 : qv;
+                            const uint32_t e = (uint32_t(c) << 16) | __half_as_ushort(__float2half_rn(float(qv) * srow));
+                            if ((c >> 5) & 1) list[o1++] = e;
+                            else list[o0++] = e;
+                        }
+                        list[n0] = kSentinel;
+                        list[n0 + 1] = kSentinel;
+                        list[kout + 2] = kSentinel;
+                        list[kout + 3] = kSentinel;
+                        reinterpret_cast<int*>(smem + off_start1(buf))[mt * kTcM + t] = n0 + 2;
+                    }
+                }
+                mbar_arrive(bar + kBarSideFree);
+                mbar_arrive(bar + kBarListReady + buf);
+            }
+            if (i >= 1) {
+                int r0;
+                TcJob job;
+                item(i - 1, r0, job);
+                const int n_mma = (job.n + 15) & ~15;
+                const bool ok = __all_sync(0xffffffffu, wait(kBarAccFull, uint32_t((i - 1) & 1)));
+                tc_fence_after();
+                if (ok) {
+                    const int ra = r0 + t, rb = r0 + kTcM + t;   // rows of the two accumulators (two w2 tiles)
+                    for (int col = 0; col < n_mma; col += 16) {
+                        float v1[16], v3[16];
+                        tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(col), v1);
+                        tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(kTcChunk + col), v3);
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const int j = col + k;
+                            if (j < job.n) {
+                                float* o = A.out + int64_t(job.n0 + j) * A.rows;
+                                if (GLU) {
+                                    o[ra] = __fdividef(v1[k], 1.0f + __expf(-v1[k])) * v3[k];
+                                } else {
+                                    o[ra] = v1[k];
+                                    o[rb] = v3[k];
+                                }
+                            }
                         }
                     }
                 }
+                tc_fence_before();
+                mbar_arrive(bar + kBarAccEmpty);
             }
         }
     }
@@ -420,8 +552,9 @@ int launch_tc(const CUtensorMap& map, const TcArgs& a, int max_jobs, cudaStream_
     const TcSmem S = tc_smem(outliers_per_row(a.cols));
     int rc = ensure_smem(reinterpret_cast<const void*>(tc_tile_kernel<GLU>), S.bytes);
     if (rc != GALE_OK) return rc;
-    const int rows_per_cta = GLU ? kTcM : 2 * kTcM;
-    dim3 grid(unsigned(a.rows / rows_per_cta), unsigned(max_jobs));
+    const int64_t items = int64_t(a.rows / (GLU ? kTcM : 2 * kTcM)) * max_jobs;   // at most
+    const int grid = int(items < sm_count() ? items : sm_count());
+    if (grid == 0) return GALE_OK;
     tc_tile_kernel<GLU><<<grid, kTcThreads, S.bytes, st>>>(map, a);
     GALE_LAUNCH_CHECK();
     return GALE_OK;
