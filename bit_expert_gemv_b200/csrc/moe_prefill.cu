@@ -3,8 +3,7 @@
 // cores (tcgen05, accumulators in TMEM).
 //
 //   route   : stable counting sort of the (token, slot) pairs by expert
-//   jobs    : every expert's slots cut into chunks (128 tokens for w1/w3,
-//             256 for w2)
+//   jobs    : every expert's slots cut into chunks of 128 tokens
 //   gather  : x of every pair, in permuted order, rotated (FWHT-1024) to fp16
 //   w1/w3   : per (128-row tile, chunk): the packed signs are expanded in
 //             registers to fp16 +-s_blk (exact), the outliers patched in
@@ -12,7 +11,7 @@
 //             straight into TMEM; the tokens come in by TMA as the B operand;
 //             both products accumulate in TMEM; SwiGLU epilogue
 //   rotate  : h -> fp16 FWHT-1024
-//   w2      : the same tile kernel with one matrix
+//   w2      : the same tile kernel over pairs of 128-row tiles of w2
 //   combine : gate-weighted sum in fixed k order (+ residual, RMSNorm)
 //
 // A in TMEM keeps the shared-memory traffic to the B operand alone: the
