@@ -28,7 +28,8 @@ GALE_FLAG_RESIDUAL_RMSNORM = 1
 # every symbol include/gale.h declares
 EXPORTS = (
     "gale_status_string", "gale_pack_layout", "gale_expert_bytes", "gale_pack", "gale_unpack",
-    "gale_fwht1024", "gale_expert_gemv", "gale_route_permute", "gale_moe_workspace_size",
+    "gale_fwht1024", "gale_expert_gemv", "gale_route_permute", "gale_route_permute_scratch_bytes",
+    "gale_route_permute_grid", "gale_moe_workspace_size",
     "gale_moe_forward", "gale_moe_forward_noalloc", "gale_selftest_scratch_bytes", "gale_selftest",
     "gale_moe_host_staging_bytes", "gale_moe_host_workspace_size", "gale_moe_forward_host",
 )
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
             "gale_expert_gemv": (i32, [ctypes.POINTER(gale_matrix), ctypes.POINTER(gale_matrix), vp, i32,
                                        vp, i32, vp]),
             "gale_route_permute": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp]),
+            "gale_route_permute_scratch_bytes": (sz, [i32, i32, i32]),
+            "gale_route_permute_grid": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
             "gale_moe_workspace_size": (sz, [ctypes.POINTER(gale_layer), i32, i32]),
             "gale_moe_forward": (i32, [ctypes.POINTER(gale_layer), vp, vp, vp, i32, i32, vp, i32, i32,
                                        ctypes.c_float, vp, sz, vp]),
@@ -174,6 +177,19 @@ def gale_route_permute(ids, n_experts: int, counts, offsets, perm, status, strea
     B, K = ids.shape
     _check(lib().gale_route_permute(_ptr(ids), B, K, n_experts, _ptr(counts), _ptr(offsets), _ptr(perm),
                                     _ptr(status), _stream(stream)), "gale_route_permute")
+
+
+def gale_route_permute_scratch_bytes(B: int, K: int, n_experts: int) -> int:
+    return int(lib().gale_route_permute_scratch_bytes(B, K, n_experts))
+
+
+def gale_route_permute_grid(ids, n_experts: int, counts, offsets, perm, status, scratch, stream=None):
+    """The many-CTA routing permute (same results as gale_route_permute);
+    `scratch` is a device byte tensor of gale_route_permute_scratch_bytes()."""
+    B, K = ids.shape
+    _check(lib().gale_route_permute_grid(_ptr(ids), B, K, n_experts, _ptr(counts), _ptr(offsets), _ptr(perm),
+                                         _ptr(status), _ptr(scratch), scratch.numel() * scratch.element_size(),
+                                         _stream(stream)), "gale_route_permute_grid")
 
 
 def make_layer(base, expert_stride: int, n_experts: int, d_model: int, d_ff: int) -> gale_layer:

@@ -576,6 +576,7 @@ PrefillWs carve_prefill_ws(void* ws, const gale_layer& L, int B, int K) {
     w.offsets = reinterpret_cast<int32_t*>(take(4 * (int64_t(L.n_experts) + 1)));
     w.perm = reinterpret_cast<int32_t*>(take(4 * P));
     w.pos_of_pair = reinterpret_cast<int32_t*>(take(4 * P));
+    w.route_scratch = take(int64_t(route_grid_scratch_bytes(B, K, L.n_experts)));
     w.max_jobs = int(L.n_experts + P / kTcChunk + 1);
     w.jobs = take(int64_t(sizeof(TcJob)) * w.max_jobs);
     w.n_jobs = reinterpret_cast<int32_t*>(take(8));
@@ -614,7 +615,7 @@ int launch_moe_prefill(const gale_layer& L, const uint16_t* x, const int32_t* id
     ra.perm = w.perm;
     ra.pos_of_pair = w.pos_of_pair;
     ra.status = w.status;
-    int rc = launch_route_permute(ra, st);
+    int rc = launch_route_permute_grid(ra, w.route_scratch, st);
     if (rc != GALE_OK) return rc;
     prefill_jobs_kernel<<<1, 1024, 0, st>>>(w.counts, w.offsets, L.n_experts, static_cast<TcJob*>(w.jobs), w.n_jobs);
     GALE_LAUNCH_CHECK();

@@ -13,6 +13,7 @@ struct PrefillWs {
     int32_t* offsets;       // [E+1]
     int32_t* perm;          // [B*K]
     int32_t* pos_of_pair;   // [B*K]
+    void* route_scratch;    // range counts of the many-CTA routing permute
     void* jobs;             // [max_jobs] (expert, first slot, tokens), chunks of 128 slots
     int32_t* n_jobs;        // [1]
     int max_jobs;

@@ -144,6 +144,145 @@ __global__ void __launch_bounds__(1024) route_permute_kernel(RouteArgs a) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Many-CTA form for large batches (the one-CTA kernel above runs on one SM).
+// Warp range r holds the kGridWarpPairs pairs from r * kGridWarpPairs, walked
+// in kBlockSteps steps with one batch of id loads.  route_count_kernel writes
+// every range's per-expert counts [rows][E]; route_scan_kernel turns them, in
+// (expert, range) order, into each range's first position per expert
+// relative to the expert's offset, and writes counts and offsets;
+// route_place_kernel places every pair at its range's base + its running
+// rank.  The order is the same stable one.
+constexpr int kGridWarps = 8;                    // warps (ranges) per block
+constexpr int kGridWarpPairs = 32 * kBlockSteps;
+
+namespace {
+__host__ __device__ inline int64_t grid_rows(int64_t BK) { return (BK + kGridWarpPairs - 1) / kGridWarpPairs; }
+}  // namespace
+
+size_t route_grid_scratch_bytes(int B, int K, int E) {
+    return size_t(grid_rows(int64_t(B) * K)) * size_t(E) * 4;
+}
+
+// The validated experts of one warp range, handed to `f(p, e, grp)` step by
+// step (e < 0: dropped or past the end; grp: the lanes of the step with the
+// same e).
+template <typename F>
+__device__ __forceinline__ void walk_range(const RouteArgs& a, int p0, int p1, F f) {
+    const int lane = threadIdx.x & 31, BK = a.B * a.K;
+    int prev;
+    {
+        const int q = p0 - 32 + lane;
+        prev = (q >= 0 && q < BK) ? __ldg(a.ids + q) : -1;
+    }
+    int idb[kBlockSteps];
+    load_block(a, p0, p1, idb);
+#pragma unroll
+    for (int j = 0; j < kBlockSteps; ++j) {
+        const int base = p0 + 32 * j;
+        if (base >= p1) break;
+        const int e = step_experts(a, base, p1, idb[j], prev);
+        prev = idb[j];
+        const unsigned grp = __match_any_sync(0xffffffffu, e);
+        f(base + lane, e, grp);
+    }
+}
+
+__global__ void __launch_bounds__(kGridWarps * 32) route_count_kernel(RouteArgs a, int32_t* __restrict__ cnt) {
+    extern __shared__ int wc[];   // [kGridWarps][E]
+    const int E = a.E, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int BK = a.B * a.K;
+    const int64_t rows = grid_rows(BK);
+    for (int i = threadIdx.x; i < kGridWarps * E; i += blockDim.x) wc[i] = 0;
+    __syncthreads();
+    const int64_t r = int64_t(blockIdx.x) * kGridWarps + warp;
+    if (r < rows) {
+        const int p0 = int(r) * kGridWarpPairs, p1 = min(BK, p0 + kGridWarpPairs);
+        walk_range(a, p0, p1, [&](int p, int e, unsigned grp) {
+            if (p < p1 && e < 0) set_status(a.status, GALE_ERR_ARG);
+            if (e >= 0 && lane == __ffs(grp) - 1) wc[warp * E + e] += __popc(grp);
+            __syncwarp();
+        });
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kGridWarps * E; i += blockDim.x) {
+        const int w = i / E;
+        const int64_t rw = int64_t(blockIdx.x) * kGridWarps + w;
+        if (rw < rows) cnt[rw * E + (i - w * E)] = wc[i];
+    }
+}
+
+// One CTA: thread e runs down expert e's column of range counts.
+__global__ void __launch_bounds__(1024) route_scan_kernel(RouteArgs a, int32_t* __restrict__ cnt) {
+    __shared__ int s1[1024];
+    const int E = a.E, tid = threadIdx.x;
+    const int64_t rows = grid_rows(int64_t(a.B) * a.K);
+    int run = 0;
+    if (tid < E) {
+#pragma unroll 8
+        for (int64_t r = 0; r < rows; ++r) {
+            const int v = cnt[r * E + tid];
+            cnt[r * E + tid] = run;
+            run += v;
+        }
+    }
+    s1[tid] = tid < E ? run : 0;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {
+        const int v = tid >= off ? s1[tid - off] : 0;
+        __syncthreads();
+        s1[tid] += v;
+        __syncthreads();
+    }
+    if (tid < E) {
+        if (a.counts) a.counts[tid] = run;
+        a.offsets[tid] = s1[tid] - run;
+        if (tid == E - 1) a.offsets[E] = s1[tid];
+    }
+}
+
+__global__ void __launch_bounds__(kGridWarps * 32) route_place_kernel(RouteArgs a, const int32_t* __restrict__ base) {
+    extern __shared__ int wb[];   // [kGridWarps][E]: next position of each expert in each range
+    const int E = a.E, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int BK = a.B * a.K;
+    const int64_t rows = grid_rows(BK);
+    for (int i = threadIdx.x; i < kGridWarps * E; i += blockDim.x) {
+        const int w = i / E, e = i - w * E;
+        const int64_t rw = int64_t(blockIdx.x) * kGridWarps + w;
+        wb[i] = rw < rows ? base[rw * E + e] + a.offsets[e] : 0;
+    }
+    __syncthreads();
+    const int64_t r = int64_t(blockIdx.x) * kGridWarps + warp;
+    if (r >= rows) return;
+    const int p0 = int(r) * kGridWarpPairs, p1 = min(BK, p0 + kGridWarpPairs);
+    walk_range(a, p0, p1, [&](int p, int e, unsigned grp) {
+        if (e >= 0) {
+            const int pos = wb[warp * E + e] + __popc(grp & ((1u << lane) - 1u));
+            a.perm[pos] = p;
+            if (a.pos_of_pair) a.pos_of_pair[p] = pos;
+        }
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(grp) - 1) wb[warp * E + e] += __popc(grp);
+        __syncwarp();
+    });
+}
+
+int launch_route_permute_grid(const RouteArgs& a, void* scratch, cudaStream_t st) {
+    const int64_t BK = int64_t(a.B) * a.K;
+    if (BK == 0) return launch_route_permute(a, st);
+    if (!a.offsets) return GALE_ERR_ARG;
+    int32_t* cnt = static_cast<int32_t*>(scratch);
+    const unsigned blocks = unsigned((grid_rows(BK) + kGridWarps - 1) / kGridWarps);
+    const size_t smem = size_t(kGridWarps) * a.E * sizeof(int);
+    route_count_kernel<<<blocks, kGridWarps * 32, smem, st>>>(a, cnt);
+    GALE_LAUNCH_CHECK();
+    route_scan_kernel<<<1, 1024, 0, st>>>(a, cnt);
+    GALE_LAUNCH_CHECK();
+    route_place_kernel<<<blocks, kGridWarps * 32, smem, st>>>(a, cnt);
+    GALE_LAUNCH_CHECK();
+    return GALE_OK;
+}
+
 int launch_route_permute(const RouteArgs& a, cudaStream_t st) {
     const size_t smem = (size_t(32) * a.E + 2048) * sizeof(int);
     if (smem > 48 * 1024)
@@ -177,4 +316,34 @@ extern "C" int gale_route_permute(const int32_t* ids, int B, int K, int E, int32
     a.perm = perm;
     a.status = status;
     return gale::launch_route_permute(a, st);
+}
+
+extern "C" size_t gale_route_permute_scratch_bytes(int B, int K, int E) {
+    if (B < 0 || K < 1 || K > 16 || E < 1 || E > 1024) return 0;
+    return gale::route_grid_scratch_bytes(B, K, E);
+}
+
+extern "C" int gale_route_permute_grid(const int32_t* ids, int B, int K, int E, int32_t* counts,
+                                       int32_t* offsets, int32_t* perm, int32_t* status, void* scratch,
+                                       size_t scratch_bytes, void* stream) {
+    if (B < 0 || K < 1 || K > 16 || E < 1 || E > 1024 || !counts || !offsets || !status)
+        return GALE_ERR_ARG;
+    if (B > 0 && (!ids || !perm || !scratch)) return GALE_ERR_ARG;
+    if (!gale::aligned(ids, 4) || !gale::aligned(counts, 4) || !gale::aligned(offsets, 4) ||
+        !gale::aligned(perm, 4) || !gale::aligned(status, 4) || !gale::aligned(scratch, 4))
+        return GALE_ERR_ALIGN;
+    if (int64_t(B) * K > (1 << 30)) return GALE_ERR_UNSUPPORTED;
+    if (scratch_bytes < gale::route_grid_scratch_bytes(B, K, E)) return GALE_ERR_WORKSPACE;
+    cudaStream_t st = gale::as_stream(stream);
+    GALE_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+    gale::RouteArgs a{};
+    a.ids = ids;
+    a.B = B;
+    a.K = K;
+    a.E = E;
+    a.counts = counts;
+    a.offsets = offsets;
+    a.perm = perm;
+    a.status = status;
+    return gale::launch_route_permute_grid(a, scratch, st);
 }

@@ -18,4 +18,8 @@ struct RouteArgs {
 
 int launch_route_permute(const RouteArgs& a, cudaStream_t st);
 
+// Many-CTA form (three launches); `scratch` holds route_grid_scratch_bytes().
+size_t route_grid_scratch_bytes(int B, int K, int E);
+int launch_route_permute_grid(const RouteArgs& a, void* scratch, cudaStream_t st);
+
 }  // namespace gale

@@ -165,6 +165,20 @@ int gale_expert_gemv(const gale_matrix* W, const gale_matrix* W3, const float* x
 int gale_route_permute(const int32_t* ids, int B, int K, int E, int32_t* counts,
                        int32_t* offsets, int32_t* perm, int32_t* status, void* stream);
 
+/* The same permute spread over many CTAs, for large batches (the form above
+ * runs in one CTA on one SM): identical arguments, results (bit for bit),
+ * status and errors, plus
+ *   scratch       : device, 4-byte aligned, at least
+ *                   gale_route_permute_scratch_bytes(B, K, E) bytes; needs no
+ *                   initialisation and holds nothing after the call
+ *   scratch_bytes : its size; GALE_ERR_WORKSPACE if too small.
+ * Three kernel launches: per-range expert counts (ranges of 256 pairs), a
+ * scan in (expert, range) order, placement. */
+size_t gale_route_permute_scratch_bytes(int B, int K, int E);   /* 0 on invalid sizes */
+int gale_route_permute_grid(const int32_t* ids, int B, int K, int E, int32_t* counts,
+                            int32_t* offsets, int32_t* perm, int32_t* status, void* scratch,
+                            size_t scratch_bytes, void* stream);
+
 /* ---------------------------------------------------------------------------
  * One routed-expert MoE layer.
  * ------------------------------------------------------------------------- */

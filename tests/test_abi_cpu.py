@@ -57,6 +57,14 @@ def test_host_argument_validation():
     assert lib.gale_fwht1024(6, 0, 8, 0, 1, 1024, None) == G.GALE_ERR_ALIGN
     assert lib.gale_expert_gemv(None, None, None, 1, None, 0, None) == G.GALE_ERR_ARG
     assert lib.gale_route_permute(None, 1, 0, 256, None, None, None, None, None) == G.GALE_ERR_ARG
+    # the many-CTA permute: scratch of one int per (256-pair range, expert), checked before any CUDA call
+    assert G.gale_route_permute_scratch_bytes(4096, 6, 256) == 96 * 256 * 4
+    assert G.gale_route_permute_scratch_bytes(1, 6, 256) == 256 * 4
+    assert G.gale_route_permute_scratch_bytes(0, 6, 256) == 0
+    assert G.gale_route_permute_scratch_bytes(4, 17, 256) == 0
+    assert lib.gale_route_permute_grid(None, 1, 0, 256, None, None, None, None, None, 0, None) == G.GALE_ERR_ARG
+    assert lib.gale_route_permute_grid(16, 4, 6, 256, 16, 16, 16, 16, 16, 1023, None) == G.GALE_ERR_WORKSPACE
+    assert lib.gale_route_permute_grid(16, 4, 6, 256, 16, 16, 16, 16, 18, 1024, None) == G.GALE_ERR_ALIGN
     assert lib.gale_selftest(None, None) == G.GALE_ERR_ARG
     assert G.status_string(G.GALE_ERR_TIMEOUT).startswith("GALE_ERR_TIMEOUT")
 

@@ -156,16 +156,28 @@ def test_gemv_unit_scale_integer_exact(rows, cols):
 # routing permute
 # ----------------------------------------------------------------------------
 
+def _route(ids, E, counts, offsets, perm, status, grid):
+    """gale_route_permute, or its many-CTA form with a scratch buffer."""
+    if grid:
+        B, K = ids.shape
+        scratch = torch.empty(G.gale_route_permute_scratch_bytes(B, K, E), dtype=torch.uint8, device="cuda")
+        G.gale_route_permute_grid(to_dev(ids), E, counts, offsets, perm, status, scratch)
+    else:
+        G.gale_route_permute(to_dev(ids), E, counts, offsets, perm, status)
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("grid", [False, True])
 @pytest.mark.parametrize("B,K,E,skew", [(1, 6, 256, 0.0), (8, 6, 256, 0.0), (64, 6, 256, 0.5),
-                                         (4096, 6, 256, 0.5), (3, 2, 4, 0.0), (200, 16, 1024, 0.0)])
-def test_route_permute_bit_exact(B, K, E, skew):
+                                         (4096, 6, 256, 0.5), (3, 2, 4, 0.0), (200, 16, 1024, 0.0),
+                                         (20000, 6, 256, 0.5)])
+def test_route_permute_bit_exact(B, K, E, skew, grid):
     ids, _ = gs.route_topk(gs.router_logits(B, E, tag=B, bias_sigma=skew), K)
     counts = torch.empty(E, dtype=torch.int32, device="cuda")
     offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
     perm = torch.empty(B * K, dtype=torch.int32, device="cuda")
     status = torch.ones(1, dtype=torch.int32, device="cuda")
-    G.gale_route_permute(to_dev(ids), E, counts, offsets, perm, status)
-    torch.cuda.synchronize()
+    _route(ids, E, counts, offsets, perm, status, grid)
     wc, wo, wp = O.route_permute(ids, E)
     assert int(status.item()) == 0
     assert np.array_equal(counts.cpu().numpy(), wc)
@@ -186,31 +198,34 @@ def test_route_permute_flags_bad_ids():
     assert int(counts.sum().item()) == 7      # the repeated 3 and the id 300 are dropped
 
 
-def test_route_permute_drops_repeats_at_walk_boundaries():
+@pytest.mark.parametrize("grid", [False, True])
+def test_route_permute_drops_repeats_at_walk_boundaries(grid):
     """Repeated ids planted where a token's pairs straddle the boundaries of
     the kernel's walk: B = 4001, K = 6 gives 32 warp ranges of 751 pairs,
     walked 32 pairs a step and eight steps per batch of loads.  Token 125
     straddles warp ranges 0 / 1 (pair 751), token 5 a step boundary (pair 32),
-    token 167 the batch boundary of range 1 (pair 751 + 256 = 1007).  The
-    later pair of each repeat is dropped; the rest is the stable sort by
-    (expert, pair), checked against a plain sort of the valid pairs."""
+    token 167 the batch boundary of range 1 (pair 751 + 256 = 1007), token 42
+    the batch boundary of range 0 (pair 256), which is also the boundary of
+    the many-CTA form's first 256-pair range.  The later pair of each repeat
+    is dropped; the rest is the stable sort by (expert, pair), checked
+    against a plain sort of the valid pairs."""
     B, K, E = 4001, 6, 256
     ids, _ = gs.route_topk(gs.router_logits(B, E, tag=4001, bias_sigma=0.5), K)
     ids = ids.copy()
     ids[125, 1] = ids[125, 0]   # pairs 750 | 751
     ids[5, 3] = ids[5, 0]       # pairs 30 | 33
     ids[167, 5] = ids[167, 1]   # pairs 1003 | 1007
+    ids[42, 5] = ids[42, 0]     # pairs 252 | 257
     flat = ids.reshape(-1)
     valid = [p for p in range(B * K) if flat[p] not in flat[p - p % K:p]]
-    assert len(valid) == B * K - 3
+    assert len(valid) == B * K - 4
     want_counts = np.bincount(flat[valid], minlength=E).astype(np.int32)
     want_perm = np.array(sorted(valid, key=lambda p: (flat[p], p)), np.int32)
     counts = torch.empty(E, dtype=torch.int32, device="cuda")
     offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
     perm = torch.full((B * K,), -7, dtype=torch.int32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    G.gale_route_permute(to_dev(ids), E, counts, offsets, perm, status)
-    torch.cuda.synchronize()
+    _route(ids, E, counts, offsets, perm, status, grid)
     assert int(status.item()) == G.GALE_ERR_ARG
     assert np.array_equal(counts.cpu().numpy(), want_counts)
     assert np.array_equal(offsets.cpu().numpy(), np.concatenate([[0], np.cumsum(want_counts)]).astype(np.int32))
