@@ -413,6 +413,72 @@ def test_rmsnorm():
     assert abs(O.rmsnorm(c, 1e-6)[0] - 2.0 / math.sqrt(4.0 + 1e-6)) < 1e-15
 
 
+
+def _chain_hand_case(a: float, i: int, experts, eps: float):
+    """A chain step whose every quantity has a closed form (d_model = d_ff = 1024).
+
+    x[c] = a * (-1)^popcount(i & c), so the rotated input is 32 a e_i (H times its
+    own column i is 1024 e_i, times 1/32).  Expert (alpha, beta, gamma, gate) has
+    dense W1 = alpha and W3 = beta on column i only, and W2 = gamma on column 0
+    only: g1 = 32 a alpha and g3 = 32 a beta on every row, h is the constant
+    silu(g1) g3, its rotation is 32 h e_0 (H times the all-ones vector is
+    1024 e_0), and every output row is 32 gamma h.  Returns (x, dense experts,
+    ids, gates, expected output written out by hand with the math module)."""
+    d = 1024
+    col = np.array([(-1) ** bin(i & c).count("1") for c in range(d)], np.float64)
+    x = a * col
+    dense, Y = [], 0.0
+    for alpha, beta, gamma, gate in experts:
+        W1 = np.zeros((d, d)); W1[:, i] = alpha
+        W3 = np.zeros((d, d)); W3[:, i] = beta
+        W2 = np.zeros((d, d)); W2[:, 0] = gamma
+        dense.append([W1, W3, W2])
+        g1, g3 = 32.0 * a * alpha, 32.0 * a * beta
+        h = g1 / (1.0 + math.exp(-g1)) * g3
+        Y += gate * 32.0 * gamma * h
+    # v = x + Y; mean(v^2) = a^2 + Y^2 because column i != 0 of H sums to zero
+    ms = a * a + Y * Y
+    want = (x + Y) / math.sqrt(ms + eps)
+    ids = np.arange(len(experts), dtype=np.int32)[None, :]
+    gates = np.array([[e[3] for e in experts]], np.float32)
+    return x, dense, ids, gates, want
+
+
+@pytest.mark.parametrize("a,eps", [(2.0 ** -10, 1e-6), (0.5, 1e-6), (2.0 ** -10, 0.0)])
+def test_chain_step_closed_form(a, eps):
+    # two experts with gates that are exact in fp32; a = 2^-10 makes mean(v^2)
+    # the size of eps, so eps outside the square root would be seen
+    experts = [(0.75, -0.5, 0.125, 0.625), (-0.25, 1.5, -0.0625, 0.375)]
+    x, dense, ids, gates, want = _chain_hand_case(a, 37, experts, eps)
+    got = O.chain_step(lambda e: dense[e], x[None, :], ids, gates, eps)[0]
+    assert np.max(np.abs(got - want)) <= 1e-12 * np.max(np.abs(want))
+    # the pin tells the plausible slips apart: each differs from the hand value
+    y = O.moe_layer(lambda e: dense[e], x[None, :], ids, gates)[0]
+    slips = {
+        "residual dropped": O.rmsnorm(y, eps),
+        "norm before the add": O.rmsnorm(x, eps) + y,
+        "eps outside the root": (x + y) / (np.sqrt(np.mean((x + y) ** 2)) + eps),
+        "norm of y, x added after": x + O.rmsnorm(y, eps),
+    }
+    for name, v in slips.items():
+        if name == "eps outside the root" and (eps == 0.0 or a * a > 1e-4):
+            continue   # only the small case, where mean(v^2) is the size of eps, sees it
+        assert np.max(np.abs(v - want)) > 1e-4 * np.max(np.abs(want)), name
+
+
+def test_chain_step_zero_gates_is_rmsnorm_of_x():
+    # with every gate 0 the layer adds nothing: the step is RMSNorm(x) exactly
+    rng = np.random.default_rng(5)
+    d = 1024
+    dense = [[rng.standard_normal((d, d)) for _ in range(3)] for _ in range(2)]
+    x = rng.standard_normal((3, d)).astype(np.float32).astype(np.float64)
+    ids = np.array([[0, 1], [1, 0], [0, 1]], np.int32)
+    gates = np.zeros((3, 2), np.float32)
+    got = O.chain_step(lambda e: dense[e], x, ids, gates, 1e-6)
+    for t in range(3):
+        want = x[t] / math.sqrt(sum(float(v) * float(v) for v in x[t]) / d + 1e-6)
+        assert np.max(np.abs(got[t] - want)) <= 1e-14 * np.max(np.abs(want))
+
 # ----------------------------------------------------------------------------
 # seeded generator (inputs, not oracle arithmetic)
 # ----------------------------------------------------------------------------
