@@ -39,8 +39,21 @@ CHAIN_LAYERS = 43
 # kernels of this library launched per decode step (the cooperative layer kernel)
 DECODE_LAUNCHES = 1
 # dram read + write bytes of one decode launch at this workload, from an ncu
-# capture of the current kernel (None once the kernel has changed since)
-DECODE_TRAFFIC = 25_196_800
+# capture (profiles/moe_decode_kernel_b1.md), and the sha256 prefix of the
+# kernel source it was taken on: the bench reports it only while the source is
+# unchanged, and null after any edit until the capture is taken again.
+DECODE_TRAFFIC = None
+DECODE_TRAFFIC_SRC = ""
+KERNEL_SRC = os.path.join(ROOT, "bit_expert_gemv_b200", "csrc", "moe_decode.cu")
+
+
+def decode_traffic():
+    import hashlib
+    if DECODE_TRAFFIC is None:
+        return None
+    with open(KERNEL_SRC, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    return DECODE_TRAFFIC if h == DECODE_TRAFFIC_SRC else None
 WORKLOAD = ("moe_layer_decode: 256 GALE-1bit experts (w1/w3 [2048x4096], w2 [4096x2048]), "
             "top-6 softmax routing, bf16 hidden [B x 4096]")
 
@@ -60,6 +73,18 @@ def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return rank, world, local
+
+
+def relaunch_replicas(n: int):
+    """`bench.py --gpus N` started without torchrun: run the same command as N
+    replica processes under torch.distributed.run (one per GPU)."""
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    os.execv(sys.executable, cmd)
 
 
 def max_over_ranks(values, world, device):
@@ -262,6 +287,36 @@ def run_gpu(args):
         d2h = B * D_MODEL * 4
         return total, h2d, d2h
 
+    def measure_single(steps, warmup):
+        """One GALE expert on one token, x fp32 N(0,1) [4096]: FWHT of x, the
+        fused w1/w3 GEMV + SwiGLU, FWHT of h, the w2 GEMV (expert 0 of the
+        resident layer), L2 flushed before every step (outside the events)."""
+        l1 = G.gale_pack_layout(D_FF, D_MODEL)["total"]
+        w1, w3, w2 = buf[0:], buf[l1:], buf[2 * l1:]
+        xs = [torch.from_numpy(gs.x_f32(D_MODEL, tag=95_000 + i)).cuda().view(1, D_MODEL)
+              for i in range(steps + warmup)]
+        xr = torch.empty(1, D_MODEL, dtype=torch.float32, device="cuda")
+        h = torch.empty(1, D_FF, dtype=torch.float32, device="cuda")
+        y = torch.empty(1, D_MODEL, dtype=torch.float32, device="cuda")
+
+        def step(x):
+            G.gale_fwht1024(x, xr)
+            G.gale_expert_gemv(w1, D_FF, D_MODEL, xr, h, W3=w3, mode=G.GALE_MODE_SWIGLU)
+            G.gale_fwht1024(h, h)
+            G.gale_expert_gemv(w2, D_MODEL, D_FF, h, y)
+
+        for i in range(warmup):
+            step(xs[i])
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step(xs[warmup + i])
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) * 1e-3 for a, b in ev)
+
     def measure_chain(steps, warmup, n_layers=CHAIN_LAYERS):
         """Decode batch 1 through n_layers layers of 256 resident experts each:
         x_{l+1} = bf16(RMSNorm(x_l + MoE_l(x_l))), fresh seeded routing per
@@ -337,6 +392,7 @@ def run_gpu(args):
     # decode batch 64 with per-expert popularity bias N(0, 0.5) (skewed tokens per expert)
     t64, bytes64, _ = measure(64, max(args.steps // 2, 3), args.warmup, 25_000, bias_sigma=0.5)
     te, h2d, d2h = measure_e2e(1, args.steps, args.warmup, 30_000)
+    ts = measure_single(args.steps, args.warmup)
     # prefill: 4096 tokens, skewed routing (tensor-core tile path)
     pf_steps = max(3, min(args.steps // 5, 10))
     tp, _, _ = measure(PREFILL_B, pf_steps, 3, 40_000, bias_sigma=0.5, n_x=2)
@@ -345,7 +401,7 @@ def run_gpu(args):
     clocks_info = clocks.stop()
 
     # max over ranks of the device time
-    t1, t8, t64, te, tp, tc = max_over_ranks([t1, t8, t64, te, tp, tc], world, "cuda")
+    t1, t8, t64, te, tp, tc, ts = max_over_ranks([t1, t8, t64, te, tp, tc, ts], world, "cuda")
     tokens, value = job_throughput(1, args.steps, world, t1)
     gbs = bytes1 * world / t1 / 1e9
     peak, tpeak, peak_kind = peaks()
@@ -355,15 +411,17 @@ def run_gpu(args):
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * t1 / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "s8x3 fixed-point activations x 1-bit signs, s32 accumulate, fp32 scales and sums",
+        "data": "synthetic",
         "config": {"workload": WORKLOAD, "B": 1, "experts": N_EXPERTS, "top_k": TOP_K,
                    "d_model": D_MODEL, "d_ff": D_FF, "packed_bytes_per_expert": expert_bytes,
                    "l2": "flushed between timed steps (write of 2x L2, outside the events)",
                    "routing": "fresh seeded routing every step", "parallelism": f"replicas{world}"},
         "hbm_gbs": gbs,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": DECODE_TRAFFIC, "peak_kind": peak_kind,
-                     "kernel": "moe_decode_kernel (the whole layer is this one launch)",
+                     "frac": achieved / peak, "traffic": decode_traffic(), "peak_kind": peak_kind,
+                     "kernel": "moe_decode_kernel (batch 1: the whole layer is this one launch)",
                      "algorithmic_bytes_per_launch": bytes1 / args.steps},
         "b8": {"tokens_per_s": 8 * max(args.steps // 2, 3) * world / t8,
                "hbm_gbs": bytes8 * world / t8 / 1e9, "frac": bytes8 * world / t8 / 1e9 / peak},
@@ -381,6 +439,11 @@ def run_gpu(args):
                     "tflops": pf_flops * pf_steps / tp / 1e12, "peak_tflops": tpeak,
                     "frac": pf_flops * pf_steps / tp / 1e12 / tpeak, "bound": "tensor",
                     "flops_per_step": pf_flops, "steps": pf_steps},
+        "single_expert": {"workload": "one GALE expert, one token, fp32 x [4096] (w1/w3 [2048x4096], w2 [4096x2048]):"
+                                      " FWHT, w1/w3 GEMV + SwiGLU, FWHT, w2 GEMV (4 launches), L2 flushed",
+                          "tokens_per_s": args.steps * world / ts, "us_per_step": 1e6 * ts / args.steps,
+                          "hbm_gbs": expert_bytes * args.steps * world / ts / 1e9,
+                          "frac": expert_bytes * args.steps * world / ts / 1e9 / peak, "launches_per_step": 4},
         "e2e": {"value": tokens / te, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": DECODE_LAUNCHES * args.steps,
         "clocks": clocks_info,
@@ -435,34 +498,59 @@ def _threads():
         return os.cpu_count() or 1
 
 
-def oracle_step(O, B, tag):
-    lg = gs.router_logits(B, N_EXPERTS, tag=tag)
-    ids, gates = gs.route_topk(lg, TOP_K)
-    _, xv = gs.hidden_bf16(B, D_MODEL, tag=tag)
-    cache = {}
+def oracle_inputs(O, n: int, tag0: int):
+    """n decode-batch-1 steps of seeded routing and hidden states, with every
+    expert they touch generated and packed by the oracle's own packer; all of
+    this happens before any timing."""
+    steps = []
+    for i in range(n):
+        ids, gates = gs.route_topk(gs.router_logits(1, N_EXPERTS, tag=tag0 + i), TOP_K)
+        _, xv = gs.hidden_bf16(1, D_MODEL, tag=tag0 + i)
+        packed = {int(e): [O.pack(c) for c in gs.expert_canonical(D_MODEL, D_FF, expert=int(e))]
+                  for e in np.unique(ids)}
+        steps.append((xv, ids, gates, packed))
+    return steps
 
-    def dense(e):
-        if e not in cache:
-            cs = gs.expert_canonical(D_MODEL, D_FF, expert=e)
-            cache[e] = [O.dequant_packed(O.pack(c), c["rows"], c["cols"]) for c in cs]
-        return cache[e]
 
-    O.moe_layer(dense, xv, ids, gates)
-    return B
+def oracle_step(O, step):
+    """The oracle on one prepared step: unpack and dense fp64 dequantisation
+    of the six experts, FWHT, SwiGLU, w2 and the gate-weighted combine."""
+    xv, ids, gates, packed = step
+    shapes = [(D_FF, D_MODEL), (D_FF, D_MODEL), (D_MODEL, D_FF)]
+    dense = {e: [O.dequant_packed(b, r, c) for b, (r, c) in zip(v, shapes)] for e, v in packed.items()}
+    O.moe_layer(dense.__getitem__, xv, ids, gates)
+    return 1
 
 
 def cpu_baseline(budget_s: float):
+    """The oracle as it stands on the host cores: half the budget on all BLAS
+    threads, half on one thread (experts generated and packed beforehand)."""
     from oracle import gale_oracle as O
-    t0 = time.perf_counter()
-    toks = 0
-    n = 0
-    while time.perf_counter() - t0 < budget_s and n < 64:
-        toks += oracle_step(O, 1, 50_000 + n)
-        n += 1
-    dt = time.perf_counter() - t0
-    return {"value": toks / dt, "unit": UNIT, "cores": _threads(), "kind": "oracle",
-            "sample": f"{n} decode-B1 layer steps (6 experts each, unpack + dense fp64 dequant + FWHT + "
-                      f"SwiGLU + combine), {dt:.1f} s"}
+    from threadpoolctl import threadpool_limits
+    inputs = oracle_inputs(O, 8, 50_000)
+    oracle_step(O, inputs[0])   # first touch of the allocator's pages, untimed
+    res = {}
+    for label, limit in (("all", None), ("one", 1)):
+        ctx = threadpool_limits(limit) if limit else None
+        if ctx:
+            ctx.__enter__()
+        try:
+            cores = _threads()
+            t0 = time.perf_counter()
+            n = 0
+            while (time.perf_counter() - t0 < budget_s / 2 or n == 0) and n < len(inputs):
+                oracle_step(O, inputs[(n + 1) % len(inputs)])
+                n += 1
+            res[label] = (n / (time.perf_counter() - t0), cores, n)
+        finally:
+            if ctx:
+                ctx.__exit__(None, None, None)
+    v, cores, n = res["all"]
+    v1, _, n1 = res["one"]
+    return {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} decode-B1 layer steps on {cores} threads and {n1} on one (6 experts each: unpack, "
+                      f"dense fp64 dequant, FWHT, SwiGLU, w2, combine; experts packed before the clock)",
+            "single_thread": {"value": v1, "unit": UNIT, "cores": 1}}
 
 
 def run_reference(args):
@@ -470,11 +558,12 @@ def run_reference(args):
     if rank != 0:
         return
     from oracle import gale_oracle as O
+    inputs = oracle_inputs(O, min(args.steps, 8), 70_000)
     for s in range(args.warmup):
-        oracle_step(O, 1, 60_000 + s)
+        oracle_step(O, inputs[s % len(inputs)])
     t0 = time.perf_counter()
     for s in range(args.steps):
-        oracle_step(O, 1, 70_000 + s)
+        oracle_step(O, inputs[s % len(inputs)])
     dt = time.perf_counter() - t0
     value = args.steps / dt
     print(json.dumps({
@@ -484,7 +573,7 @@ def run_reference(args):
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "B": 1, "experts": N_EXPERTS, "top_k": TOP_K},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads(), "kind": "oracle",
-                         "sample": f"{args.steps} decode-B1 layer steps"},
+                         "sample": f"{args.steps} decode-B1 layer steps (experts packed before the clock)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -504,6 +593,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        relaunch_replicas(args.gpus)
     if args.impl == "reference":
         run_reference(args)
     elif args.only:

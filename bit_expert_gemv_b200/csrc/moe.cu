@@ -9,6 +9,7 @@
 #include "gemv_simple.cuh"
 #include "moe.cuh"
 #include "moe_decode.cuh"
+#include "moe_stream.cuh"
 #include "moe_prefill.cuh"
 #include "route.cuh"
 
@@ -17,6 +18,11 @@ namespace gale {
 constexpr int kGWarps = 8;
 constexpr int kGRowsPerWarp = 8;
 constexpr int kGRowsPerCta = kGWarps * kGRowsPerWarp;
+
+// One or two tokens take the small-batch decode kernel (measured faster there
+// than the streaming kernel, whose per-CTA planning and phase hand-off cost
+// more than they save at this size).
+bool small_batch(const gale_layer& L, int B, int K) { return B >= 1 && B <= 2 && decode_supported(L, B, K); }
 
 MoeWs carve_ws(void* ws, const gale_layer& L, int B, int K) {
     MoeWs w{};
@@ -217,7 +223,8 @@ extern "C" size_t gale_moe_workspace_size(const gale_layer* layer, int B, int K)
     size_t n = gale::carve_ws(nullptr, *layer, B, K).bytes;
     // each batch takes exactly one path; its workspace also holds the status word
     size_t p = 0;
-    if (gale::decode_supported(*layer, B, K)) p = gale::carve_decode_ws(nullptr, *layer, B, K).bytes;
+    if (gale::small_batch(*layer, B, K)) p = gale::carve_decode_ws(nullptr, *layer, B, K).bytes;
+    else if (gale::stream_supported(*layer, B, K)) p = gale::carve_stream_ws(nullptr, *layer, B, K).bytes;
     else if (gale::prefill_supported(*layer, B, K)) p = gale::carve_prefill_ws(nullptr, *layer, B, K).bytes;
     return p > n ? p : n;
 }
@@ -236,22 +243,26 @@ extern "C" int gale_moe_forward(const gale_layer* layer, const uint16_t* x, cons
     if (!ws) return GALE_ERR_WORKSPACE;
     const gale_layer& L = *layer;
     MoeWs w = carve_ws(ws, L, B, K);
-    const bool decode = decode_supported(L, B, K);
-    const bool prefill = !decode && prefill_supported(L, B, K);
-    if (ws_bytes < w.bytes || (decode && ws_bytes < carve_decode_ws(nullptr, L, B, K).bytes) ||
+    const bool small = small_batch(L, B, K);
+    const bool decode = !small && stream_supported(L, B, K);
+    const bool prefill = !small && !decode && prefill_supported(L, B, K);
+    if (ws_bytes < w.bytes || (small && ws_bytes < carve_decode_ws(nullptr, L, B, K).bytes) ||
+        (decode && ws_bytes < carve_stream_ws(nullptr, L, B, K).bytes) ||
         (prefill && ws_bytes < carve_prefill_ws(nullptr, L, B, K).bytes))
         return GALE_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return GALE_ERR_ALIGN;
     cudaStream_t st = as_stream(stream);
-    // the status word and the decode kernel's grid-barrier counters
-    GALE_CUDA_TRY(cudaMemsetAsync(w.status, 0, 8 * sizeof(int32_t), st));
+    // the status word (and the small-batch kernel's grid-barrier counters)
+    if (!decode || B == 0) GALE_CUDA_TRY(cudaMemsetAsync(w.status, 0, 8 * sizeof(int32_t), st));
     if (B == 0) return GALE_OK;
     if (!x || !ids || !gates || !out) return GALE_ERR_ARG;
     if (!aligned(x, 4) || !aligned(ids, 4) || !aligned(gates, 4) || !aligned(out, 4)) return GALE_ERR_ALIGN;
     const int64_t BK = int64_t(B) * K;
     if (BK > (1 << 24)) return GALE_ERR_UNSUPPORTED;
-    // decode batches: tensor-core streaming kernels
-    if (decode) return launch_moe_decode(L, x, ids, gates, B, K, out, out_dtype, fuse, eps, ws, st);
+    // one or two tokens: the small-batch decode kernel
+    if (small) return launch_moe_decode(L, x, ids, gates, B, K, out, out_dtype, fuse, eps, ws, st);
+    // other decode batches: the streaming kernel (it clears its own status word and counters)
+    if (decode) return launch_moe_stream(L, x, ids, gates, B, K, out, out_dtype, fuse, eps, ws, st);
     // larger batches: tcgen05 tensor-core tiles
     if (prefill) return launch_moe_prefill(L, x, ids, gates, B, K, out, out_dtype, fuse, eps, ws, st);
 

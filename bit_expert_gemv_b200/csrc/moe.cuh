@@ -50,5 +50,6 @@ struct CombineArgs {
 };
 
 int validate_layer(const gale_layer* L);
+bool small_batch(const gale_layer& L, int B, int K);
 
 }  // namespace gale

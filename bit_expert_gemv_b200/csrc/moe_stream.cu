@@ -1,0 +1,1236 @@
+// Decode path of gale_moe_forward: the routed-expert layer for batches of up
+// to 384 (token, expert) pairs as one persistent kernel, one CTA per SM,
+// launched cooperatively (all CTAs resident: CTAs wait on each other's h).
+//
+// Work.  The (token, k) pairs are grouped by expert, stable in pair order,
+// and every expert's pairs are cut into segments of at most two (one MMA
+// column group).  A unit is
+//   phase 1: (segment, 16 rows of w1 and the same 16 rows of w3), full width;
+//   phase 2: (segment, 64 rows of w2), full width.
+// Each phase's unit list is cut into one contiguous range per CTA.
+//
+// Roles inside a CTA (15 consumer warps and one producer warp):
+//  - producer: streams the packed rows of the CTA's units, phase 1 then
+//    phase 2, into a ring of stages: the sign rows as one TMA tensor box with
+//    128-byte swizzle, block scales, row scales, outlier columns and values
+//    as bulk copies.  It waits only for a stage to be released, so the w2 rows
+//    arrive while w1/w3 are still being computed; at batch 1 the ring holds
+//    nearly a CTA's whole share of the layer.
+//  - consumers: take pieces from one queue in unit order.  A unit has one
+//    piece per (1024-column chunk, 32 rows) on the int8 tensor cores and two
+//    outlier pieces.  The warp that finishes a unit's last piece sums the
+//    partial sums in a fixed order and writes the rows:
+//      phase 1: h = silu(w1 x) * (w3 x) into the workspace, then counts the
+//               tile into the readiness counter of its (segment, 1024-block);
+//      phase 2: the expert outputs o, then counts the unit into the
+//               (token, 64-row block) counter; the last of a token's experts
+//               sums the K outputs in fixed k order with the gates, and with
+//               the fused norm the last block of a token applies the residual
+//               and RMSNorm.
+//    Activations (x in phase 1, h in phase 2) are rotated by the blocked
+//    FWHT-1024 into one of two slots by the consumer warps, one group of
+//    segments at a time: consecutive phase-1 segments with the same tokens
+//    share a slot (at batch 1 a CTA rotates x once).  A phase-2 slot waits
+//    until the segment's h blocks are complete in every CTA.
+//
+// Arithmetic of a tile (mma.sync m16n8k32, int8, exact int32 sums).  For row
+// r and a 128-column block b,  sum_c sign(r,c) x_c = X_b - 2 P_b  with
+// P_b = sum_{c in b, bit(r,c)=1} x_c.  A sign word w of 32 columns gives the
+// A operand of bit position s as w & (0x01010101 << s), whose bytes are
+// bit * a(s), a(s) = 2^s for s < 7 and -128 for s = 7.  Each 1024-block of an
+// activation is held in fixed point, X_c = round(u_c S / a(c mod 8)) with u
+// the unnormalised transform and S a power of two such that |u S| <= 2^20,
+// as three int8 digits (X = d1 2^14 + d2 2^7 + d3), one MMA column per digit
+// and token; the block sums X_b are exact integers of the same values.  The
+// outlier corrections (q s_row - sign s_blk) x_c read x_c from an fp16 copy
+// of u S / 64 (per-block scale, so it cannot overflow).
+//
+// Code size matters here: code run once per launch is fetched cold, so the
+// helpers are single out-of-line copies with rolled loops.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "moe_stream.cuh"
+#include "ptx.cuh"
+#include "tma.cuh"
+
+namespace gale {
+
+namespace {
+
+constexpr int kCW = 15;                       // consumer warps (16 warps in all: 128 registers each)
+constexpr int kThreads = (kCW + 1) * 32;      // + the producer warp
+constexpr int kSegTok = 2;                    // pairs per segment
+constexpr int kMaxStages = 12;
+constexpr int kMaxLocalSeg = 64;
+constexpr int kSmemBytes = 227 * 1024;
+constexpr int kR1 = 16;                       // rows of w1 (and of w3) per phase-1 unit
+constexpr int kR2 = 64;                       // rows of w2 per phase-2 unit
+constexpr int kPartBytes = 192 * kSegTok * 4; // partial sums of a stage: 192 rows x 2 tokens
+constexpr uint64_t kWaitNs = 2000000000ull;   // bound of every wait
+
+struct StreamArgs {
+    const char* base;
+    int64_t stride;
+    int E, d_model, d_ff, B, K;
+    int64_t off_w[3];       // w1, w3, w2 inside a record
+    const uint16_t* x;
+    const int32_t* ids;
+    const float* gates;
+    void* out;
+    int out_dtype, fuse_norm;
+    float eps;
+    StreamWs ws;
+};
+
+// Byte offsets inside a stage for each phase (the rest of the stage after
+// the data is the partial-sum area).
+struct StageMap {
+    int sb, sr, idx, q;     // block scales, row scales, outlier columns, values
+    int sb_bytes;           // block scales of one matrix
+    int idx_bytes;          // outlier columns of one matrix
+    int q_bytes;            // room for the values of one matrix
+};
+
+// Activation layout of one token in a slot (bytes): digits [cols/128][3][4][32],
+// int32 128-block sums, fp32 1024-block factors sigma = 1/(32 S), fp16 copy of
+// u S / 64 in column order, fp32 factors 2 / S of that copy.
+struct TokMap {
+    int xsum, sig, x16, f16, bytes;
+};
+
+struct Plan {
+    int C1, C2;                  // columns of w1/w3 (d_model) and of w2 (d_ff)
+    int nch1, nch2;              // 1024-column chunks
+    int k1, k2;                  // outliers per row
+    int tiles1, tiles2;          // units per segment in each phase
+    int pp1, pp2;                // pieces per unit
+    TokMap t1, t2;
+    StageMap m1, m2;
+    int part;                    // partial area offset in a stage
+    int stage_bytes;
+    Layout L1, L2;
+};
+
+__host__ __device__ inline int align_i(int n, int a) { return (n + a - 1) / a * a; }
+
+__host__ __device__ inline TokMap make_tokmap(int C) {
+    TokMap t;
+    t.xsum = 3 * C;
+    t.sig = t.xsum + C / 32;
+    t.x16 = align_i(t.sig + 4 * (C / 1024), 16);
+    t.f16 = t.x16 + 2 * C;
+    t.bytes = align_i(t.f16 + 4 * (C / 1024), 128);
+    return t;
+}
+
+__host__ __device__ inline Plan make_stream_plan(int d_model, int d_ff) {
+    Plan p{};
+    p.C1 = d_model;
+    p.C2 = d_ff;
+    p.nch1 = d_model / 1024;
+    p.nch2 = d_ff / 1024;
+    p.k1 = outliers_per_row(d_model);
+    p.k2 = outliers_per_row(d_ff);
+    p.tiles1 = d_ff / kR1;
+    p.tiles2 = d_model / kR2;
+    p.pp1 = p.nch1 + 2;
+    p.pp2 = 2 * p.nch2 + 2;
+    p.t1 = make_tokmap(d_model);
+    p.t2 = make_tokmap(d_ff);
+    // phase 1: signs [mat 2][chunk][16 rows][128 B]
+    p.m1.sb_bytes = kR1 * (p.C1 / 64);
+    p.m1.idx_bytes = kR1 * p.k1 * 2;
+    p.m1.q_bytes = align_i(kR1 * p.k1 / 2, 16) + 16;
+    p.m1.sb = 2 * p.nch1 * 2048;
+    p.m1.sr = p.m1.sb + 2 * p.m1.sb_bytes;
+    p.m1.idx = p.m1.sr + 2 * 32;
+    p.m1.q = p.m1.idx + 2 * align_i(p.m1.idx_bytes, 16);
+    const int end1 = p.m1.q + 2 * p.m1.q_bytes;
+    // phase 2: signs [chunk][64 rows][128 B]
+    p.m2.sb_bytes = kR2 * (p.C2 / 64);
+    p.m2.idx_bytes = kR2 * p.k2 * 2;
+    p.m2.q_bytes = align_i(kR2 * p.k2 / 2, 16) + 16;
+    p.m2.sb = p.nch2 * kR2 * 128;
+    p.m2.sr = p.m2.sb + p.m2.sb_bytes;
+    p.m2.idx = p.m2.sr + align_i(kR2 * 2, 16);
+    p.m2.q = p.m2.idx + align_i(p.m2.idx_bytes, 16);
+    const int end2 = p.m2.q + p.m2.q_bytes;
+    p.part = align_i(end1 > end2 ? end1 : end2, 128);
+    p.stage_bytes = align_i(p.part + kPartBytes, 1024);
+    p.L1 = make_layout(d_ff, d_model);
+    p.L2 = make_layout(d_model, d_ff);
+    return p;
+}
+
+// Shared control block.
+struct Ctl {
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
+    int next_piece;
+    int abort;
+    int stage_done[kMaxStages];
+    int slot_grp[2];       // group of segments held (or being built) by each slot
+    int slot_claim[2];     // (group << 16) | activation pieces claimed for that group
+    int slot_done[2];      // and finished
+    int n_valid, n_seg, bad;
+    int u1b, u1e, u2b, u2e;      // this CTA's unit ranges (global unit indices)
+    int s1b, s2b, nl1, nl, ngrp; // first segment of each range, local segments of phase 1, in all; groups
+    int stages, slot_bytes, ring;
+    int issued;                  // units whose copies the producer issued
+    int grp_of[kMaxLocalSeg];    // group of each local segment
+    int grp_seg[kMaxLocalSeg];   // the local segment whose pairs define each group
+    int grp_left[kMaxLocalSeg];  // units of each group not finished yet
+    int sorted[kDecodeMaxPairsStream];   // pair index at each sorted position
+    int seg[kDecodeMaxPairsStream];      // packed (expert << 12) | (first << 3) | n
+    uint32_t vmask[kDecodeMaxPairsStream];  // per token: bit k = pair (t, k) valid
+    int wsum[32];
+};
+
+__device__ __forceinline__ int seg_e(int s) { return s >> 12; }
+__device__ __forceinline__ int seg_first(int s) { return (s >> 3) & 511; }
+__device__ __forceinline__ int seg_n(int s) { return s & 7; }
+
+__device__ __forceinline__ float h2f(uint32_t bits) { return __half2float(__ushort_as_half(uint16_t(bits))); }
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) { return __uint_as_float(lds_u32(addr)); }
+__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sts_u16(uint32_t addr, uint16_t v) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) { sts_u32(addr, __float_as_uint(v)); }
+
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ int vload(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
+
+// Signed bit field of `len` bits at `pos`.
+__device__ __forceinline__ int bfe_s32(uint32_t v, uint32_t pos, uint32_t len) {
+    int r;
+    asm("bfe.s32 %0, %1, %2, %3;" : "=r"(r) : "r"(v), "r"(pos), "r"(len));
+    return r;
+}
+
+// Bounded waits that leave the issue slots to the warps doing work: a
+// shared-memory counter of this CTA or a global counter of other CTAs is
+// re-read after a short sleep; an mbarrier phase is awaited with the
+// hardware's suspend hint.  Each returns false on abort or after kWaitNs.
+__device__ __noinline__ bool wait_smem(const int* p, int v, bool eq, const int* abort) {
+    unsigned ns = 64;
+    uint64_t t0 = 0;
+#pragma unroll 1
+    for (int it = 0;; ++it) {
+        const int x = vload(p);
+        if (eq ? x == v : x >= v) return true;
+        if (vload(abort)) return false;
+        if (it == 0) t0 = globaltimer_ns();
+        else if (globaltimer_ns() - t0 > kWaitNs) return false;
+        __nanosleep(ns);
+        if (ns < 512) ns <<= 1;
+    }
+}
+
+__device__ __noinline__ bool wait_global(const int32_t* p, int v, const int* abort) {
+    unsigned ns = 64;
+    uint64_t t0 = 0;
+#pragma unroll 1
+    for (int it = 0;; ++it) {
+        if (ld_acquire(p) >= v) return true;
+        if (vload(abort)) return false;
+        if (it == 0) t0 = globaltimer_ns();
+        else if (globaltimer_ns() - t0 > kWaitNs) return false;
+        __nanosleep(ns);
+        if (ns < 512) ns <<= 1;
+    }
+}
+
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, uint64_t limit = kWaitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_sleep(bar, parity))
+        if (globaltimer_ns() - t0 > limit) return false;
+    return true;
+}
+
+// a(s) of bit position s inside a byte of a sign word
+__device__ __forceinline__ int a_of(int s) { return s < 7 ? (1 << s) : -128; }
+
+// ----------------------------------------------------------------------------
+// routing and the CTA's plan (every thread of the CTA)
+// ----------------------------------------------------------------------------
+
+// Routing scratch (expert id and sort key of every pair) lives at the end of
+// shared memory, which the ring reaches only after the plan is made.
+struct RouteScratch {
+    int ids[kDecodeMaxPairsStream];
+    int key[kDecodeMaxPairsStream];
+};
+constexpr int kScratchOff = kSmemBytes - 1024 - int(sizeof(RouteScratch));
+
+// Runs once per launch on the critical path before the first copy, so the
+// code stays short and rolled (it is fetched cold).  Up to 32 pairs, one warp
+// routes with shuffles alone; larger batches use the whole block.
+__device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, RouteScratch& rs) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int BK = A.B * A.K, K = A.K;
+    if (tid < kMaxStages) {
+        c.stage_done[tid] = 0;
+        mbar_init(&c.full[tid], 1);
+        mbar_init(&c.empty[tid], 1);
+    }
+    if (tid < kMaxLocalSeg) c.grp_left[tid] = 0;
+    if (tid == 32) {
+        c.issued = 0;
+        c.next_piece = 0;
+        c.slot_grp[0] = 0;
+        c.slot_grp[1] = 1;
+        c.slot_claim[0] = 0 << 16;
+        c.slot_claim[1] = 1 << 16;
+        c.slot_done[0] = c.slot_done[1] = 0;
+        fence_mbar_init();
+    }
+    if (BK <= 32) {
+        if (warp == 0) {
+            const int p = lane;
+            const int e = p < BK ? __ldg(A.ids + p) : -1;
+            if (lane < A.B) c.vmask[lane] = 0u;
+            const int t = p / K, k = p - t * K;
+            bool valid = p < BK && e >= 0 && e < A.E;
+#pragma unroll 1
+            for (int j = 1; j < K; ++j) {
+                const int ej = __shfl_sync(0xffffffffu, e, (p - j) & 31);
+                if (j <= k && ej == e) valid = false;   // a repeated id drops the later pair
+            }
+            const int key = valid ? (e << 9) | p : 0x7FFFFFFF;
+            int r = 0;
+#pragma unroll 1
+            for (int q = 0; q < 32; ++q) r += __shfl_sync(0xffffffffu, key, q) < key;
+            __syncwarp();
+            if (valid) {
+                atomicOr(&c.vmask[t], 1u << k);
+                c.sorted[r] = p;
+            }
+            const unsigned vb = __ballot_sync(0xffffffffu, valid);
+            const int nv = __popc(vb);
+            const unsigned bad = __ballot_sync(0xffffffffu, p < BK && !valid);
+            if (lane == 0) c.bad = bad != 0u;
+            __syncwarp();
+            // sorted position `lane`: its expert, run starts and segments of two
+            const int sp = lane < nv ? c.sorted[lane] : 0;
+            const int se = __shfl_sync(0xffffffffu, e, sp);
+            const int prev = __shfl_up_sync(0xffffffffu, se, 1);
+            const unsigned rsb = __ballot_sync(0xffffffffu, lane < nv && (lane == 0 || prev != se));
+            const unsigned le = (2u << lane) - 1u;   // lanes <= this one
+            const int rstart = 31 - __clz(rsb & le);
+            const unsigned later = rsb & ~le;
+            const int rend = later ? __ffs(later) - 1 : nv;
+            const bool start = lane < nv && ((lane - rstart) % kSegTok) == 0;
+            const unsigned sgb = __ballot_sync(0xffffffffu, start);
+            if (start) c.seg[__popc(sgb & (le >> 1))] = (se << 12) | (lane << 3) | min(kSegTok, rend - lane);
+            if (lane == 0) {
+                c.n_valid = nv;
+                c.n_seg = __popc(sgb);
+            }
+        }
+    } else {
+        if (tid < A.B) c.vmask[tid] = 0u;
+        if (tid < BK) rs.ids[tid] = __ldg(A.ids + tid);
+        if (tid == 0) {
+            c.n_valid = 0;
+            c.bad = 0;
+        }
+        __syncthreads();
+        bool valid = false;
+        if (tid < BK) {
+            const int e = rs.ids[tid];
+            const int t = tid / K, k = tid - t * K;
+            valid = e >= 0 && e < A.E;
+#pragma unroll 1
+            for (int j = tid - k; j < tid; ++j)
+                if (rs.ids[j] == e) valid = false;   // a repeated id drops the later pair
+            rs.key[tid] = valid ? (e << 9) | tid : 0x7FFFFFFF;
+            if (valid) atomicOr(&c.vmask[t], 1u << k);
+            else c.bad = 1;
+        }
+        const unsigned vb = __ballot_sync(0xffffffffu, valid);
+        if (lane == 0 && vb) atomicAdd(&c.n_valid, __popc(vb));
+        __syncthreads();
+        if (valid) {
+            const int k = rs.key[tid];
+            int r = 0;
+#pragma unroll 1
+            for (int j = 0; j < BK; ++j) r += rs.key[j] < k;
+            c.sorted[r] = tid;
+        }
+        __syncthreads();
+        // segments: every kSegTok pairs of an expert's run; the run of the pair
+        // at sorted position tid starts at lo and the segment ends before hi
+        const int nv = c.n_valid;
+        bool start = false;
+        int packed = 0;
+        if (tid < nv) {
+            const int e = rs.ids[c.sorted[tid]];
+            int lo = tid, hi = tid + 1;
+#pragma unroll 1
+            while (lo > 0 && rs.ids[c.sorted[lo - 1]] == e) --lo;
+#pragma unroll 1
+            while (hi < nv && rs.ids[c.sorted[hi]] == e && hi - tid < kSegTok) ++hi;
+            start = (tid - lo) % kSegTok == 0;
+            packed = (e << 12) | (tid << 3) | (hi - tid);
+        }
+        const unsigned sb = __ballot_sync(0xffffffffu, start);
+        if (lane == 0) c.wsum[warp] = __popc(sb);
+        __syncthreads();
+        if (start) {
+            int sid = __popc(sb & ((1u << lane) - 1u));
+#pragma unroll 1
+            for (int w = 0; w < warp; ++w) sid += c.wsum[w];
+            c.seg[sid] = packed;
+        }
+        if (tid == 0) {
+            int ns = 0;
+#pragma unroll 1
+            for (int w = 0; w < kThreads / 32; ++w) ns += c.wsum[w];
+            c.n_seg = ns;
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        // every unit costs the same (a segment is one MMA column group): the
+        // CTA's ranges are equal shares of each phase's unit list
+        const unsigned G = gridDim.x, i = blockIdx.x;
+        const unsigned n1 = unsigned(c.n_seg * P.tiles1), n2 = unsigned(c.n_seg * P.tiles2);
+        c.u1b = int(n1 * i / G);
+        c.u1e = int(n1 * (i + 1) / G);
+        c.u2b = int(n2 * i / G);
+        c.u2e = int(n2 * (i + 1) / G);
+        c.s1b = c.u1b / P.tiles1;
+        c.s2b = c.u2b / P.tiles2;
+        const int nl1 = c.u1e > c.u1b ? (c.u1e - 1) / P.tiles1 - c.s1b + 1 : 0;
+        const int nl2 = c.u2e > c.u2b ? (c.u2e - 1) / P.tiles2 - c.s2b + 1 : 0;
+        c.nl1 = nl1;
+        c.nl = nl1 + nl2;
+        if (c.nl > kMaxLocalSeg) {
+            c.abort = 1;
+            c.nl = kMaxLocalSeg;
+        }
+        // groups: consecutive phase-1 segments with the same tokens share one slot
+        int g = -1, prev_t0 = -1, prev_t1 = -1;
+#pragma unroll 1
+        for (int q = 0; q < c.nl; ++q) {
+            const bool p1 = q < nl1;
+            const int s2 = p1 ? c.s1b + q : c.s2b + (q - nl1);
+            const int sg = c.seg[s2];
+            const int n = seg_n(sg), f = seg_first(sg);
+            const int t0 = c.sorted[f] / K, t1 = n > 1 ? c.sorted[f + 1] / K : -1;
+            if (!(p1 && q > 0 && t0 == prev_t0 && t1 == prev_t1)) {
+                ++g;
+                c.grp_seg[g] = q;
+            }
+            c.grp_of[q] = g;
+            prev_t0 = p1 ? t0 : -1;
+            prev_t1 = p1 ? t1 : -1;
+            const int tiles = p1 ? P.tiles1 : P.tiles2;
+            const int lo = max(s2 * tiles, p1 ? c.u1b : c.u2b), hi = min((s2 + 1) * tiles, p1 ? c.u1e : c.u2e);
+            c.grp_left[g] += hi - lo;
+        }
+        c.ngrp = g + 1;
+        // a slot holds kSegTok tokens of either phase
+        c.slot_bytes = kSegTok * (P.t1.bytes > P.t2.bytes ? P.t1.bytes : P.t2.bytes);
+        c.ring = align_i(align_i(int(sizeof(Ctl)), 1024) + 2 * c.slot_bytes, 1024);
+        const int st = (kSmemBytes - 1024 - c.ring) / P.stage_bytes;
+        c.stages = st > kMaxStages ? kMaxStages : st;
+        if (c.stages < 2) c.abort = 1;
+        if (blockIdx.x == 0 && c.bad) set_status(A.ws.status, GALE_ERR_ARG);
+        if (blockIdx.x == 0 && c.abort) set_status(A.ws.status, GALE_ERR_UNSUPPORTED);
+    }
+    __syncthreads();
+}
+
+// ----------------------------------------------------------------------------
+// activations: rotate one 1024-block of a token and write its digits
+// ----------------------------------------------------------------------------
+
+// Register layout of a warp-held 1024-block: lane l, register r holds element
+//   (l & 7) + 8 (r & 3) + 32 (l >> 3) + 128 (r >> 2),
+// so that lane l = q + 8 tig holds, in registers 4 bb .. 4 bb + 3, the four
+// elements 128 bb + 32 tig + 8 i + q (i = 0..3): byte i of digit word
+// (bb, tig, q).  Digit storage per 128-column block b:
+// [digit j (3)][tig (4)][32 bytes], register q of lane-quad tig at bytes
+// 4q..4q+3, which is the B fragment of the MMAs of bit positions q.
+__device__ __forceinline__ int elem_of(int lane, int r) {
+    return (lane & 7) + 8 * (r & 3) + 32 * (lane >> 3) + 128 * (r >> 2);
+}
+
+// Largest power of two S with m * S <= 2^20 (1 when m is 0).
+__device__ __forceinline__ float fixed_scale_of(float m) {
+    if (!(m > 0.f)) return 1.0f;
+    int e;
+    frexpf(1048576.0f / m, &e);
+    return ldexpf(1.0f, e - 1);
+}
+
+// round(u) (|u| < 2^22) and its three int8 digits.
+__device__ __forceinline__ int round_digits(float u, uint32_t& d1, uint32_t& d2, uint32_t& d3) {
+    const int X = __float_as_int(__fadd_rn(u, 12582912.0f)) - 0x4B400000;
+    const int p1 = (X + 8192) >> 14;
+    const int r = X - (p1 << 14);
+    const int p2 = (r + 64) >> 7;
+    const int p3 = r - (p2 << 7);
+    d1 = uint32_t(p1) & 0xFFu;
+    d2 = uint32_t(p2) & 0xFFu;
+    d3 = uint32_t(p3) & 0xFFu;
+    return X;
+}
+
+// One 1024-block `blk` of a token's activation (bf16 x, or fp32 h) into the
+// slot area `dst` of that token.  Runs a few times per launch and per SM, so
+// the loops that do not need registers indexed at compile time stay rolled.
+__device__ __noinline__ void build_block(const void* src, int bf16, int blk, uint32_t dst, TokMap tm) {
+    const int lane = threadIdx.x & 31;
+    float v[32];
+    if (bf16) {
+        const uint16_t* s = static_cast<const uint16_t*>(src) + 1024 * blk;
+#pragma unroll
+        for (int r = 0; r < 32; ++r) v[r] = bf16_to_f32(__ldg(s + elem_of(lane, r)));
+    } else {
+        const float* s = static_cast<const float*>(src) + 1024 * blk;
+#pragma unroll
+        for (int r = 0; r < 32; ++r) v[r] = __ldcg(s + elem_of(lane, r));
+    }
+    // butterflies over the lane bits: lower lane v + o, upper lane o - v
+#pragma unroll 1
+    for (int st = 0; st < 5; ++st) {
+        const float sg = ((lane >> st) & 1) ? -1.0f : 1.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = fmaf(v[i], sg, __shfl_xor_sync(0xffffffffu, v[i], 1 << st));
+    }
+    // butterflies over the register bits
+#pragma unroll
+    for (int st = 0; st < 5; ++st) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (i & (1 << st)) continue;
+            const float a = v[i], b = v[i | (1 << st)];
+            v[i] = a + b;
+            v[i | (1 << st)] = a - b;
+        }
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int r = 0; r < 32; ++r) m = fmaxf(m, fabsf(v[r]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float S = fixed_scale_of(m);           // the unnormalised transform is 32x the rotation
+    // fp16 copy of u S / 64 (|u S| <= 2^20) in column order, for the outliers
+    const float s16 = S * 0.015625f;
+#pragma unroll
+    for (int r = 0; r < 32; ++r)
+        sts_u16(dst + tm.x16 + 2 * (1024 * blk + elem_of(lane, r)), __half_as_ushort(__float2half_rn(v[r] * s16)));
+    const int q = lane & 7, tig = lane >> 3;
+    const float sc = S * (q < 7 ? __int_as_float((127 - q) << 23) : -0.0078125f);   // S / a(q)
+    const int aq = a_of(q);
+    uint32_t a = dst + (blk * 8) * 384 + tig * 32 + q * 4;
+    const uint32_t xs_a = dst + tm.xsum + 4 * (blk * 8);
+#pragma unroll 1
+    for (int bb = 0; bb < 8; ++bb) {
+        uint32_t w0 = 0u, w1 = 0u, w2 = 0u;
+        int xs = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t d1, d2, d3;
+            xs += round_digits(v[i] * sc, d1, d2, d3);
+            w0 |= d1 << (8 * i);
+            w1 |= d2 << (8 * i);
+            w2 |= d3 << (8 * i);
+        }
+        sts_u32(a, w0);
+        sts_u32(a + 128, w1);
+        sts_u32(a + 256, w2);
+        a += 384;
+        const int tot = __reduce_add_sync(0xffffffffu, xs * aq);
+        if (lane == 0) sts_u32(xs_a + 4 * bb, uint32_t(tot));
+#pragma unroll
+        for (int i = 0; i < 28; ++i) v[i] = v[i + 4];
+    }
+    // x_rot = u / 32 = X a / (32 S); the fp16 copy times 2 / S
+    if (lane == 0) {
+        sts_f32(dst + tm.sig + 4 * blk, 1.0f / (32.0f * S));
+        sts_f32(dst + tm.f16 + 4 * blk, 2.0f / S);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// pieces
+// ----------------------------------------------------------------------------
+
+// Two 16-row tiles (sign rows at sg0 / sg1, swizzled: 16-byte chunk bb of row
+// r at chunk bb ^ (r & 7), rows 128 bytes apart; block scales at sb0 / sb1,
+// row pitch sbp bytes) times the 1024-column chunk c of up to two tokens.
+// Writes  sigma_c (sum_{b in c} s_blk (X_b - 2 P_b))  of row r of tile m,
+// token t to part[(pr_m + r) * 2 + t].
+__device__ __noinline__ void mma_piece(uint32_t sg0, uint32_t sg1, uint32_t sb0, uint32_t sb1, int sbp, int c,
+                                       uint32_t slot, int tstride, TokMap tm, int ntok, uint32_t part, int pr0,
+                                       int pr1) {
+    const uint32_t sg[2] = {sg0, sg1}, sb[2] = {sb0, sb1};
+    const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+    // B fragment of this lane: MMA column g = (token g / 3, digit g % 3), columns 6 and 7 unused
+    const bool bl = g < 3 || (g < 6 && ntok > 1);
+    const uint32_t bsrc = slot + (g >= 3 ? tstride : 0) + (g % 3) * 128 + tig * 32;
+    float acc[2][4];
+#pragma unroll
+    for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
+    const uint32_t woff = g * 128 + tig * 4;
+    // sign words and block scales of the next block are loaded one block ahead
+    uint32_t nw[2][2];
+    float ns[2][2];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        nw[m][0] = lds_u32(sg[m] + woff + (g << 4));
+        nw[m][1] = lds_u32(sg[m] + woff + (g << 4) + 1024);
+        ns[m][0] = h2f(lds_u16(sb[m] + g * sbp + 16 * c));
+        ns[m][1] = h2f(lds_u16(sb[m] + (g + 8) * sbp + 16 * c));
+    }
+#pragma unroll 1
+    for (int bb = 0; bb < 8; ++bb) {
+        const int b = c * 8 + bb;
+        uint4 q0 = make_uint4(0u, 0u, 0u, 0u), q1 = make_uint4(0u, 0u, 0u, 0u);
+        if (bl) {
+            q0 = lds_v4(bsrc + b * 384);
+            q1 = lds_v4(bsrc + b * 384 + 16);
+        }
+        uint32_t w[2][2];
+        float sc[2][2];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            w[m][0] = nw[m][0];
+            w[m][1] = nw[m][1];
+            sc[m][0] = ns[m][0];
+            sc[m][1] = ns[m][1];
+        }
+        if (bb < 7) {
+            const uint32_t wo = woff + (((bb + 1) ^ g) << 4);
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                nw[m][0] = lds_u32(sg[m] + wo);
+                nw[m][1] = lds_u32(sg[m] + wo + 1024);
+                ns[m][0] = h2f(lds_u16(sb[m] + g * sbp + 2 * (b + 1)));
+                ns[m][1] = h2f(lds_u16(sb[m] + (g + 8) * sbp + 2 * (b + 1)));
+            }
+        }
+        const uint32_t breg[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            int cc[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm) {
+                const uint32_t m0 = 0x01010101u << (2 * mm), m1 = m0 << 1;
+                mma_s8(cc, w[m][0] & m0, w[m][1] & m0, w[m][0] & m1, w[m][1] & m1, breg[2 * mm], breg[2 * mm + 1]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[m][i] = fmaf(sc[m][i >> 1], float(cc[i]), acc[m][i]);
+        }
+    }
+    // P of (row, token) from the three digit columns of the token, summed over
+    // the lane quad; lane (g, tig) then owns row g + 8 (tig >> 1), token tig & 1.
+    const int orow = g + 8 * (tig >> 1), tok = tig & 1;
+    const uint32_t tb = slot + tok * tstride;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        float p[4];   // (row g, tok 0), (row g, tok 1), (row g+8, tok 0), (row g+8, tok 1)
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh) {
+            const float a = acc[m][2 * rh], b2 = acc[m][2 * rh + 1];
+            p[2 * rh] = tig == 0 ? fmaf(16384.0f, a, 128.0f * b2) : (tig == 1 ? a : 0.f);
+            p[2 * rh + 1] = tig == 1 ? 16384.0f * b2 : (tig == 2 ? fmaf(128.0f, a, b2) : 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            p[i] += __shfl_xor_sync(0xffffffffu, p[i], 1);
+            p[i] += __shfl_xor_sync(0xffffffffu, p[i], 2);
+        }
+        const float P = tig == 0 ? p[0] : tig == 1 ? p[1] : tig == 2 ? p[2] : p[3];
+        if (tok < ntok) {
+            const uint4 sv = lds_v4(sb[m] + orow * sbp + 16 * c);
+            const uint4 x0 = lds_v4(tb + tm.xsum + 32 * c), x1 = lds_v4(tb + tm.xsum + 32 * c + 16);
+            const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+            const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            float xt = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                xt = fmaf(h2f(sw[i] & 0xFFFFu), float(int(xw[2 * i])), xt);
+                xt = fmaf(h2f(sw[i] >> 16), float(int(xw[2 * i + 1])), xt);
+            }
+            const float sig = lds_f32(tb + tm.sig + 4 * c);
+            sts_f32(part + (((m ? pr1 : pr0) + orow) * 2 + tok) * 4, sig * fmaf(-2.0f, P, xt));
+        }
+    }
+}
+
+// Outlier corrections of one row over outliers j0 <= j < j1:
+//   sum_j (q_j s_row - sign_j s_blk) x_{c_j}
+// for up to two tokens (the MMA part counted the sign weight at c_j); written
+// to out (two floats).
+struct RowRef {
+    uint32_t idx;       // outlier columns of the row (uint16)
+    uint32_t qb;        // byte holding nibble 0 of the values counted from n0
+    int n0;             // nibble index of the row's value 0 relative to qb
+    uint32_t sign;      // the row's 128-byte line in chunk 0 of the swizzled sign area
+    int chunk_stride;   // bytes between chunks in the sign area
+    int sw;             // row & 7
+    uint32_t sblk;      // the row's block scales
+    float srow;
+};
+
+__device__ __noinline__ void outlier_row(const RowRef R, int j0, int j1, int C, uint32_t slot, int tstride,
+                                         TokMap tm, int ntok, uint32_t out) {
+    float corr0 = 0.f, corr1 = 0.f;
+    const uint32_t x0 = slot + tm.x16, x1 = slot + tstride + tm.x16;
+    const uint32_t f0 = slot + tm.f16, f1 = slot + tstride + tm.f16;
+#pragma unroll 2
+    for (int j = j0; j < j1; ++j) {
+        const int col = int(lds_u16(R.idx + 2 * j));
+        if (col >= C) continue;   // only records that failed validation
+        const int n = R.n0 + j;
+        const int qv = bfe_s32(lds_u8(R.qb + (n >> 1)), (n & 1) * 4, 4);
+        const uint32_t word = lds_u32(R.sign + (col >> 10) * R.chunk_stride + ((((col >> 7) & 7) ^ R.sw) << 4) +
+                                      ((col >> 3) & 12));
+        const float sb = h2f(lds_u16(R.sblk + 2 * (col >> 7)));
+        const float wq = fmaf(float(qv), R.srow, ((word >> (col & 31)) & 1u) ? sb : -sb);
+        const int ch4 = 4 * (col >> 10);
+        corr0 = fmaf(wq * lds_f32(f0 + ch4), h2f(lds_u16(x0 + 2 * col)), corr0);
+        if (ntok > 1) corr1 = fmaf(wq * lds_f32(f1 + ch4), h2f(lds_u16(x1 + 2 * col)), corr1);
+    }
+    sts_f32(out, corr0);
+    sts_f32(out + 4, corr1);
+}
+
+// ----------------------------------------------------------------------------
+// finishing a unit
+// ----------------------------------------------------------------------------
+
+__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
+// RMSNorm of token t once all its 64-row blocks are combined: v (x + y) is
+// in the workspace, the blocks' sums of squares in ssq.
+__device__ __noinline__ void normalize_token(const StreamArgs& A, int t) {
+    const int lane = threadIdx.x & 31;
+    const int d = A.d_model, nb = d / 64;
+    __threadfence();
+    float ss = 0.f;
+#pragma unroll 1
+    for (int i = lane; i < nb; i += 32) ss += __ldcg(A.ws.ssq + t * nb + i);
+    ss = warp_sum(ss);
+    const float inv = rsqrtf(ss / float(d) + A.eps);
+    const float4* v = reinterpret_cast<const float4*>(A.ws.v + t * d);
+    uint2* o = reinterpret_cast<uint2*>(static_cast<uint16_t*>(A.out) + t * d);
+#pragma unroll 4
+    for (int i = lane; i < d / 4; i += 32) {
+        const float4 a = __ldcg(v + i);
+        uint2 w;
+        w.x = uint32_t(f32_to_bf16(a.x * inv)) | (uint32_t(f32_to_bf16(a.y * inv)) << 16);
+        w.y = uint32_t(f32_to_bf16(a.z * inv)) | (uint32_t(f32_to_bf16(a.w * inv)) << 16);
+        o[i] = w;
+    }
+}
+
+// y of token t over the 64 rows of block `tile`, once all its experts' o are
+// in: the K outputs in fixed k order, eight loads in flight at a time.
+__device__ __noinline__ void combine_block(const StreamArgs& A, const Ctl& c, int t, int tile) {
+    const int lane = threadIdx.x & 31;
+    const int d = A.d_model, K = A.K, nb = d / 64;
+    __threadfence();
+    const uint32_t vm = c.vmask[t];
+    float y0 = 0.f, y1 = 0.f;
+#pragma unroll 1
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        float g[8], o0[8], o1[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int k = k0 + j;
+            const bool ok = k < K && ((vm >> k) & 1u);
+            const float* o = A.ws.o + (t * K + (ok ? k : 0)) * d + tile * 64 + lane;
+            g[j] = ok ? __ldg(A.gates + t * K + k) : 0.f;
+            o0[j] = ok ? __ldcg(o) : 0.f;
+            o1[j] = ok ? __ldcg(o + 32) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            y0 = fmaf(g[j], o0[j], y0);
+            y1 = fmaf(g[j], o1[j], y1);
+        }
+    }
+    const int r0 = t * d + tile * 64 + lane;
+    if (!A.fuse_norm) {
+        if (A.out_dtype == GALE_F32) {
+            static_cast<float*>(A.out)[r0] = y0;
+            static_cast<float*>(A.out)[r0 + 32] = y1;
+        } else {
+            static_cast<uint16_t*>(A.out)[r0] = f32_to_bf16(y0);
+            static_cast<uint16_t*>(A.out)[r0 + 32] = f32_to_bf16(y1);
+        }
+        return;
+    }
+    const float v0 = bf16_to_f32(__ldg(A.x + r0)) + y0;
+    const float v1 = bf16_to_f32(__ldg(A.x + r0 + 32)) + y1;
+    A.ws.v[r0] = v0;
+    A.ws.v[r0 + 32] = v1;
+    const float ss = warp_sum(fmaf(v0, v0, v1 * v1));
+    if (lane == 0) A.ws.ssq[t * nb + tile] = ss;
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+        __threadfence();
+        last = atomicAdd(A.ws.tokcnt + t, 1) == nb - 1;
+    }
+    if (__shfl_sync(0xffffffffu, last, 0)) normalize_token(A, t);
+}
+
+// Tokens with no valid pair: y = 0 (out = 0, or the norm of x alone).
+__device__ __noinline__ void empty_token(const StreamArgs& A, int t) {
+    const int lane = threadIdx.x & 31;
+    const int d = A.d_model;
+    float ss = 0.f;
+#pragma unroll 1
+    for (int r = lane; r < d; r += 32) {
+        const float v = bf16_to_f32(__ldg(A.x + t * d + r));
+        ss = fmaf(v, v, ss);
+    }
+    const float inv = rsqrtf(warp_sum(ss) / float(d) + A.eps);
+#pragma unroll 1
+    for (int r = lane; r < d; r += 32) {
+        if (A.fuse_norm) static_cast<uint16_t*>(A.out)[t * d + r] = f32_to_bf16(bf16_to_f32(__ldg(A.x + t * d + r)) * inv);
+        else if (A.out_dtype == GALE_F32) static_cast<float*>(A.out)[t * d + r] = 0.f;
+        else static_cast<uint16_t*>(A.out)[t * d + r] = 0;
+    }
+}
+
+// ----------------------------------------------------------------------------
+// the kernel
+// ----------------------------------------------------------------------------
+
+struct UnitRef {
+    bool p1;
+    int U, s, q, tile, e, n, first, st, par;
+};
+
+__device__ __forceinline__ UnitRef unit_ref(const Ctl& c, const Plan& P, int u) {
+    UnitRef r;
+    const int n1 = c.u1e - c.u1b;
+    r.p1 = u < n1;
+    if (r.p1) {
+        r.U = c.u1b + u;
+        r.s = r.U / P.tiles1;
+        r.tile = r.U - r.s * P.tiles1;
+        r.q = r.s - c.s1b;
+    } else {
+        r.U = c.u2b + (u - n1);
+        r.s = r.U / P.tiles2;
+        r.tile = r.U - r.s * P.tiles2;
+        r.q = c.nl1 + r.s - c.s2b;
+    }
+    const int sg = c.seg[r.s];
+    r.e = seg_e(sg);
+    r.n = seg_n(sg);
+    r.first = seg_first(sg);
+    r.st = u % c.stages;
+    r.par = (u / c.stages) & 1;
+    return r;
+}
+
+// One activation piece `cl` (token cl / blocks, 1024-block cl % blocks) of
+// group g into its slot.  A phase-2 piece first waits until the segment's h
+// block is complete in every CTA (bounded).
+__device__ __noinline__ void act_piece(const StreamArgs& A, const Plan& P, Ctl& c, int g, int cl, uint32_t slot) {
+    const int lane = threadIdx.x & 31;
+    const int q = c.grp_seg[g];
+    const bool p1 = q < c.nl1;
+    const int s = p1 ? c.s1b + q : c.s2b + (q - c.nl1);
+    const int sg = c.seg[s];
+    const int nb = p1 ? P.nch1 : P.nch2;
+    const int tk = cl / nb, blk = cl - tk * nb;
+    const int pair = c.sorted[seg_first(sg) + tk];
+    if (p1) {
+        build_block(A.x + (pair / A.K) * A.d_model, 1, blk, slot + uint32_t(tk * P.t1.bytes), P.t1);
+    } else {
+        int v = 1;
+        if (lane == 0) v = wait_global(A.ws.hcnt + s * P.nch2 + blk, 1024 / kR1, &c.abort);
+        v = __shfl_sync(0xffffffffu, v, 0);
+        if (!v) {
+            set_status(A.ws.status, GALE_ERR_TIMEOUT);
+            atomicExch(&c.abort, 1);
+        }
+        build_block(A.ws.h + pair * A.d_ff, 0, blk, slot + uint32_t(tk * P.t2.bytes), P.t2);
+    }
+}
+
+// Whether the phase-2 activation piece `cl` of group g could start now (its
+// h block complete); phase-1 pieces always can.
+__device__ __forceinline__ bool act_ready(const StreamArgs& A, const Plan& P, const Ctl& c, int g, int cl) {
+    const int q = c.grp_seg[g];
+    if (q < c.nl1) return true;
+    const int s = c.s2b + (q - c.nl1);
+    return ld_acquire(A.ws.hcnt + s * P.nch2 + cl % P.nch2) >= 1024 / kR1;
+}
+
+__device__ __forceinline__ int grp_need(const Ctl& c, const Plan& P, int g) {
+    const int q = c.grp_seg[g];
+    const bool p1 = q < c.nl1;
+    const int sg = c.seg[p1 ? c.s1b + q : c.s2b + (q - c.nl1)];
+    return seg_n(sg) * (p1 ? P.nch1 : P.nch2);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_constant__ CUtensorMap map2,
+                  const StreamArgs A, const Plan P) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_align1024(smem_raw);
+    Ctl& c = *reinterpret_cast<Ctl*>(smem);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == kCW * 32) {
+        prefetch_tensormap(&map13);
+        prefetch_tensormap(&map2);
+    }
+    if (tid == 0) c.abort = 0;
+    route_and_plan(A, P, c, *reinterpret_cast<RouteScratch*>(smem + kScratchOff));
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t slot_base = s_base + uint32_t(align_i(int(sizeof(Ctl)), 1024));
+    const uint32_t ring = s_base + uint32_t(c.ring);
+    const int S = c.stages;
+    const int n1 = c.u1e - c.u1b, n2 = c.u2e - c.u2b;
+    const int nunits = n1 + n2;
+    int32_t* status = A.ws.status;
+
+    if (warp == kCW) {
+        // ---------------- producer ----------------
+        if (lane == 0 && !c.abort) {
+#pragma unroll 1
+            for (int u = 0; u < nunits; ++u) {
+                const UnitRef R = unit_ref(c, P, u);
+                if (u >= S && !wait_phase(&c.empty[R.st], R.par ^ 1)) {
+                    set_status(status, GALE_ERR_TIMEOUT);
+                    atomicExch(&c.abort, 1);
+                    break;
+                }
+                if (vload(&c.abort)) break;
+                uint8_t* stage = smem + (ring - s_base) + size_t(R.st) * P.stage_bytes;
+                uint64_t* bar = &c.full[R.st];
+                const char* rec = A.base + int64_t(R.e) * A.stride;
+                const int rows = R.p1 ? kR1 : kR2;
+                const int k = R.p1 ? P.k1 : P.k2;
+                const StageMap& M = R.p1 ? P.m1 : P.m2;
+                const Layout& L = R.p1 ? P.L1 : P.L2;
+                const int nmat = R.p1 ? 2 : 1;
+                const int64_t qs = int64_t(R.tile) * rows * k / 2;   // first value byte
+                const int64_t qa = qs & ~int64_t(15), qe = align_up(qs + int64_t(rows) * k / 2, 16);
+                const uint32_t qbytes = uint32_t(qe - qa);
+                const uint32_t per_mat = uint32_t(M.sb_bytes) + uint32_t(rows * 2) + uint32_t(M.idx_bytes) + qbytes;
+                mbar_arrive_expect_tx(bar, uint32_t(nmat * (R.p1 ? P.nch1 : P.nch2) * rows * 128) + nmat * per_mat);
+                tma_load_5d(stage, R.p1 ? &map13 : &map2, bar, 0, R.tile * rows, 0, 0, R.e);
+#pragma unroll 1
+                for (int m = 0; m < nmat; ++m) {
+                    const char* mat = rec + A.off_w[R.p1 ? m : 2];
+                    bulk_load(stage + M.sb + m * M.sb_bytes, mat + L.off_sblk + int64_t(R.tile) * M.sb_bytes,
+                              M.sb_bytes, bar);
+                    bulk_load(stage + M.sr + m * 32, mat + L.off_srow + int64_t(R.tile) * rows * 2, rows * 2, bar);
+                    bulk_load(stage + M.idx + m * align_i(M.idx_bytes, 16),
+                              mat + L.off_idx + int64_t(R.tile) * M.idx_bytes, M.idx_bytes, bar);
+                    bulk_load(stage + M.q + m * M.q_bytes, mat + L.off_q + qa, qbytes, bar);
+                }
+                c.issued = u + 1;
+            }
+        }
+    } else {
+        // ---------------- consumers ----------------
+        // tokens without a valid pair get their output here (nothing combines them)
+#pragma unroll 1
+        for (int t = blockIdx.x * kCW + warp; t < A.B; t += gridDim.x * kCW)
+            if (c.vmask[t] == 0u) empty_token(A, t);
+        const int tot_pieces = n1 * P.pp1 + n2 * P.pp2;
+        const int nhb = P.nch2;
+#pragma unroll 1
+        for (;;) {
+            int pc = 0;
+            if (lane == 0) pc = atomicAdd(&c.next_piece, 1);
+            pc = __shfl_sync(0xffffffffu, pc, 0);
+            if (pc >= tot_pieces || vload(&c.abort)) break;
+            const bool p1 = pc < n1 * P.pp1;
+            const int u = p1 ? pc / P.pp1 : n1 + (pc - n1 * P.pp1) / P.pp2;
+            const int sub = p1 ? pc - (pc / P.pp1) * P.pp1 : (pc - n1 * P.pp1) % P.pp2;
+            const UnitRef R = unit_ref(c, P, u);
+            // ---- the activations of the unit's group, in slot g & 1 ----
+            const int g = c.grp_of[R.q];
+            const int sl = g & 1;
+            const int need = grp_need(c, P, g);
+            const int tstride = R.p1 ? P.t1.bytes : P.t2.bytes;
+            const uint32_t slot = slot_base + uint32_t(sl * c.slot_bytes);
+            {
+                bool ok = wait_smem(&c.slot_grp[sl], g, true, &c.abort);
+#pragma unroll 1
+                while (ok && vload(&c.slot_done[sl]) < need) {
+                    // the slot cannot move on while this unit is unfinished,
+                    // so the claim word is the group's
+                    int cl = 0;
+                    if (lane == 0) cl = atomicAdd(&c.slot_claim[sl], 1) & 0xFFFF;
+                    cl = __shfl_sync(0xffffffffu, cl, 0);
+                    if (cl < need) {
+                        act_piece(A, P, c, g, cl, slot);
+                        __syncwarp();
+                        __threadfence_block();
+                        if (lane == 0) atomicAdd(&c.slot_done[sl], 1);
+                    } else {
+                        ok = wait_smem(&c.slot_done[sl], need, false, &c.abort);
+                    }
+                }
+                if (!ok) {
+                    if (!vload(&c.abort)) set_status(status, GALE_ERR_TIMEOUT);
+                    atomicExch(&c.abort, 1);
+                    break;
+                }
+                __threadfence_block();
+            }
+            // ---- the unit's rows ----
+            if (!wait_phase(&c.full[R.st], R.par)) {
+                set_status(status, GALE_ERR_TIMEOUT);
+                atomicExch(&c.abort, 1);
+                break;
+            }
+            const uint32_t stage = ring + uint32_t(R.st * P.stage_bytes);
+            const uint32_t part = stage + P.part;
+            if (R.p1) {
+                const int nch = P.nch1;
+                if (sub < nch) {
+                    mma_piece(stage + uint32_t(sub * 2048), stage + uint32_t((nch + sub) * 2048), stage + P.m1.sb,
+                              stage + P.m1.sb + P.m1.sb_bytes, P.C1 / 64, sub, slot, tstride, P.t1, R.n,
+                              part + uint32_t(sub * 32 * 8), 0, 16);
+                } else {
+                    const int o = sub - nch;
+                    const int m = lane >> 4, r = lane & 15;
+                    RowRef RR;
+                    RR.idx = stage + P.m1.idx + m * align_i(P.m1.idx_bytes, 16) + r * P.k1 * 2;
+                    const int64_t qs = int64_t(R.tile) * kR1 * P.k1 / 2;
+                    RR.qb = stage + P.m1.q + m * P.m1.q_bytes + uint32_t(qs & 15);
+                    RR.n0 = r * P.k1;
+                    RR.sign = stage + uint32_t(m * nch * 2048 + r * 128);
+                    RR.chunk_stride = 2048;
+                    RR.sw = r & 7;
+                    RR.sblk = stage + P.m1.sb + m * P.m1.sb_bytes + r * (P.C1 / 64);
+                    RR.srow = h2f(lds_u16(stage + P.m1.sr + m * 32 + 2 * r));
+                    const int jh = (P.k1 + 1) / 2;
+                    outlier_row(RR, o ? jh : 0, o ? P.k1 : jh, P.C1, slot, tstride, P.t1, R.n,
+                                part + uint32_t(((nch + o) * 32 + lane) * 8));
+                }
+            } else {
+                const int nch = P.nch2;
+                if (sub < 2 * nch) {
+                    const int ch = sub % nch, half = sub / nch;
+                    const int sbp = P.C2 / 64;
+                    mma_piece(stage + uint32_t(ch * kR2 * 128 + (2 * half) * 2048),
+                              stage + uint32_t(ch * kR2 * 128 + (2 * half + 1) * 2048),
+                              stage + P.m2.sb + uint32_t((2 * half) * 16 * sbp),
+                              stage + P.m2.sb + uint32_t((2 * half + 1) * 16 * sbp), sbp, ch, slot, tstride, P.t2,
+                              R.n, part + uint32_t(ch * 64 * 8), half * 32, half * 32 + 16);
+                } else {
+                    const int o = sub - 2 * nch;
+                    const int r = o * 32 + lane;
+                    RowRef RR;
+                    RR.idx = stage + P.m2.idx + r * P.k2 * 2;
+                    RR.qb = stage + P.m2.q;
+                    RR.n0 = r * P.k2;
+                    RR.sign = stage + uint32_t(r * 128);
+                    RR.chunk_stride = kR2 * 128;
+                    RR.sw = r & 7;
+                    RR.sblk = stage + P.m2.sb + r * (P.C2 / 64);
+                    RR.srow = h2f(lds_u16(stage + P.m2.sr + 2 * r));
+                    outlier_row(RR, 0, P.k2, P.C2, slot, tstride, P.t2, R.n, part + uint32_t((nch * 64 + r) * 8));
+                }
+            }
+            // ---- the last piece of the unit finishes it ----
+            __syncwarp();
+            __threadfence_block();
+            int last = 0;
+            if (lane == 0) last = atomicAdd(&c.stage_done[R.st], 1) == (R.p1 ? P.pp1 : P.pp2) - 1;
+            if (__shfl_sync(0xffffffffu, last, 0)) {
+                __threadfence_block();
+                if (R.p1) {
+                    // h rows: silu(w1 x) * (w3 x); slices 0..nch-1 (chunks), nch, nch+1 (outliers)
+                    const int nsl = P.nch1 + 2;
+#pragma unroll 1
+                    for (int i = lane; i < kR1 * R.n; i += 32) {
+                        const int r = i & 15, t = i >> 4;
+                        float g1 = 0.f, g3 = 0.f;
+#pragma unroll 1
+                        for (int s2 = 0; s2 < nsl; ++s2) {
+                            g1 += lds_f32(part + uint32_t(((s2 * 32 + r) * 2 + t) * 4));
+                            g3 += lds_f32(part + uint32_t(((s2 * 32 + 16 + r) * 2 + t) * 4));
+                        }
+                        const int pair = c.sorted[R.first + t];
+                        A.ws.h[pair * A.d_ff + R.tile * kR1 + r] = silu_fast(g1) * g3;
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        __threadfence();
+                        atomicAdd(A.ws.hcnt + R.s * nhb + (R.tile * kR1) / 1024, 1);
+                    }
+                } else {
+                    // o rows; slices 0..nch-1 (chunks), nch (outliers)
+                    const int nsl = P.nch2 + 1;
+#pragma unroll 1
+                    for (int i = lane; i < kR2 * R.n; i += 32) {
+                        const int r = i & 63, t = i >> 6;
+                        float y = 0.f;
+#pragma unroll 1
+                        for (int s2 = 0; s2 < nsl; ++s2) y += lds_f32(part + uint32_t(((s2 * 64 + r) * 2 + t) * 4));
+                        const int pair = c.sorted[R.first + t];
+                        A.ws.o[pair * A.d_model + R.tile * kR2 + r] = y;
+                    }
+                    __syncwarp();
+                    if (lane == 0) __threadfence();
+                    __syncwarp();
+                    const int nb = A.d_model / 64;
+#pragma unroll 1
+                    for (int t = 0; t < R.n; ++t) {
+                        const int tk = c.sorted[R.first + t] / A.K;
+                        int lastc = 0;
+                        if (lane == 0)
+                            lastc = atomicAdd(A.ws.comb + tk * nb + R.tile, 1) == __popc(c.vmask[tk]) - 1;
+                        if (__shfl_sync(0xffffffffu, lastc, 0)) combine_block(A, c, tk, R.tile);
+                    }
+                }
+                // release the stage and count the unit into its group
+                __syncwarp();
+                if (lane == 0) {
+                    c.stage_done[R.st] = 0;
+                    __threadfence_block();
+                    mbar_arrive(&c.empty[R.st]);
+                    if (atomicSub(&c.grp_left[g], 1) == 1 && g + 2 < c.ngrp) {
+                        c.slot_claim[sl] = (g + 2) << 16;
+                        c.slot_done[sl] = 0;
+                        __threadfence_block();
+                        atomicExch(&c.slot_grp[sl], g + 2);
+                    }
+                }
+            }
+            // ---- work ahead: one activation piece of the next group, if its
+            //      slot is free and (phase 2) its h block is complete ----
+            const int gn = g + 1;
+            if (gn < c.ngrp && vload(&c.slot_grp[gn & 1]) == gn) {
+                const int sln = gn & 1;
+                const int needn = grp_need(c, P, gn);
+                // claim only if the claim word still belongs to group gn: a
+                // warp ahead holds no unit of gn, so the slot may move on
+                int cl = needn;
+                if (lane == 0) {
+                    const int v = vload(&c.slot_claim[sln]);
+                    if ((v >> 16) == gn && (v & 0xFFFF) < needn && act_ready(A, P, c, gn, v & 0xFFFF) &&
+                        atomicCAS(&c.slot_claim[sln], v, v + 1) == v)
+                        cl = v & 0xFFFF;
+                }
+                cl = __shfl_sync(0xffffffffu, cl, 0);
+                if (cl < needn) {
+                    act_piece(A, P, c, gn, cl, slot_base + uint32_t(sln * c.slot_bytes));
+                    __syncwarp();
+                    __threadfence_block();
+                    if (lane == 0) atomicAdd(&c.slot_done[sln], 1);
+                }
+            }
+        }
+    }
+    // every copy the producer issued has landed before the CTA exits
+    __syncthreads();
+    if (tid == 0 && vload(&c.abort)) {
+        const int iss = c.issued;
+#pragma unroll 1
+        for (int u = iss - S > 0 ? iss - S : 0; u < iss; ++u) wait_phase(&c.full[u % S], (u / S) & 1, 100000000ull);
+    }
+}
+
+}  // namespace
+
+StreamWs carve_stream_ws(void* ws, const gale_layer& L, int B, int K) {
+    StreamWs w{};
+    char* p = static_cast<char*>(ws);
+    int64_t o = 0;
+    auto take = [&](int64_t bytes) {
+        char* q = p ? p + o : nullptr;
+        o = align_up(o + bytes, 256);
+        return q;
+    };
+    const int64_t BK = int64_t(B) * K, dm = L.d_model, df = L.d_ff;
+    const int64_t nb = dm / 64;
+    // counters first: one memset clears them all
+    w.status = reinterpret_cast<int32_t*>(take(256));
+    w.hcnt = reinterpret_cast<int32_t*>(take(4 * BK * (df / 1024)));
+    w.comb = reinterpret_cast<int32_t*>(take(4 * int64_t(B) * nb));
+    w.tokcnt = reinterpret_cast<int32_t*>(take(4 * int64_t(B)));
+    w.counter_bytes = size_t(o);
+    w.ssq = reinterpret_cast<float*>(take(4 * int64_t(B) * nb));
+    w.h = reinterpret_cast<float*>(take(4 * BK * df));
+    w.o = reinterpret_cast<float*>(take(4 * BK * dm));
+    w.v = reinterpret_cast<float*>(take(4 * int64_t(B) * dm));
+    w.bytes = size_t(o);
+    return w;
+}
+
+bool stream_supported(const gale_layer& L, int B, int K) {
+    if (B < 1 || K > 16 || int64_t(B) * K > kDecodeMaxPairsStream || L.n_experts > 1023) return false;
+    if (L.d_model % 1024 || L.d_ff % 1024 || L.d_model > 4096 || L.d_ff > 2048) return false;
+    const Plan P = make_stream_plan(L.d_model, L.d_ff);
+    const int ctl = align_i(int(sizeof(Ctl)), 1024);
+    const int slot = kSegTok * (P.t1.bytes > P.t2.bytes ? P.t1.bytes : P.t2.bytes);
+    return kSmemBytes - 1024 - align_i(ctl + 2 * slot, 1024) >= 2 * P.stage_bytes;
+}
+
+int launch_moe_stream(const gale_layer& L, const uint16_t* x, const int32_t* ids, const float* gates, int B, int K,
+                      void* out, int out_dtype, bool fuse_norm, float eps, void* ws, cudaStream_t st) {
+    StreamArgs A{};
+    A.base = static_cast<const char*>(L.base);
+    A.stride = L.expert_stride;
+    A.E = L.n_experts;
+    A.d_model = L.d_model;
+    A.d_ff = L.d_ff;
+    A.B = B;
+    A.K = K;
+    const Plan P = make_stream_plan(L.d_model, L.d_ff);
+    A.off_w[0] = 0;
+    A.off_w[1] = P.L1.total;
+    A.off_w[2] = 2 * P.L1.total;
+    A.x = x;
+    A.ids = ids;
+    A.gates = gates;
+    A.out = out;
+    A.out_dtype = out_dtype;
+    A.fuse_norm = fuse_norm ? 1 : 0;
+    A.eps = eps;
+    A.ws = carve_stream_ws(ws, L, B, K);
+    GALE_CUDA_TRY(cudaMemsetAsync(A.ws.status, 0, A.ws.counter_bytes, st));
+    CUtensorMap map13, map2;
+    int rc = cached_sign_map5b(&map13, A.base, L.d_ff, L.d_model, 2, P.L1.total, L.n_experts, L.expert_stride, kR1, 2);
+    if (rc == GALE_OK)
+        rc = cached_sign_map5b(&map2, A.base + A.off_w[2], L.d_model, L.d_ff, 1, P.L1.total, L.n_experts,
+                               L.expert_stride, kR2, 1);
+    if (rc != GALE_OK) return rc;
+    rc = ensure_smem(reinterpret_cast<const void*>(moe_stream_kernel), kSmemBytes);
+    if (rc != GALE_OK) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(sm_count()));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = size_t(kSmemBytes);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, moe_stream_kernel, map13, map2, A, P) == cudaSuccess ? GALE_OK : GALE_ERR_CUDA;
+}
+
+}  // namespace gale

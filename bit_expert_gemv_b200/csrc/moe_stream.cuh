@@ -1,0 +1,28 @@
+// Decode path of the MoE layer (batches of up to 384 (token, expert) pairs):
+// one persistent streaming kernel; workspace layout and host entry.
+#pragma once
+#include "common.cuh"
+
+namespace gale {
+
+constexpr int kDecodeMaxPairsStream = 384;   // B * K handled by the streaming kernel
+
+struct StreamWs {
+    int32_t* status;      // device status word
+    int32_t* hcnt;        // [segments][d_ff/1024] finished 16-row tiles of h per 1024-block
+    int32_t* comb;        // [B][d_model/64] experts finished per (token, 64-row block)
+    int32_t* tokcnt;      // [B] row blocks combined per token (RMSNorm)
+    size_t counter_bytes; // status .. tokcnt, cleared by one memset per call
+    float* ssq;           // [B][d_model/64] sums of squares of v per block
+    float* h;             // [B*K][d_ff] SwiGLU output of every pair (pair index t*K + k)
+    float* o;             // [B*K][d_model] expert output of every pair
+    float* v;             // [B][d_model] x + y before the norm
+    size_t bytes;
+};
+
+StreamWs carve_stream_ws(void* ws, const gale_layer& L, int B, int K);
+bool stream_supported(const gale_layer& L, int B, int K);
+int launch_moe_stream(const gale_layer& L, const uint16_t* x, const int32_t* ids, const float* gates, int B, int K,
+                      void* out, int out_dtype, bool fuse_norm, float eps, void* ws, cudaStream_t st);
+
+}  // namespace gale

@@ -72,10 +72,27 @@ int make_sign_map5(CUtensorMap* m, const void* first_matrix, int rows, int cols,
     return r == CUDA_SUCCESS ? GALE_OK : GALE_ERR_CUDA;
 }
 
+// The same 5-D view with a box over `box_mats` matrices at once (every
+// matrix of the view when box_mats == n_mat): a box of (32 words, box_rows
+// rows, every piece, box_mats matrices) lands as [matrix][piece][row][128 B].
+int make_sign_map5b(CUtensorMap* m, const void* first_matrix, int rows, int cols, int n_mat, int64_t mat_stride,
+                    int experts, int64_t stride, int box_rows, int box_mats) {
+    auto fn = encode_fn();
+    if (!fn) return GALE_ERR_CUDA;
+    cuuint64_t dims[5] = {32, cuuint64_t(rows), cuuint64_t(cols / 1024), cuuint64_t(n_mat), cuuint64_t(experts)};
+    cuuint64_t strides[4] = {cuuint64_t(cols / 8), 128, cuuint64_t(mat_stride), cuuint64_t(stride)};
+    cuuint32_t box[5] = {32, cuuint32_t(box_rows), cuuint32_t(cols / 1024), cuuint32_t(box_mats), 1};
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 5, const_cast<void*>(first_matrix), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GALE_OK : GALE_ERR_CUDA;
+}
+
 namespace {
 struct Map5Entry {
     const void* base;
-    int rows, cols, n_mat, experts, box_rows;
+    int rows, cols, n_mat, experts, box_rows, box_mats;
     int64_t mat_stride, stride;
     CUtensorMap map;
 };
@@ -86,16 +103,23 @@ thread_local int g_map5_next = 0;
 
 int cached_sign_map5(CUtensorMap* out, const void* first_matrix, int rows, int cols, int n_mat, int64_t mat_stride,
                      int experts, int64_t stride, int box_rows) {
+    return cached_sign_map5b(out, first_matrix, rows, cols, n_mat, mat_stride, experts, stride, box_rows, 1);
+}
+
+int cached_sign_map5b(CUtensorMap* out, const void* first_matrix, int rows, int cols, int n_mat, int64_t mat_stride,
+                      int experts, int64_t stride, int box_rows, int box_mats) {
     for (int i = 0; i < kMap5Cache; ++i) {
         const Map5Entry& e = g_maps5[i];
         if (e.base == first_matrix && e.rows == rows && e.cols == cols && e.n_mat == n_mat &&
-            e.experts == experts && e.box_rows == box_rows && e.mat_stride == mat_stride && e.stride == stride) {
+            e.experts == experts && e.box_rows == box_rows && e.box_mats == box_mats && e.mat_stride == mat_stride &&
+            e.stride == stride) {
             *out = e.map;
             return GALE_OK;
         }
     }
-    Map5Entry e{first_matrix, rows, cols, n_mat, experts, box_rows, mat_stride, stride, {}};
-    const int rc = make_sign_map5(&e.map, first_matrix, rows, cols, n_mat, mat_stride, experts, stride, box_rows);
+    Map5Entry e{first_matrix, rows, cols, n_mat, experts, box_rows, box_mats, mat_stride, stride, {}};
+    const int rc = make_sign_map5b(&e.map, first_matrix, rows, cols, n_mat, mat_stride, experts, stride, box_rows,
+                                   box_mats);
     if (rc != GALE_OK) return rc;
     g_maps5[g_map5_next] = e;
     g_map5_next = (g_map5_next + 1) % kMap5Cache;

@@ -18,6 +18,10 @@ int make_sign_map5(CUtensorMap* m, const void* first_matrix, int rows, int cols,
                    int experts, int64_t stride, int box_rows);
 int cached_sign_map5(CUtensorMap* out, const void* first_matrix, int rows, int cols, int n_mat, int64_t mat_stride,
                      int experts, int64_t stride, int box_rows);
+int make_sign_map5b(CUtensorMap* m, const void* first_matrix, int rows, int cols, int n_mat, int64_t mat_stride,
+                    int experts, int64_t stride, int box_rows, int box_mats);
+int cached_sign_map5b(CUtensorMap* out, const void* first_matrix, int rows, int cols, int n_mat, int64_t mat_stride,
+                      int experts, int64_t stride, int box_rows, int box_mats);
 // Raise a kernel's dynamic shared-memory limit once per device.
 int ensure_smem(const void* kernel, int bytes);
 
