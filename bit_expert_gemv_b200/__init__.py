@@ -20,6 +20,7 @@ GALE_ERR_WORKSPACE = -3
 GALE_ERR_CUDA = -4
 GALE_ERR_TIMEOUT = -5
 GALE_ERR_UNSUPPORTED = -6
+GALE_ERR_SELFTEST = -7
 
 GALE_F32, GALE_BF16, GALE_F16 = 0, 1, 2
 GALE_MODE_PLAIN, GALE_MODE_SWIGLU = 0, 1

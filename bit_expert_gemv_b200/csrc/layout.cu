@@ -28,6 +28,7 @@ extern "C" const char* gale_status_string(int status) {
         case GALE_ERR_CUDA: return "GALE_ERR_CUDA: CUDA runtime call or launch failed";
         case GALE_ERR_TIMEOUT: return "GALE_ERR_TIMEOUT: bounded device wait ran out";
         case GALE_ERR_UNSUPPORTED: return "GALE_ERR_UNSUPPORTED: shape or device not supported";
+        case GALE_ERR_SELFTEST: return "GALE_ERR_SELFTEST: a self-check result differs from its expected value";
         default: return "GALE: unknown status";
     }
 }

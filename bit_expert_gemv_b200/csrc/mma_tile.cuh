@@ -123,14 +123,15 @@ __host__ __device__ inline StageLayout stage_layout(int C) {
 }
 
 // The token vectors a tile job multiplies: up to two tokens, each with its
-// digits, 128-block sums, reconstruction factor 1/S and rotated values (fp32
-// in global memory, or fp16 in shared memory) for the outliers.
+// digits, 128-block sums, reconstruction factor 1/S and, for the outliers,
+// its rotated values (fp32 in global memory, or an fp16 copy of v S / 64 in
+// shared memory).
 struct TokRef {
     const uint8_t* pieces;   // nullptr: no token in this slot
     const float* xsum;
     const float* xr;         // fp32 rotated vector (global), or null
     float sigma;             // 1 / S
-    const __half* x16;       // fp16 rotated vector (shared), or null
+    const __half* x16;       // fp16 copy of the rotated vector times S / 64 (shared), or null
 };
 
 // Issue the TMA / bulk loads of tile (rows r0.., expert coordinate e) of a
@@ -262,206 +263,6 @@ __device__ __forceinline__ void tile_compute(uint8_t* stage, const MatView& m, i
         const float* col = scratch + row * 8 + 3 * t;
         const float P = tok[t].pieces ? tok[t].sigma * (col[0] * 16384.0f + col[1] * 128.0f + col[2]) : 0.f;
         y[t] = v - 2.0f * P;
-    }
-    __syncwarp();
-}
-
-// ---------------------------------------------------------------------------
-// Register layout of a warp-held 1024-block used for building digits: lane l
-// register r holds element
-//     (l & 7) + 8 (r & 3) + 32 (l >> 3) + 128 (r >> 2),
-// so that lane l = q + 8 tig holds, in registers 4 bb .. 4 bb + 3, the four
-// elements 128 bb + 32 tig + 8 i + q (i = 0..3) of digit word (bb, tig, q).
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ int piece_elem(int lane, int r) {
-    return (lane & 7) + 8 * (r & 3) + 32 * (lane >> 3) + 128 * (r >> 2);
-}
-
-// Digits, the eight 128-block sums and the fp16 copy of one rotated
-// 1024-block in the layout above (values already scaled by 1/32).
-__device__ __forceinline__ void pieces_from_regs(const float (&v)[32], float S, uint8_t* pieces_blk,
-                                                 float* xsum_blk, __half* x16_blk) {
-    const int lane = threadIdx.x & 31;
-    const int q = lane & 7, tig = lane >> 3;
-    const float scale = S * inv_a(q);
-#pragma unroll
-    for (int r = 0; r < 32; ++r) x16_blk[piece_elem(lane, r)] = __float2half_rn(v[r]);
-#pragma unroll
-    for (int bb = 0; bb < 8; ++bb) {
-        const float s = warp_sum(v[4 * bb] + v[4 * bb + 1] + v[4 * bb + 2] + v[4 * bb + 3]);
-        if (lane == 0) xsum_blk[bb] = s;
-        uint32_t word[kPieces] = {0u, 0u, 0u};
-#pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) {
-            uint32_t d1, d2, d3;
-            fixed_digits(v[4 * bb + i4] * scale, d1, d2, d3);
-            word[0] |= d1 << (8 * i4);
-            word[1] |= d2 << (8 * i4);
-            word[2] |= d3 << (8 * i4);
-        }
-        uint32_t* dst = reinterpret_cast<uint32_t*>(pieces_blk + bb * kPieceBlockBytes + tig * 32 + q * 4);
-#pragma unroll
-        for (int j = 0; j < kPieces; ++j) dst[j * 32] = word[j];
-    }
-}
-
-// Largest |x| over a warp-held block (all lanes get it).
-__device__ __forceinline__ float block_absmax(const float (&v)[32]) {
-    float m = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    return m;
-}
-
-// Bytes that issue_tile_copies moves for tile (rows r0..) of matrix m.
-__device__ __forceinline__ uint32_t tile_tx_bytes(const MatView& m, int r0) {
-    const int nrows = min(16, m.rows - r0);
-    const uint32_t idx_bytes = uint32_t(align_up(int64_t(nrows) * m.k * 2, 16));
-    const char* q_src = reinterpret_cast<const char*>(m.q) + int64_t(r0) * m.k / 2;
-    const int q_delta = int(reinterpret_cast<uintptr_t>(q_src) & 15);
-    const uint32_t q_bytes = uint32_t(align_up(q_delta + (int64_t(nrows) * m.k + 1) / 2, 16));
-    return uint32_t(2 * m.cols + 16 * (m.cols / 64)) + (m.k ? idx_bytes + q_bytes + 32u : 0u);
-}
-
-// The copies of issue_tile without arming the barrier (the caller arms it
-// once for all the tiles of a job); the 16 row scales go to L.srow (32 bytes:
-// the record continues past the section, so the copy stays inside it).
-__device__ inline void issue_tile_copies(uint8_t* stage, uint64_t* bar, const CUtensorMap* smap,
-                                         const CUtensorMap* bmap, const MatView& m, int e, int r0) {
-    const StageLayout L = stage_layout(m.cols);
-    const int nrows = min(16, m.rows - r0);
-    for (int ch = 0; ch < m.cols / 1024; ++ch) tma_load_3d(stage + L.signs + ch * 2048, smap, bar, ch * 32, r0, e);
-    tma_load_3d(stage + L.scales, bmap, bar, 0, r0, e);
-    if (m.k) {
-        const uint32_t idx_bytes = uint32_t(align_up(int64_t(nrows) * m.k * 2, 16));
-        const char* q_src = reinterpret_cast<const char*>(m.q) + int64_t(r0) * m.k / 2;
-        const int q_delta = int(reinterpret_cast<uintptr_t>(q_src) & 15);
-        const uint32_t q_bytes = uint32_t(align_up(q_delta + (int64_t(nrows) * m.k + 1) / 2, 16));
-        bulk_load(stage + L.idx, m.idx + int64_t(r0) * m.k, idx_bytes, bar);
-        bulk_load(stage + L.q, q_src - q_delta, q_bytes, bar);
-        bulk_load(stage + L.srow, m.s_row + r0, 32, bar);
-    }
-}
-
-// One 1024-column chunk `ch` of a staged 16-row tile, for up to two tokens
-// whose digits, sums and fp16 values live in shared memory.  On return lanes
-// 0..15 hold the chunk's contribution to row r0 + lane for tokens 0 and 1:
-//   sum_{b in chunk} s_blk (X_b - 2 P_b) + sum_{outliers in chunk} (q s_row - sign s_blk) x_c.
-// Contributions of the chunks of a row add up to the row result.
-__device__ __forceinline__ void chunk_compute(uint8_t* tile, const MatView& m, int r0, int ch,
-                                              const TokRef (&tok)[2], float* scratch, float (&part)[2]) {
-    const int lane = threadIdx.x & 31;
-    const int C = m.cols, nb = C / 128, k = m.k;
-    const StageLayout L = stage_layout(C);
-    const uint32_t t_s = smem_u32(tile);
-    const uint32_t signs_s = t_s + L.signs, sblk_s = t_s + L.scales, idx_s = t_s + L.idx;
-    const int nrows = min(16, m.rows - r0);
-    const int q_delta = int(reinterpret_cast<uintptr_t>(reinterpret_cast<const char*>(m.q) + int64_t(r0) * k / 2) & 15);
-    const uint32_t qn_s = t_s + L.q + q_delta;
-    const int row = lane & 15, half = lane >> 4;
-    const bool has0 = tok[0].pieces != nullptr, has1 = tok[1].pieces != nullptr;
-    const uint32_t x16_0 = has0 ? smem_u32(tok[0].x16) : 0u, x16_1 = has1 ? smem_u32(tok[1].x16) : 0u;
-
-    // 1. outliers of this chunk: the row's columns are ascending, so the
-    //    chunk's outliers are the range [lo, hi) found by binary search; the
-    //    two half-warps split it.
-    float corr0 = 0.f, corr1 = 0.f;
-    if (row < nrows && k) {
-        const uint32_t ri = idx_s + 2 * row * k;
-        int a0 = 0, a1 = k;   // first j with idx >= 1024 ch
-        while (a0 < a1) {
-            const int mid = (a0 + a1) >> 1;
-            if (int(lds_u16(ri + 2 * mid)) < (ch << 10)) a0 = mid + 1;
-            else a1 = mid;
-        }
-        const int lo = a0;
-        a1 = k;               // first j with idx >= 1024 (ch + 1)
-        while (a0 < a1) {
-            const int mid = (a0 + a1) >> 1;
-            if (int(lds_u16(ri + 2 * mid)) < ((ch + 1) << 10)) a0 = mid + 1;
-            else a1 = mid;
-        }
-        const int hi = a0;
-        const int mid = (lo + hi + 1) >> 1;
-        const int j0 = half ? mid : lo, j1 = half ? hi : mid;
-        const float srow = __half2float(__ushort_as_half(uint16_t(lds_u16(t_s + L.srow + 2 * row))));
-        for (int j = j0; j < j1; ++j) {
-            const int c = int(lds_u16(ri + 2 * j));
-            const int n = row * k + j;
-            const int qb = int(lds_u8(qn_s + (n >> 1))) >> ((n & 1) * 4);
-            const int qv = (qb & 15) - ((qb & 8) << 1);
-            const int w = (c >> 5) & 31;
-            const uint32_t word =
-                lds_u32(signs_s + ch * 2048 + row * 128 + (((w >> 2) ^ (row & 7)) << 4) + (w & 3) * 4);
-            const float sb = __half2float(__ushort_as_half(uint16_t(lds_u16(sblk_s + 2 * (row * nb + (c >> 7))))));
-            const float wq = fmaf(float(qv), srow, ((word >> (c & 31)) & 1u) ? sb : -sb);
-            if (has0) corr0 = fmaf(wq, __half2float(__ushort_as_half(uint16_t(lds_u16(x16_0 + 2 * c)))), corr0);
-            if (has1) corr1 = fmaf(wq, __half2float(__ushort_as_half(uint16_t(lds_u16(x16_1 + 2 * c)))), corr1);
-        }
-    }
-    // 2. block-scale-weighted 128-block sums of x over the chunk (4 blocks per half)
-    float xt0 = 0.f, xt1 = 0.f;
-#pragma unroll
-    for (int bb = 0; bb < 4; ++bb) {
-        const int b = ch * 8 + half * 4 + bb;
-        const float s = __half2float(__ushort_as_half(uint16_t(lds_u16(sblk_s + 2 * (row * nb + b)))));
-        if (has0) xt0 = fmaf(s, tok[0].xsum[b], xt0);
-        if (has1) xt1 = fmaf(s, tok[1].xsum[b], xt1);
-    }
-
-    // 3. tensor-core loop over the chunk's eight 128-column blocks
-    const int g = lane >> 2, tig = lane & 3;
-    const bool bsrc = g < 6 && (g < 3 ? has0 : has1);
-    const uint32_t src = bsrc ? smem_u32(g < 3 ? tok[0].pieces : tok[1].pieces) + (g % 3) * 128 + tig * 32 : 0u;
-    const uint32_t w_base = signs_s + ch * 2048 + g * 128 + tig * 4;
-    const uint32_t sc_base = sblk_s + 2 * (ch * 8);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-    for (int bp = 0; bp < 4; ++bp) {
-        int c2[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
-        const uint32_t sc_g = lds_u32(sc_base + 2 * (g * nb + 2 * bp));
-        const uint32_t sc_g8 = lds_u32(sc_base + 2 * ((g + 8) * nb + 2 * bp));
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            const int bb = 2 * bp + h2;
-            uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
-            if (bsrc) {
-                const uint32_t a = src + (ch * 8 + bb) * kPieceBlockBytes;
-                q0 = lds_v4(a);
-                q1 = lds_v4(a + 16);
-            }
-            const uint32_t wa = w_base + ((bb ^ (g & 7)) << 4);
-            const uint32_t wg = lds_u32(wa), wg8 = lds_u32(wa + 1024);
-            const uint32_t breg[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-            for (int mm = 0; mm < 4; ++mm) {
-                uint32_t a0, a1, a2, a3;
-                a_regs(wg, wg8, mm, a0, a1, a2, a3);
-                mma_s8(c2[h2], a0, a1, a2, a3, breg[2 * mm], breg[2 * mm + 1]);
-            }
-        }
-        const float2 sg = __half22float2(*reinterpret_cast<const __half2*>(&sc_g));
-        const float2 sg8 = __half22float2(*reinterpret_cast<const __half2*>(&sc_g8));
-        acc[0] = fmaf(sg.x, float(c2[0][0]), fmaf(sg.y, float(c2[1][0]), acc[0]));
-        acc[1] = fmaf(sg.x, float(c2[0][1]), fmaf(sg.y, float(c2[1][1]), acc[1]));
-        acc[2] = fmaf(sg8.x, float(c2[0][2]), fmaf(sg8.y, float(c2[1][2]), acc[2]));
-        acc[3] = fmaf(sg8.x, float(c2[0][3]), fmaf(sg8.y, float(c2[1][3]), acc[3]));
-    }
-    // 4. gather the 8 columns of every row through shared memory
-    scratch[g * 8 + 2 * tig] = acc[0];
-    scratch[g * 8 + 2 * tig + 1] = acc[1];
-    scratch[(g + 8) * 8 + 2 * tig] = acc[2];
-    scratch[(g + 8) * 8 + 2 * tig + 1] = acc[3];
-    __syncwarp();
-    {
-        float v0 = xt0 + corr0, v1 = xt1 + corr1;
-        v0 += __shfl_xor_sync(0xffffffffu, v0, 16);
-        v1 += __shfl_xor_sync(0xffffffffu, v1, 16);
-        const float* col = scratch + row * 8;
-        part[0] = has0 ? v0 - 2.0f * tok[0].sigma * (col[0] * 16384.0f + col[1] * 128.0f + col[2]) : 0.f;
-        part[1] = has1 ? v1 - 2.0f * tok[1].sigma * (col[3] * 16384.0f + col[4] * 128.0f + col[5]) : 0.f;
     }
     __syncwarp();
 }

@@ -526,15 +526,18 @@ __device__ __forceinline__ void ensure_cached(const DecArgs& A, const Shape& sh,
         for (int w = e * nblk; w < (e + 1) * nblk; ++w) m = fmaxf(m, M.red[w]);
         const float S = fixed_scale(m);
         const int b = blk * 8 + (lane >> 2), tig = lane & 3;
-        // fp16 copy (for the outliers) and the 128-block sums
+        // fp16 copy of v S / 64 (|v S| <= 2^20, so it cannot overflow whatever
+        // the size of the vector; the outlier sums are scaled back by 64 / S)
+        // and the 128-block sums
         uint4* x16 = reinterpret_cast<uint4*>(dst + C * kPieces + (C / 128) * 4) + blk * 128 + lane * 4;
+        const float s64 = S * 0.015625f;
         float sum = 0.f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             uint32_t hw[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const __half2 h2 = __floats2half2_rn(v[8 * i + 2 * j], v[8 * i + 2 * j + 1]);
+                const __half2 h2 = __floats2half2_rn(v[8 * i + 2 * j] * s64, v[8 * i + 2 * j + 1] * s64);
                 hw[j] = *reinterpret_cast<const uint32_t*>(&h2);
                 sum += v[8 * i + 2 * j] + v[8 * i + 2 * j + 1];
             }
@@ -689,6 +692,7 @@ __device__ __forceinline__ void row_outliers(const uint8_t* tile, const JobTile&
     const bool has0 = tok[0].pieces != nullptr, has1 = tok[1].pieces != nullptr;
     const __half* x0 = tok[0].x16;
     const __half* x1 = tok[1].x16;
+    float c0 = 0.f, c1 = 0.f;   // in units of the fp16 copies (v S / 64)
     for (int jb = sub; jb < k; jb += 6 * step) {
         int c[6];
         bool use[6];
@@ -710,10 +714,12 @@ __device__ __forceinline__ void row_outliers(const uint8_t* tile, const JobTile&
             const float sb = __half2float(sblk[c[u] >> 7]);
             float wq = fmaf(float(qv), srow, ((word >> (c[u] & 31)) & 1u) ? sb : -sb);
             wq = use[u] ? wq : 0.f;
-            if (has0) corr0 = fmaf(wq, __half2float(x0[c[u]]), corr0);
-            if (has1) corr1 = fmaf(wq, __half2float(x1[c[u]]), corr1);
+            if (has0) c0 = fmaf(wq, __half2float(x0[c[u]]), c0);
+            if (has1) c1 = fmaf(wq, __half2float(x1[c[u]]), c1);
         }
     }
+    if (has0) corr0 = fmaf(c0, 64.0f * tok[0].sigma, corr0);
+    if (has1) corr1 = fmaf(c1, 64.0f * tok[1].sigma, corr1);
 }
 
 // ----------------------------------------------------------------------------

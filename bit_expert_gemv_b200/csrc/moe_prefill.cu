@@ -56,6 +56,7 @@ struct TcArgs {
     const TcJob* jobs;
     const int32_t* n_jobs;
     float* out;                // [slots][rows] fp32
+    const float* unscale;      // [slots] factor of each slot's fp16 activation tile
     int32_t* status;
 };
 
@@ -150,18 +151,58 @@ __global__ void __launch_bounds__(1024) prefill_jobs_kernel(const int32_t* count
         jobs[first + i] = TcJob{e, offsets[e] + i * kTcChunk, min(kTcChunk, n_e - i * kTcChunk)};
 }
 
-// x of every pair in permuted order, rotated, as fp16: one warp per (token,
-// 1024-block) rotates the block once and writes it to the slot of each of the
-// token's routed pairs (pairs with an invalid expert id have no slot).
+// fp16 activation tiles carry a power-of-two scale per slot so that no value
+// overflows (or falls below the normal range) whatever the size of the input:
+// with m the row's largest |value| before the rotation, every rotated value
+// is at most 32 m (1/32 times a sum of 1024 terms), so the stored value
+// u * 2^k with 32 m 2^k in (2^13, 2^14] fits with room to spare; the tile
+// epilogue multiplies its sums by 2^-k (exact).
+__device__ __forceinline__ float slot_scale(float m) {
+    if (!(m > 0.f) || !(m < 3.0e38f)) return 1.0f;   // zero (or non-finite) rows keep scale 1
+    int e;
+    frexpf(32.0f * m, &e);                           // 32 m = f 2^e, f in [0.5, 1)
+    return ldexpf(1.0f, 14 - e);
+}
+
+// Largest |value| of row `src` (bf16 bits or fp32) of length d, all lanes of the warp.
+__device__ __forceinline__ float row_absmax(const void* src, bool bf16, int d) {
+    const int lane = threadIdx.x & 31;
+    float m = 0.f;
+    if (bf16) {
+        const uint2* p = static_cast<const uint2*>(src);
+#pragma unroll 4
+        for (int i = lane; i < d / 4; i += 32) {
+            const uint2 w = p[i];
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_to_f32(uint16_t(w.x))), fabsf(bf16_to_f32(uint16_t(w.x >> 16)))),
+                               fmaxf(fabsf(bf16_to_f32(uint16_t(w.y))), fabsf(bf16_to_f32(uint16_t(w.y >> 16))))));
+        }
+    } else {
+        const float4* p = static_cast<const float4*>(src);
+#pragma unroll 4
+        for (int i = lane; i < d / 4; i += 32) {
+            const float4 v = __ldcg(p + i);
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    return m;
+}
+
+// x of every pair in permuted order, rotated, as scaled fp16: one warp per
+// (token, 1024-block) rotates the block once and writes it to the slot of
+// each of the token's routed pairs (pairs with an invalid expert id have no
+// slot); the warps of block 0 write the slots' unscaling factors.
 __global__ void __launch_bounds__(256) gather_rotate_kernel(const uint16_t* __restrict__ x,
                                                             const int32_t* __restrict__ pos_of_pair, int B, int K,
-                                                            int d, __half* __restrict__ y) {
+                                                            int d, __half* __restrict__ y, float* __restrict__ unscale) {
     const int lane = threadIdx.x & 31;
     const int64_t wid = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
     const int nb = d / 1024;
     if (wid >= int64_t(B) * nb) return;
     const int64_t t = wid / nb;
     const int blk = int(wid - t * nb);
+    const float sc = slot_scale(row_absmax(x + t * d, true, d));
     const uint16_t* src = x + t * d + blk * 1024;
     float v[32];
 #pragma unroll
@@ -169,7 +210,7 @@ __global__ void __launch_bounds__(256) gather_rotate_kernel(const uint16_t* __re
     fwht1024_warp(v, lane);
     __half hv[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) hv[i] = __float2half_rn(v[i] * (1.0f / 32.0f));
+    for (int i = 0; i < 32; ++i) hv[i] = __float2half_rn(v[i] * (sc * (1.0f / 32.0f)));
 #pragma unroll 1
     for (int k = 0; k < K; ++k) {
         const int64_t s = pos_of_pair[t * K + k];
@@ -177,7 +218,30 @@ __global__ void __launch_bounds__(256) gather_rotate_kernel(const uint16_t* __re
         __half* dst = y + s * d + blk * 1024;
 #pragma unroll
         for (int i = 0; i < 32; ++i) dst[32 * i + lane] = hv[i];
+        if (blk == 0 && lane == 0) unscale[s] = 1.0f / sc;
     }
+}
+
+// h of every slot rotated into scaled fp16 (the w2 operand), one warp per
+// (slot, 1024-block); the warps of block 0 write the slots' unscaling factors.
+__global__ void __launch_bounds__(256) rotate_h_kernel(const float* __restrict__ h, int64_t P, int d,
+                                                       __half* __restrict__ y, float* __restrict__ unscale) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
+    const int nb = d / 1024;
+    if (wid >= P * nb) return;
+    const int64_t s = wid / nb;
+    const int blk = int(wid - s * nb);
+    const float sc = slot_scale(row_absmax(h + s * d, false, d));
+    const float* src = h + s * d + blk * 1024;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __ldcg(src + 32 * i + lane);
+    fwht1024_warp(v, lane);
+    __half* dst = y + s * d + blk * 1024;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) dst[32 * i + lane] = __float2half_rn(v[i] * (sc * (1.0f / 32.0f)));
+    if (blk == 0 && lane == 0) unscale[s] = 1.0f / sc;
 }
 
 // The 16 fp16 pairs of 32 weights: sign word w (bit c set = column c negative)
@@ -521,11 +585,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_tile_kernel(const __grid_con
                             const int j = col + k;
                             if (j < job.n) {
                                 float* o = A.out + int64_t(job.n0 + j) * A.rows;
+                                const float u = __ldg(A.unscale + job.n0 + j);
+                                const float a1 = v1[k] * u, a3 = v3[k] * u;
                                 if (GLU) {
-                                    o[ra] = __fdividef(v1[k], 1.0f + __expf(-v1[k])) * v3[k];
+                                    o[ra] = __fdividef(a1, 1.0f + __expf(-a1)) * a3;
                                 } else {
-                                    o[ra] = v1[k];
-                                    o[rb] = v3[k];
+                                    o[ra] = a1;
+                                    o[rb] = a3;
                                 }
                             }
                         }
@@ -581,6 +647,8 @@ PrefillWs carve_prefill_ws(void* ws, const gale_layer& L, int B, int K) {
     w.jobs = take(int64_t(sizeof(TcJob)) * w.max_jobs);
     w.n_jobs = reinterpret_cast<int32_t*>(take(8));
     w.x16 = reinterpret_cast<__half*>(take(2 * P * dm));
+    w.x_unscale = reinterpret_cast<float*>(take(4 * P));
+    w.h_unscale = reinterpret_cast<float*>(take(4 * P));
     w.h = reinterpret_cast<float*>(take(4 * P * df));
     w.h16 = reinterpret_cast<__half*>(take(2 * P * df));
     w.o = reinterpret_cast<float*>(take(4 * P * dm));
@@ -622,7 +690,7 @@ int launch_moe_prefill(const gale_layer& L, const uint16_t* x, const int32_t* id
     {
         const int64_t warps = int64_t(B) * (L.d_model / 1024);
         gather_rotate_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, st>>>(x, w.pos_of_pair, B, K, L.d_model,
-                                                                                  w.x16);
+                                                                                  w.x16, w.x_unscale);
         GALE_LAUNCH_CHECK();
     }
     const int64_t l1 = make_layout(L.d_ff, L.d_model).total;
@@ -641,11 +709,15 @@ int launch_moe_prefill(const gale_layer& L, const uint16_t* x, const int32_t* id
     a.rows = L.d_ff;
     a.cols = L.d_model;
     a.out = w.h;
+    a.unscale = w.x_unscale;
     rc = launch_tc<true>(xm, a, w.max_jobs, st);
     if (rc != GALE_OK) return rc;
-    // rotate h
-    rc = gale_fwht1024(w.h, GALE_F32, w.h16, GALE_F16, P, L.d_ff, st);
-    if (rc != GALE_OK) return rc;
+    // rotate h into scaled fp16
+    {
+        const int64_t warps = P * (L.d_ff / 1024);
+        rotate_h_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, st>>>(w.h, P, L.d_ff, w.h16, w.h_unscale);
+        GALE_LAUNCH_CHECK();
+    }
     CUtensorMap hm;
     rc = act_map(&hm, w.h16, L.d_ff, P, kTcChunk);
     if (rc != GALE_OK) return rc;
@@ -655,6 +727,7 @@ int launch_moe_prefill(const gale_layer& L, const uint16_t* x, const int32_t* id
     a.rows = L.d_model;
     a.cols = L.d_ff;
     a.out = w.o;
+    a.unscale = w.h_unscale;
     rc = launch_tc<false>(hm, a, w.max_jobs, st);
     if (rc != GALE_OK) return rc;
     return launch_moe_combine(w.o, w.pos_of_pair, gates, x, B, K, L.d_model, out, out_dtype, fuse_norm, eps,

@@ -17,9 +17,11 @@ struct PrefillWs {
     void* jobs;             // [max_jobs] (expert, first slot, tokens), chunks of 128 slots
     int32_t* n_jobs;        // [1]
     int max_jobs;
-    __half* x16;            // [B*K][d_model] rotated x of each pair, permuted order
+    __half* x16;            // [B*K][d_model] rotated x of each pair, permuted order, scaled
+    float* x_unscale;       // [B*K] factor that undoes each slot's x16 scale
+    float* h_unscale;       // [B*K] the same for h16
     float* h;               // [B*K][d_ff]
-    __half* h16;            // [B*K][d_ff] rotated h
+    __half* h16;            // [B*K][d_ff] rotated h, scaled per slot
     float* o;               // [B*K][d_model]
     float* scratch;         // [B][d_model]
     size_t bytes;

@@ -23,16 +23,23 @@ std::mutex g_scratch_mu;
 
 // Device address of the scratch array on the current device.  The array's
 // name in host code is only a host-side stand-in; the device address comes
-// from cudaGetSymbolAddress, queried once per device with that device current.
-int scratch_address(void** out) {
+// from cudaGetSymbolAddress with that device current.  It is looked up again
+// on every call made outside stream capture (a context that was reset and
+// created again may place the array elsewhere); a call inside a capture uses
+// the address of the last uncaptured call on the device.
+int scratch_address(cudaStream_t st, void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return GALE_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return GALE_ERR_UNSUPPORTED;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return GALE_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    if (cs == cudaStreamCaptureStatusNone) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GALE_ERR_CUDA;
         g_scratch_addr[dev] = p;
+    } else if (!g_scratch_addr[dev]) {
+        return GALE_ERR_UNSUPPORTED;   // no uncaptured call on this device yet
     }
     *out = g_scratch_addr[dev];
     return GALE_OK;
@@ -51,7 +58,7 @@ extern "C" int gale_moe_forward_noalloc(const gale_layer* layer, const uint16_t*
     if (need > size_t(GALE_NOALLOC_SCRATCH_BYTES)) return GALE_ERR_WORKSPACE;
     if (status && !gale::aligned(status, 4)) return GALE_ERR_ALIGN;
     void* ws = nullptr;
-    rc = scratch_address(&ws);
+    rc = scratch_address(gale::as_stream(stream), &ws);
     if (rc != GALE_OK) return rc;
     rc = gale_moe_forward(layer, x, ids, gates, B, K, out, out_dtype, flags, eps, ws,
                           size_t(GALE_NOALLOC_SCRATCH_BYTES), stream);

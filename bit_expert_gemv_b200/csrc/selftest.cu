@@ -104,9 +104,9 @@ extern "C" int gale_selftest(void* scratch, void* stream) {
             int c = idx[r * k + j];
             want += (long(q[r * k + j]) - (signs[r * kC + c] ? -1 : 1)) * long(x[c]);
         }
-        if (y[r] != float(want)) return GALE_ERR_UNSUPPORTED;
+        if (y[r] != float(want)) return GALE_ERR_SELFTEST;
     }
     for (int c = 0; c < kC; ++c)
-        if (fabsf(xr[c] - x[kC + c]) > 1e-5f) return GALE_ERR_UNSUPPORTED;
+        if (fabsf(xr[c] - x[kC + c]) > 1e-5f) return GALE_ERR_SELFTEST;
     return GALE_OK;
 }

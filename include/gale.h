@@ -43,6 +43,7 @@ extern "C" {
 #define GALE_ERR_CUDA        -4   /* a CUDA runtime call or launch failed */
 #define GALE_ERR_TIMEOUT     -5   /* a bounded device-side wait ran out */
 #define GALE_ERR_UNSUPPORTED -6   /* shape or device not supported */
+#define GALE_ERR_SELFTEST    -7   /* gale_selftest: a GPU result differs from the expected value */
 
 /* element types */
 #define GALE_F32  0
@@ -236,9 +237,12 @@ int gale_moe_forward(const gale_layer* layer, const uint16_t* x, const int32_t* 
  *  - status: optional device int32; when non-NULL the call ends by copying
  *    the device status word there (same codes as gale_moe_forward's);
  *  - the library allocates and frees nothing (no cudaMalloc, no cudaFree);
- *  - the first call on each device looks up the array's device address with
- *    that device current and caches it: make that first call before any
- *    stream capture;
+ *  - every call made outside stream capture looks the array's device
+ *    address up again with the calling device current (so the address stays
+ *    right after a cudaDeviceReset or any other re-creation of the primary
+ *    context); a call made while its stream is being captured uses the
+ *    address of the last uncaptured call on that device, so make at least
+ *    one call on the device before capturing, and again after a reset;
  *  - all calls on a device share the one array and it keeps the previous
  *    call's contents (each call clears what must start at zero): calls that
  *    overlap on the GPU, from any stream or thread, race and give undefined
@@ -282,7 +286,8 @@ int gale_moe_forward_host(const gale_layer* layer, const uint16_t* x, const int3
  * verify themselves at startup" -- without any fallback).  Synchronous:
  * allocates nothing itself but needs `scratch` of gale_selftest_scratch_bytes()
  * device bytes.  Returns GALE_OK when the GPU results match the host-side
- * expectations built into the library. */
+ * expectations built into the library, GALE_ERR_SELFTEST when one differs,
+ * and the usual codes for launch or argument failures. */
 size_t gale_selftest_scratch_bytes(void);
 int gale_selftest(void* scratch, void* stream);
 

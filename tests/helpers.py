@@ -18,6 +18,54 @@ def rel_l2(a, b) -> float:
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
+def rel_l2_rows(a, b) -> np.ndarray:
+    """Relative L2 error of every row (token) of a against b."""
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return np.linalg.norm(a - b, axis=-1) / np.maximum(np.linalg.norm(b, axis=-1), 1e-300)
+
+
+def assert_tokens(got, want, tol=REL_L2_TOL, what=""):
+    """Per-token parity: every row within `tol` relative L2; rows the oracle
+    gives as exact zeros must be exact zeros."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert got.shape == want.shape, what
+    assert np.isfinite(got).all(), what
+    zero = np.all(want == 0.0, axis=-1)
+    assert np.all(got[zero] == 0.0), f"{what}: rows {np.nonzero(zero)[0][:8]} should be exactly zero"
+    if (~zero).any():
+        e = rel_l2_rows(got[~zero], want[~zero])
+        worst = int(np.argmax(e))
+        assert e.max() < tol, f"{what}: token {np.nonzero(~zero)[0][worst]} rel-L2 {e.max():.3g} >= {tol}"
+
+
+def bf16_round(v) -> np.ndarray:
+    """fp64 values rounded to bf16 (round to nearest even), back as fp64."""
+    return gs.bf16_bits_to_f32(gs.f32_to_bf16_bits(np.asarray(v, dtype=np.float32))).astype(np.float64)
+
+
+def edge_hidden(B: int, d: int, kind: str, tag: int):
+    """bf16 hidden states with a hard case planted: "spikes" puts three
+    features of every token at 300x the rms, "zero" makes the middle token all
+    zeros, "scaled" multiplies every value by 1000.  Returns (bits, values)."""
+    _, v = gs.hidden_bf16(B, d, tag=tag)
+    v = v.astype(np.float32).copy()
+    if kind == "spikes":
+        rng = np.random.default_rng(tag)
+        for t in range(B):
+            cols = rng.choice(d, size=3, replace=False)
+            v[t, cols] = 300.0 * np.sign(v[t, cols] + 0.5)
+    elif kind == "zero":
+        v[B // 2] = 0.0
+    elif kind == "scaled":
+        v *= 1000.0
+    else:
+        raise ValueError(kind)
+    bits = gs.f32_to_bf16_bits(v)
+    return bits, gs.bf16_bits_to_f32(bits)
+
+
 def to_dev(a, dtype=None):
     import torch
     t = torch.from_numpy(np.ascontiguousarray(a))
