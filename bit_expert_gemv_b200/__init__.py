@@ -33,6 +33,7 @@ EXPORTS = (
     "gale_route_permute_grid", "gale_moe_workspace_size",
     "gale_moe_forward", "gale_moe_forward_noalloc", "gale_selftest_scratch_bytes", "gale_selftest",
     "gale_moe_host_staging_bytes", "gale_moe_host_workspace_size", "gale_moe_forward_host",
+    "gale_debug_set_failure", "gale_route_topk",
 )
 
 GALE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
             "gale_moe_host_workspace_size": (sz, [ctypes.POINTER(gale_layer), i32, i32]),
             "gale_moe_forward_host": (i32, [ctypes.POINTER(gale_layer), vp, vp, vp, i32, i32, vp, i32, i32,
                                             ctypes.c_float, vp, sz, vp, sz, vp]),
+            "gale_debug_set_failure": (i32, [ctypes.c_uint64, i32]),
+            "gale_route_topk": (i32, [vp, i32, i32, i32, vp, vp, vp]),
             "gale_selftest_scratch_bytes": (sz, []),
             "gale_selftest": (i32, [vp, vp]),
         }
@@ -193,6 +196,13 @@ def gale_route_permute_grid(ids, n_experts: int, counts, offsets, perm, status, 
                                          _stream(stream)), "gale_route_permute_grid")
 
 
+def gale_route_topk(logits, ids, gates, stream=None):
+    """Top-K experts of every token (K = ids.shape[1]) and their softmax gates."""
+    B, E = logits.shape
+    _check(lib().gale_route_topk(_ptr(logits), B, E, ids.shape[1], _ptr(ids), _ptr(gates), _stream(stream)),
+           "gale_route_topk")
+
+
 def make_layer(base, expert_stride: int, n_experts: int, d_model: int, d_ff: int) -> gale_layer:
     return gale_layer(_ptr(base), expert_stride, n_experts, d_model, d_ff, 0)
 
@@ -239,6 +249,12 @@ def gale_moe_forward_host(layer: gale_layer, x, ids, gates, out, ws, staging, fl
                                        _dtype_code(out), flags, eps, _ptr(ws), ws.numel() * ws.element_size(),
                                        _ptr(staging), staging.numel() * staging.element_size(), _stream(stream)),
            "gale_moe_forward_host")
+
+
+def gale_debug_set_failure(wait_limit_ns: int, withhold_cta: int):
+    """Failure-path testing: bound of the streaming decode kernel's device
+    waits (0 = default 2 s) and a CTA whose h tiles are never counted (-1 = none)."""
+    _check(lib().gale_debug_set_failure(int(wait_limit_ns), int(withhold_cta)), "gale_debug_set_failure")
 
 
 def gale_selftest_scratch_bytes() -> int:

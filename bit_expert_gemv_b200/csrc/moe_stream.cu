@@ -67,7 +67,7 @@ constexpr int kSmemBytes = 227 * 1024;
 constexpr int kR1 = 16;                       // rows of w1 (and of w3) per phase-1 unit
 constexpr int kR2 = 64;                       // rows of w2 per phase-2 unit
 constexpr int kPartBytes = 192 * kSegTok * 4; // partial sums of a stage: 192 rows x 2 tokens
-constexpr uint64_t kWaitNs = 2000000000ull;   // bound of every wait
+constexpr uint64_t kWaitNs = 2000000000ull;   // default bound of every wait
 
 struct StreamArgs {
     const char* base;
@@ -80,6 +80,8 @@ struct StreamArgs {
     void* out;
     int out_dtype, fuse_norm;
     float eps;
+    uint64_t wait_ns;       // bound of every wait
+    int withhold_cta;       // failure-path testing: this CTA never counts its h tiles (-1: none)
     StreamWs ws;
 };
 
@@ -178,6 +180,7 @@ struct Ctl {
     int s1b, s2b, nl1, nl, ngrp; // first segment of each range, local segments of phase 1, in all; groups
     int stages, slot_bytes, ring;
     int issued;                  // units whose copies the producer issued
+    uint64_t wait_ns;            // bound of every wait
     int grp_of[kMaxLocalSeg];    // group of each local segment
     int grp_seg[kMaxLocalSeg];   // the local segment whose pairs define each group
     int grp_left[kMaxLocalSeg];  // units of each group not finished yet
@@ -220,8 +223,8 @@ __device__ __forceinline__ int bfe_s32(uint32_t v, uint32_t pos, uint32_t len) {
 // Bounded waits that leave the issue slots to the warps doing work: a
 // shared-memory counter of this CTA or a global counter of other CTAs is
 // re-read after a short sleep; an mbarrier phase is awaited with the
-// hardware's suspend hint.  Each returns false on abort or after kWaitNs.
-__device__ __noinline__ bool wait_smem(const int* p, int v, bool eq, const int* abort) {
+// hardware's suspend hint.  Each returns false on abort or after `limit` ns.
+__device__ __noinline__ bool wait_smem(const int* p, int v, bool eq, const int* abort, uint64_t limit) {
     unsigned ns = 64;
     uint64_t t0 = 0;
 #pragma unroll 1
@@ -230,13 +233,13 @@ __device__ __noinline__ bool wait_smem(const int* p, int v, bool eq, const int* 
         if (eq ? x == v : x >= v) return true;
         if (vload(abort)) return false;
         if (it == 0) t0 = globaltimer_ns();
-        else if (globaltimer_ns() - t0 > kWaitNs) return false;
+        else if (globaltimer_ns() - t0 > limit) return false;
         __nanosleep(ns);
         if (ns < 512) ns <<= 1;
     }
 }
 
-__device__ __noinline__ bool wait_global(const int32_t* p, int v, const int* abort) {
+__device__ __noinline__ bool wait_global(const int32_t* p, int v, const int* abort, uint64_t limit) {
     unsigned ns = 64;
     uint64_t t0 = 0;
 #pragma unroll 1
@@ -244,13 +247,13 @@ __device__ __noinline__ bool wait_global(const int32_t* p, int v, const int* abo
         if (ld_acquire(p) >= v) return true;
         if (vload(abort)) return false;
         if (it == 0) t0 = globaltimer_ns();
-        else if (globaltimer_ns() - t0 > kWaitNs) return false;
+        else if (globaltimer_ns() - t0 > limit) return false;
         __nanosleep(ns);
         if (ns < 512) ns <<= 1;
     }
 }
 
-__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, uint64_t limit = kWaitNs) {
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, uint64_t limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait_sleep(bar, parity))
@@ -287,6 +290,7 @@ __device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, Route
     if (tid < kMaxLocalSeg) c.grp_left[tid] = 0;
     if (tid == 32) {
         c.issued = 0;
+        c.wait_ns = A.wait_ns;
         c.next_piece = 0;
         c.slot_grp[0] = 0;
         c.slot_grp[1] = 1;
@@ -862,7 +866,7 @@ __device__ __noinline__ void act_piece(const StreamArgs& A, const Plan& P, Ctl& 
         build_block(A.x + (pair / A.K) * A.d_model, 1, blk, slot + uint32_t(tk * P.t1.bytes), P.t1);
     } else {
         int v = 1;
-        if (lane == 0) v = wait_global(A.ws.hcnt + s * P.nch2 + blk, 1024 / kR1, &c.abort);
+        if (lane == 0) v = wait_global(A.ws.hcnt + s * P.nch2 + blk, 1024 / kR1, &c.abort, c.wait_ns);
         v = __shfl_sync(0xffffffffu, v, 0);
         if (!v) {
             set_status(A.ws.status, GALE_ERR_TIMEOUT);
@@ -915,7 +919,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
 #pragma unroll 1
             for (int u = 0; u < nunits; ++u) {
                 const UnitRef R = unit_ref(c, P, u);
-                if (u >= S && !wait_phase(&c.empty[R.st], R.par ^ 1)) {
+                if (u >= S && !wait_phase(&c.empty[R.st], R.par ^ 1, c.wait_ns)) {
                     set_status(status, GALE_ERR_TIMEOUT);
                     atomicExch(&c.abort, 1);
                     break;
@@ -973,7 +977,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
             const int tstride = R.p1 ? P.t1.bytes : P.t2.bytes;
             const uint32_t slot = slot_base + uint32_t(sl * c.slot_bytes);
             {
-                bool ok = wait_smem(&c.slot_grp[sl], g, true, &c.abort);
+                bool ok = wait_smem(&c.slot_grp[sl], g, true, &c.abort, c.wait_ns);
 #pragma unroll 1
                 while (ok && vload(&c.slot_done[sl]) < need) {
                     // the slot cannot move on while this unit is unfinished,
@@ -987,7 +991,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
                         __threadfence_block();
                         if (lane == 0) atomicAdd(&c.slot_done[sl], 1);
                     } else {
-                        ok = wait_smem(&c.slot_done[sl], need, false, &c.abort);
+                        ok = wait_smem(&c.slot_done[sl], need, false, &c.abort, c.wait_ns);
                     }
                 }
                 if (!ok) {
@@ -998,7 +1002,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
                 __threadfence_block();
             }
             // ---- the unit's rows ----
-            if (!wait_phase(&c.full[R.st], R.par)) {
+            if (!wait_phase(&c.full[R.st], R.par, c.wait_ns)) {
                 set_status(status, GALE_ERR_TIMEOUT);
                 atomicExch(&c.abort, 1);
                 break;
@@ -1076,7 +1080,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
                         A.ws.h[pair * A.d_ff + R.tile * kR1 + r] = silu_fast(g1) * g3;
                     }
                     __syncwarp();
-                    if (lane == 0) {
+                    if (lane == 0 && int(blockIdx.x) != A.withhold_cta) {
                         __threadfence();
                         atomicAdd(A.ws.hcnt + R.s * nhb + (R.tile * kR1) / 1024, 1);
                     }
@@ -1153,6 +1157,10 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
     }
 }
 
+// Failure-path testing settings (process-wide, see gale_debug_set_failure).
+uint64_t g_wait_ns = kWaitNs;
+int g_withhold_cta = -1;
+
 }  // namespace
 
 StreamWs carve_stream_ws(void* ws, const gale_layer& L, int B, int K) {
@@ -1210,6 +1218,8 @@ int launch_moe_stream(const gale_layer& L, const uint16_t* x, const int32_t* ids
     A.out_dtype = out_dtype;
     A.fuse_norm = fuse_norm ? 1 : 0;
     A.eps = eps;
+    A.wait_ns = g_wait_ns;
+    A.withhold_cta = g_withhold_cta;
     A.ws = carve_stream_ws(ws, L, B, K);
     GALE_CUDA_TRY(cudaMemsetAsync(A.ws.status, 0, A.ws.counter_bytes, st));
     CUtensorMap map13, map2;
@@ -1234,3 +1244,9 @@ int launch_moe_stream(const gale_layer& L, const uint16_t* x, const int32_t* ids
 }
 
 }  // namespace gale
+
+extern "C" int gale_debug_set_failure(uint64_t wait_limit_ns, int withhold_cta) {
+    gale::g_wait_ns = wait_limit_ns ? wait_limit_ns : gale::kWaitNs;
+    gale::g_withhold_cta = withhold_cta;
+    return GALE_OK;
+}

@@ -347,3 +347,81 @@ extern "C" int gale_route_permute_grid(const int32_t* ids, int B, int K, int E, 
     a.status = status;
     return gale::launch_route_permute_grid(a, scratch, st);
 }
+
+// ----------------------------------------------------------------------------
+// router: top-K experts by logit and their softmax gates
+// ----------------------------------------------------------------------------
+
+namespace gale {
+namespace {
+
+// One warp per token.  Lane l holds the logits of experts l, l + 32, ...;
+// each of the K rounds takes the warp-wide (largest logit, lowest index) not
+// yet taken, and lane k keeps round k's pick.  NaN logits count as -inf.
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int B, int E, int K,
+                                                         int32_t* __restrict__ ids, float* __restrict__ gates) {
+    const int lane = threadIdx.x & 31;
+    const int t = int((blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5);
+    if (t >= B) return;
+    const float* l = logits + int64_t(t) * E;
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const int e = lane + 32 * j;
+        const float x = e < E ? __ldg(l + e) : -INFINITY;
+        v[j] = x == x ? x : -INFINITY;
+    }
+    uint32_t taken = 0u;
+    float mine = -INFINITY;
+    int mine_id = -1;
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+        float bv = -INFINITY;
+        int bi = 0x7FFFFFFF;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E && !((taken >> j) & 1u) && (v[j] > bv || (v[j] == bv && e < bi))) {
+                bv = v[j];
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        if (lane == k) {
+            mine = bv;
+            mine_id = bi;
+        }
+    }
+    // softmax over the K picks (lane 0 holds the largest)
+    const float m = __shfl_sync(0xffffffffu, mine, 0);
+    const float ex = lane < K ? expf(mine - m) : 0.f;
+    const float sum = warp_sum(ex);
+    if (lane < K) {
+        ids[int64_t(t) * K + lane] = mine_id;
+        gates[int64_t(t) * K + lane] = ex / sum;
+    }
+}
+
+}  // namespace
+}  // namespace gale
+
+extern "C" int gale_route_topk(const float* logits, int B, int E, int K, int32_t* ids, float* gates, void* stream) {
+    if (B < 0 || E < 1 || E > 1024 || K < 1 || K > 16 || K > E) return GALE_ERR_ARG;
+    if (B == 0) return GALE_OK;
+    if (!logits || !ids || !gates) return GALE_ERR_ARG;
+    if (!gale::aligned(logits, 4) || !gale::aligned(ids, 4) || !gale::aligned(gates, 4)) return GALE_ERR_ALIGN;
+    const int64_t threads = int64_t(B) * 32;
+    gale::route_topk_kernel<<<unsigned((threads + 255) / 256), 256, 0, gale::as_stream(stream)>>>(logits, B, E, K, ids,
+                                                                                                 gates);
+    GALE_LAUNCH_CHECK();
+    return GALE_OK;
+}

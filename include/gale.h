@@ -181,6 +181,20 @@ int gale_route_permute_grid(const int32_t* ids, int B, int K, int E, int32_t* co
                             size_t scratch_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Router: the top-K experts of every token and their gates (the cards' "top-6
+ * of 256 experts" per token; the gates are the softmax over the K selected
+ * logits, as the benchmark configuration normalises them).
+ *   logits : device fp32 [B][E]
+ *   ids    : device int32 [B][K], experts by descending logit; on equal logits
+ *            the lower expert index comes first; NaN logits rank as -inf
+ *   gates  : device fp32 [B][K], exp(l_k - l_max) / sum over the K picks (fp32)
+ * 1 <= K <= 16, K <= E <= 1024, B >= 0 (0 is a no-op).  One launch, one warp
+ * per token; the outputs feed gale_moe_forward directly.
+ * Errors: GALE_ERR_ARG (sizes, NULL pointers), GALE_ERR_ALIGN.
+ * ------------------------------------------------------------------------- */
+int gale_route_topk(const float* logits, int B, int E, int K, int32_t* ids, float* gates, void* stream);
+
+/* ---------------------------------------------------------------------------
  * One routed-expert MoE layer.
  * ------------------------------------------------------------------------- */
 typedef struct {
@@ -281,6 +295,19 @@ int gale_moe_forward_host(const gale_layer* layer, const uint16_t* x, const int3
                           const float* gates, int B, int K, void* out, int out_dtype, int flags,
                           float eps, void* ws, size_t ws_bytes, void* staging, size_t staging_bytes,
                           void* stream);
+
+/* Failure-path testing hook; an interface addition of this library with no
+ * counterpart on the GALE cards.  Applies to later gale_moe_forward calls of
+ * this process that take the streaming decode kernel (3 to 64 tokens):
+ *   wait_limit_ns : bound of every device-side wait of the kernel, in ns
+ *                   (0 restores the default of 2 s);
+ *   withhold_cta  : a CTA index whose finished h tiles are never counted
+ *                   (-1: none), so that the phase-2 waits of the CTAs that
+ *                   need those tiles run out: the call then reports
+ *                   GALE_ERR_TIMEOUT in its status word, every CTA drains its
+ *                   copies and returns, and the output is unspecified.
+ * Process-wide and not thread-safe; meant for tests of the failure path. */
+int gale_debug_set_failure(uint64_t wait_limit_ns, int withhold_cta);
 
 /* Built-in parity self-check on tiny shapes (the card's "optional fast paths
  * verify themselves at startup" -- without any fallback).  Synchronous:

@@ -251,8 +251,34 @@ def chain_step(dense_of, x_bf16_values: np.ndarray, ids, gates, eps: float = 1e-
 
 
 # ----------------------------------------------------------------------------
-# routing permute
+# router and routing permute
 # ----------------------------------------------------------------------------
+
+def route_topk(logits: np.ndarray, k: int):
+    """Top-k routing of every token: the k experts of largest fp32 logit, in
+    descending order (a lower expert index first on equal logits), and their
+    gates, the softmax over the k selected logits taken in fp64 and rounded
+    to fp32.
+
+    Reading: the cards give "top-6 of 256 experts" per token; the benchmark
+    configuration normalises the gates over the selected six.  Written as a
+    plain sort of (-logit, index) and exp / sum.
+    """
+    lg = np.asarray(logits, dtype=np.float32)
+    B, E = lg.shape
+    ids = np.zeros((B, k), dtype=np.int32)
+    gates = np.zeros((B, k), dtype=np.float32)
+    for t in range(B):
+        order = sorted(range(E), key=lambda e: (-float(lg[t, e]), e))[:k]
+        sel = [float(lg[t, e]) for e in order]
+        m = max(sel)
+        ex = [math.exp(v - m) for v in sel]
+        tot = sum(ex)
+        ids[t] = order
+        gates[t] = [v / tot for v in ex]
+    return ids, gates
+
+
 
 def route_permute(ids: np.ndarray, n_experts: int):
     """Group the (token, slot) pairs by expert, stable in (token, slot) order.

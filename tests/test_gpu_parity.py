@@ -469,3 +469,36 @@ def test_moe_prefill_full_size(full_layer, skew):
 def test_selftest():
     scratch = torch.empty(G.gale_selftest_scratch_bytes(), dtype=torch.uint8, device="cuda")
     assert G.gale_selftest(scratch) == G.GALE_OK
+
+
+# ----------------------------------------------------------------------------
+# router
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,E,K,skew", [(1, 256, 6, 0.0), (8, 256, 6, 0.0), (64, 256, 6, 0.5), (4096, 256, 6, 0.5),
+                                         (5, 16, 16, 0.0), (33, 1000, 8, 0.0), (7, 1024, 1, 0.0)])
+def test_route_topk_matches_oracle(B, E, K, skew):
+    """Ids bit-exact, gates within 1e-6, against the oracle's router."""
+    lg = gs.router_logits(B, E, tag=6000 + B, bias_sigma=skew)
+    ids = torch.empty(B, K, dtype=torch.int32, device="cuda")
+    gates = torch.empty(B, K, dtype=torch.float32, device="cuda")
+    G.gale_route_topk(to_dev(lg), ids, gates)
+    torch.cuda.synchronize()
+    wi, wg = O.route_topk(lg, K)
+    assert np.array_equal(ids.cpu().numpy(), wi)
+    assert np.max(np.abs(gates.cpu().numpy().astype(np.float64) - wg)) < 1e-6
+
+
+def test_route_topk_ties_and_nan():
+    """Equal logits go to the lower expert index; NaN ranks last."""
+    lg = np.array([[0.5, 2.0, 2.0, np.nan, 2.0, -1.0, 0.5, 0.5]] * 3, np.float32)
+    lg[1, 1] = np.nan
+    lg[2] = 1.0
+    ids = torch.empty(3, 4, dtype=torch.int32, device="cuda")
+    gates = torch.empty(3, 4, dtype=torch.float32, device="cuda")
+    G.gale_route_topk(to_dev(lg), ids, gates)
+    torch.cuda.synchronize()
+    assert ids.cpu().numpy().tolist() == [[1, 2, 4, 0], [2, 4, 0, 6], [0, 1, 2, 3]]
+    wi, wg = O.route_topk(np.nan_to_num(lg, nan=-np.inf), 4)
+    assert np.array_equal(ids.cpu().numpy(), wi)
+    assert np.max(np.abs(gates.cpu().numpy().astype(np.float64) - wg)) < 1e-6

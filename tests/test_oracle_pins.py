@@ -390,6 +390,40 @@ def test_route_topk_gates_sum_to_one():
         assert np.all(np.diff(lg[t, ids[t]]) <= 0)
 
 
+def test_oracle_route_topk_by_hand_and_ties():
+    # equal logits: the lower expert index comes first
+    lg = np.array([[1.0, 3.0, 3.0, 2.0, -1.0]], np.float32)
+    ids, g = O.route_topk(lg, 2)
+    assert ids.tolist() == [[1, 2]]
+    assert g.tolist() == [[0.5, 0.5]]
+    ids, g = O.route_topk(lg, 3)
+    assert ids.tolist() == [[1, 2, 3]]
+    e = [1.0, 1.0, math.exp(-1.0)]
+    want = [v / sum(e) for v in e]
+    assert np.max(np.abs(g[0].astype(np.float64) - want)) < 1e-7
+
+
+def test_oracle_route_topk_brute_force():
+    """Against every k-subset of a small expert set: the selected set is the
+    one whose sorted logits are largest (lexicographic), gates follow the
+    closed form exp(l_i - l_j) for their ratios and sum to one."""
+    import itertools
+    rng = np.random.default_rng(3)
+    for t in range(20):
+        E, k = 7, 3
+        lg = rng.integers(-3, 4, size=(1, E)).astype(np.float32)   # many ties
+        ids, g = O.route_topk(lg, k)
+        best = max(itertools.combinations(range(E), k),
+                   key=lambda c: (sorted((float(lg[0, e]) for e in c), reverse=True), [-e for e in sorted(c)]))
+        assert sorted(ids[0].tolist()) == sorted(best)
+        vals = lg[0, ids[0]].astype(np.float64)
+        assert np.all(np.diff(vals) <= 0)
+        assert abs(float(g[0].astype(np.float64).sum()) - 1.0) < 1e-6
+        for i in range(k):
+            for j in range(k):
+                assert abs(g[0, i] / g[0, j] - math.exp(vals[i] - vals[j])) < 1e-5
+
+
 def test_route_permute_brute_force():
     ids = np.array([[3, 1, 0], [1, 3, 2], [0, 1, 3], [3, 2, 1]], np.int32)
     counts, offsets, perm = O.route_permute(ids, 5)
