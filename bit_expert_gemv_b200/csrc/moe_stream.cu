@@ -33,17 +33,19 @@
 //    share a slot (at batch 1 a CTA rotates x once).  A phase-2 slot waits
 //    until the segment's h blocks are complete in every CTA.
 //
-// Arithmetic of a tile (mma.sync m16n8k32, int8, exact int32 sums).  For row
-// r and a 128-column block b,  sum_c sign(r,c) x_c = X_b - 2 P_b  with
+// Arithmetic of a tile (mma.sync m16n8k32, s8 x u8, exact int32 sums).  For
+// row r and a 128-column block b,  sum_c sign(r,c) x_c = X_b - 2 P_b  with
 // P_b = sum_{c in b, bit(r,c)=1} x_c.  A sign word w of 32 columns gives the
 // A operand of bit position s as w & (0x01010101 << s), whose bytes are
 // bit * a(s), a(s) = 2^s for s < 7 and -128 for s = 7.  Each 1024-block of an
 // activation is held in fixed point, X_c = round(u_c S / a(c mod 8)) with u
-// the unnormalised transform and S a power of two such that |u S| <= 2^20,
-// as three int8 digits (X = d1 2^14 + d2 2^7 + d3), one MMA column per digit
-// and token; the block sums X_b are exact integers of the same values.  The
-// outlier corrections (q s_row - sign s_blk) x_c read x_c from an fp16 copy
-// of u S / 64 (per-block scale, so it cannot overflow).
+// the unnormalised transform and S a power of two such that |u S| <= 2^20;
+// Y_c = X_c + 2^20 (0 <= Y_c <= 2^21) is stored as three unsigned bytes, one
+// MMA column per byte and token, plus a column of ones that counts
+// sum a(s) bit, so that the 2^20 offset cancels exactly in int32.  The block
+// sums X_b are exact integers of the same values.  The outlier corrections
+// (q s_row - sign s_blk) x_c read x_c from an fp16 copy of u S / 64
+// (per-block scale, so it cannot overflow).
 //
 // Code size matters here: code run once per launch is fetched cold, so the
 // helpers are single out-of-line copies with rolled loops.
@@ -68,6 +70,16 @@ constexpr int kR1 = 16;                       // rows of w1 (and of w3) per phas
 constexpr int kR2 = 64;                       // rows of w2 per phase-2 unit
 constexpr int kPartBytes = 192 * kSegTok * 4; // partial sums of a stage: 192 rows x 2 tokens
 constexpr uint64_t kWaitNs = 2000000000ull;   // default bound of every wait
+
+// Division by a run-time constant d >= 2 as a multiply-high: exact for
+// n * d < 2^32 (n below 2^23 here, d at most a few hundred).
+struct FastDiv {
+    uint32_t d, m;
+};
+__host__ __device__ inline FastDiv make_div(uint32_t d) {
+    return FastDiv{d, uint32_t((0x100000000ull + d - 1) / d)};
+}
+__device__ __forceinline__ int fdiv(int n, FastDiv f) { return int(__umulhi(uint32_t(n), f.m)); }
 
 struct StreamArgs {
     const char* base;
@@ -112,9 +124,11 @@ struct Plan {
     int part;                    // partial area offset in a stage
     int stage_bytes;
     Layout L1, L2;
+    FastDiv dt1, dt2, dpp1, dpp2;   // division by tiles1, tiles2, pp1, pp2
 };
 
 __host__ __device__ inline int align_i(int n, int a) { return (n + a - 1) / a * a; }
+
 
 __host__ __device__ inline TokMap make_tokmap(int C) {
     TokMap t;
@@ -162,6 +176,10 @@ __host__ __device__ inline Plan make_stream_plan(int d_model, int d_ff) {
     p.stage_bytes = align_i(p.part + kPartBytes, 1024);
     p.L1 = make_layout(d_ff, d_model);
     p.L2 = make_layout(d_model, d_ff);
+    p.dt1 = make_div(uint32_t(p.tiles1));
+    p.dt2 = make_div(uint32_t(p.tiles2));
+    p.dpp1 = make_div(uint32_t(p.pp1));
+    p.dpp2 = make_div(uint32_t(p.pp2));
     return p;
 }
 
@@ -176,9 +194,11 @@ struct Ctl {
     int slot_claim[2];     // (group << 16) | activation pieces claimed for that group
     int slot_done[2];      // and finished
     int n_valid, n_seg, bad;
+    int nmax;                    // most pairs in one segment (sizes the slots)
     int u1b, u1e, u2b, u2e;      // this CTA's unit ranges (global unit indices)
     int s1b, s2b, nl1, nl, ngrp; // first segment of each range, local segments of phase 1, in all; groups
     int stages, slot_bytes, ring;
+    FastDiv dst;                 // division by stages
     int issued;                  // units whose copies the producer issued
     uint64_t wait_ns;            // bound of every wait
     int grp_of[kMaxLocalSeg];    // group of each local segment
@@ -212,13 +232,6 @@ __device__ __forceinline__ int ld_acquire(const int32_t* p) {
 }
 
 __device__ __forceinline__ int vload(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
-
-// Signed bit field of `len` bits at `pos`.
-__device__ __forceinline__ int bfe_s32(uint32_t v, uint32_t pos, uint32_t len) {
-    int r;
-    asm("bfe.s32 %0, %1, %2, %3;" : "=r"(r) : "r"(v), "r"(pos), "r"(len));
-    return r;
-}
 
 // Bounded waits that leave the issue slots to the warps doing work: a
 // shared-memory counter of this CTA or a global counter of other CTAs is
@@ -297,6 +310,7 @@ __device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, Route
         c.slot_claim[0] = 0 << 16;
         c.slot_claim[1] = 1 << 16;
         c.slot_done[0] = c.slot_done[1] = 0;
+        c.nmax = 1;
         fence_mbar_init();
     }
     if (BK <= 32) {
@@ -336,10 +350,13 @@ __device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, Route
             const int rend = later ? __ffs(later) - 1 : nv;
             const bool start = lane < nv && ((lane - rstart) % kSegTok) == 0;
             const unsigned sgb = __ballot_sync(0xffffffffu, start);
-            if (start) c.seg[__popc(sgb & (le >> 1))] = (se << 12) | (lane << 3) | min(kSegTok, rend - lane);
+            const int sn = start ? min(kSegTok, rend - lane) : 0;
+            if (start) c.seg[__popc(sgb & (le >> 1))] = (se << 12) | (lane << 3) | sn;
+            const int nmax = __reduce_max_sync(0xffffffffu, sn);
             if (lane == 0) {
                 c.n_valid = nv;
                 c.n_seg = __popc(sgb);
+                c.nmax = nmax > 1 ? nmax : 1;
             }
         }
     } else {
@@ -392,6 +409,7 @@ __device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, Route
         if (lane == 0) c.wsum[warp] = __popc(sb);
         __syncthreads();
         if (start) {
+            if ((packed & 7) > 1) atomicMax(&c.nmax, packed & 7);
             int sid = __popc(sb & ((1u << lane) - 1u));
 #pragma unroll 1
             for (int w = 0; w < warp; ++w) sid += c.wsum[w];
@@ -445,12 +463,16 @@ __device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, Route
             c.grp_left[g] += hi - lo;
         }
         c.ngrp = g + 1;
-        // a slot holds kSegTok tokens of either phase
-        c.slot_bytes = kSegTok * (P.t1.bytes > P.t2.bytes ? P.t1.bytes : P.t2.bytes);
+        // a slot holds the tokens of the largest segment, of either phase
+        c.slot_bytes = c.nmax * (P.t1.bytes > P.t2.bytes ? P.t1.bytes : P.t2.bytes);
         c.ring = align_i(align_i(int(sizeof(Ctl)), 1024) + 2 * c.slot_bytes, 1024);
         const int st = (kSmemBytes - 1024 - c.ring) / P.stage_bytes;
         c.stages = st > kMaxStages ? kMaxStages : st;
-        if (c.stages < 2) c.abort = 1;
+        if (c.stages < 2) {
+            c.abort = 1;
+            c.stages = 2;
+        }
+        c.dst = make_div(uint32_t(c.stages));
         if (blockIdx.x == 0 && c.bad) set_status(A.ws.status, GALE_ERR_ARG);
         if (blockIdx.x == 0 && c.abort) set_status(A.ws.status, GALE_ERR_UNSUPPORTED);
     }
@@ -466,8 +488,9 @@ __device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, Route
 // so that lane l = q + 8 tig holds, in registers 4 bb .. 4 bb + 3, the four
 // elements 128 bb + 32 tig + 8 i + q (i = 0..3): byte i of digit word
 // (bb, tig, q).  Digit storage per 128-column block b:
-// [digit j (3)][tig (4)][32 bytes], register q of lane-quad tig at bytes
-// 4q..4q+3, which is the B fragment of the MMAs of bit positions q.
+// [digit j (3: bits 16..23, 8..15, 0..7 of Y)][tig (4)][32 bytes], register q
+// of lane-quad tig at bytes 4q..4q+3, which is the B fragment of the MMAs of
+// bit positions q.
 __device__ __forceinline__ int elem_of(int lane, int r) {
     return (lane & 7) + 8 * (r & 3) + 32 * (lane >> 3) + 128 * (r >> 2);
 }
@@ -478,19 +501,6 @@ __device__ __forceinline__ float fixed_scale_of(float m) {
     int e;
     frexpf(1048576.0f / m, &e);
     return ldexpf(1.0f, e - 1);
-}
-
-// round(u) (|u| < 2^22) and its three int8 digits.
-__device__ __forceinline__ int round_digits(float u, uint32_t& d1, uint32_t& d2, uint32_t& d3) {
-    const int X = __float_as_int(__fadd_rn(u, 12582912.0f)) - 0x4B400000;
-    const int p1 = (X + 8192) >> 14;
-    const int r = X - (p1 << 14);
-    const int p2 = (r + 64) >> 7;
-    const int p3 = r - (p2 << 7);
-    d1 = uint32_t(p1) & 0xFFu;
-    d2 = uint32_t(p2) & 0xFFu;
-    d3 = uint32_t(p3) & 0xFFu;
-    return X;
 }
 
 // One 1024-block `blk` of a token's activation (bf16 x, or fp32 h) into the
@@ -540,28 +550,24 @@ __device__ __noinline__ void build_block(const void* src, int bf16, int blk, uin
     const int q = lane & 7, tig = lane >> 3;
     const float sc = S * (q < 7 ? __int_as_float((127 - q) << 23) : -0.0078125f);   // S / a(q)
     const int aq = a_of(q);
-    uint32_t a = dst + (blk * 8) * 384 + tig * 32 + q * 4;
+    const uint32_t a = dst + (blk * 8) * 384 + tig * 32 + q * 4;
     const uint32_t xs_a = dst + tm.xsum + 4 * (blk * 8);
-#pragma unroll 1
-    for (int bb = 0; bb < 8; ++bb) {
-        uint32_t w0 = 0u, w1 = 0u, w2 = 0u;
-        int xs = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t d1, d2, d3;
-            xs += round_digits(v[i] * sc, d1, d2, d3);
-            w0 |= d1 << (8 * i);
-            w1 |= d2 << (8 * i);
-            w2 |= d3 << (8 * i);
-        }
-        sts_u32(a, w0);
-        sts_u32(a + 128, w1);
-        sts_u32(a + 256, w2);
-        a += 384;
+    for (int bb = 0; bb < 8; ++bb) {
+        // fmaf(v, S / a, 2^23 + 2^20) rounds v S / a to an integer X (|X| <= 2^20)
+        // and leaves Y = X + 2^20 in the low 24 bits: its bytes are the digits
+        uint32_t y[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) y[i] = __float_as_uint(fmaf(v[4 * bb + i], sc, 9437184.0f));
+        const uint32_t lo01 = __byte_perm(y[0], y[1], 0x5140), lo23 = __byte_perm(y[2], y[3], 0x5140);
+        const uint32_t hi01 = __byte_perm(y[0], y[1], 0x0062), hi23 = __byte_perm(y[2], y[3], 0x0062);
+        sts_u32(a + bb * 384, __byte_perm(hi01, hi23, 0x5410));         // bits 16..23
+        sts_u32(a + bb * 384 + 128, __byte_perm(lo01, lo23, 0x7632));   // bits 8..15
+        sts_u32(a + bb * 384 + 256, __byte_perm(lo01, lo23, 0x5410));   // bits 0..7
+        // sum of the four X (each float word is 0x4B100000 + X)
+        const int xs = int(y[0] + y[1] + y[2] + y[3] - 0x2C400000u);
         const int tot = __reduce_add_sync(0xffffffffu, xs * aq);
         if (lane == 0) sts_u32(xs_a + 4 * bb, uint32_t(tot));
-#pragma unroll
-        for (int i = 0; i < 28; ++i) v[i] = v[i + 4];
     }
     // x_rot = u / 32 = X a / (32 S); the fp16 copy times 2 / S
     if (lane == 0) {
@@ -579,110 +585,106 @@ __device__ __noinline__ void build_block(const void* src, int bf16, int blk, uin
 // row pitch sbp bytes) times the 1024-column chunk c of up to two tokens.
 // Writes  sigma_c (sum_{b in c} s_blk (X_b - 2 P_b))  of row r of tile m,
 // token t to part[(pr_m + r) * 2 + t].
+//
+// MMA column n = 4 t + j of token t: j = 0 the digit of bits 16..23 of
+// Y = X + 2^20, j = 1 a column of ones, j = 2 and 3 the digits of bits 8..15
+// and 0..7.  Per block a lane combines its two columns exactly in int32:
+// lanes of even tig  D16 - 16 ONES  (the 2^20 offset times ONES, over 2^16),
+// lanes of odd tig   256 D8 + D0,  so that P_b = 2^16 (even) + (odd).
+// The eight blocks are unrolled; the sixteen block scales a lane needs (its
+// two rows of each tile) come in four 16-byte loads before the loop.
 __device__ __noinline__ void mma_piece(uint32_t sg0, uint32_t sg1, uint32_t sb0, uint32_t sb1, int sbp, int c,
                                        uint32_t slot, int tstride, TokMap tm, int ntok, uint32_t part, int pr0,
                                        int pr1) {
     const uint32_t sg[2] = {sg0, sg1}, sb[2] = {sb0, sb1};
     const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
-    // B fragment of this lane: MMA column g = (token g / 3, digit g % 3), columns 6 and 7 unused
-    const bool bl = g < 3 || (g < 6 && ntok > 1);
-    const uint32_t bsrc = slot + (g >= 3 ? tstride : 0) + (g % 3) * 128 + tig * 32;
-    float acc[2][4];
-#pragma unroll
-    for (int m = 0; m < 2; ++m)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
-    const uint32_t woff = g * 128 + tig * 4;
-    // sign words and block scales of the next block are loaded one block ahead
-    uint32_t nw[2][2];
-    float ns[2][2];
+    const int j = g & 3;
+    const bool ones = j == 1;
+    const bool bl = !ones && (g < 4 || ntok > 1);
+    const uint32_t bsrc = slot + (g >> 2) * tstride + (j == 0 ? 0 : j - 1) * 128 + tig * 32 + c * 8 * 384;
+    const uint32_t bfill = ones ? 0x01010101u : 0u;
+    const int mA = (tig & 1) ? 256 : 1, mB = (tig & 1) ? 1 : -16;
+    uint4 sv[2][2];   // [tile][row g, row g + 8]: the chunk's eight fp16 block scales
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-        nw[m][0] = lds_u32(sg[m] + woff + (g << 4));
-        nw[m][1] = lds_u32(sg[m] + woff + (g << 4) + 1024);
-        ns[m][0] = h2f(lds_u16(sb[m] + g * sbp + 16 * c));
-        ns[m][1] = h2f(lds_u16(sb[m] + (g + 8) * sbp + 16 * c));
+        sv[m][0] = lds_v4(sb[m] + g * sbp + 16 * c);
+        sv[m][1] = lds_v4(sb[m] + (g + 8) * sbp + 16 * c);
     }
+    float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    const uint32_t woff = g * 128 + tig * 4;
+    // two blocks per iteration (the scale pair of both is one 32-bit word of
+    // sv, which moves down by one component per iteration)
 #pragma unroll 1
-    for (int bb = 0; bb < 8; ++bb) {
-        const int b = c * 8 + bb;
-        uint4 q0 = make_uint4(0u, 0u, 0u, 0u), q1 = make_uint4(0u, 0u, 0u, 0u);
-        if (bl) {
-            q0 = lds_v4(bsrc + b * 384);
-            q1 = lds_v4(bsrc + b * 384 + 16);
-        }
-        uint32_t w[2][2];
-        float sc[2][2];
+    for (int bp = 0; bp < 4; ++bp) {
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            w[m][0] = nw[m][0];
-            w[m][1] = nw[m][1];
-            sc[m][0] = ns[m][0];
-            sc[m][1] = ns[m][1];
-        }
-        if (bb < 7) {
-            const uint32_t wo = woff + (((bb + 1) ^ g) << 4);
+        for (int h = 0; h < 2; ++h) {
+            const int bb = 2 * bp + h;
+            uint4 q0 = make_uint4(bfill, bfill, bfill, bfill), q1 = q0;
+            if (bl) {
+                q0 = lds_v4(bsrc + bb * 384);
+                q1 = lds_v4(bsrc + bb * 384 + 16);
+            }
+            const uint32_t wo = woff + ((bb ^ g) << 4);
+            uint32_t w[2][2];
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
-                nw[m][0] = lds_u32(sg[m] + wo);
-                nw[m][1] = lds_u32(sg[m] + wo + 1024);
-                ns[m][0] = h2f(lds_u16(sb[m] + g * sbp + 2 * (b + 1)));
-                ns[m][1] = h2f(lds_u16(sb[m] + (g + 8) * sbp + 2 * (b + 1)));
+                w[m][0] = lds_u32(sg[m] + wo);
+                w[m][1] = lds_u32(sg[m] + wo + 1024);
+            }
+            const uint32_t breg[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                // bit positions 0..3 and 4..7 as two independent MMA chains
+                int ca[4] = {0, 0, 0, 0}, cb[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int mm = 0; mm < 2; ++mm) {
+                    const uint32_t m0 = 0x01010101u << (2 * mm), m1 = m0 << 1;
+                    const uint32_t n0 = m0 << 4, n1 = m1 << 4;
+                    mma_s8u8(ca, w[m][0] & m0, w[m][1] & m0, w[m][0] & m1, w[m][1] & m1, breg[2 * mm],
+                             breg[2 * mm + 1]);
+                    mma_s8u8(cb, w[m][0] & n0, w[m][1] & n0, w[m][0] & n1, w[m][1] & n1, breg[2 * mm + 4],
+                             breg[2 * mm + 5]);
+                }
+                const float s0 = h2f(h ? sv[m][0].x >> 16 : sv[m][0].x);
+                const float s1 = h2f(h ? sv[m][1].x >> 16 : sv[m][1].x);
+                acc[m][0] = fmaf(s0, float((ca[0] + cb[0]) * mA + (ca[1] + cb[1]) * mB), acc[m][0]);
+                acc[m][1] = fmaf(s1, float((ca[2] + cb[2]) * mA + (ca[3] + cb[3]) * mB), acc[m][1]);
             }
         }
-        const uint32_t breg[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            int cc[4] = {0, 0, 0, 0};
+        for (int m = 0; m < 2; ++m)
 #pragma unroll
-            for (int mm = 0; mm < 4; ++mm) {
-                const uint32_t m0 = 0x01010101u << (2 * mm), m1 = m0 << 1;
-                mma_s8(cc, w[m][0] & m0, w[m][1] & m0, w[m][0] & m1, w[m][1] & m1, breg[2 * mm], breg[2 * mm + 1]);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[m][i] = fmaf(sc[m][i >> 1], float(cc[i]), acc[m][i]);
-        }
+            for (int r = 0; r < 2; ++r) sv[m][r] = make_uint4(sv[m][r].y, sv[m][r].z, sv[m][r].w, sv[m][r].x);
     }
-    // P of (row, token) from the three digit columns of the token, summed over
-    // the lane quad; lane (g, tig) then owns row g + 8 (tig >> 1), token tig & 1.
-    const int orow = g + 8 * (tig >> 1), tok = tig & 1;
+    // P of rows g and g + 8 from the lane pair (tig even: high part, odd: low
+    // part); the even lane then owns row g, the odd lane row g + 8, of token
+    // tig >> 1.
+    const int odd = tig & 1, tok = tig >> 1;
+    const int orow = g + 8 * odd;
     const uint32_t tb = slot + tok * tstride;
+    const uint4 x0 = lds_v4(tb + tm.xsum + 32 * c), x1 = lds_v4(tb + tm.xsum + 32 * c + 16);
+    const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    const float sig = lds_f32(tb + tm.sig + 4 * c);
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-        float p[4];   // (row g, tok 0), (row g, tok 1), (row g+8, tok 0), (row g+8, tok 1)
-#pragma unroll
-        for (int rh = 0; rh < 2; ++rh) {
-            const float a = acc[m][2 * rh], b2 = acc[m][2 * rh + 1];
-            p[2 * rh] = tig == 0 ? fmaf(16384.0f, a, 128.0f * b2) : (tig == 1 ? a : 0.f);
-            p[2 * rh + 1] = tig == 1 ? 16384.0f * b2 : (tig == 2 ? fmaf(128.0f, a, b2) : 0.f);
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            p[i] += __shfl_xor_sync(0xffffffffu, p[i], 1);
-            p[i] += __shfl_xor_sync(0xffffffffu, p[i], 2);
-        }
-        const float P = tig == 0 ? p[0] : tig == 1 ? p[1] : tig == 2 ? p[2] : p[3];
+        const float o0 = __shfl_xor_sync(0xffffffffu, acc[m][0], 1);
+        const float o1 = __shfl_xor_sync(0xffffffffu, acc[m][1], 1);
+        const float P = odd ? fmaf(65536.0f, o1, acc[m][1]) : fmaf(65536.0f, acc[m][0], o0);
         if (tok < ntok) {
-            const uint4 sv = lds_v4(sb[m] + orow * sbp + 16 * c);
-            const uint4 x0 = lds_v4(tb + tm.xsum + 32 * c), x1 = lds_v4(tb + tm.xsum + 32 * c + 16);
-            const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
-            const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            const uint4 sc = odd ? sv[m][1] : sv[m][0];
+            const uint32_t sw[4] = {sc.x, sc.y, sc.z, sc.w};
             float xt = 0.f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 xt = fmaf(h2f(sw[i] & 0xFFFFu), float(int(xw[2 * i])), xt);
                 xt = fmaf(h2f(sw[i] >> 16), float(int(xw[2 * i + 1])), xt);
             }
-            const float sig = lds_f32(tb + tm.sig + 4 * c);
             sts_f32(part + (((m ? pr1 : pr0) + orow) * 2 + tok) * 4, sig * fmaf(-2.0f, P, xt));
         }
     }
 }
 
-// Outlier corrections of one row over outliers j0 <= j < j1:
-//   sum_j (q_j s_row - sign_j s_blk) x_{c_j}
-// for up to two tokens (the MMA part counted the sign weight at c_j); written
-// to out (two floats).
+// Where one row's outlier records, sign line and block scales sit in a stage.
 struct RowRef {
     uint32_t idx;       // outlier columns of the row (uint16)
     uint32_t qb;        // byte holding nibble 0 of the values counted from n0
@@ -694,25 +696,51 @@ struct RowRef {
     float srow;
 };
 
+// One outlier of the row: the value nibble q (offset binary q + 8 in `nib`)
+// and column `col` (col >= C: a record that failed validation, counted as 0).
+__device__ __forceinline__ void outlier_one(const RowRef& R, uint32_t col, uint32_t nib, int C, uint32_t x0,
+                                            uint32_t f0, int tstride, int ntok, float& corr0, float& corr1) {
+    const bool ok = col < uint32_t(C);
+    const uint32_t cc = ok ? col : 0u;
+    // value: float(q) through the exponent field of 2^23 (exact for small integers)
+    const float q = __uint_as_float(nib ^ 0x4B000008u) - 8388616.0f;
+    // the sign word holding column cc (swizzled 16-byte chunk of the row's line)
+    const uint32_t word = lds_u32(R.sign + (cc >> 10) * uint32_t(R.chunk_stride) +
+                                  (((cc >> 3) & 0x7Cu) ^ (uint32_t(R.sw) << 4)));
+    const uint32_t sbits = lds_u16(R.sblk + ((cc >> 6) & ~1u));
+    // - sign s_blk: +s_blk where the bit is 1 (weight -1), -s_blk where it is 0
+    const float nsb = __uint_as_float(__float_as_uint(h2f(sbits)) ^ ((~__funnelshift_r(word, word, cc)) << 31));
+    const float wq = ok ? fmaf(q, R.srow, nsb) : 0.f;
+    const uint32_t fo = 4u * (cc >> 10);
+    corr0 = fmaf(wq * lds_f32(f0 + fo), h2f(lds_u16(x0 + 2u * cc)), corr0);
+    if (ntok > 1)
+        corr1 = fmaf(wq * lds_f32(f0 + uint32_t(tstride) + fo), h2f(lds_u16(x0 + uint32_t(tstride) + 2u * cc)), corr1);
+}
+
+// Outlier corrections of one row over outliers j0 <= j < j1:
+//   sum_j (q_j s_row - sign_j s_blk) x_{c_j}
+// for up to two tokens (the MMA part counted the sign weight at c_j); written
+// to out (two floats).  Values are read a byte (two nibbles) at a time.
 __device__ __noinline__ void outlier_row(const RowRef R, int j0, int j1, int C, uint32_t slot, int tstride,
                                          TokMap tm, int ntok, uint32_t out) {
     float corr0 = 0.f, corr1 = 0.f;
-    const uint32_t x0 = slot + tm.x16, x1 = slot + tstride + tm.x16;
-    const uint32_t f0 = slot + tm.f16, f1 = slot + tstride + tm.f16;
-#pragma unroll 2
-    for (int j = j0; j < j1; ++j) {
-        const int col = int(lds_u16(R.idx + 2 * j));
-        if (col >= C) continue;   // only records that failed validation
-        const int n = R.n0 + j;
-        const int qv = bfe_s32(lds_u8(R.qb + (n >> 1)), (n & 1) * 4, 4);
-        const uint32_t word = lds_u32(R.sign + (col >> 10) * R.chunk_stride + ((((col >> 7) & 7) ^ R.sw) << 4) +
-                                      ((col >> 3) & 12));
-        const float sb = h2f(lds_u16(R.sblk + 2 * (col >> 7)));
-        const float wq = fmaf(float(qv), R.srow, ((word >> (col & 31)) & 1u) ? sb : -sb);
-        const int ch4 = 4 * (col >> 10);
-        corr0 = fmaf(wq * lds_f32(f0 + ch4), h2f(lds_u16(x0 + 2 * col)), corr0);
-        if (ntok > 1) corr1 = fmaf(wq * lds_f32(f1 + ch4), h2f(lds_u16(x1 + 2 * col)), corr1);
+    const uint32_t x0 = slot + tm.x16, f0 = slot + tm.f16;
+    int j = j0;
+    int n = R.n0 + j0;   // nibble index of outlier j, counted from byte qb
+    if (j < j1 && (n & 1)) {
+        outlier_one(R, lds_u16(R.idx + 2 * j), lds_u8(R.qb + (n >> 1)) >> 4, C, x0, f0, tstride, ntok, corr0, corr1);
+        ++j;
+        ++n;
     }
+#pragma unroll 2
+    for (; j + 1 < j1; j += 2, n += 2) {
+        const uint32_t qb = lds_u8(R.qb + (n >> 1));
+        const uint32_t c0 = lds_u16(R.idx + 2 * j), c1 = lds_u16(R.idx + 2 * j + 2);
+        outlier_one(R, c0, qb & 0xFu, C, x0, f0, tstride, ntok, corr0, corr1);
+        outlier_one(R, c1, qb >> 4, C, x0, f0, tstride, ntok, corr0, corr1);
+    }
+    if (j < j1)
+        outlier_one(R, lds_u16(R.idx + 2 * j), lds_u8(R.qb + (n >> 1)) & 0xFu, C, x0, f0, tstride, ntok, corr0, corr1);
     sts_f32(out, corr0);
     sts_f32(out + 4, corr1);
 }
@@ -728,7 +756,6 @@ __device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f 
 __device__ __noinline__ void normalize_token(const StreamArgs& A, int t) {
     const int lane = threadIdx.x & 31;
     const int d = A.d_model, nb = d / 64;
-    __threadfence();
     float ss = 0.f;
 #pragma unroll 1
     for (int i = lane; i < nb; i += 32) ss += __ldcg(A.ws.ssq + t * nb + i);
@@ -751,7 +778,6 @@ __device__ __noinline__ void normalize_token(const StreamArgs& A, int t) {
 __device__ __noinline__ void combine_block(const StreamArgs& A, const Ctl& c, int t, int tile) {
     const int lane = threadIdx.x & 31;
     const int d = A.d_model, K = A.K, nb = d / 64;
-    __threadfence();
     const uint32_t vm = c.vmask[t];
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll 1
@@ -791,11 +817,11 @@ __device__ __noinline__ void combine_block(const StreamArgs& A, const Ctl& c, in
     if (lane == 0) A.ws.ssq[t * nb + tile] = ss;
     __syncwarp();
     int last = 0;
-    if (lane == 0) {
-        __threadfence();
-        last = atomicAdd(A.ws.tokcnt + t, 1) == nb - 1;
+    if (lane == 0) last = atom_acq_rel_add(A.ws.tokcnt + t, 1) == nb - 1;
+    if (__shfl_sync(0xffffffffu, last, 0)) {
+        __syncwarp();
+        normalize_token(A, t);
     }
-    if (__shfl_sync(0xffffffffu, last, 0)) normalize_token(A, t);
 }
 
 // Tokens with no valid pair: y = 0 (out = 0, or the norm of x alone).
@@ -832,12 +858,12 @@ __device__ __forceinline__ UnitRef unit_ref(const Ctl& c, const Plan& P, int u) 
     r.p1 = u < n1;
     if (r.p1) {
         r.U = c.u1b + u;
-        r.s = r.U / P.tiles1;
+        r.s = fdiv(r.U, P.dt1);
         r.tile = r.U - r.s * P.tiles1;
         r.q = r.s - c.s1b;
     } else {
         r.U = c.u2b + (u - n1);
-        r.s = r.U / P.tiles2;
+        r.s = fdiv(r.U, P.dt2);
         r.tile = r.U - r.s * P.tiles2;
         r.q = c.nl1 + r.s - c.s2b;
     }
@@ -845,8 +871,9 @@ __device__ __forceinline__ UnitRef unit_ref(const Ctl& c, const Plan& P, int u) 
     r.e = seg_e(sg);
     r.n = seg_n(sg);
     r.first = seg_first(sg);
-    r.st = u % c.stages;
-    r.par = (u / c.stages) & 1;
+    const int lap = fdiv(u, c.dst);
+    r.st = u - lap * c.stages;
+    r.par = lap & 1;
     return r;
 }
 
@@ -868,6 +895,7 @@ __device__ __noinline__ void act_piece(const StreamArgs& A, const Plan& P, Ctl& 
         int v = 1;
         if (lane == 0) v = wait_global(A.ws.hcnt + s * P.nch2 + blk, 1024 / kR1, &c.abort, c.wait_ns);
         v = __shfl_sync(0xffffffffu, v, 0);
+        __syncwarp();
         if (!v) {
             set_status(A.ws.status, GALE_ERR_TIMEOUT);
             atomicExch(&c.abort, 1);
@@ -882,7 +910,7 @@ __device__ __forceinline__ bool act_ready(const StreamArgs& A, const Plan& P, co
     const int q = c.grp_seg[g];
     if (q < c.nl1) return true;
     const int s = c.s2b + (q - c.nl1);
-    return ld_acquire(A.ws.hcnt + s * P.nch2 + cl % P.nch2) >= 1024 / kR1;
+    return vload(A.ws.hcnt + s * P.nch2 + cl % P.nch2) >= 1024 / kR1;
 }
 
 __device__ __forceinline__ int grp_need(const Ctl& c, const Plan& P, int g) {
@@ -967,8 +995,10 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
             pc = __shfl_sync(0xffffffffu, pc, 0);
             if (pc >= tot_pieces || vload(&c.abort)) break;
             const bool p1 = pc < n1 * P.pp1;
-            const int u = p1 ? pc / P.pp1 : n1 + (pc - n1 * P.pp1) / P.pp2;
-            const int sub = p1 ? pc - (pc / P.pp1) * P.pp1 : (pc - n1 * P.pp1) % P.pp2;
+            const int pr = p1 ? pc : pc - n1 * P.pp1;
+            const int ur = fdiv(pr, p1 ? P.dpp1 : P.dpp2);
+            const int u = p1 ? ur : n1 + ur;
+            const int sub = pr - ur * (p1 ? P.pp1 : P.pp2);
             const UnitRef R = unit_ref(c, P, u);
             // ---- the activations of the unit's group, in slot g & 1 ----
             const int g = c.grp_of[R.q];
@@ -977,7 +1007,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
             const int tstride = R.p1 ? P.t1.bytes : P.t2.bytes;
             const uint32_t slot = slot_base + uint32_t(sl * c.slot_bytes);
             {
-                bool ok = wait_smem(&c.slot_grp[sl], g, true, &c.abort, c.wait_ns);
+                bool ok = vload(&c.slot_grp[sl]) == g || wait_smem(&c.slot_grp[sl], g, true, &c.abort, c.wait_ns);
 #pragma unroll 1
                 while (ok && vload(&c.slot_done[sl]) < need) {
                     // the slot cannot move on while this unit is unfinished,
@@ -1057,56 +1087,42 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
                     outlier_row(RR, 0, P.k2, P.C2, slot, tstride, P.t2, R.n, part + uint32_t((nch * 64 + r) * 8));
                 }
             }
-            // ---- the last piece of the unit finishes it ----
+            // ---- the last piece of the unit finishes it: the partial sums
+            //      go to registers, the stage goes back to the producer, then
+            //      the rows are written and published ----
             __syncwarp();
             __threadfence_block();
             int last = 0;
             if (lane == 0) last = atomicAdd(&c.stage_done[R.st], 1) == (R.p1 ? P.pp1 : P.pp2) - 1;
             if (__shfl_sync(0xffffffffu, last, 0)) {
                 __threadfence_block();
+                constexpr int kY = kSegTok * kR2 / 32;
+                float hv = 0.f, yv[kY];
                 if (R.p1) {
-                    // h rows: silu(w1 x) * (w3 x); slices 0..nch-1 (chunks), nch, nch+1 (outliers)
-                    const int nsl = P.nch1 + 2;
-#pragma unroll 1
-                    for (int i = lane; i < kR1 * R.n; i += 32) {
-                        const int r = i & 15, t = i >> 4;
+                    // h row lane & 15 of token lane >> 4: silu(w1 x) * (w3 x) over
+                    // slices 0..nch-1 (chunks), nch, nch+1 (outliers)
+                    if (lane < kR1 * R.n) {
+                        const int r = lane & 15, t = lane >> 4;
                         float g1 = 0.f, g3 = 0.f;
 #pragma unroll 1
-                        for (int s2 = 0; s2 < nsl; ++s2) {
+                        for (int s2 = 0; s2 < P.nch1 + 2; ++s2) {
                             g1 += lds_f32(part + uint32_t(((s2 * 32 + r) * 2 + t) * 4));
                             g3 += lds_f32(part + uint32_t(((s2 * 32 + 16 + r) * 2 + t) * 4));
                         }
-                        const int pair = c.sorted[R.first + t];
-                        A.ws.h[pair * A.d_ff + R.tile * kR1 + r] = silu_fast(g1) * g3;
-                    }
-                    __syncwarp();
-                    if (lane == 0 && int(blockIdx.x) != A.withhold_cta) {
-                        __threadfence();
-                        atomicAdd(A.ws.hcnt + R.s * nhb + (R.tile * kR1) / 1024, 1);
+                        hv = silu_fast(g1) * g3;
                     }
                 } else {
-                    // o rows; slices 0..nch-1 (chunks), nch (outliers)
-                    const int nsl = P.nch2 + 1;
-#pragma unroll 1
-                    for (int i = lane; i < kR2 * R.n; i += 32) {
-                        const int r = i & 63, t = i >> 6;
+                    // o rows over slices 0..nch-1 (chunks), nch (outliers)
+#pragma unroll
+                    for (int i = 0; i < kY; ++i) {
+                        const int it = lane + 32 * i, r = it & 63, t = it >> 6;
                         float y = 0.f;
+                        if (it < kR2 * R.n) {
 #pragma unroll 1
-                        for (int s2 = 0; s2 < nsl; ++s2) y += lds_f32(part + uint32_t(((s2 * 64 + r) * 2 + t) * 4));
-                        const int pair = c.sorted[R.first + t];
-                        A.ws.o[pair * A.d_model + R.tile * kR2 + r] = y;
-                    }
-                    __syncwarp();
-                    if (lane == 0) __threadfence();
-                    __syncwarp();
-                    const int nb = A.d_model / 64;
-#pragma unroll 1
-                    for (int t = 0; t < R.n; ++t) {
-                        const int tk = c.sorted[R.first + t] / A.K;
-                        int lastc = 0;
-                        if (lane == 0)
-                            lastc = atomicAdd(A.ws.comb + tk * nb + R.tile, 1) == __popc(c.vmask[tk]) - 1;
-                        if (__shfl_sync(0xffffffffu, lastc, 0)) combine_block(A, c, tk, R.tile);
+                            for (int s2 = 0; s2 < P.nch2 + 1; ++s2)
+                                y += lds_f32(part + uint32_t(((s2 * 64 + r) * 2 + t) * 4));
+                        }
+                        yv[i] = y;
                     }
                 }
                 // release the stage and count the unit into its group
@@ -1122,11 +1138,45 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
                         atomicExch(&c.slot_grp[sl], g + 2);
                     }
                 }
+                if (R.p1) {
+                    if (lane < kR1 * R.n) {
+                        const int pair = c.sorted[R.first + (lane >> 4)];
+                        A.ws.h[pair * A.d_ff + R.tile * kR1 + (lane & 15)] = hv;
+                    }
+                    __syncwarp();
+                    if (lane == 0 && int(blockIdx.x) != A.withhold_cta)
+                        red_release_add(A.ws.hcnt + R.s * nhb + (R.tile * kR1) / 1024, 1);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kY; ++i) {
+                        const int it = lane + 32 * i;
+                        if (it < kR2 * R.n) {
+                            const int pair = c.sorted[R.first + (it >> 6)];
+                            A.ws.o[pair * A.d_model + R.tile * kR2 + (it & 63)] = yv[i];
+                        }
+                    }
+                    __syncwarp();
+                    const int nb = A.d_model / 64;
+#pragma unroll 1
+                    for (int t = 0; t < R.n; ++t) {
+                        const int tk = c.sorted[R.first + t] / A.K;
+                        int lastc = 0;
+                        if (lane == 0)
+                            lastc = atom_acq_rel_add(A.ws.comb + tk * nb + R.tile, 1) == __popc(c.vmask[tk]) - 1;
+                        if (__shfl_sync(0xffffffffu, lastc, 0)) {
+                            __syncwarp();
+                            combine_block(A, c, tk, R.tile);
+                        }
+                    }
+                }
             }
             // ---- work ahead: one activation piece of the next group, if its
             //      slot is free and (phase 2) its h block is complete ----
+            // (a phase-2 group only once this CTA's phase-1 pieces are nearly
+            // all taken: its readiness test reads a global counter)
             const int gn = g + 1;
-            if (gn < c.ngrp && vload(&c.slot_grp[gn & 1]) == gn) {
+            if (gn < c.ngrp && (!R.p1 || c.grp_seg[gn] < c.nl1 || pc + 2 * kCW >= n1 * P.pp1) &&
+                vload(&c.slot_grp[gn & 1]) == gn) {
                 const int sln = gn & 1;
                 const int needn = grp_need(c, P, gn);
                 // claim only if the claim word still belongs to group gn: a
