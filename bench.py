@@ -36,6 +36,8 @@ UNIT = "tokens/s"
 D_MODEL, D_FF, N_EXPERTS, TOP_K = 4096, 2048, 256, 6
 PREFILL_B = 4096
 CHAIN_LAYERS = 43
+# rows of the 4-bit non-expert GEMV line (x d_model columns: 138 MB of 4-bit weights)
+W4_ROWS = 65536
 # kernels of this library launched per decode step (the cooperative layer kernel)
 DECODE_LAUNCHES = 1
 # dram read + write bytes of one decode launch at this workload, from an ncu
@@ -317,6 +319,38 @@ def run_gpu(args):
         torch.cuda.synchronize()
         return sum(a.elapsed_time(b) * 1e-3 for a, b in ev)
 
+    def measure_w4(steps, warmup, B):
+        """The 4-bit non-expert weight GEMV (symmetric int4, 128-block fp16
+        scales): one [W4_ROWS x D_MODEL] matrix quantized on the device from
+        seeded N(0, 0.02) weights, B bf16 tokens, L2 flushed before every
+        step (outside the events).  Returns (seconds, bytes per step)."""
+        L = G.gale_w4_layout(W4_ROWS, D_MODEL)
+        packed = torch.empty(L.total, dtype=torch.uint8, device="cuda")
+        key = gs.stream_key(73, 0)
+        w = torch.empty(W4_ROWS, D_MODEL, dtype=torch.float32, device="cuda")
+        rows_per = 4096
+        for r0 in range(0, W4_ROWS, rows_per):   # drawn in slices of rows
+            w[r0:r0 + rows_per] = (gs.normal_torch(key, rows_per * D_MODEL, start=r0 * D_MODEL) * 0.02).view(
+                rows_per, D_MODEL)
+        G.gale_w4_quantize(w, packed)
+        del w
+        xs = [torch.from_numpy(gs.hidden_bf16(B, D_MODEL, tag=97_000 + i)[0]).view(torch.int16).cuda()
+              for i in range(steps + warmup)]
+        y = torch.empty(B, W4_ROWS, dtype=torch.float32, device="cuda")
+        ws = torch.empty(G.gale_w4_workspace_size(W4_ROWS, D_MODEL, B), dtype=torch.uint8, device="cuda")
+        for i in range(warmup):
+            G.gale_w4_gemv(packed, W4_ROWS, D_MODEL, xs[i], y, ws)
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            G.gale_w4_gemv(packed, W4_ROWS, D_MODEL, xs[warmup + i], y, ws)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        t = sum(a.elapsed_time(b) * 1e-3 for a, b in ev)
+        return t, L.total + B * D_MODEL * 2 + B * W4_ROWS * 4
+
     def measure_chain(steps, warmup, n_layers=CHAIN_LAYERS):
         """Decode batch 1 through n_layers layers of 256 resident experts each:
         x_{l+1} = bf16(RMSNorm(x_l + MoE_l(x_l))), fresh seeded routing per
@@ -393,6 +427,8 @@ def run_gpu(args):
     t64, bytes64, _ = measure(64, max(args.steps // 2, 3), args.warmup, 25_000, bias_sigma=0.5)
     te, h2d, d2h = measure_e2e(1, args.steps, args.warmup, 30_000)
     ts = measure_single(args.steps, args.warmup)
+    tw1, w4b1 = measure_w4(args.steps, args.warmup, 1)
+    tw8, w4b8 = measure_w4(args.steps, args.warmup, 8)
     # prefill: 4096 tokens, skewed routing (tensor-core tile path)
     pf_steps = max(3, min(args.steps // 5, 10))
     tp, _, _ = measure(PREFILL_B, pf_steps, 3, 40_000, bias_sigma=0.5, n_x=2)
@@ -401,7 +437,7 @@ def run_gpu(args):
     clocks_info = clocks.stop()
 
     # max over ranks of the device time
-    t1, t8, t64, te, tp, tc, ts = max_over_ranks([t1, t8, t64, te, tp, tc, ts], world, "cuda")
+    t1, t8, t64, te, tp, tc, ts, tw1, tw8 = max_over_ranks([t1, t8, t64, te, tp, tc, ts, tw1, tw8], world, "cuda")
     tokens, value = job_throughput(1, args.steps, world, t1)
     gbs = bytes1 * world / t1 / 1e9
     peak, tpeak, peak_kind = peaks()
@@ -445,6 +481,14 @@ def run_gpu(args):
                           "tokens_per_s": args.steps * world / ts, "us_per_step": 1e6 * ts / args.steps,
                           "hbm_gbs": expert_bytes * args.steps * world / ts / 1e9,
                           "frac": expert_bytes * args.steps * world / ts / 1e9 / peak, "launches_per_step": 4},
+        "w4_gemv": {"workload": f"4-bit non-expert weight GEMV: symmetric int4, fp16 scale per 128-block, "
+                                f"[{W4_ROWS} x {D_MODEL}] (quantized on the device from seeded N(0, 0.02)), "
+                                f"bf16 tokens, L2 flushed (2 launches: activation digits, GEMV)",
+                    "b1": {"us_per_step": 1e6 * tw1 / args.steps, "hbm_gbs": w4b1 * args.steps * world / tw1 / 1e9,
+                           "frac": w4b1 * args.steps * world / tw1 / 1e9 / peak, "bytes_per_step": w4b1},
+                    "b8": {"us_per_step": 1e6 * tw8 / args.steps, "hbm_gbs": w4b8 * args.steps * world / tw8 / 1e9,
+                           "frac": w4b8 * args.steps * world / tw8 / 1e9 / peak, "bytes_per_step": w4b8},
+                    "bound": "hbm"},
         "e2e": {"value": tokens / te, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": DECODE_LAUNCHES * args.steps,
         "clocks": clocks_info,

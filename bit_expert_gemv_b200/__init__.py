@@ -34,6 +34,7 @@ EXPORTS = (
     "gale_moe_forward", "gale_moe_forward_noalloc", "gale_selftest_scratch_bytes", "gale_selftest",
     "gale_moe_host_staging_bytes", "gale_moe_host_workspace_size", "gale_moe_forward_host",
     "gale_debug_set_failure", "gale_route_topk",
+    "gale_w4_layout", "gale_w4_quantize", "gale_w4_workspace_size", "gale_w4_gemv",
 )
 
 GALE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -53,6 +54,12 @@ class gale_layout(ctypes.Structure):
 
 class gale_matrix(ctypes.Structure):
     _fields_ = [("packed", ctypes.c_void_p), ("rows", ctypes.c_int32), ("cols", ctypes.c_int32)]
+
+
+class gale_w4_layout_t(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("q_offset", ctypes.c_int64),
+                ("q_bytes", ctypes.c_int64), ("s_offset", ctypes.c_int64), ("s_bytes", ctypes.c_int64),
+                ("total", ctypes.c_int64)]
 
 
 class gale_layer(ctypes.Structure):
@@ -95,6 +102,10 @@ def lib() -> ctypes.CDLL:
                                             ctypes.c_float, vp, sz, vp, sz, vp]),
             "gale_debug_set_failure": (i32, [ctypes.c_uint64, i32]),
             "gale_route_topk": (i32, [vp, i32, i32, i32, vp, vp, vp]),
+            "gale_w4_layout": (i32, [i64, i64, ctypes.POINTER(gale_w4_layout_t)]),
+            "gale_w4_quantize": (i32, [vp, i64, i64, vp, vp]),
+            "gale_w4_workspace_size": (sz, [i64, i64, i32]),
+            "gale_w4_gemv": (i32, [vp, i64, i64, vp, i32, vp, vp, sz, vp]),
             "gale_selftest_scratch_bytes": (sz, []),
             "gale_selftest": (i32, [vp, vp]),
         }
@@ -201,6 +212,29 @@ def gale_route_topk(logits, ids, gates, stream=None):
     B, E = logits.shape
     _check(lib().gale_route_topk(_ptr(logits), B, E, ids.shape[1], _ptr(ids), _ptr(gates), _stream(stream)),
            "gale_route_topk")
+
+
+def gale_w4_layout(rows: int, cols: int) -> gale_w4_layout_t:
+    out = gale_w4_layout_t()
+    _check(lib().gale_w4_layout(rows, cols, ctypes.byref(out)), "gale_w4_layout")
+    return out
+
+
+def gale_w4_quantize(w, packed, stream=None):
+    """Quantize a device fp32 [rows, cols] matrix into the W4 g128 layout (packed: device bytes)."""
+    rows, cols = w.shape
+    _check(lib().gale_w4_quantize(_ptr(w), rows, cols, _ptr(packed), _stream(stream)), "gale_w4_quantize")
+
+
+def gale_w4_workspace_size(rows: int, cols: int, B: int) -> int:
+    return int(lib().gale_w4_workspace_size(rows, cols, B))
+
+
+def gale_w4_gemv(packed, rows: int, cols: int, x, y, ws, stream=None):
+    """y [B, rows] fp32 = x [B, cols] (bf16 bits) times the W4 matrix transposed."""
+    B = x.shape[0]
+    _check(lib().gale_w4_gemv(_ptr(packed), rows, cols, _ptr(x), B, _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
+                              _stream(stream)), "gale_w4_gemv")
 
 
 def make_layer(base, expert_stride: int, n_experts: int, d_model: int, d_ff: int) -> gale_layer:

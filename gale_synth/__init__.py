@@ -245,6 +245,18 @@ def _t_normal(keys, n):
     return torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(2.0 * torch.pi * u2)
 
 
+def normal_torch(key: int, n: int, device="cuda", start: int = 0):
+    """Elements start .. start + n of the N(0, 1) stream `key` as an fp64
+    tensor on a torch device (Box-Muller of the same SplitMix64 draws as
+    ``normal``; the device's fp64 log and cos may round a last bit apart)."""
+    import torch
+    k = torch.tensor([key - (1 << 64) if key >= (1 << 63) else key], dtype=torch.int64, device=device)
+    i = torch.arange(start, start + n, dtype=torch.int64, device=device)
+    u1 = _t_uniform(k, 2 * i)
+    u2 = _t_uniform(k, 2 * i + 1)
+    return torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(2.0 * torch.pi * u2)
+
+
 def _t_keys(fields_list, device):
     import torch
     ks = [stream_key(*f) for f in fields_list]

@@ -309,6 +309,60 @@ int gale_moe_forward_host(const gale_layer* layer, const uint16_t* x, const int3
  * Process-wide and not thread-safe; meant for tests of the failure path. */
 int gale_debug_set_failure(uint64_t wait_limit_ns, int withhold_cta);
 
+/* ---------------------------------------------------------------------------
+ * 4-bit non-expert weights (W4, g128).  The DeepSeek-V4-Pro-671B-GALE-1bit-v4
+ * card (paragraph under the weights table) keeps attention and shared-expert
+ * weights as symmetric int4 per 128-block with fp16 scales; the
+ * DeepSeek-V4-Flash card ("What is in the pack", non-expert row) keeps them
+ * 4-bit in VRAM.  Readings: codes q in [-7, 7]; per (row, 128-column block)
+ * s = fp16(amax / 7) (fp32 division, round to nearest even) and
+ * q = clamp(rint(w / s), -7, 7) in fp32 with ties to even (q = 0 when s = 0).
+ * Layout of one [rows x cols] matrix (cols % 128 == 0):
+ *   q at q_offset = 0 : [rows][cols/2] bytes, two's complement nibbles, the
+ *                       low nibble holding the even column
+ *   s at s_offset     : fp16 [rows][cols/128], 256-byte aligned
+ *   total             : 256-byte aligned.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+    int64_t rows, cols;
+    int64_t q_offset, q_bytes;
+    int64_t s_offset, s_bytes;
+    int64_t total;
+} gale_w4_layout_t;
+
+/* Host only.  Errors: GALE_ERR_ARG (NULL out, rows < 1, cols < 128 or not a
+ * multiple of 128). */
+int gale_w4_layout(int64_t rows, int64_t cols, gale_w4_layout_t* out);
+
+/* Quantizes a dense fp32 matrix into the layout above (bit-exact with the
+ * readings: the same fp32 decisions).
+ *   w      : device fp32 [rows][cols], 16-byte aligned
+ *   packed : device, gale_w4_layout(...).total bytes, 256-byte aligned; owned
+ *            by the caller, fully written (padding bytes excepted)
+ * One launch, one warp per (row, block).  Errors: GALE_ERR_ARG, GALE_ERR_ALIGN. */
+int gale_w4_quantize(const float* w, int64_t rows, int64_t cols, void* packed, void* stream);
+
+/* y = x W^T for 1..8 tokens (decode):
+ *   y[t][r] = sum_c s[r][c/128] q[r][c] x[t][c]
+ *   packed : device, the layout above, 256-byte aligned
+ *   x      : device bf16 bits [B][cols]
+ *   y      : device fp32 [B][rows] (overwritten)
+ *   ws     : device, 256-byte aligned, gale_w4_workspace_size(rows, cols, B)
+ *            bytes; needs no initialisation and holds nothing afterwards.
+ * rows % 16 == 0, cols % 1024 == 0, 1 <= B <= 8, and the activation digits
+ * 6 ceil(B/2) (cols + 16) bytes plus 67,584 bytes within 227 KB of shared
+ * memory (GALE_ERR_UNSUPPORTED beyond: cols <= 6144 at 7-8 tokens, 8192 at
+ * 5-6, 13312 at 3-4, 26624 at 1-2).  Activations are held in
+ * fixed point per 1024 columns (21 bits, three int8 digits) and multiplied on
+ * the int8 tensor cores with exact int32 sums; scales and sums in fp32.  Two
+ * launches (activation digits, then one 16-row tile per CTA reading every
+ * weight byte once for all B tokens).
+ * Errors: GALE_ERR_ARG (shape, NULL), GALE_ERR_ALIGN, GALE_ERR_WORKSPACE,
+ * GALE_ERR_UNSUPPORTED (shared memory, above). */
+size_t gale_w4_workspace_size(int64_t rows, int64_t cols, int B);   /* 0 on invalid sizes */
+int gale_w4_gemv(const void* packed, int64_t rows, int64_t cols, const uint16_t* x, int B, float* y, void* ws,
+                 size_t ws_bytes, void* stream);
+
 /* Built-in parity self-check on tiny shapes (the card's "optional fast paths
  * verify themselves at startup" -- without any fallback).  Synchronous:
  * allocates nothing itself but needs `scratch` of gale_selftest_scratch_bytes()
