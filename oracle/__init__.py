@@ -8,3 +8,4 @@ from .gale_oracle import *  # noqa: F401,F403
 from . import gale_oracle  # noqa: F401
 from .w4_oracle import *  # noqa: F401,F403,E402
 from . import w4_oracle  # noqa: F401,E402
+from . import encoder_oracle  # noqa: F401,E402
