@@ -34,7 +34,7 @@ EXPORTS = (
     "gale_moe_forward", "gale_moe_forward_noalloc", "gale_selftest_scratch_bytes", "gale_selftest",
     "gale_moe_host_staging_bytes", "gale_moe_host_workspace_size", "gale_moe_forward_host",
     "gale_debug_set_failure", "gale_route_topk",
-    "gale_w4_layout", "gale_w4_quantize", "gale_w4_workspace_size", "gale_w4_gemv",
+    "gale_w4_layout", "gale_w4_quantize", "gale_w4_workspace_size", "gale_w4_gemv", "gale_encode",
 )
 
 GALE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -102,6 +102,7 @@ def lib() -> ctypes.CDLL:
                                             ctypes.c_float, vp, sz, vp, sz, vp]),
             "gale_debug_set_failure": (i32, [ctypes.c_uint64, i32]),
             "gale_route_topk": (i32, [vp, i32, i32, i32, vp, vp, vp]),
+            "gale_encode": (i32, [vp, i32, i32, vp, vp]),
             "gale_w4_layout": (i32, [i64, i64, ctypes.POINTER(gale_w4_layout_t)]),
             "gale_w4_quantize": (i32, [vp, i64, i64, vp, vp]),
             "gale_w4_workspace_size": (sz, [i64, i64, i32]),
@@ -212,6 +213,12 @@ def gale_route_topk(logits, ids, gates, stream=None):
     B, E = logits.shape
     _check(lib().gale_route_topk(_ptr(logits), B, E, ids.shape[1], _ptr(ids), _ptr(gates), _stream(stream)),
            "gale_route_topk")
+
+
+def gale_encode(w, dst, stream=None):
+    """Encode a device fp32 [rows, cols] matrix into one packed GALE record (dst: device bytes)."""
+    rows, cols = w.shape
+    _check(lib().gale_encode(_ptr(w), rows, cols, _ptr(dst), _stream(stream)), "gale_encode")
 
 
 def gale_w4_layout(rows: int, cols: int) -> gale_w4_layout_t:

@@ -310,6 +310,31 @@ int gale_moe_forward_host(const gale_layer* layer, const uint16_t* x, const int3
 int gale_debug_set_failure(uint64_t wait_limit_ns, int withhold_cta);
 
 /* ---------------------------------------------------------------------------
+ * Encoder: a dense fp32 matrix -> one packed record (the layout above), the
+ * plain encoder of the DeepSeek-V4-Pro-671B-GALE-1bit-v4 card ("the v3 pack
+ * rounded each weight to its sign"; the v4 error-feedback sign choice needs
+ * real activations and is not this call).  Readings, in the pages' order:
+ *   rotation : W_rot = W H, i.e. a blocked FWHT-1024 of every row, in fp64,
+ *              butterfly stages h = 1, 2, ..., 512 (a + b lower, a - b upper),
+ *              then times 1/32;
+ *   signs    : bit 1 where W_rot < 0 (every column, outliers included);
+ *   outliers : the k columns of largest |W_rot| (the lower column first on
+ *              equal magnitudes), stored ascending; s_row = fp16(max|W_rot|/7)
+ *              and q = clamp(rint(W_rot / s_row), -7, 7) in fp64 (0 if s_row
+ *              is 0);
+ *   s_blk    : fp16 of the mean |W_rot| over the block's columns that are not
+ *              outliers (the least-squares scale of their signs), summed in
+ *              column order in fp64; 0 for a block of outliers only.
+ *   w   : device fp32 [rows][cols], 4-byte aligned
+ *   dst : device, gale_layout.total bytes, 16-byte aligned (fully written;
+ *         padding zero)
+ * 1024 <= cols <= 16384, cols % 1024 == 0.  One launch (one CTA per row) after
+ * a memset of dst.  Errors: GALE_ERR_ARG, GALE_ERR_ALIGN, GALE_ERR_UNSUPPORTED
+ * (cols > 16384: the row is held in shared memory in fp64).
+ * ------------------------------------------------------------------------- */
+int gale_encode(const float* w, int rows, int cols, void* dst, void* stream);
+
+/* ---------------------------------------------------------------------------
  * 4-bit non-expert weights (W4, g128).  The DeepSeek-V4-Pro-671B-GALE-1bit-v4
  * card (paragraph under the weights table) keeps attention and shared-expert
  * weights as symmetric int4 per 128-block with fp16 scales; the
