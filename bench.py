@@ -44,8 +44,8 @@ DECODE_LAUNCHES = 1
 # capture (profiles/moe_decode_kernel_b1.md), and the sha256 prefix of the
 # kernel source it was taken on: the bench reports it only while the source is
 # unchanged, and null after any edit until the capture is taken again.
-DECODE_TRAFFIC = None
-DECODE_TRAFFIC_SRC = ""
+DECODE_TRAFFIC = 25_199_104
+DECODE_TRAFFIC_SRC = "212e84e48af81dae"
 KERNEL_SRC = os.path.join(ROOT, "bit_expert_gemv_b200", "csrc", "moe_decode.cu")
 
 
