@@ -502,12 +502,44 @@ def run_gpu(args):
         print(json.dumps(result), flush=True)
 
 
+def run_profile_w4(args):
+    """ncu driver of the 4-bit GEMV: the [W4_ROWS x D_MODEL] matrix of the bench
+    line, --warmup calls, an L2 flush, then --steps calls with --batch tokens."""
+    import torch
+    import bit_expert_gemv_b200 as G
+    G.lib()
+    B = args.batch
+    L = G.gale_w4_layout(W4_ROWS, D_MODEL)
+    packed = torch.empty(L.total, dtype=torch.uint8, device="cuda")
+    w = torch.empty(W4_ROWS, D_MODEL, dtype=torch.float32, device="cuda")
+    for r0 in range(0, W4_ROWS, 4096):
+        w[r0:r0 + 4096] = (gs.normal_torch(gs.stream_key(73, 0), 4096 * D_MODEL, start=r0 * D_MODEL) * 0.02).view(
+            4096, D_MODEL)
+    G.gale_w4_quantize(w, packed)
+    del w
+    x = torch.from_numpy(gs.hidden_bf16(B, D_MODEL, tag=97_000)[0]).view(torch.int16).cuda()
+    y = torch.empty(B, W4_ROWS, dtype=torch.float32, device="cuda")
+    ws = torch.empty(G.gale_w4_workspace_size(W4_ROWS, D_MODEL, B), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        G.gale_w4_gemv(packed, W4_ROWS, D_MODEL, x, y, ws)
+    torch.cuda.synchronize()
+    flush.zero_()
+    torch.cuda.synchronize()
+    for _ in range(args.steps):
+        G.gale_w4_gemv(packed, W4_ROWS, D_MODEL, x, y, ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": "w4", "batch": B, "steps": args.steps}), flush=True)
+
+
 def run_profile(args):
     """A short fixed sequence for ncu captures: build the layer, run
     --warmup calls, flush L2, run --steps calls (decode: unbiased routing;
     prefill: per-expert bias N(0, 0.5)), print the device status."""
     import torch
     import bit_expert_gemv_b200 as G
+    if args.only == "w4":
+        return run_profile_w4(args)
     G.lib()
     buf, stride = build_layer(torch, G)
     layer = G.make_layer(buf, stride, N_EXPERTS, D_MODEL, D_FF)
@@ -632,7 +664,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-chain", action="store_true", help="skip the 43-layer chain measurement")
-    ap.add_argument("--only", choices=["decode", "prefill"], default=None,
+    ap.add_argument("--only", choices=["decode", "prefill", "w4"], default=None,
                     help="profiling driver: warm-up, an L2 flush, then --steps layer calls of one path")
     ap.add_argument("--batch", type=int, default=1, help="tokens per step with --only")
     args = ap.parse_args()
