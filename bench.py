@@ -414,9 +414,37 @@ def run_gpu(args):
             ev[s][1].record(stream)
         torch.cuda.synchronize()
         t = sum(a.elapsed_time(b) * 1e-3 for a, b in ev)
+        # the same stack as one persistent launch (gale_moe_chain) after one
+        # router launch for every layer: two launches per token
+        first = layers[0]
+        wsc = torch.empty(G.gale_moe_chain_workspace_size(first, n_layers, 1, TOP_K), dtype=torch.uint8,
+                          device="cuda")
+        xo = torch.empty(1, D_MODEL, dtype=torch.bfloat16, device="cuda")
+        lg2 = cur_lg.view(n_layers, N_EXPERTS)
+        ids2 = cur_ids.view(n_layers, TOP_K)
+        g2 = cur_g.view(n_layers, TOP_K)
+
+        def token_chain():
+            G.gale_route_topk(lg2, ids2, g2)
+            G.gale_moe_chain(first, n_layers, lb, x0, cur_ids, cur_g, xo, wsc)
+
+        for s in range(warmup):
+            cur_lg.copy_(logits[s])
+            token_chain()
+        torch.cuda.synchronize()
+        if int(wsc[:4].view(torch.int32).item()) != 0:
+            raise RuntimeError("device status after persistent chain warm-up")
+        evc = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for s in range(steps):
+            cur_lg.copy_(logits[warmup + s])
+            evc[s][0].record(stream)
+            token_chain()
+            evc[s][1].record(stream)
+        torch.cuda.synchronize()
+        tk = sum(a.elapsed_time(b) * 1e-3 for a, b in evc)
         del big
         torch.cuda.empty_cache()
-        return t, distinct * expert_bytes, graph is not None
+        return t, distinct * expert_bytes, graph is not None, tk
 
     # nvidia-smi samples the clocks through every timed measurement below
     clocks = Clocks(local)
@@ -433,11 +461,13 @@ def run_gpu(args):
     pf_steps = max(3, min(args.steps // 5, 10))
     tp, _, _ = measure(PREFILL_B, pf_steps, 3, 40_000, bias_sigma=0.5, n_x=2)
     ch_steps = max(3, min(args.steps // 5, 10))
-    tc, bytes_c, ch_graph = measure_chain(ch_steps, 3) if not args.no_chain else (float("nan"), 0, False)
+    tc, bytes_c, ch_graph, tck = measure_chain(ch_steps, 3) if not args.no_chain else (float("nan"), 0, False,
+                                                                                         float("nan"))
     clocks_info = clocks.stop()
 
     # max over ranks of the device time
-    t1, t8, t64, te, tp, tc, ts, tw1, tw8 = max_over_ranks([t1, t8, t64, te, tp, tc, ts, tw1, tw8], world, "cuda")
+    t1, t8, t64, te, tp, tc, ts, tw1, tw8, tck = max_over_ranks([t1, t8, t64, te, tp, tc, ts, tw1, tw8, tck], world,
+                                                                 "cuda")
     tokens, value = job_throughput(1, args.steps, world, t1)
     gbs = bytes1 * world / t1 / 1e9
     peak, tpeak, peak_kind = peaks()
@@ -470,7 +500,13 @@ def run_gpu(args):
                                 f"between layers, bf16 hidden state",
                     "tokens_per_s": ch_steps * world / tc, "ms_per_token": 1e3 * tc / ch_steps,
                     "hbm_gbs": bytes_c * world / tc / 1e9, "frac": bytes_c * world / tc / 1e9 / peak,
-                    "cuda_graph": ch_graph, "steps": ch_steps},
+                    "cuda_graph": ch_graph, "steps": ch_steps,
+                    "persistent": {"launches_per_token": 2,
+                                   "what": "one router launch for all layers, then gale_moe_chain (one cooperative "
+                                           "launch for the 43 layers)",
+                                   "tokens_per_s": ch_steps * world / tck, "ms_per_token": 1e3 * tck / ch_steps,
+                                   "hbm_gbs": bytes_c * world / tck / 1e9,
+                                   "frac": bytes_c * world / tck / 1e9 / peak}},
         "prefill": {"workload": "4096 tokens, top-6 with per-expert bias N(0, 0.5) (skewed), same 256 experts",
                     "tokens_per_s": PREFILL_B * pf_steps * world / tp, "ms_per_step": 1e3 * tp / pf_steps,
                     "tflops": pf_flops * pf_steps / tp / 1e12, "peak_tflops": tpeak,

@@ -35,6 +35,7 @@ EXPORTS = (
     "gale_moe_host_staging_bytes", "gale_moe_host_workspace_size", "gale_moe_forward_host",
     "gale_debug_set_failure", "gale_route_topk",
     "gale_w4_layout", "gale_w4_quantize", "gale_w4_workspace_size", "gale_w4_gemv", "gale_encode",
+    "gale_moe_chain", "gale_moe_chain_workspace_size",
 )
 
 GALE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -103,6 +104,9 @@ def lib() -> ctypes.CDLL:
             "gale_debug_set_failure": (i32, [ctypes.c_uint64, i32]),
             "gale_route_topk": (i32, [vp, i32, i32, i32, vp, vp, vp]),
             "gale_encode": (i32, [vp, i32, i32, vp, vp]),
+            "gale_moe_chain_workspace_size": (sz, [ctypes.POINTER(gale_layer), i32, i32, i32]),
+            "gale_moe_chain": (i32, [ctypes.POINTER(gale_layer), i32, i64, vp, vp, vp, i32, i32, vp, ctypes.c_float,
+                                     vp, sz, vp]),
             "gale_w4_layout": (i32, [i64, i64, ctypes.POINTER(gale_w4_layout_t)]),
             "gale_w4_quantize": (i32, [vp, i64, i64, vp, vp]),
             "gale_w4_workspace_size": (sz, [i64, i64, i32]),
@@ -213,6 +217,19 @@ def gale_route_topk(logits, ids, gates, stream=None):
     B, E = logits.shape
     _check(lib().gale_route_topk(_ptr(logits), B, E, ids.shape[1], _ptr(ids), _ptr(gates), _stream(stream)),
            "gale_route_topk")
+
+
+def gale_moe_chain_workspace_size(first: gale_layer, n_layers: int, B: int, K: int) -> int:
+    return int(lib().gale_moe_chain_workspace_size(ctypes.byref(first), n_layers, B, K))
+
+
+def gale_moe_chain(first: gale_layer, n_layers: int, layer_stride: int, x0, ids, gates, out, ws, eps: float = 1e-6,
+                   stream=None):
+    """x_L of a stack of n_layers layers: x_{l+1} = bf16(RMSNorm(x_l + MoE_l(x_l))); ids/gates [n_layers, B, K]."""
+    B, K = ids.shape[1], ids.shape[2]
+    _check(lib().gale_moe_chain(ctypes.byref(first), n_layers, layer_stride, _ptr(x0), _ptr(ids), _ptr(gates), B, K,
+                                _ptr(out), eps, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "gale_moe_chain")
 
 
 def gale_encode(w, dst, stream=None):

@@ -320,3 +320,30 @@ extern "C" int gale_moe_forward(const gale_layer* layer, const uint16_t* x, cons
     // x_rot is dead by now; reused for v = x + y
     return launch_moe_combine(w.o, w.pos_of_pair, gates, x, B, K, L.d_model, out, out_dtype, fuse, eps, w.x_rot, st);
 }
+
+extern "C" size_t gale_moe_chain_workspace_size(const gale_layer* first, int n_layers, int B, int K) {
+    if (gale::validate_layer(first) != GALE_OK || n_layers < 1 || n_layers > 4096 || B < 1 || K < 1 || K > 16 ||
+        !gale::stream_supported(*first, B, K))
+        return 0;
+    return gale::carve_stream_ws(nullptr, *first, B, K, n_layers).bytes;
+}
+
+extern "C" int gale_moe_chain(const gale_layer* first, int n_layers, int64_t layer_stride, const uint16_t* x0,
+                              const int32_t* ids, const float* gates, int B, int K, uint16_t* out, float eps,
+                              void* ws, size_t ws_bytes, void* stream) {
+    using namespace gale;
+    int rc = validate_layer(first);
+    if (rc != GALE_OK) return rc;
+    const gale_layer& L = *first;
+    if (n_layers < 1 || n_layers > 4096 || B < 1 || K < 1 || K > 16 || K > L.n_experts || !(eps >= 0.f))
+        return GALE_ERR_ARG;
+    if (layer_stride < int64_t(L.n_experts) * L.expert_stride || layer_stride % L.expert_stride)
+        return GALE_ERR_ARG;
+    if (!stream_supported(L, B, K)) return GALE_ERR_UNSUPPORTED;
+    if (!x0 || !ids || !gates || !out) return GALE_ERR_ARG;
+    if (!ws || ws_bytes < carve_stream_ws(nullptr, L, B, K, n_layers).bytes) return GALE_ERR_WORKSPACE;
+    if (!aligned(ws, 256) || !aligned(x0, 4) || !aligned(ids, 4) || !aligned(gates, 4) || !aligned(out, 4))
+        return GALE_ERR_ALIGN;
+    return launch_moe_stream(L, x0, ids, gates, B, K, out, GALE_BF16, true, eps, ws, as_stream(stream), n_layers,
+                             layer_stride / L.expert_stride);
+}

@@ -94,6 +94,10 @@ struct StreamArgs {
     float eps;
     uint64_t wait_ns;       // bound of every wait
     int withhold_cta;       // failure-path testing: this CTA never counts its h tiles (-1: none)
+    int n_layers;           // layers of a chain (1: one layer)
+    int64_t layer_experts;  // expert records between consecutive layers
+    int64_t e_off;          // first expert record of the current layer
+    int32_t* xready;        // tokens of the current layer whose output is written
     StreamWs ws;
 };
 
@@ -199,7 +203,8 @@ struct Ctl {
     int s1b, s2b, nl1, nl, ngrp; // first segment of each range, local segments of phase 1, in all; groups
     int stages, slot_bytes, ring;
     FastDiv dst;                 // division by stages
-    int issued;                  // units whose copies the producer issued
+    int issued;                  // units whose copies the producer issued (all layers)
+    int ubase;                   // units of this CTA in the layers before the current one
     uint64_t wait_ns;            // bound of every wait
     int grp_of[kMaxLocalSeg];    // group of each local segment
     int grp_seg[kMaxLocalSeg];   // the local segment whose pairs define each group
@@ -295,14 +300,8 @@ constexpr int kScratchOff = kSmemBytes - 1024 - int(sizeof(RouteScratch));
 __device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, RouteScratch& rs) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int BK = A.B * A.K, K = A.K;
-    if (tid < kMaxStages) {
-        c.stage_done[tid] = 0;
-        mbar_init(&c.full[tid], 1);
-        mbar_init(&c.empty[tid], 1);
-    }
     if (tid < kMaxLocalSeg) c.grp_left[tid] = 0;
     if (tid == 32) {
-        c.issued = 0;
         c.wait_ns = A.wait_ns;
         c.next_piece = 0;
         c.slot_grp[0] = 0;
@@ -310,8 +309,9 @@ __device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, Route
         c.slot_claim[0] = 0 << 16;
         c.slot_claim[1] = 1 << 16;
         c.slot_done[0] = c.slot_done[1] = 0;
-        c.nmax = 1;
-        fence_mbar_init();
+        // slots for the tokens of the largest possible segment: the ring keeps
+        // its number of stages across the layers of a chain
+        c.nmax = A.B < kSegTok ? A.B : kSegTok;
     }
     if (BK <= 32) {
         if (warp == 0) {
@@ -352,11 +352,9 @@ __device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, Route
             const unsigned sgb = __ballot_sync(0xffffffffu, start);
             const int sn = start ? min(kSegTok, rend - lane) : 0;
             if (start) c.seg[__popc(sgb & (le >> 1))] = (se << 12) | (lane << 3) | sn;
-            const int nmax = __reduce_max_sync(0xffffffffu, sn);
             if (lane == 0) {
                 c.n_valid = nv;
                 c.n_seg = __popc(sgb);
-                c.nmax = nmax > 1 ? nmax : 1;
             }
         }
     } else {
@@ -409,7 +407,6 @@ __device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, Route
         if (lane == 0) c.wsum[warp] = __popc(sb);
         __syncthreads();
         if (start) {
-            if ((packed & 7) > 1) atomicMax(&c.nmax, packed & 7);
             int sid = __popc(sb & ((1u << lane) - 1u));
 #pragma unroll 1
             for (int w = 0; w < warp; ++w) sid += c.wsum[w];
@@ -512,7 +509,7 @@ __device__ __noinline__ void build_block(const void* src, int bf16, int blk, uin
     if (bf16) {
         const uint16_t* s = static_cast<const uint16_t*>(src) + 1024 * blk;
 #pragma unroll
-        for (int r = 0; r < 32; ++r) v[r] = bf16_to_f32(__ldg(s + elem_of(lane, r)));
+        for (int r = 0; r < 32; ++r) v[r] = bf16_to_f32(__ldcg(s + elem_of(lane, r)));
     } else {
         const float* s = static_cast<const float*>(src) + 1024 * blk;
 #pragma unroll
@@ -771,6 +768,9 @@ __device__ __noinline__ void normalize_token(const StreamArgs& A, int t) {
         w.y = uint32_t(f32_to_bf16(a.z * inv)) | (uint32_t(f32_to_bf16(a.w * inv)) << 16);
         o[i] = w;
     }
+    // the token's output (a chain's next input) is complete
+    __syncwarp();
+    if (lane == 0) red_release_add(A.xready, 1);
 }
 
 // y of token t over the 64 rows of block `tile`, once all its experts' o are
@@ -809,8 +809,8 @@ __device__ __noinline__ void combine_block(const StreamArgs& A, const Ctl& c, in
         }
         return;
     }
-    const float v0 = bf16_to_f32(__ldg(A.x + r0)) + y0;
-    const float v1 = bf16_to_f32(__ldg(A.x + r0 + 32)) + y1;
+    const float v0 = bf16_to_f32(__ldcg(A.x + r0)) + y0;
+    const float v1 = bf16_to_f32(__ldcg(A.x + r0 + 32)) + y1;
     A.ws.v[r0] = v0;
     A.ws.v[r0 + 32] = v1;
     const float ss = warp_sum(fmaf(v0, v0, v1 * v1));
@@ -831,16 +831,18 @@ __device__ __noinline__ void empty_token(const StreamArgs& A, int t) {
     float ss = 0.f;
 #pragma unroll 1
     for (int r = lane; r < d; r += 32) {
-        const float v = bf16_to_f32(__ldg(A.x + t * d + r));
+        const float v = bf16_to_f32(__ldcg(A.x + t * d + r));
         ss = fmaf(v, v, ss);
     }
     const float inv = rsqrtf(warp_sum(ss) / float(d) + A.eps);
 #pragma unroll 1
     for (int r = lane; r < d; r += 32) {
-        if (A.fuse_norm) static_cast<uint16_t*>(A.out)[t * d + r] = f32_to_bf16(bf16_to_f32(__ldg(A.x + t * d + r)) * inv);
+        if (A.fuse_norm) static_cast<uint16_t*>(A.out)[t * d + r] = f32_to_bf16(bf16_to_f32(__ldcg(A.x + t * d + r)) * inv);
         else if (A.out_dtype == GALE_F32) static_cast<float*>(A.out)[t * d + r] = 0.f;
         else static_cast<uint16_t*>(A.out)[t * d + r] = 0;
     }
+    __syncwarp();
+    if (lane == 0) red_release_add(A.xready, 1);
 }
 
 // ----------------------------------------------------------------------------
@@ -871,8 +873,9 @@ __device__ __forceinline__ UnitRef unit_ref(const Ctl& c, const Plan& P, int u) 
     r.e = seg_e(sg);
     r.n = seg_n(sg);
     r.first = seg_first(sg);
-    const int lap = fdiv(u, c.dst);
-    r.st = u - lap * c.stages;
+    const int gu = c.ubase + u;   // the ring's running unit index (all layers)
+    const int lap = fdiv(gu, c.dst);
+    r.st = gu - lap * c.stages;
     r.par = lap & 1;
     return r;
 }
@@ -931,12 +934,41 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
         prefetch_tensormap(&map13);
         prefetch_tensormap(&map2);
     }
-    if (tid == 0) c.abort = 0;
-    route_and_plan(A, P, c, *reinterpret_cast<RouteScratch*>(smem + kScratchOff));
+    // the ring's barriers and counters live across the layers of a chain
+    if (tid < kMaxStages) {
+        c.stage_done[tid] = 0;
+        mbar_init(&c.full[tid], 1);
+        mbar_init(&c.empty[tid], 1);
+    }
+    if (tid == 0) {
+        c.abort = 0;
+        c.issued = 0;
+        c.ubase = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    int S = 2;
+#pragma unroll 1
+    for (int layer = 0; layer < A.n_layers; ++layer) {
+    // the layer's arguments: its pairs, its input and output, its counters
+    StreamArgs Al = A;
+    {
+        const int64_t lpairs = int64_t(layer) * A.B * A.K;
+        Al.ids = A.ids + lpairs;
+        Al.gates = A.gates + lpairs;
+        Al.e_off = int64_t(layer) * A.layer_experts;
+        Al.x = layer == 0 ? A.x : A.ws.xbuf + int64_t((layer - 1) & 1) * A.B * A.d_model;
+        Al.out = layer == A.n_layers - 1 ? A.out : static_cast<void*>(A.ws.xbuf + int64_t(layer & 1) * A.B * A.d_model);
+        Al.ws.hcnt = A.ws.hcnt + layer * A.ws.layer_ints;
+        Al.ws.comb = A.ws.comb + layer * A.ws.layer_ints;
+        Al.ws.tokcnt = A.ws.tokcnt + layer * A.ws.layer_ints;
+        Al.xready = A.ws.xready + layer;
+    }
+    route_and_plan(Al, P, c, *reinterpret_cast<RouteScratch*>(smem + kScratchOff));
     const uint32_t s_base = smem_u32(smem);
     const uint32_t slot_base = s_base + uint32_t(align_i(int(sizeof(Ctl)), 1024));
     const uint32_t ring = s_base + uint32_t(c.ring);
-    const int S = c.stages;
+    S = c.stages;
     const int n1 = c.u1e - c.u1b, n2 = c.u2e - c.u2b;
     const int nunits = n1 + n2;
     int32_t* status = A.ws.status;
@@ -947,7 +979,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
 #pragma unroll 1
             for (int u = 0; u < nunits; ++u) {
                 const UnitRef R = unit_ref(c, P, u);
-                if (u >= S && !wait_phase(&c.empty[R.st], R.par ^ 1, c.wait_ns)) {
+                if (c.ubase + u >= S && !wait_phase(&c.empty[R.st], R.par ^ 1, c.wait_ns)) {
                     set_status(status, GALE_ERR_TIMEOUT);
                     atomicExch(&c.abort, 1);
                     break;
@@ -955,7 +987,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
                 if (vload(&c.abort)) break;
                 uint8_t* stage = smem + (ring - s_base) + size_t(R.st) * P.stage_bytes;
                 uint64_t* bar = &c.full[R.st];
-                const char* rec = A.base + int64_t(R.e) * A.stride;
+                const char* rec = A.base + (Al.e_off + R.e) * A.stride;
                 const int rows = R.p1 ? kR1 : kR2;
                 const int k = R.p1 ? P.k1 : P.k2;
                 const StageMap& M = R.p1 ? P.m1 : P.m2;
@@ -966,7 +998,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
                 const uint32_t qbytes = uint32_t(qe - qa);
                 const uint32_t per_mat = uint32_t(M.sb_bytes) + uint32_t(rows * 2) + uint32_t(M.idx_bytes) + qbytes;
                 mbar_arrive_expect_tx(bar, uint32_t(nmat * (R.p1 ? P.nch1 : P.nch2) * rows * 128) + nmat * per_mat);
-                tma_load_5d(stage, R.p1 ? &map13 : &map2, bar, 0, R.tile * rows, 0, 0, R.e);
+                tma_load_5d(stage, R.p1 ? &map13 : &map2, bar, 0, R.tile * rows, 0, 0, int(Al.e_off) + R.e);
 #pragma unroll 1
                 for (int m = 0; m < nmat; ++m) {
                     const char* mat = rec + A.off_w[R.p1 ? m : 2];
@@ -977,7 +1009,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
                               mat + L.off_idx + int64_t(R.tile) * M.idx_bytes, M.idx_bytes, bar);
                     bulk_load(stage + M.q + m * M.q_bytes, mat + L.off_q + qa, qbytes, bar);
                 }
-                c.issued = u + 1;
+                c.issued = c.ubase + u + 1;
             }
         }
     } else {
@@ -985,7 +1017,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
         // tokens without a valid pair get their output here (nothing combines them)
 #pragma unroll 1
         for (int t = blockIdx.x * kCW + warp; t < A.B; t += gridDim.x * kCW)
-            if (c.vmask[t] == 0u) empty_token(A, t);
+            if (c.vmask[t] == 0u) empty_token(Al, t);
         const int tot_pieces = n1 * P.pp1 + n2 * P.pp2;
         const int nhb = P.nch2;
 #pragma unroll 1
@@ -1016,7 +1048,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
                     if (lane == 0) cl = atomicAdd(&c.slot_claim[sl], 1) & 0xFFFF;
                     cl = __shfl_sync(0xffffffffu, cl, 0);
                     if (cl < need) {
-                        act_piece(A, P, c, g, cl, slot);
+                        act_piece(Al, P, c, g, cl, slot);
                         __syncwarp();
                         __threadfence_block();
                         if (lane == 0) atomicAdd(&c.slot_done[sl], 1);
@@ -1145,7 +1177,7 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
                     }
                     __syncwarp();
                     if (lane == 0 && int(blockIdx.x) != A.withhold_cta)
-                        red_release_add(A.ws.hcnt + R.s * nhb + (R.tile * kR1) / 1024, 1);
+                        red_release_add(Al.ws.hcnt + R.s * nhb + (R.tile * kR1) / 1024, 1);
                 } else {
 #pragma unroll
                     for (int i = 0; i < kY; ++i) {
@@ -1162,21 +1194,21 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
                         const int tk = c.sorted[R.first + t] / A.K;
                         int lastc = 0;
                         if (lane == 0)
-                            lastc = atom_acq_rel_add(A.ws.comb + tk * nb + R.tile, 1) == __popc(c.vmask[tk]) - 1;
+                            lastc = atom_acq_rel_add(Al.ws.comb + tk * nb + R.tile, 1) == __popc(c.vmask[tk]) - 1;
                         if (__shfl_sync(0xffffffffu, lastc, 0)) {
                             __syncwarp();
-                            combine_block(A, c, tk, R.tile);
+                            combine_block(Al, c, tk, R.tile);
                         }
                     }
                 }
             }
             // ---- work ahead: one activation piece of the next group, if its
             //      slot is free and (phase 2) its h block is complete ----
-            // (a phase-2 group only once this CTA's phase-1 pieces are nearly
-            // all taken: its readiness test reads a global counter)
+            // (a phase-2 group only from a phase-2 piece: its readiness test
+            // reads a global counter, a round trip that a phase-1 piece would
+            // add to every hand-off)
             const int gn = g + 1;
-            if (gn < c.ngrp && (!R.p1 || c.grp_seg[gn] < c.nl1 || pc + 2 * kCW >= n1 * P.pp1) &&
-                vload(&c.slot_grp[gn & 1]) == gn) {
+            if (gn < c.ngrp && (!R.p1 || c.grp_seg[gn] < c.nl1) && vload(&c.slot_grp[gn & 1]) == gn) {
                 const int sln = gn & 1;
                 const int needn = grp_need(c, P, gn);
                 // claim only if the claim word still belongs to group gn: a
@@ -1184,13 +1216,13 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
                 int cl = needn;
                 if (lane == 0) {
                     const int v = vload(&c.slot_claim[sln]);
-                    if ((v >> 16) == gn && (v & 0xFFFF) < needn && act_ready(A, P, c, gn, v & 0xFFFF) &&
+                    if ((v >> 16) == gn && (v & 0xFFFF) < needn && act_ready(Al, P, c, gn, v & 0xFFFF) &&
                         atomicCAS(&c.slot_claim[sln], v, v + 1) == v)
                         cl = v & 0xFFFF;
                 }
                 cl = __shfl_sync(0xffffffffu, cl, 0);
                 if (cl < needn) {
-                    act_piece(A, P, c, gn, cl, slot_base + uint32_t(sln * c.slot_bytes));
+                    act_piece(Al, P, c, gn, cl, slot_base + uint32_t(sln * c.slot_bytes));
                     __syncwarp();
                     __threadfence_block();
                     if (lane == 0) atomicAdd(&c.slot_done[sln], 1);
@@ -1198,6 +1230,20 @@ moe_stream_kernel(const __grid_constant__ CUtensorMap map13, const __grid_consta
             }
         }
     }
+    // ---- end of the layer: the next one starts once every token's output
+    //      (its input) is written by whichever CTAs finished them ----
+    __syncthreads();
+    if (tid == 0) {
+        c.ubase += nunits;
+        if (layer + 1 < A.n_layers && !vload(&c.abort) &&
+            !wait_global(Al.xready, A.B, &c.abort, c.wait_ns)) {
+            set_status(status, GALE_ERR_TIMEOUT);
+            atomicExch(&c.abort, 1);
+        }
+    }
+    __syncthreads();
+    if (vload(&c.abort)) break;
+    }   // layers
     // every copy the producer issued has landed before the CTA exits
     __syncthreads();
     if (tid == 0 && vload(&c.abort)) {
@@ -1213,7 +1259,7 @@ int g_withhold_cta = -1;
 
 }  // namespace
 
-StreamWs carve_stream_ws(void* ws, const gale_layer& L, int B, int K) {
+StreamWs carve_stream_ws(void* ws, const gale_layer& L, int B, int K, int n_layers) {
     StreamWs w{};
     char* p = static_cast<char*>(ws);
     int64_t o = 0;
@@ -1224,16 +1270,21 @@ StreamWs carve_stream_ws(void* ws, const gale_layer& L, int B, int K) {
     };
     const int64_t BK = int64_t(B) * K, dm = L.d_model, df = L.d_ff;
     const int64_t nb = dm / 64;
-    // counters first: one memset clears them all
+    // counters first: one memset clears them all.  Per layer, [hcnt | comb | tokcnt].
     w.status = reinterpret_cast<int32_t*>(take(256));
-    w.hcnt = reinterpret_cast<int32_t*>(take(4 * BK * (df / 1024)));
-    w.comb = reinterpret_cast<int32_t*>(take(4 * int64_t(B) * nb));
-    w.tokcnt = reinterpret_cast<int32_t*>(take(4 * int64_t(B)));
+    const int64_t nh = BK * (df / 1024), nc = int64_t(B) * nb;
+    w.layer_ints = align_up(nh + nc + B, 64);
+    int32_t* cnt = reinterpret_cast<int32_t*>(take(4 * w.layer_ints * n_layers));
+    w.hcnt = cnt;
+    w.comb = cnt ? cnt + nh : nullptr;
+    w.tokcnt = cnt ? cnt + nh + nc : nullptr;
+    w.xready = reinterpret_cast<int32_t*>(take(4 * int64_t(n_layers)));
     w.counter_bytes = size_t(o);
     w.ssq = reinterpret_cast<float*>(take(4 * int64_t(B) * nb));
     w.h = reinterpret_cast<float*>(take(4 * BK * df));
     w.o = reinterpret_cast<float*>(take(4 * BK * dm));
     w.v = reinterpret_cast<float*>(take(4 * int64_t(B) * dm));
+    w.xbuf = n_layers > 1 ? reinterpret_cast<uint16_t*>(take(2 * 2 * int64_t(B) * dm)) : nullptr;
     w.bytes = size_t(o);
     return w;
 }
@@ -1248,7 +1299,8 @@ bool stream_supported(const gale_layer& L, int B, int K) {
 }
 
 int launch_moe_stream(const gale_layer& L, const uint16_t* x, const int32_t* ids, const float* gates, int B, int K,
-                      void* out, int out_dtype, bool fuse_norm, float eps, void* ws, cudaStream_t st) {
+                      void* out, int out_dtype, bool fuse_norm, float eps, void* ws, cudaStream_t st, int n_layers,
+                      int64_t layer_experts) {
     StreamArgs A{};
     A.base = static_cast<const char*>(L.base);
     A.stride = L.expert_stride;
@@ -1270,12 +1322,20 @@ int launch_moe_stream(const gale_layer& L, const uint16_t* x, const int32_t* ids
     A.eps = eps;
     A.wait_ns = g_wait_ns;
     A.withhold_cta = g_withhold_cta;
-    A.ws = carve_stream_ws(ws, L, B, K);
+    A.n_layers = n_layers;
+    A.layer_experts = n_layers > 1 ? layer_experts : 0;
+    A.e_off = 0;
+    A.ws = carve_stream_ws(ws, L, B, K, n_layers);
+    A.xready = A.ws.xready;
     GALE_CUDA_TRY(cudaMemsetAsync(A.ws.status, 0, A.ws.counter_bytes, st));
     CUtensorMap map13, map2;
-    int rc = cached_sign_map5b(&map13, A.base, L.d_ff, L.d_model, 2, P.L1.total, L.n_experts, L.expert_stride, kR1, 2);
+    // one map over the expert records of every layer (a chain's layers are
+    // records l * layer_experts + e of the same array)
+    const int64_t n_rec = int64_t(n_layers - 1) * A.layer_experts + L.n_experts;
+    if (n_rec > 0x7FFFFFFF) return GALE_ERR_UNSUPPORTED;
+    int rc = cached_sign_map5b(&map13, A.base, L.d_ff, L.d_model, 2, P.L1.total, int(n_rec), L.expert_stride, kR1, 2);
     if (rc == GALE_OK)
-        rc = cached_sign_map5b(&map2, A.base + A.off_w[2], L.d_model, L.d_ff, 1, P.L1.total, L.n_experts,
+        rc = cached_sign_map5b(&map2, A.base + A.off_w[2], L.d_model, L.d_ff, 1, P.L1.total, int(n_rec),
                                L.expert_stride, kR2, 1);
     if (rc != GALE_OK) return rc;
     rc = ensure_smem(reinterpret_cast<const void*>(moe_stream_kernel), kSmemBytes);

@@ -296,6 +296,35 @@ int gale_moe_forward_host(const gale_layer* layer, const uint16_t* x, const int3
                           float eps, void* ws, size_t ws_bytes, void* staging, size_t staging_bytes,
                           void* stream);
 
+/* ---------------------------------------------------------------------------
+ * A stack of layers in one launch (decode): for l = 0 .. n_layers-1,
+ *   x_{l+1} = bf16( RMSNorm( x_l + MoE_l(x_l) ) )   (unit weight, eps)
+ * with MoE_l the layer of gale_moe_forward on ids[l], gates[l]; out = x_L.
+ * The DeepSeek-V4-Pro-671B-GALE-1bit-v4 card's A100 paragraph names the
+ * batch-1 floor: expert unpacks plus about 200 small kernel launches per
+ * layer; here a whole stack is one persistent cooperative kernel.  Each layer
+ * starts once every token's output of the previous one is written (a
+ * counter per layer, bounded wait), and the weight ring streams on across
+ * the layers.
+ *   first        : layer 0; layer l's expert e is record l * (layer_stride /
+ *                  first->expert_stride) + e of the records starting at
+ *                  first->base (every layer the same shape and record size;
+ *                  layer_stride a multiple of expert_stride, at least
+ *                  n_experts * expert_stride)
+ *   x0           : device bf16 [B][d_model]
+ *   ids, gates   : device int32 / fp32 [n_layers][B][K] (as gale_moe_forward)
+ *   out          : device bf16 [B][d_model], x_L
+ *   ws           : device, 256-byte aligned, gale_moe_chain_workspace_size()
+ *                  bytes; its first int32 is the status word (as for
+ *                  gale_moe_forward)
+ * 1 <= n_layers <= 4096; the batches of the streaming decode kernel
+ * (B * K <= 384, d_model <= 4096, d_ff <= 2048), else GALE_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------- */
+size_t gale_moe_chain_workspace_size(const gale_layer* first, int n_layers, int B, int K);
+int gale_moe_chain(const gale_layer* first, int n_layers, int64_t layer_stride, const uint16_t* x0,
+                   const int32_t* ids, const float* gates, int B, int K, uint16_t* out, float eps, void* ws,
+                   size_t ws_bytes, void* stream);
+
 /* Failure-path testing hook; an interface addition of this library with no
  * counterpart on the GALE cards.  Applies to later gale_moe_forward calls of
  * this process that take the streaming decode kernel (3 to 64 tokens):
