@@ -1,6 +1,9 @@
 // Decode path of gale_moe_forward: the routed-expert layer for batches of up
 // to 384 (token, expert) pairs as one persistent kernel, one CTA per SM,
 // launched cooperatively (all CTAs resident: CTAs wait on each other's h).
+// The same kernel runs a stack of layers (gale_moe_chain): it loops over the
+// layers, each with its own counters, and starts layer l + 1 once every
+// token's output of layer l (its input) has been written.
 //
 // Work.  The (token, k) pairs are grouped by expert, stable in pair order,
 // and every expert's pairs are cut into segments of at most two (one MMA
