@@ -59,7 +59,8 @@ def _stack(n_layers, E, d, dff):
 
 
 @pytest.mark.parametrize("n_layers,E,d,dff,B,K", [(4, 8, 4096, 2048, 1, 6), (5, 16, 2048, 1024, 3, 4),
-                                                  (3, 12, 4096, 2048, 8, 6), (2, 16, 2048, 1024, 2, 16)])
+                                                  (3, 12, 4096, 2048, 8, 6), (2, 16, 2048, 1024, 2, 16),
+                                                  (3, 32, 2048, 1024, 32, 6)])
 def test_chain_kernel(n_layers, E, d, dff, B, K):
     """gale_moe_chain (one persistent launch for the whole stack):
     - from three tokens on, bit-identical to the same layers run one call at a
