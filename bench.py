@@ -307,17 +307,25 @@ def run_gpu(args):
             G.gale_fwht1024(h, h)
             G.gale_expert_gemv(w2, D_MODEL, D_FF, h, y)
 
-        for i in range(warmup):
-            step(xs[i])
-        torch.cuda.synchronize()
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-        for i in range(steps):
-            flush.zero_()
-            ev[i][0].record(stream)
-            step(xs[warmup + i])
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        return sum(a.elapsed_time(b) * 1e-3 for a, b in ev)
+        wsf = torch.empty(G.gale_expert_forward_workspace_size(layer, 1), dtype=torch.uint8, device="cuda")
+
+        def fused(x):
+            G.gale_expert_forward(layer, 0, x, y, wsf)
+
+        times = []
+        for fn in (step, fused):
+            for i in range(warmup):
+                fn(xs[i])
+            torch.cuda.synchronize()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            for i in range(steps):
+                flush.zero_()
+                ev[i][0].record(stream)
+                fn(xs[warmup + i])
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            times.append(sum(a.elapsed_time(b) * 1e-3 for a, b in ev))
+        return times[0], times[1]
 
     def measure_w4(steps, warmup, B):
         """The 4-bit non-expert weight GEMV (symmetric int4, 128-block fp16
@@ -454,7 +462,7 @@ def run_gpu(args):
     # decode batch 64 with per-expert popularity bias N(0, 0.5) (skewed tokens per expert)
     t64, bytes64, _ = measure(64, max(args.steps // 2, 3), args.warmup, 25_000, bias_sigma=0.5)
     te, h2d, d2h = measure_e2e(1, args.steps, args.warmup, 30_000)
-    ts = measure_single(args.steps, args.warmup)
+    ts, tsf = measure_single(args.steps, args.warmup)
     tw1, w4b1 = measure_w4(args.steps, args.warmup, 1)
     tw8, w4b8 = measure_w4(args.steps, args.warmup, 8)
     # prefill: 4096 tokens, skewed routing (tensor-core tile path)
@@ -466,8 +474,8 @@ def run_gpu(args):
     clocks_info = clocks.stop()
 
     # max over ranks of the device time
-    t1, t8, t64, te, tp, tc, ts, tw1, tw8, tck = max_over_ranks([t1, t8, t64, te, tp, tc, ts, tw1, tw8, tck], world,
-                                                                 "cuda")
+    t1, t8, t64, te, tp, tc, ts, tw1, tw8, tck, tsf = max_over_ranks([t1, t8, t64, te, tp, tc, ts, tw1, tw8, tck, tsf],
+                                                                      world, "cuda")
     tokens, value = job_throughput(1, args.steps, world, t1)
     gbs = bytes1 * world / t1 / 1e9
     peak, tpeak, peak_kind = peaks()
@@ -512,11 +520,15 @@ def run_gpu(args):
                     "tflops": pf_flops * pf_steps / tp / 1e12, "peak_tflops": tpeak,
                     "frac": pf_flops * pf_steps / tp / 1e12 / tpeak, "bound": "tensor",
                     "flops_per_step": pf_flops, "steps": pf_steps},
-        "single_expert": {"workload": "one GALE expert, one token, fp32 x [4096] (w1/w3 [2048x4096], w2 [4096x2048]):"
-                                      " FWHT, w1/w3 GEMV + SwiGLU, FWHT, w2 GEMV (4 launches), L2 flushed",
-                          "tokens_per_s": args.steps * world / ts, "us_per_step": 1e6 * ts / args.steps,
-                          "hbm_gbs": expert_bytes * args.steps * world / ts / 1e9,
-                          "frac": expert_bytes * args.steps * world / ts / 1e9 / peak, "launches_per_step": 4},
+        "single_expert": {"workload": "one GALE expert, one token, fp32 x [4096] (w1/w3 [2048x4096], w2 [4096x2048]), "
+                                      "L2 flushed: gale_expert_forward (one launch)",
+                          "tokens_per_s": args.steps * world / tsf, "us_per_step": 1e6 * tsf / args.steps,
+                          "hbm_gbs": expert_bytes * args.steps * world / tsf / 1e9,
+                          "frac": expert_bytes * args.steps * world / tsf / 1e9 / peak, "launches_per_step": 1,
+                          "four_launches": {"what": "FWHT, w1/w3 GEMV + SwiGLU, FWHT, w2 GEMV (gale_fwht1024, "
+                                                    "gale_expert_gemv)",
+                                            "us_per_step": 1e6 * ts / args.steps,
+                                            "frac": expert_bytes * args.steps * world / ts / 1e9 / peak}},
         "w4_gemv": {"workload": f"4-bit non-expert weight GEMV: symmetric int4, fp16 scale per 128-block, "
                                 f"[{W4_ROWS} x {D_MODEL}] (quantized on the device from seeded N(0, 0.02)), "
                                 f"bf16 tokens, L2 flushed (2 launches: activation digits, GEMV)",

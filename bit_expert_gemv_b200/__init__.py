@@ -35,7 +35,7 @@ EXPORTS = (
     "gale_moe_host_staging_bytes", "gale_moe_host_workspace_size", "gale_moe_forward_host",
     "gale_debug_set_failure", "gale_route_topk",
     "gale_w4_layout", "gale_w4_quantize", "gale_w4_workspace_size", "gale_w4_gemv", "gale_encode",
-    "gale_moe_chain", "gale_moe_chain_workspace_size",
+    "gale_moe_chain", "gale_moe_chain_workspace_size", "gale_expert_forward", "gale_expert_forward_workspace_size",
 )
 
 GALE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -105,6 +105,8 @@ def lib() -> ctypes.CDLL:
             "gale_route_topk": (i32, [vp, i32, i32, i32, vp, vp, vp]),
             "gale_encode": (i32, [vp, i32, i32, vp, vp]),
             "gale_moe_chain_workspace_size": (sz, [ctypes.POINTER(gale_layer), i32, i32, i32]),
+            "gale_expert_forward_workspace_size": (sz, [ctypes.POINTER(gale_layer), i32]),
+            "gale_expert_forward": (i32, [ctypes.POINTER(gale_layer), i32, vp, i32, vp, vp, sz, vp]),
             "gale_moe_chain": (i32, [ctypes.POINTER(gale_layer), i32, i64, vp, vp, vp, i32, i32, vp, ctypes.c_float,
                                      vp, sz, vp]),
             "gale_w4_layout": (i32, [i64, i64, ctypes.POINTER(gale_w4_layout_t)]),
@@ -217,6 +219,17 @@ def gale_route_topk(logits, ids, gates, stream=None):
     B, E = logits.shape
     _check(lib().gale_route_topk(_ptr(logits), B, E, ids.shape[1], _ptr(ids), _ptr(gates), _stream(stream)),
            "gale_route_topk")
+
+
+def gale_expert_forward_workspace_size(layer: gale_layer, B: int) -> int:
+    return int(lib().gale_expert_forward_workspace_size(ctypes.byref(layer), B))
+
+
+def gale_expert_forward(layer: gale_layer, expert: int, x, out, ws, stream=None):
+    """out [B, d_model] fp32 = the SwiGLU forward of one expert on fp32 x [B, d_model] (one launch)."""
+    B = x.shape[0]
+    _check(lib().gale_expert_forward(ctypes.byref(layer), expert, _ptr(x), B, _ptr(out), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)), "gale_expert_forward")
 
 
 def gale_moe_chain_workspace_size(first: gale_layer, n_layers: int, B: int, K: int) -> int:

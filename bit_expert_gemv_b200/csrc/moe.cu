@@ -347,3 +347,22 @@ extern "C" int gale_moe_chain(const gale_layer* first, int n_layers, int64_t lay
     return launch_moe_stream(L, x0, ids, gates, B, K, out, GALE_BF16, true, eps, ws, as_stream(stream), n_layers,
                              layer_stride / L.expert_stride);
 }
+
+extern "C" size_t gale_expert_forward_workspace_size(const gale_layer* layer, int B) {
+    if (gale::validate_layer(layer) != GALE_OK || B < 1 || !gale::stream_supported(*layer, B, 1)) return 0;
+    return gale::carve_stream_ws(nullptr, *layer, B, 1).bytes;
+}
+
+extern "C" int gale_expert_forward(const gale_layer* layer, int expert, const float* x, int B, float* out, void* ws,
+                                   size_t ws_bytes, void* stream) {
+    using namespace gale;
+    int rc = validate_layer(layer);
+    if (rc != GALE_OK) return rc;
+    const gale_layer& L = *layer;
+    if (expert < 0 || expert >= L.n_experts || B < 1 || !x || !out) return GALE_ERR_ARG;
+    if (!stream_supported(L, B, 1)) return GALE_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < carve_stream_ws(nullptr, L, B, 1).bytes) return GALE_ERR_WORKSPACE;
+    if (!aligned(ws, 256) || !aligned(x, 4) || !aligned(out, 4)) return GALE_ERR_ALIGN;
+    return launch_moe_stream(L, nullptr, nullptr, nullptr, B, 1, out, GALE_F32, false, 0.f, ws, as_stream(stream), 1, 0,
+                             x, expert);
+}

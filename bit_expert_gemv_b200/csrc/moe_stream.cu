@@ -101,6 +101,8 @@ struct StreamArgs {
     int64_t layer_experts;  // expert records between consecutive layers
     int64_t e_off;          // first expert record of the current layer
     int32_t* xready;        // tokens of the current layer whose output is written
+    const float* xf;        // fp32 activations in place of x (one expert's forward), or null
+    int fixed_e;            // >= 0: every token's one pair is this expert with gate 1 (ids and gates unused)
     StreamWs ws;
 };
 
@@ -319,7 +321,7 @@ __device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, Route
     if (BK <= 32) {
         if (warp == 0) {
             const int p = lane;
-            const int e = p < BK ? __ldg(A.ids + p) : -1;
+            const int e = p < BK ? (A.fixed_e >= 0 ? A.fixed_e : __ldg(A.ids + p)) : -1;
             if (lane < A.B) c.vmask[lane] = 0u;
             const int t = p / K, k = p - t * K;
             bool valid = p < BK && e >= 0 && e < A.E;
@@ -362,7 +364,7 @@ __device__ void route_and_plan(const StreamArgs& A, const Plan& P, Ctl& c, Route
         }
     } else {
         if (tid < A.B) c.vmask[tid] = 0u;
-        if (tid < BK) rs.ids[tid] = __ldg(A.ids + tid);
+        if (tid < BK) rs.ids[tid] = A.fixed_e >= 0 ? A.fixed_e : __ldg(A.ids + tid);
         if (tid == 0) {
             c.n_valid = 0;
             c.bad = 0;
@@ -791,7 +793,7 @@ __device__ __noinline__ void combine_block(const StreamArgs& A, const Ctl& c, in
             const int k = k0 + j;
             const bool ok = k < K && ((vm >> k) & 1u);
             const float* o = A.ws.o + (t * K + (ok ? k : 0)) * d + tile * 64 + lane;
-            g[j] = ok ? __ldg(A.gates + t * K + k) : 0.f;
+            g[j] = ok ? (A.fixed_e >= 0 ? 1.f : __ldg(A.gates + t * K + k)) : 0.f;
             o0[j] = ok ? __ldcg(o) : 0.f;
             o1[j] = ok ? __ldcg(o + 32) : 0.f;
         }
@@ -896,7 +898,10 @@ __device__ __noinline__ void act_piece(const StreamArgs& A, const Plan& P, Ctl& 
     const int tk = cl / nb, blk = cl - tk * nb;
     const int pair = c.sorted[seg_first(sg) + tk];
     if (p1) {
-        build_block(A.x + (pair / A.K) * A.d_model, 1, blk, slot + uint32_t(tk * P.t1.bytes), P.t1);
+        if (A.xf)
+            build_block(A.xf + (pair / A.K) * A.d_model, 0, blk, slot + uint32_t(tk * P.t1.bytes), P.t1);
+        else
+            build_block(A.x + (pair / A.K) * A.d_model, 1, blk, slot + uint32_t(tk * P.t1.bytes), P.t1);
     } else {
         int v = 1;
         if (lane == 0) v = wait_global(A.ws.hcnt + s * P.nch2 + blk, 1024 / kR1, &c.abort, c.wait_ns);
@@ -1303,7 +1308,7 @@ bool stream_supported(const gale_layer& L, int B, int K) {
 
 int launch_moe_stream(const gale_layer& L, const uint16_t* x, const int32_t* ids, const float* gates, int B, int K,
                       void* out, int out_dtype, bool fuse_norm, float eps, void* ws, cudaStream_t st, int n_layers,
-                      int64_t layer_experts) {
+                      int64_t layer_experts, const float* xf, int fixed_e) {
     StreamArgs A{};
     A.base = static_cast<const char*>(L.base);
     A.stride = L.expert_stride;
@@ -1326,6 +1331,8 @@ int launch_moe_stream(const gale_layer& L, const uint16_t* x, const int32_t* ids
     A.wait_ns = g_wait_ns;
     A.withhold_cta = g_withhold_cta;
     A.n_layers = n_layers;
+    A.xf = xf;
+    A.fixed_e = fixed_e;
     A.layer_experts = n_layers > 1 ? layer_experts : 0;
     A.e_off = 0;
     A.ws = carve_stream_ws(ws, L, B, K, n_layers);

@@ -30,6 +30,6 @@ bool stream_supported(const gale_layer& L, int B, int K);
 // that start at L.base.
 int launch_moe_stream(const gale_layer& L, const uint16_t* x, const int32_t* ids, const float* gates, int B, int K,
                       void* out, int out_dtype, bool fuse_norm, float eps, void* ws, cudaStream_t st,
-                      int n_layers = 1, int64_t layer_experts = 0);
+                      int n_layers = 1, int64_t layer_experts = 0, const float* xf = nullptr, int fixed_e = -1);
 
 }  // namespace gale

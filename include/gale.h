@@ -297,6 +297,22 @@ int gale_moe_forward_host(const gale_layer* layer, const uint16_t* x, const int3
                           void* stream);
 
 /* ---------------------------------------------------------------------------
+ * One expert's SwiGLU forward in one launch (the single-expert configuration
+ * of the GALE cards' format table: w1/w3 [d_ff x d_model], w2 [d_model x
+ * d_ff], fp32 activations):
+ *   out[t] = W2 H( silu(W1 H x[t]) * (W3 H x[t]) )      (expert `expert` of layer)
+ *   x   : device fp32 [B][d_model]        out : device fp32 [B][d_model]
+ *   ws  : device, 256-byte aligned, gale_expert_forward_workspace_size()
+ *         bytes; its first int32 is the status word
+ * The batches of the streaming decode kernel (B <= 384, d_model <= 4096,
+ * d_ff <= 2048), else GALE_ERR_UNSUPPORTED.  gale_expert_gemv is the
+ * one-matrix call.
+ * ------------------------------------------------------------------------- */
+size_t gale_expert_forward_workspace_size(const gale_layer* layer, int B);
+int gale_expert_forward(const gale_layer* layer, int expert, const float* x, int B, float* out, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * A stack of layers in one launch (decode): for l = 0 .. n_layers-1,
  *   x_{l+1} = bf16( RMSNorm( x_l + MoE_l(x_l) ) )   (unit weight, eps)
  * with MoE_l the layer of gale_moe_forward on ids[l], gates[l]; out = x_L.

@@ -4,6 +4,8 @@ Bit-exact for packing, dense dequantisation and the routing permute; within
 a relative L2 error of 2e-3 (bf16 activations, fp32 accumulation) for the
 expert GEMV, the SwiGLU expert and the MoE layer; FWHT within fp32 rounding.
 """
+import ctypes
+
 import numpy as np
 import pytest
 
@@ -502,3 +504,28 @@ def test_route_topk_ties_and_nan():
     wi, wg = O.route_topk(np.nan_to_num(lg, nan=-np.inf), 4)
     assert np.array_equal(ids.cpu().numpy(), wi)
     assert np.max(np.abs(gates.cpu().numpy().astype(np.float64) - wg)) < 1e-6
+
+
+@pytest.mark.parametrize("shape,e,B", [("small", 3, 1), ("small", 15, 2), ("small", 0, 5), ("full", 7, 1),
+                                       ("full", 200, 3)])
+def test_expert_forward(small_layer, full_layer, shape, e, B):
+    """One expert's SwiGLU forward on fp32 tokens in one launch
+    (gale_expert_forward) against the oracle's expert_forward, per token."""
+    L = small_layer if shape == "small" else full_layer
+    x = np.stack([gs.x_f32(L.d_model, tag=1000 + 10 * B + t) for t in range(B)])
+    ws = torch.empty(G.gale_expert_forward_workspace_size(L.desc, B), dtype=torch.uint8, device="cuda")
+    out = torch.full((B, L.d_model), float("nan"), device="cuda")
+    G.gale_expert_forward(L.desc, e, to_dev(x), out, ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    assert_tokens(out.cpu().numpy(), O.expert_forward(L.dense(e), x.astype(np.float64)), what=f"expert {e} B={B}")
+
+
+def test_expert_forward_rejects_bad_expert(small_layer):
+    L = small_layer
+    x = torch.zeros(1, L.d_model, device="cuda")
+    out = torch.zeros(1, L.d_model, device="cuda")
+    ws = torch.empty(G.gale_expert_forward_workspace_size(L.desc, 1), dtype=torch.uint8, device="cuda")
+    rc = G.lib().gale_expert_forward(ctypes.byref(L.desc), L.E, x.data_ptr(), 1, out.data_ptr(), ws.data_ptr(),
+                                     ws.numel(), None)
+    assert rc == G.GALE_ERR_ARG
