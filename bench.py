@@ -345,7 +345,7 @@ def run_gpu(args):
         xs = [torch.from_numpy(gs.hidden_bf16(B, D_MODEL, tag=97_000 + i)[0]).view(torch.int16).cuda()
               for i in range(steps + warmup)]
         y = torch.empty(B, W4_ROWS, dtype=torch.float32, device="cuda")
-        ws = torch.empty(G.gale_w4_workspace_size(W4_ROWS, D_MODEL, B), dtype=torch.uint8, device="cuda")
+        ws = torch.zeros(G.gale_w4_workspace_size(W4_ROWS, D_MODEL, B), dtype=torch.uint8, device="cuda")
         for i in range(warmup):
             G.gale_w4_gemv(packed, W4_ROWS, D_MODEL, xs[i], y, ws)
         torch.cuda.synchronize()
@@ -531,7 +531,7 @@ def run_gpu(args):
                                             "frac": expert_bytes * args.steps * world / ts / 1e9 / peak}},
         "w4_gemv": {"workload": f"4-bit non-expert weight GEMV: symmetric int4, fp16 scale per 128-block, "
                                 f"[{W4_ROWS} x {D_MODEL}] (quantized on the device from seeded N(0, 0.02)), "
-                                f"bf16 tokens, L2 flushed (2 launches: activation digits, GEMV)",
+                                f"bf16 tokens, L2 flushed (one launch)",
                     "b1": {"us_per_step": 1e6 * tw1 / args.steps, "hbm_gbs": w4b1 * args.steps * world / tw1 / 1e9,
                            "frac": w4b1 * args.steps * world / tw1 / 1e9 / peak, "bytes_per_step": w4b1},
                     "b8": {"us_per_step": 1e6 * tw8 / args.steps, "hbm_gbs": w4b8 * args.steps * world / tw8 / 1e9,
@@ -567,7 +567,7 @@ def run_profile_w4(args):
     del w
     x = torch.from_numpy(gs.hidden_bf16(B, D_MODEL, tag=97_000)[0]).view(torch.int16).cuda()
     y = torch.empty(B, W4_ROWS, dtype=torch.float32, device="cuda")
-    ws = torch.empty(G.gale_w4_workspace_size(W4_ROWS, D_MODEL, B), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(G.gale_w4_workspace_size(W4_ROWS, D_MODEL, B), dtype=torch.uint8, device="cuda")
     flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device="cuda")
     for _ in range(args.warmup):
         G.gale_w4_gemv(packed, W4_ROWS, D_MODEL, x, y, ws)

@@ -11,11 +11,12 @@
 // column), then fp16 scales [rows][cols / 128], each section 256-byte aligned.
 //
 // GEMV (decode, 1..8 tokens).  y[t, r] = sum_c s(r, c / 128) q(r, c) x(t, c).
-// The weights are streamed once with 16-byte loads and fed, still packed, to
-// the int8 tensor cores: a 32-bit word of eight nibbles gives two A registers
+// One launch: the weights are streamed once by bulk copies into a ring of
+// shared-memory stages and fed, still packed, to the int8 tensor cores: a 32-bit word of eight nibbles gives two A registers
 // of (q + 8) as unsigned bytes, (w & 0x0F0F0F0F) ^ 0x08080808 and the same of
-// w >> 4, one LOP3 each.  The activations are prepared once per call in fixed
-// point: per 1024-column chunk a power-of-two S with max |x S| <= 2^20,
+// w >> 4, one LOP3 each.  The activations are prepared in fixed point by
+// every CTA while its first copies are in flight: per 1024-column
+// chunk a power-of-two S with max |x S| <= 2^20,
 // X = rint(x S) as three balanced int8 digits (X = 2^14 d1 + 2^7 d2 + d3).  A
 // block's MMA sum over (q + 8) X is corrected exactly in int32 by the block
 // sum of X (times 8), then scaled by s in fp32; 1/S is applied per chunk.
@@ -33,10 +34,7 @@ namespace {
 constexpr int kW4Block = 128;
 constexpr int kW4Chunk = 1024;
 constexpr int kW4Rows = 16;       // rows of a CTA tile
-constexpr int kW4MaxStages = 4;   // shared-memory stages per warp (fewer when the activations need room)
-constexpr int kW4KBlk = 4;        // 128-column blocks per streamed unit
-constexpr int kW4UnitW = kW4Rows * kW4KBlk * 64;            // code bytes of a unit (4 KB)
-constexpr int kW4UnitBytes = kW4UnitW + kW4Rows * kW4KBlk * 2;   // + scales (128 B)
+constexpr int kW4MaxStages = 8;   // ring stages of a CTA (fewer when the activations need room)
 constexpr int kW4SmemMax = 227 * 1024;
 
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -78,39 +76,59 @@ __global__ void __launch_bounds__(256) w4_quantize_kernel(const float* __restric
     if (lane == 0) s[r * nb + b] = sh;
 }
 
-// Activation digits of one (token, 1024-column chunk) per warp.  Lane
-// l = 8 tig + 2 i + par writes, for each block bb of the chunk and digit j,
-// the word of the four columns 128 bb + 32 tig + 8 i + 2 e + par (e = 0..3),
-// at xd + ((t * 3 + j) * nblk + block) * 128 + tig * 32 + i * 8 + par * 4:
-// the B fragment of MMA i for the lanes of quad index tig.
-__global__ void __launch_bounds__(256) w4_xprep_kernel(const uint16_t* __restrict__ x, int B, int64_t cols,
-                                                      uint8_t* __restrict__ xd, int32_t* __restrict__ xsum,
-                                                      float* __restrict__ xsig) {
-    const int64_t nch = cols / kW4Chunk, nblk = cols / kW4Block;
-    const int64_t item = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    if (item >= int64_t(B) * nch) return;
-    const int lane = threadIdx.x & 31;
-    const int t = int(item / nch);
-    const int64_t ch = item - int64_t(t) * nch;
+// Launch parameters of the GEMV.  Shared memory, in this order: nst ring
+// stages (the 16 code rows, then 16 scale rows of `spitch` bytes from byte
+// `sreg` of the stage), the activation digits (6 NP rows of `xpitch` bytes), the block sums
+// of X (int32 [2 NP][cols / 128]), 1 / S (fp32 [2 NP][cols / 1024]), the
+// per-warp partial sums (fp32 [2][NWC][NP][32]), then 2 nst mbarriers and an
+// abort flag.  Offsets in bytes from the start of dynamic shared memory.
+struct W4Args {
+    const uint8_t* q;
+    const __half* s;
+    const uint16_t* x;
+    float* y;
+    int32_t* status;
+    int64_t rows, cols;
+    int B, nst, uc;                 // tokens, ring stages, columns of a unit
+    // whole rows (a tile is one unit): codes as 8 copies of two rows, pair p at
+    // p ppitch (ppitch = cols + 64: consecutive pairs 64 bytes apart modulo
+    // 128), scales as one copy; else one copy per row at ppitch / 2 and one per
+    // row of scales at a padded spitch.  Row g of a stage starts at
+    // (g >> 1) ppitch + (g & 1) rstride.
+    int whole, ppitch, rstride, spitch, sreg, xpitch, stage_bytes;
+    int off_x, off_xsum, off_xsig, off_red, off_bar;
+};
+
+// Activation digits of one (token t, 1024-column chunk ch) by one warp, into
+// shared memory.  Lane l = 8 tig + 2 i + par writes, for each block bb of the
+// chunk and digit j, the word of the four columns 128 bb + 32 tig + 8 i +
+// 2 e + par (e = 0..3) at row (3 t + j), byte 128 block + 32 tig + 8 i + 4 par:
+// the B fragment of MMA i for the lanes of quad index tig.  Tokens t >= B
+// (the pad of an odd count) get zero digits and zero sums.
+__device__ __forceinline__ void w4_prep_chunk(const W4Args& a, uint8_t* smem, int t, int ch, int lane) {
     const int tig = lane >> 3, i = (lane >> 1) & 3, par = lane & 1;
-    const uint16_t* xs = x + int64_t(t) * cols + ch * kW4Chunk + 32 * tig + 8 * i + par;
+    const int nblk = int(a.cols / kW4Block), nch = int(a.cols / kW4Chunk);
     float v[8][4];
     float m = 0.f;
+    const uint16_t* xs = a.x + int64_t(t) * a.cols + int64_t(ch) * kW4Chunk + 32 * tig + 8 * i + par;
 #pragma unroll
     for (int bb = 0; bb < 8; ++bb)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            v[bb][e] = bf16_to_f32(__ldg(xs + 128 * bb + 2 * e));
+            v[bb][e] = t < a.B ? bf16_to_f32(__ldg(xs + 128 * bb + 2 * e)) : 0.f;
             m = fmaxf(m, fabsf(v[bb][e]));
         }
     m = warp_max(m);
     // largest power of two S with m S <= 2^20 (1 for a zero chunk; at most 2^100)
+    // (m = f 2^e2 with 0.5 <= f < 1 gives e2 = biased exponent - 126; a
+    // subnormal m takes e2 = -126, which the cap at 2^100 makes exact)
     float S = 1.0f;
     if (m > 0.f) {
-        int e2;
-        frexpf(m, &e2);                       // m = f 2^e2, 0.5 <= f < 1
-        S = ldexpf(1.0f, min(20 - e2, 100));  // m S < 2^20
+        const int e2 = int((__float_as_uint(m) >> 23) & 0xFFu) - 126;
+        S = __uint_as_float(uint32_t(min(20 - e2, 100) + 127) << 23);   // m S < 2^20
     }
+    uint8_t* xd = smem + a.off_x;
+    int32_t* xsum = reinterpret_cast<int32_t*>(smem + a.off_xsum);
 #pragma unroll
     for (int bb = 0; bb < 8; ++bb) {
         uint32_t wd[3] = {0u, 0u, 0u};
@@ -127,100 +145,138 @@ __global__ void __launch_bounds__(256) w4_xprep_kernel(const uint16_t* __restric
             wd[1] |= (uint32_t(d2) & 0xFFu) << (8 * e);
             wd[2] |= (uint32_t(d3) & 0xFFu) << (8 * e);
         }
-        const int64_t blk = ch * 8 + bb;
+        const int blk = ch * 8 + bb;
 #pragma unroll
         for (int j = 0; j < 3; ++j)
-            *reinterpret_cast<uint32_t*>(xd + ((int64_t(t) * 3 + j) * nblk + blk) * 128 + tig * 32 + i * 8 + par * 4) =
-                wd[j];
+            *reinterpret_cast<uint32_t*>(xd + (t * 3 + j) * a.xpitch + blk * 128 + tig * 32 + i * 8 + par * 4) = wd[j];
         const int tot = __reduce_add_sync(0xffffffffu, sx);
-        if (lane == 0) xsum[int64_t(t) * nblk + blk] = tot;
+        if (lane == 0) xsum[t * nblk + blk] = tot;
     }
-    if (lane == 0) xsig[int64_t(t) * nch + ch] = 1.0f / S;
+    if (lane == 0) reinterpret_cast<float*>(smem + a.off_xsig)[t * nch + ch] = 1.0f / S;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-// wait until at most n - 1 groups of this thread are pending (n = 2..4)
-__device__ __forceinline__ void cp_wait_stages(int n) {
-    if (n == 4) asm volatile("cp.async.wait_group 3;" ::: "memory");
-    else if (n == 3) asm volatile("cp.async.wait_group 2;" ::: "memory");
-    else asm volatile("cp.async.wait_group 1;" ::: "memory");
+__device__ __forceinline__ void w4_fail(const W4Args& a, volatile int* abort_flag) {
+    *abort_flag = 1;
+    atomicExch(a.status, GALE_ERR_TIMEOUT);
 }
 
-// Persistent GEMV: every warp owns whole 16-row tiles (tile = global warp +
-// k x all warps) and streams each tile in units of four 128-column blocks
-// (4 KB of codes + 128 B of scales) through its own ring of `nst` shared-memory
-// stages, filled with 16-byte asynchronous copies nst - 1 units ahead of the
-// arithmetic.  In a stage, row r's 16-byte chunk c (block c / 4, quad lane
-// c % 4) sits at chunk c ^ (r & 7) of the row's 256 bytes, so the eight rows
-// a load touches fall in eight different bank groups.  The activation digits
-// of all 2 NP tokens are copied into shared memory once (one block-wide
-// barrier at the start), rows of (token, digit) `xpitch` bytes apart.  NP
-// column groups of two tokens (tokens 2p, 2p + 1) share the A registers of a
-// block.
-template <int NP, int NW>
-__global__ void __launch_bounds__(NW * 32, 1) w4_gemv_kernel(const uint8_t* __restrict__ q,
-                                                             const __half* __restrict__ s, int64_t cols, int B,
-                                                             const uint8_t* __restrict__ xd,
-                                                             const int32_t* __restrict__ xsum,
-                                                             const float* __restrict__ xsig, float* __restrict__ y,
-                                                             int64_t rows, int nst, int xpitch) {
-    extern __shared__ __align__(16) uint8_t w4_smem[];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, tig = lane & 3;
-    const int nblk = int(cols / kW4Block), nch = int(cols / kW4Chunk);
-    const int nk = nblk / kW4KBlk;                            // units per tile
-    const int64_t ntiles = rows / kW4Rows;
-    const int64_t gw = int64_t(blockIdx.x) * NW + warp, nw = int64_t(gridDim.x) * NW;
-    const int64_t my_tiles = gw < ntiles ? (ntiles - gw + nw - 1) / nw : 0;
-    const uint32_t ring = smem_u32(w4_smem) + uint32_t(warp * nst * kW4UnitBytes);
-    const uint32_t xs = smem_u32(w4_smem) + uint32_t(NW * nst * kW4UnitBytes);
-    const int swz = g & 7;
-    const int64_t rowb = cols / 2;                            // code bytes of a row
-    // the activation digits, once: 6 NP rows of cols bytes
-    {
-        const int nrow = 6 * NP, per_row = int(cols / 16);
-        for (int i = threadIdx.x; i < nrow * per_row; i += blockDim.x) {
-            const int r = i / per_row, c = i - r * per_row;
-            cp_async16(xs + uint32_t(r * xpitch + 16 * c), xd + int64_t(r) * cols + 16 * c);
+// Persistent GEMV, one CTA per SM: CTA c owns the 16-row tiles c, c + grid,
+// ...; a tile is read as units of 16 rows x `uc` columns (the last unit of a
+// row may be narrower).  Warp NWC copies each unit into the next ring stage
+// with bulk copies (lane r < 16: code row r, `uc` / 2 contiguous bytes; lane
+// 16 + r: that row's `uc` / 128 scales), each row at a padded pitch so the
+// eight rows of an A fragment fall in distinct bank groups.  The NWC consumer
+// warps form two groups of NWG = NWC / 2 that take alternate tiles (group k:
+// the CTA's tiles k, k + 2, ...), so one group's per-unit hand-off overlaps
+// the other's arithmetic.  Warp w of a group multiplies columns
+// [w sw, (w + 1) sw) of every unit of its tiles (sw = uc / NWG, inside one
+// 1024-column chunk) and frees the stage; at the end of a tile the NWG
+// partial sums of every (row, token) are added in warp order by one warp of
+// the group.
+// The activation digits are built by the consumer warps at the start, while
+// the first copies are in flight.  NP column groups of two tokens (tokens
+// 2p, 2p + 1) share the A registers of a block.  Every wait is bounded: on
+// time-out the status word takes GALE_ERR_TIMEOUT, the other waits are
+// skipped, and the copy warp waits (bounded) for its copies in flight.
+template <int NP, int NWC, int NBW>
+__global__ void __launch_bounds__((NWC + 1) * 32, 1) w4_gemv_kernel(const W4Args a) {
+    extern __shared__ __align__(128) uint8_t w4_smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nblk = int(a.cols / kW4Block), nch = int(a.cols / kW4Chunk);
+    const int64_t ntiles = a.rows / kW4Rows;
+    const int64_t my_tiles = int64_t(blockIdx.x) < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int upt = int((a.cols + a.uc - 1) / a.uc);          // units per tile
+    const int nst = a.nst;
+    uint64_t* full = reinterpret_cast<uint64_t*>(w4_smem + a.off_bar);
+    uint64_t* empty = full + nst;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + nst);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < nst; ++i) {
+            mbar_init(full + i, 1);
+            mbar_init(empty + i, NWC / 2);
         }
-        cp_commit();
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        __syncthreads();
+        *abort_flag = 0;
+        fence_mbar_init();
     }
+    __syncthreads();
+
+    if (warp == NWC) {
+        // ---- copy warp ----
+        const int64_t my_units = my_tiles * upt;
+        const int r = lane & 15;
+        int64_t gu = 0;
+        int st = 0, u = 0;
+        // parity of the empty phase a stage's next reuse waits for: the first
+        // reuse (units nst .. 2 nst - 1) waits for phase 0, and so on
+        uint32_t eph = 1;
+        int64_t tile = blockIdx.x;
+#pragma unroll 1
+        for (; gu < my_units; ++gu) {
+            if (*abort_flag) break;
+            if (gu >= nst) {
+                bool ok = true;
+                if (lane == 0) ok = mbar_wait(empty + st, eph);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) {
+                    if (lane == 0) w4_fail(a, abort_flag);
+                    break;
+                }
+            }
+            const int wid = int(min(int64_t(a.uc), a.cols - int64_t(u) * a.uc));
+            uint8_t* stage = w4_smem + st * a.stage_bytes;
+            if (lane == 0) mbar_arrive_expect_tx(full + st, uint32_t(16 * (wid / 2 + wid / 64)));
+            __syncwarp();
+            if (a.whole) {
+                if (lane < 8)
+                    bulk_load(stage + lane * a.ppitch, a.q + (tile * kW4Rows + 2 * lane) * (a.cols / 2),
+                              uint32_t(a.cols), full + st);
+                else if (lane == 8)
+                    bulk_load(stage + a.sreg, a.s + tile * kW4Rows * nblk, uint32_t(16 * nblk * 2), full + st);
+            } else {
+                const int64_t row = tile * kW4Rows + r;
+                if (lane < 16)
+                    bulk_load(stage + (r >> 1) * a.ppitch + (r & 1) * a.rstride,
+                              a.q + row * (a.cols / 2) + int64_t(u) * (a.uc / 2), uint32_t(wid / 2), full + st);
+                else
+                    bulk_load(stage + a.sreg + r * a.spitch, a.s + row * nblk + int64_t(u) * (a.uc / kW4Block),
+                              uint32_t(wid / 64), full + st);
+            }
+            if (++st == nst) {
+                st = 0;
+                eph ^= 1;
+            }
+            if (++u == upt) {
+                u = 0;
+                tile += gridDim.x;
+            }
+        }
+        // the copies of the last units issued land before the CTA may exit
+        if (lane == 0) {
+            const int64_t first = gu > nst ? gu - nst : 0;
+            for (int64_t v = first; v < gu; ++v)
+                if (!mbar_wait(full + (v % nst), uint32_t((v / nst) & 1))) {
+                    w4_fail(a, abort_flag);
+                    break;
+                }
+        }
+        return;
+    }
+
+    // ---- consumer warps ----
+    for (int it = warp; it < 2 * NP * nch; it += NWC) w4_prep_chunk(a, w4_smem, it / nch, it % nch, lane);
+    named_bar_sync(3, NWC * 32);
     if (my_tiles == 0) return;
 
-    // issue pointer: (tile i_t, unit i_k) into stage i_s; this lane's own chunks
-    int64_t i_t = 0;
-    int i_k = 0, i_s = 0;
-    auto issue_next = [&]() {
-        if (i_t < my_tiles) {
-            const int64_t r0 = (gw + i_t * nw) * kW4Rows;
-            const uint32_t base = ring + uint32_t(i_s * kW4UnitBytes);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int row = g + 8 * h;
-                const uint8_t* src = q + (r0 + row) * rowb + 64 * (i_k * kW4KBlk) + 16 * tig;
-#pragma unroll
-                for (int j = 0; j < kW4KBlk; ++j)
-                    cp_async16(base + uint32_t(row * 256 + (((4 * j + tig) ^ swz) << 4)), src + 64 * j);
-                if (tig == 0) cp_async8(base + uint32_t(kW4UnitW + row * 8), s + (r0 + row) * nblk + i_k * kW4KBlk);
-            }
-            if (++i_k == nk) {
-                i_k = 0;
-                ++i_t;
-            }
-            if (++i_s == nst) i_s = 0;
-        }
-        cp_commit();
-    };
-#pragma unroll 1
-    for (int i = 0; i < nst - 1; ++i) issue_next();
+    constexpr int NWG = NWC / 2;                // warps of a consumer group
+    const int grp = warp / NWG, wg = warp - grp * NWG;
+
+    const int g = lane >> 2, tig = lane & 3;
+    constexpr int sw = NBW * kW4Block;          // columns of this warp's slice of a unit (uc = NWG sw)
+    const uint32_t sbase = smem_u32(w4_smem);
+    const uint32_t xs = sbase + uint32_t(a.off_x);
+    const int32_t* xsum = reinterpret_cast<const int32_t*>(w4_smem + a.off_xsum);
+    const float* xsig = reinterpret_cast<const float*>(w4_smem + a.off_xsig);
+    float* red = reinterpret_cast<float*>(w4_smem + a.off_red);
     // B fragment of this lane: column g = (token g / 3 of the group, digit g % 3); 6, 7 unused
     const bool bl = g < 6;
     const int tk = g / 3, dg = g % 3;
@@ -232,94 +288,124 @@ __global__ void __launch_bounds__(NW * 32, 1) w4_gemv_kernel(const uint8_t* __re
     // digits -> value: token 0 = 2^14 n0 + 2^7 n1 + n2, token 1 = 2^14 n3 + 2^7 n4 + n5
     const float wa = tig == 0 ? 16384.0f : tig == 1 ? 1.0f : tig == 2 ? 128.0f : 0.f;    // weight of column 2 tig
     const float wc = tig == 0 ? 128.0f : tig == 1 ? 16384.0f : tig == 2 ? 1.0f : 0.f;    // of column 2 tig + 1
-    const uint32_t xrow = xs + uint32_t((tk * 3 + dg) * xpitch + tig * 32);
-    float acc[NP][4], tot[NP][4];
-    int c_s = 0;
+    const uint32_t xrow = xs + uint32_t((tk * 3 + dg) * a.xpitch + tig * 32);
+    // row g, this slice, chunk tig (row g + 8 is four pairs further)
+    const uint32_t aoff = uint32_t((g >> 1) * a.ppitch + (g & 1) * a.rstride + wg * (sw / 2) + 16 * tig);
+    const uint32_t boff = uint32_t(4 * a.ppitch);
+    const uint32_t soff = uint32_t(a.sreg + g * a.spitch + 2 * wg * NBW);
+    bool live = true;   // false once a wait ran out: the remaining waits are skipped
+    // stage and phase parity of the group's next unit (unit index ti upt + u of the CTA)
+    int st = (grp * upt) % nst;
+    uint32_t ph = uint32_t(((grp * upt) / nst) & 1);
 #pragma unroll 1
-    for (int64_t t_i = 0; t_i < my_tiles; ++t_i) {
+    for (int64_t ti = grp; ti < my_tiles; ti += 2) {
+        float tot[NP][4];
 #pragma unroll
         for (int p = 0; p < NP; ++p)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) acc[p][i] = tot[p][i] = 0.f;
+            for (int i = 0; i < 4; ++i) tot[p][i] = 0.f;
 #pragma unroll 1
-        for (int kc = 0; kc < nk; ++kc) {
-            issue_next();
-            cp_wait_stages(nst);
-            __syncwarp();
-            const uint32_t base = ring + uint32_t(c_s * kW4UnitBytes);
-            if (++c_s == nst) c_s = 0;
-#pragma unroll
-            for (int j = 0; j < kW4KBlk; ++j) {
-                const int b = kc * kW4KBlk + j;
-                const uint32_t co = uint32_t(((4 * j + tig) ^ swz) << 4);
-                const uint4 ua = lds_v4(base + uint32_t(g * 256) + co);
-                const uint4 ub = lds_v4(base + uint32_t((g + 8) * 256) + co);
-                const float s0 =
-                    __half2float(__ushort_as_half(uint16_t(lds_u16(base + uint32_t(kW4UnitW + g * 8 + 2 * j)))));
-                const float s1 =
-                    __half2float(__ushort_as_half(uint16_t(lds_u16(base + uint32_t(kW4UnitW + (g + 8) * 8 + 2 * j)))));
-                const uint32_t wa4[4] = {ua.x, ua.y, ua.z, ua.w}, wb4[4] = {ub.x, ub.y, ub.z, ub.w};
-                uint32_t lo[4], lo8[4], hi[4], hi8[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    lo[i] = (wa4[i] & 0x0F0F0F0Fu) ^ 0x08080808u;
-                    hi[i] = ((wa4[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-                    lo8[i] = (wb4[i] & 0x0F0F0F0Fu) ^ 0x08080808u;
-                    hi8[i] = ((wb4[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+        for (int u = 0; u < upt; ++u) {
+            // one lane waits for the stage (the warp barrier orders the others' reads after it)
+            if (live && !*abort_flag) {
+                bool ok = true;
+                if (lane == 0) ok = mbar_wait(full + st, ph);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    if (lane == 0) w4_fail(a, abort_flag);
+                    live = false;
                 }
-#pragma unroll
-                for (int p = 0; p < NP; ++p) {
-                    uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
-                    if (bl) {
-                        const uint32_t xb = xrow + uint32_t(6 * p * xpitch + b * 128);
-                        x0 = lds_v4(xb);
-                        x1 = lds_v4(xb + 16);
-                    }
-                    // two independent MMA chains (columns of words 0, 1 and 2, 3)
-                    int ca[4] = {0, 0, 0, 0}, cb[4] = {0, 0, 0, 0};
-                    mma_u8s8(ca, lo[0], lo8[0], hi[0], hi8[0], x0.x, x0.y);
-                    mma_u8s8(cb, lo[2], lo8[2], hi[2], hi8[2], x1.x, x1.y);
-                    mma_u8s8(ca, lo[1], lo8[1], hi[1], hi8[1], x0.z, x0.w);
-                    mma_u8s8(cb, lo[3], lo8[3], hi[3], hi8[3], x1.z, x1.w);
-                    int cc[4] = {ca[0] + cb[0], ca[1] + cb[1], ca[2] + cb[2], ca[3] + cb[3]};
-                    if (cor >= 0) {
-                        const int xb8 = 8 * __ldg(xsum + (2 * p + ctok) * nblk + b);
-                        cc[cor] -= xb8;
-                        cc[cor + 2] -= xb8;
-                    }
-                    acc[p][0] = fmaf(s0, float(cc[0]), acc[p][0]);
-                    acc[p][1] = fmaf(s0, float(cc[1]), acc[p][1]);
-                    acc[p][2] = fmaf(s1, float(cc[2]), acc[p][2]);
-                    acc[p][3] = fmaf(s1, float(cc[3]), acc[p][3]);
-                }
+            } else {
+                live = false;
             }
             __syncwarp();
-            // a 1024-column chunk is two units: its sums take 1/S of each column's token
-            if (kc & 1) {
-                const int ch = kc / 2;
+            const int c0 = u * a.uc + wg * sw;                 // first column of the slice
+            if (c0 < a.cols && c0 < u * a.uc + min(int64_t(a.uc), a.cols - int64_t(u) * a.uc)) {
+                const uint32_t base = sbase + uint32_t(st * a.stage_bytes);
+                float acc[NP][4];
+#pragma unroll
+                for (int p = 0; p < NP; ++p)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[p][i] = 0.f;
+#pragma unroll
+                for (int j = 0; j < NBW; ++j) {
+                    const int b = c0 / kW4Block + j;
+                    const uint4 ua = lds_v4(base + aoff + uint32_t(64 * j));
+                    const uint4 ub = lds_v4(base + aoff + boff + uint32_t(64 * j));
+                    const float s0 = __half2float(__ushort_as_half(uint16_t(lds_u16(base + soff + uint32_t(2 * j)))));
+                    const float s1 = __half2float(
+                        __ushort_as_half(uint16_t(lds_u16(base + soff + uint32_t(8 * a.spitch + 2 * j)))));
+                    const uint32_t wa4[4] = {ua.x, ua.y, ua.z, ua.w}, wb4[4] = {ub.x, ub.y, ub.z, ub.w};
+                    uint32_t lo[4], lo8[4], hi[4], hi8[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        lo[i] = (wa4[i] & 0x0F0F0F0Fu) ^ 0x08080808u;
+                        hi[i] = ((wa4[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+                        lo8[i] = (wb4[i] & 0x0F0F0F0Fu) ^ 0x08080808u;
+                        hi8[i] = ((wb4[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+                    }
+#pragma unroll
+                    for (int p = 0; p < NP; ++p) {
+                        uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
+                        if (bl) {
+                            const uint32_t xb = xrow + uint32_t(6 * p * a.xpitch + b * 128);
+                            x0 = lds_v4(xb);
+                            x1 = lds_v4(xb + 16);
+                        }
+                        // two independent MMA chains (columns of words 0, 1 and 2, 3)
+                        int ca[4] = {0, 0, 0, 0}, cb[4] = {0, 0, 0, 0};
+                        mma_u8s8(ca, lo[0], lo8[0], hi[0], hi8[0], x0.x, x0.y);
+                        mma_u8s8(cb, lo[2], lo8[2], hi[2], hi8[2], x1.x, x1.y);
+                        mma_u8s8(ca, lo[1], lo8[1], hi[1], hi8[1], x0.z, x0.w);
+                        mma_u8s8(cb, lo[3], lo8[3], hi[3], hi8[3], x1.z, x1.w);
+                        int cc[4] = {ca[0] + cb[0], ca[1] + cb[1], ca[2] + cb[2], ca[3] + cb[3]};
+                        if (cor >= 0) {
+                            const int xb8 = 8 * xsum[(2 * p + ctok) * nblk + b];
+                            cc[cor] -= xb8;
+                            cc[cor + 2] -= xb8;
+                        }
+                        acc[p][0] = fmaf(s0, float(cc[0]), acc[p][0]);
+                        acc[p][1] = fmaf(s0, float(cc[1]), acc[p][1]);
+                        acc[p][2] = fmaf(s1, float(cc[2]), acc[p][2]);
+                        acc[p][3] = fmaf(s1, float(cc[3]), acc[p][3]);
+                    }
+                }
+                // the slice lies in one 1024-column chunk: its sums take 1/S of each column's token
+                const int ch = c0 / kW4Chunk;
 #pragma unroll
                 for (int p = 0; p < NP; ++p) {
-                    const float f0 = tc0 < 2 ? __ldg(xsig + (2 * p + tc0) * nch + ch) : 0.f;
-                    const float f1 = tc1 < 2 ? __ldg(xsig + (2 * p + tc1) * nch + ch) : 0.f;
+                    const float f0 = tc0 < 2 ? xsig[(2 * p + tc0) * nch + ch] : 0.f;
+                    const float f1 = tc1 < 2 ? xsig[(2 * p + tc1) * nch + ch] : 0.f;
                     tot[p][0] = fmaf(f0, acc[p][0], tot[p][0]);
                     tot[p][1] = fmaf(f1, acc[p][1], tot[p][1]);
                     tot[p][2] = fmaf(f0, acc[p][2], tot[p][2]);
                     tot[p][3] = fmaf(f1, acc[p][3], tot[p][3]);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) acc[p][i] = 0.f;
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + st);
+            if (++st == nst) {
+                st = 0;
+                ph ^= 1;
+            }
         }
-        // sums over the lane quad, then lane (g, tig) writes row g + 8 (tig >> 1), token tig & 1
-        const int64_t r0 = (gw + t_i * nw) * kW4Rows;
+        // skip the other group's tile
+#pragma unroll 1
+        for (int k = 0; k < upt; ++k)
+            if (++st == nst) {
+                st = 0;
+                ph ^= 1;
+            }
+        // sums over the lane quad; lane (g, tig) holds row g + 8 (tig >> 1), token tig & 1 of each group
+        const int li = int(ti >> 1);                          // the tile's index within the group
+        float* gred = red + (grp * 2 + (li & 1)) * NWG * NP * 32;
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
             float v[2][2];   // [row g, g + 8][token]
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const float a = wa * tot[p][2 * h], c = wc * tot[p][2 * h + 1];
-                float t0v = (tc0 == 0 ? a : 0.f) + (tc1 == 0 ? c : 0.f);
-                float t1v = (tc0 == 1 ? a : 0.f) + (tc1 == 1 ? c : 0.f);
+                const float x0 = wa * tot[p][2 * h], x1 = wc * tot[p][2 * h + 1];
+                float t0v = (tc0 == 0 ? x0 : 0.f) + (tc1 == 0 ? x1 : 0.f);
+                float t1v = (tc0 == 1 ? x0 : 0.f) + (tc1 == 1 ? x1 : 0.f);
                 t0v += __shfl_xor_sync(0xffffffffu, t0v, 1);
                 t0v += __shfl_xor_sync(0xffffffffu, t0v, 2);
                 t1v += __shfl_xor_sync(0xffffffffu, t1v, 1);
@@ -327,11 +413,24 @@ __global__ void __launch_bounds__(NW * 32, 1) w4_gemv_kernel(const uint8_t* __re
                 v[h][0] = t0v;
                 v[h][1] = t1v;
             }
-            const int t = 2 * p + (tig & 1);
-            if (t < B) y[int64_t(t) * rows + r0 + g + 8 * (tig >> 1)] = v[tig >> 1][tig & 1];
+            const float mine = (tig >> 1) ? ((tig & 1) ? v[1][1] : v[1][0]) : ((tig & 1) ? v[0][1] : v[0][0]);
+            gred[(wg * NP + p) * 32 + lane] = mine;
+        }
+        named_bar_sync(1 + grp, NWG * 32);
+        // one warp adds the NWG partials in warp order (a group's buffers
+        // alternate by tile, so its next tile's writes never meet this read)
+        if (wg == li % NWG) {
+            const int64_t r0 = (int64_t(blockIdx.x) + ti * gridDim.x) * kW4Rows;
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < NWG; ++w) sum += gred[(w * NP + p) * 32 + lane];
+                const int t = 2 * p + (tig & 1);
+                if (t < a.B) a.y[int64_t(t) * a.rows + r0 + g + 8 * (tig >> 1)] = sum;
+            }
         }
     }
-    cp_wait_all();
 }
 
 }  // namespace
@@ -365,90 +464,130 @@ extern "C" int gale_w4_quantize(const float* w, int64_t rows, int64_t cols, void
 }
 
 namespace {
-// workspace: digits [Bp][3][cols], block sums [Bp][cols/128], 1/S [Bp][cols/1024]
-struct W4Ws {
-    uint8_t* xd;
-    int32_t* xsum;
-    float* xsig;
-    int64_t bytes;
-};
-W4Ws carve_w4_ws(void* ws, int64_t cols, int B) {
-    const int64_t bp = B + (B & 1);
-    char* p = static_cast<char*>(ws);
-    W4Ws w{};
-    int64_t o = 0;
-    w.xd = reinterpret_cast<uint8_t*>(p ? p + o : nullptr);
-    o = gale::align_up(o + bp * 3 * cols, 256);
-    w.xsum = reinterpret_cast<int32_t*>(p ? p + o : nullptr);
-    o = gale::align_up(o + bp * (cols / 128) * 4, 256);
-    w.xsig = reinterpret_cast<float*>(p ? p + o : nullptr);
-    o = gale::align_up(o + bp * (cols / 1024) * 4, 256);
-    w.bytes = o;
-    return w;
-}
 bool w4_gemv_shape_ok(int64_t rows, int64_t cols, int B) {
     return rows >= 16 && rows % 16 == 0 && cols >= 1024 && cols % 1024 == 0 && B >= 1 && B <= 8 &&
-           rows / 16 <= 0x7FFFFFFF;
+           rows / 16 <= 0x7FFFFFFF && cols <= (int64_t(1) << 20);
 }
+
+// Shared-memory plan for NWC consumer warps: the widest unit (4096, 2048 or
+// 1024 columns, at least 128 per warp, no wider than the row needs) that
+// leaves room for three ring stages, else for two.  False when none fits.
+bool w4_plan(int64_t cols, int B, int nwc, gale::W4Args& a, int& smem) {
+    const int np = (B + 1) / 2;
+    const int nblk = int(cols / gale::kW4Block), nch = int(cols / gale::kW4Chunk);
+    a.xpitch = int(cols) + 16;
+    const int64_t xbytes = int64_t(6) * np * a.xpitch;
+    const int64_t sums = gale::align_up(int64_t(2) * np * nblk * 4, 16) + gale::align_up(int64_t(2) * np * nch * 4, 16);
+    const int64_t redb = int64_t(2) * nwc * np * 32 * 4;
+    const int64_t bars = 2 * gale::kW4MaxStages * 8 + 16;
+    for (int need = 3; need >= 2; --need) {
+        for (int uc = 4096; uc >= 1024; uc /= 2) {
+            if (uc < 64 * nwc) break;                                // a block per warp of a group
+            if (uc / 2 >= 64 * nwc && uc / 2 >= cols) continue;     // a narrower unit covers the row
+            const int whole = cols <= uc;
+            const int ppitch = whole ? int(cols) + 64 : uc + 32;
+            const int spitch = whole ? int(cols / 64) : uc / 64 + 16;
+            const int sreg = 8 * ppitch;
+            const int64_t stage = sreg + int64_t(16) * spitch;
+            const int64_t room = gale::kW4SmemMax - xbytes - sums - redb - bars;
+            if (room < need * stage) continue;
+            a.uc = uc;
+            a.whole = whole;
+            a.ppitch = ppitch;
+            a.rstride = whole ? int(cols / 2) : ppitch / 2;
+            a.spitch = spitch;
+            a.sreg = sreg;
+            a.stage_bytes = int(stage);
+            a.nst = int(room / stage < gale::kW4MaxStages ? room / stage : gale::kW4MaxStages);
+            int64_t o = int64_t(a.nst) * stage;
+            a.off_x = int(o);
+            o += xbytes;
+            a.off_xsum = int(o);
+            o += gale::align_up(int64_t(2) * np * nblk * 4, 16);
+            a.off_xsig = int(o);
+            o += gale::align_up(int64_t(2) * np * nch * 4, 16);
+            a.off_red = int(o);
+            o += redb;
+            a.off_bar = int(o);
+            o += bars;
+            smem = int(o);
+            return true;
+        }
+    }
+    return false;
+}
+
+// Consumer warps (two groups): 16 up to 4 tokens (on [65536 x 4096]: 47.1
+// against 55.3 us at 1-2 tokens, 67.6 against 90.1 us at 4), 8 from 5 (172
+// against 240 us at 8 tokens, where 16 warps' 96-register cap spills).
+int w4_nwc(int B) { return B >= 5 ? 8 : 16; }
 }  // namespace
 
 extern "C" size_t gale_w4_workspace_size(int64_t rows, int64_t cols, int B) {
     if (!w4_gemv_shape_ok(rows, cols, B)) return 0;
-    return size_t(carve_w4_ws(nullptr, cols, B).bytes);
+    return 256;   // the status word
 }
 
 extern "C" int gale_w4_gemv(const void* packed, int64_t rows, int64_t cols, const uint16_t* x, int B, float* y,
                             void* ws, size_t ws_bytes, void* stream) {
     if (!w4_gemv_shape_ok(rows, cols, B) || !packed || !x || !y) return GALE_ERR_ARG;
     if (!gale::aligned(packed, 256) || !gale::aligned(x, 2) || !gale::aligned(y, 4)) return GALE_ERR_ALIGN;
-    const W4Ws w = carve_w4_ws(ws, cols, B);
-    if (!ws || ws_bytes < size_t(w.bytes)) return GALE_ERR_WORKSPACE;
+    if (!ws || ws_bytes < 256) return GALE_ERR_WORKSPACE;
     if (!gale::aligned(ws, 256)) return GALE_ERR_ALIGN;
     gale_w4_layout_t L;
     gale_w4_layout(rows, cols, &L);
-    cudaStream_t st = gale::as_stream(stream);
-    if (B & 1) {   // the unused token of the last column group reads zeros
-        const int64_t bp = B + 1;
-        if (cudaMemsetAsync(w.xd + int64_t(B) * 3 * cols, 0, size_t(3 * cols), st) != cudaSuccess ||
-            cudaMemsetAsync(w.xsum + int64_t(B) * (cols / 128), 0, size_t(cols / 128 * 4), st) != cudaSuccess ||
-            cudaMemsetAsync(w.xsig + int64_t(B) * (cols / 1024), 0, size_t(cols / 1024 * 4), st) != cudaSuccess)
-            return GALE_ERR_CUDA;
-        (void)bp;
+    int nwc = w4_nwc(B);
+    gale::W4Args a{};
+    int smem = 0;
+    if (!w4_plan(cols, B, nwc, a, smem)) {
+        nwc = 8;   // fewer partial-sum buffers leave room for wider rows
+        if (!w4_plan(cols, B, nwc, a, smem)) return GALE_ERR_UNSUPPORTED;
     }
-    const int64_t warps = int64_t(B) * (cols / 1024);
-    gale::w4_xprep_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, st>>>(x, B, cols, w.xd, w.xsum, w.xsig);
-    GALE_LAUNCH_CHECK();
     const uint8_t* qb = static_cast<const uint8_t*>(packed);
-    const __half* sb = reinterpret_cast<const __half*>(qb + L.s_offset);
-    const int np = (B + 1) / 2;
-    // shared memory: the activation digits of 2 np tokens, then the ring
-    // stages of the 8 warps, as many (2..4) as fit (16 warps with fewer stages
-    // each measured slower on the [65536 x 4096] case: 80 against 71 us)
-    const int xpitch = int(cols) + 16;
-    const int xbytes = 6 * np * xpitch;
-    auto stages_for = [&](int warps) {
-        int n = gale::kW4MaxStages;
-        while (n >= 2 && xbytes + warps * n * gale::kW4UnitBytes > gale::kW4SmemMax) --n;
-        return n;
-    };
-    const int nw = 8;
-    const int nst = stages_for(nw);
-    if (nst < 2) return GALE_ERR_UNSUPPORTED;
-    const int smem = xbytes + nw * nst * gale::kW4UnitBytes;
-    const int64_t ctas = (rows / 16 + nw - 1) / nw;
-    const unsigned grid = unsigned(ctas < gale::sm_count() ? ctas : gale::sm_count());
-    auto launch = [&](auto kern) {
+    a.q = qb;
+    a.s = reinterpret_cast<const __half*>(qb + L.s_offset);
+    a.x = x;
+    a.y = y;
+    a.status = static_cast<int32_t*>(ws);
+    a.rows = rows;
+    a.cols = cols;
+    a.B = B;
+    cudaStream_t st = gale::as_stream(stream);
+    const int64_t tiles = rows / 16;
+    const unsigned grid = unsigned(tiles < gale::sm_count() ? tiles : gale::sm_count());
+    auto launch = [&](auto kern, int threads) {
         // (set on every call: the attribute belongs to the current device)
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return false;
-        kern<<<grid, nw * 32, smem, st>>>(qb, sb, cols, B, w.xd, w.xsum, w.xsig, y, rows, nst, xpitch);
+        kern<<<grid, threads, smem, st>>>(a);
         return true;
     };
+    const int np = (B + 1) / 2;
+    const int nbw = a.uc / (64 * nwc);   // blocks of a warp's slice (nwc / 2 warps per group)
     bool ok = false;
-    if (np == 1) ok = launch(gale::w4_gemv_kernel<1, 8>);
-    else if (np == 2) ok = launch(gale::w4_gemv_kernel<2, 8>);
-    else if (np == 3) ok = launch(gale::w4_gemv_kernel<3, 8>);
-    else ok = launch(gale::w4_gemv_kernel<4, 8>);
+    auto by_np = [&](auto k1, auto k2, auto k3, auto k4) {
+        const int threads = (nwc + 1) * 32;
+        return np == 1 ? launch(k1, threads) : np == 2 ? launch(k2, threads) : np == 3 ? launch(k3, threads)
+                                                                                 : launch(k4, threads);
+    };
+    using namespace gale;
+    if (nwc == 16) {
+        if (nbw == 4)
+            ok = by_np(w4_gemv_kernel<1, 16, 4>, w4_gemv_kernel<2, 16, 4>, w4_gemv_kernel<3, 16, 4>,
+                       w4_gemv_kernel<4, 16, 4>);
+        else if (nbw == 2)
+            ok = by_np(w4_gemv_kernel<1, 16, 2>, w4_gemv_kernel<2, 16, 2>, w4_gemv_kernel<3, 16, 2>,
+                       w4_gemv_kernel<4, 16, 2>);
+        else
+            ok = by_np(w4_gemv_kernel<1, 16, 1>, w4_gemv_kernel<2, 16, 1>, w4_gemv_kernel<3, 16, 1>,
+                       w4_gemv_kernel<4, 16, 1>);
+    } else if (nbw == 8) {
+        ok = by_np(w4_gemv_kernel<1, 8, 8>, w4_gemv_kernel<2, 8, 8>, w4_gemv_kernel<3, 8, 8>, w4_gemv_kernel<4, 8, 8>);
+    } else if (nbw == 4) {
+        ok = by_np(w4_gemv_kernel<1, 8, 4>, w4_gemv_kernel<2, 8, 4>, w4_gemv_kernel<3, 8, 4>, w4_gemv_kernel<4, 8, 4>);
+    } else {
+        ok = by_np(w4_gemv_kernel<1, 8, 2>, w4_gemv_kernel<2, 8, 2>, w4_gemv_kernel<3, 8, 2>, w4_gemv_kernel<4, 8, 2>);
+    }
     if (!ok) return GALE_ERR_CUDA;
     GALE_LAUNCH_CHECK();
     return GALE_OK;

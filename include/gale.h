@@ -418,15 +418,19 @@ int gale_w4_quantize(const float* w, int64_t rows, int64_t cols, void* packed, v
  *   x      : device bf16 bits [B][cols]
  *   y      : device fp32 [B][rows] (overwritten)
  *   ws     : device, 256-byte aligned, gale_w4_workspace_size(rows, cols, B)
- *            bytes; needs no initialisation and holds nothing afterwards.
+ *            bytes (256); its first int32 is a sticky status word: the caller
+ *            sets it to 0 once, the call never clears it and writes
+ *            GALE_ERR_TIMEOUT there if a bounded wait inside the kernel ran
+ *            out (results are then undefined).
  * rows % 16 == 0, cols % 1024 == 0, 1 <= B <= 8, and the activation digits
- * 6 ceil(B/2) (cols + 16) bytes plus 67,584 bytes within 227 KB of shared
- * memory (GALE_ERR_UNSUPPORTED beyond: cols <= 6144 at 7-8 tokens, 8192 at
- * 5-6, 13312 at 3-4, 26624 at 1-2).  Activations are held in
- * fixed point per 1024 columns (21 bits, three int8 digits) and multiplied on
- * the int8 tensor cores with exact int32 sums; scales and sums in fp32.  Two
- * launches (activation digits, then one 16-row tile per CTA reading every
- * weight byte once for all B tokens).
+ * 6 ceil(B/2) (cols + 16) bytes plus two ring stages within 227 KB of shared
+ * memory (GALE_ERR_UNSUPPORTED beyond: cols <= 8192 at 7-8 tokens, 11264 at
+ * 5-6, 16384 at 3-4, 34816 at 1-2).  Activations are held in fixed point per
+ * 1024 columns (21 bits, three int8 digits, built inside the kernel) and
+ * multiplied on the int8 tensor cores with exact int32 sums; scales and sums
+ * in fp32.  One launch: a persistent CTA per SM streams its 16-row tiles by
+ * bulk copies through a ring of shared-memory stages, reading every weight
+ * byte once for all B tokens.
  * Errors: GALE_ERR_ARG (shape, NULL), GALE_ERR_ALIGN, GALE_ERR_WORKSPACE,
  * GALE_ERR_UNSUPPORTED (shared memory, above). */
 size_t gale_w4_workspace_size(int64_t rows, int64_t cols, int B);   /* 0 on invalid sizes */

@@ -45,9 +45,10 @@ def _gemv(buf_np, rows, cols, xbits):
     packed = to_dev(buf_np)
     x = to_dev(xbits.astype(np.uint16), torch.int16)
     y = torch.full((B, rows), float("nan"), device="cuda")
-    ws = torch.empty(G.gale_w4_workspace_size(rows, cols, B), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(G.gale_w4_workspace_size(rows, cols, B), dtype=torch.uint8, device="cuda")
     G.gale_w4_gemv(packed, rows, cols, x, y, ws)
     torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
     return y.cpu().numpy()
 
 
@@ -67,8 +68,14 @@ def test_w4_quantize_bit_exact(rows, cols, scale):
 
 
 @pytest.mark.parametrize("rows,cols,B", [(16, 1024, 1), (64, 2048, 2), (128, 4096, 3), (512, 4096, 8),
-                                         (48, 3072, 5), (2048, 4096, 1), (96, 8192, 4), (32, 1024, 7)])
+                                         (48, 3072, 5), (2048, 4096, 1), (96, 8192, 4), (32, 1024, 7),
+                                         (4752, 1024, 2), (32, 7168, 6), (16, 8192, 8), (48, 16384, 3),
+                                         (16, 34816, 1)])
 def test_w4_gemv_parity(rows, cols, B):
+    """Shapes: one tile (one CTA), more tiles than SMs with a ragged last
+    round (4752 rows = 297 tiles), rows of several units with a narrower last
+    unit (7168, 16384), and the widest rows the shared memory holds at 8 and
+    at 1 token."""
     w = _weights(rows, cols, 1000 + rows + B)
     q, s = W.w4_quantize(w)
     xbits, xv = gs.hidden_bf16(B, cols, tag=rows + cols + B)
@@ -89,9 +96,10 @@ def test_w4_gemv_full_shape_sampled_rows(B):
     xbits, xv = gs.hidden_bf16(B, cols, tag=17)
     x = to_dev(xbits.astype(np.uint16), torch.int16)
     y = torch.full((B, rows), float("nan"), device="cuda")
-    ws = torch.empty(G.gale_w4_workspace_size(rows, cols, B), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(G.gale_w4_workspace_size(rows, cols, B), dtype=torch.uint8, device="cuda")
     G.gale_w4_gemv(packed, rows, cols, x, y, ws)
     torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
     sel = np.r_[0:16, 30000:30016, rows - 16:rows]
     q, s = W.w4_quantize(w[torch.from_numpy(sel).cuda()].cpu().numpy())
     assert_tokens(y.cpu().numpy()[:, sel], W.w4_gemv(q, s, xv), what=f"w4 {rows}x{cols} B={B} sampled rows")
@@ -136,8 +144,8 @@ def test_w4_argument_errors():
     assert L.gale_w4_gemv(packed.data_ptr() + 16, rows, cols, x.data_ptr(), 1, y.data_ptr(), ws.data_ptr(),
                           ws.numel(), None) == G.GALE_ERR_ALIGN
     assert G.gale_w4_workspace_size(rows, 1000, 1) == 0
-    # beyond the shared-memory limit: 8 tokens of 7168 columns
-    c2 = 7168
+    # beyond the shared-memory limit: 8 tokens of 9216 columns
+    c2 = 9216
     x8 = torch.zeros((8, c2), dtype=torch.int16, device="cuda")
     y8 = torch.zeros((8, 16), device="cuda")
     ws8 = torch.empty(G.gale_w4_workspace_size(16, c2, 8), dtype=torch.uint8, device="cuda")
