@@ -525,6 +525,9 @@ int w4_nwc(int B) { return B >= 5 ? 8 : 16; }
 
 extern "C" size_t gale_w4_workspace_size(int64_t rows, int64_t cols, int B) {
     if (!w4_gemv_shape_ok(rows, cols, B)) return 0;
+    gale::W4Args a{};
+    int smem = 0;
+    if (!w4_plan(cols, B, w4_nwc(B), a, smem) && !w4_plan(cols, B, 8, a, smem)) return 0;   // unsupported
     return 256;   // the status word
 }
 

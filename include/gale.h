@@ -433,7 +433,8 @@ int gale_w4_quantize(const float* w, int64_t rows, int64_t cols, void* packed, v
  * byte once for all B tokens.
  * Errors: GALE_ERR_ARG (shape, NULL), GALE_ERR_ALIGN, GALE_ERR_WORKSPACE,
  * GALE_ERR_UNSUPPORTED (shared memory, above). */
-size_t gale_w4_workspace_size(int64_t rows, int64_t cols, int B);   /* 0 on invalid sizes */
+size_t gale_w4_workspace_size(int64_t rows, int64_t cols, int B);   /* host only; 0 on invalid or
+                                                                        unsupported sizes */
 int gale_w4_gemv(const void* packed, int64_t rows, int64_t cols, const uint16_t* x, int B, float* y, void* ws,
                  size_t ws_bytes, void* stream);
 

@@ -84,3 +84,16 @@ def test_workspace_size_and_layer_validation():
     rc = lib.gale_moe_forward(ctypes.byref(bad), None, None, None, 1, 6, None, 5, 0, ctypes.c_float(1e-6),
                               None, 0, None)
     assert rc == G.GALE_ERR_ARG
+
+
+def test_w4_supported_sizes():
+    """The 4-bit GEMV's documented limits, from the host-only workspace query:
+    the widest row (a multiple of 1024) whose activation digits and two ring
+    stages fit the shared memory, per token count, and 0 one step beyond."""
+    limits = {1: 34816, 2: 34816, 3: 16384, 4: 16384, 5: 11264, 6: 11264, 7: 8192, 8: 8192}
+    for B, cols in limits.items():
+        assert G.gale_w4_workspace_size(16, cols, B) == 256, (B, cols)
+        assert G.gale_w4_workspace_size(16, cols + 1024, B) == 0, (B, cols)
+    assert G.gale_w4_workspace_size(16, 4096, 9) == 0
+    assert G.gale_w4_workspace_size(24, 4096, 1) == 0
+    assert G.gale_w4_workspace_size(16, 1536, 1) == 0

@@ -148,7 +148,8 @@ def test_w4_argument_errors():
     c2 = 9216
     x8 = torch.zeros((8, c2), dtype=torch.int16, device="cuda")
     y8 = torch.zeros((8, 16), device="cuda")
-    ws8 = torch.empty(G.gale_w4_workspace_size(16, c2, 8), dtype=torch.uint8, device="cuda")
+    assert G.gale_w4_workspace_size(16, c2, 8) == 0
+    ws8 = torch.zeros(256, dtype=torch.uint8, device="cuda")
     p8 = torch.zeros(G.gale_w4_layout(16, c2).total, dtype=torch.uint8, device="cuda")
     assert L.gale_w4_gemv(p8.data_ptr(), 16, c2, x8.data_ptr(), 8, y8.data_ptr(), ws8.data_ptr(), ws8.numel(),
                           None) == G.GALE_ERR_UNSUPPORTED
