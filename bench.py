@@ -349,6 +349,8 @@ def run_gpu(args):
         for i in range(warmup):
             G.gale_w4_gemv(packed, W4_ROWS, D_MODEL, xs[i], y, ws)
         torch.cuda.synchronize()
+        if int(ws[:4].view(torch.int32).item()) != 0:
+            raise RuntimeError("4-bit GEMV status after warm-up")
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         for i in range(steps):
             flush.zero_()
