@@ -306,7 +306,13 @@ int gale_moe_forward_host(const gale_layer* layer, const uint16_t* x, const int3
  *         bytes; its first int32 is the status word
  * The batches of the streaming decode kernel (B <= 384, d_model <= 4096,
  * d_ff <= 2048), else GALE_ERR_UNSUPPORTED.  gale_expert_gemv is the
- * one-matrix call.
+ * one-matrix call.  One launch, asynchronous on `stream`; the workspace and
+ * out must not be in use by another call on another stream.
+ * Errors: GALE_ERR_ARG (layer descriptor, expert outside [0, n_experts),
+ * B < 1, NULL x or out), GALE_ERR_UNSUPPORTED (above), GALE_ERR_WORKSPACE,
+ * GALE_ERR_ALIGN (ws not 256-byte, x or out not 4-byte aligned),
+ * GALE_ERR_CUDA; on the device, GALE_ERR_TIMEOUT in the status word if a
+ * bounded wait ran out.
  * ------------------------------------------------------------------------- */
 size_t gale_expert_forward_workspace_size(const gale_layer* layer, int B);
 int gale_expert_forward(const gale_layer* layer, int expert, const float* x, int B, float* out, void* ws,
