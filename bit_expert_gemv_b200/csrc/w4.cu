@@ -78,9 +78,10 @@ __global__ void __launch_bounds__(256) w4_quantize_kernel(const float* __restric
 
 // Launch parameters of the GEMV.  Shared memory, in this order: nst ring
 // stages (the 16 code rows, then 16 scale rows of `spitch` bytes from byte
-// `sreg` of the stage), the activation digits (6 NP rows of `xpitch` bytes), the block sums
-// of X (int32 [2 NP][cols / 128]), 1 / S (fp32 [2 NP][cols / 1024]), the
-// per-warp partial sums (fp32 [2][NWC][NP][32]), then 2 nst mbarriers and an
+// `sreg` of the stage), the activation digits (6 NP rows of `xpitch` bytes),
+// the block sums of X (int32 [2 NP][cols / 128]), 1 / S (fp32
+// [2 NP][cols / 1024]), the per-warp partial sums (fp32 [2 consumer groups]
+// [2 alternating buffers][NWC / 2][NP][32]), then 2 nst mbarriers and an
 // abort flag.  Offsets in bytes from the start of dynamic shared memory.
 struct W4Args {
     const uint8_t* q;
@@ -163,9 +164,10 @@ __device__ __forceinline__ void w4_fail(const W4Args& a, volatile int* abort_fla
 // Persistent GEMV, one CTA per SM: CTA c owns the 16-row tiles c, c + grid,
 // ...; a tile is read as units of 16 rows x `uc` columns (the last unit of a
 // row may be narrower).  Warp NWC copies each unit into the next ring stage
-// with bulk copies (lane r < 16: code row r, `uc` / 2 contiguous bytes; lane
-// 16 + r: that row's `uc` / 128 scales), each row at a padded pitch so the
-// eight rows of an A fragment fall in distinct bank groups.  The NWC consumer
+// with bulk copies: when a tile is one unit, lanes 0-7 copy two whole rows
+// each and lane 8 the tile's scales; else lane r < 16 copies row r's segment
+// and lane 16 + r its scales.  The row placement (see W4Args) puts the eight
+// rows of an A fragment in distinct bank groups.  The NWC consumer
 // warps form two groups of NWG = NWC / 2 that take alternate tiles (group k:
 // the CTA's tiles k, k + 2, ...), so one group's per-unit hand-off overlaps
 // the other's arithmetic.  Warp w of a group multiplies columns
